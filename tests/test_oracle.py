@@ -1,0 +1,303 @@
+"""Pins for the CPU oracle (oracle/): checks against facts fixed outside it.
+
+Each test pins the oracle to something other than itself: hand-derived
+values (tests/golden/), a second literal implementation (tests/brute.py),
+library routines in special cases that reduce to them (PyTorch's causal
+scaled-dot-product attention and autograd, in fp64), calculus (finite
+differences, softmax sum identities) and structural facts (examples are
+independent; one-block and window-1 rules).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import brute
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def rand_case(rng, lengths, H, D, scale=1.0):
+    offs = np.zeros(len(lengths) + 1, dtype=np.int32)
+    offs[1:] = np.cumsum(lengths)
+    T = int(offs[-1])
+    q = rng.standard_normal((T, H, D)) * scale
+    k = rng.standard_normal((T, H, D)) * scale
+    v = rng.standard_normal((T, H, D))
+    do = rng.standard_normal((T, H, D))
+    return offs, q, k, v, do
+
+
+# ---------------------------------------------------------------- golden ---
+
+def load_masks():
+    tables, cur = [], None
+    with open(os.path.join(GOLDEN, "masks.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            if line.startswith("mask"):
+                _, L, b, w = line.split()
+                cur = (int(L), int(b), int(w), [])
+                tables.append(cur)
+            else:
+                cur[3].append([int(c) for c in line])
+    return tables
+
+
+@pytest.mark.parametrize("table", load_masks(), ids=lambda t: f"L{t[0]}_b{t[1]}_w{t[2]}")
+def test_mask_tables_by_hand(table):
+    """q = k = 0 makes every visible key equally likely; with one-hot values
+    the output row is 1/count at exactly the visible keys."""
+    L, block, window, rows = table
+    mask = np.array(rows, dtype=np.float64)
+    assert mask.shape == (L, L)
+    offs = np.array([0, L], dtype=np.int32)
+    q = np.zeros((L, 1, 1))
+    k = np.zeros((L, 1, 1))
+    v = np.eye(L).reshape(L, 1, L)
+    q = np.zeros((L, 1, L))
+    k = np.zeros((L, 1, L))
+    out, lse = oracle.fwd(offs, q, k, v, block, window)
+    count = mask.sum(1)
+    np.testing.assert_array_equal(out[:, 0, :] > 0, mask > 0)
+    np.testing.assert_allclose(out[:, 0, :], mask / count[:, None], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse[0], np.log(count), rtol=0, atol=1e-15)
+
+
+def load_worked():
+    vals = {}
+    with open(os.path.join(GOLDEN, "worked_example.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            w, name, *xs = line.split()
+            vals[(int(w), name)] = np.array([eval(x, {"math": math}) for x in xs])
+    return vals
+
+
+@pytest.mark.parametrize("window", [1, 2])
+def test_worked_example_by_hand(window):
+    g = load_worked()
+    offs = np.array([0, 3], dtype=np.int32)
+    q = np.ones((3, 1, 1))
+    k = np.array([0.0, math.log(3), math.log(2)]).reshape(3, 1, 1)
+    v = np.array([4.0, 8.0, -1.0]).reshape(3, 1, 1)
+    do = np.ones((3, 1, 1))
+    out, lse = oracle.fwd(offs, q, k, v, 2, window)
+    dq, dk, dv = oracle.bwd(offs, q, k, v, do, 2, window)
+    for name, got in [("out", out[:, 0, 0]), ("lse", lse[0]), ("dq", dq[:, 0, 0]),
+                      ("dk", dk[:, 0, 0]), ("dv", dv[:, 0, 0])]:
+        np.testing.assert_allclose(got, g[(window, name)], rtol=0, atol=1e-14, err_msg=name)
+
+
+# ----------------------------------------------------------- brute force ---
+
+@pytest.mark.parametrize("seed", range(6))
+def test_matches_literal_brute_force(seed):
+    rng = np.random.default_rng(100 + seed)
+    block = [1, 2, 3, 5, 8, 4][seed]
+    window = [1, 2, 3, 2, 1, 3][seed]
+    D = [1, 4, 3, 4, 1, 2][seed]
+    H = 1 + seed % 2
+    lengths = [int(x) for x in rng.integers(0, 40, size=3)] + [1]
+    offs, q, k, v, _ = rand_case(rng, lengths, H, D)
+    out, lse = oracle.fwd(offs, q, k, v, block, window)
+    bout, blse = brute.fwd(offs, q, k, v, block, window)
+    np.testing.assert_allclose(out, np.array(bout).reshape(out.shape), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, np.array(blse).reshape(lse.shape), rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------- library special cases ---
+
+def sdpa_causal(q, k, v, dout):
+    """PyTorch causal attention (fp64) for one example [L, H, D]; returns out and grads."""
+    tq, tk, tv = (torch.tensor(x.transpose(1, 0, 2), dtype=torch.float64, requires_grad=True)
+                  for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True)
+    o.backward(torch.tensor(dout.transpose(1, 0, 2)))
+    t = lambda x: x.detach().numpy().transpose(1, 0, 2)
+    return t(o), t(tq.grad), t(tk.grad), t(tv.grad)
+
+
+@pytest.mark.parametrize("block,window,lengths", [
+    (16, 4, [64, 37, 1, 50]),      # window * block = 64 >= every length
+    (64, 1, [64, 10, 33]),          # one block covers everything
+    (7, 10, [70, 69, 3]),
+])
+def test_full_causal_when_window_covers_sequence(block, window, lengths):
+    rng = np.random.default_rng(7)
+    offs, q, k, v, do = rand_case(rng, lengths, 3, 8)
+    out, _ = oracle.fwd(offs, q, k, v, block, window)
+    dq, dk, dv = oracle.bwd(offs, q, k, v, do, block, window)
+    for e in range(len(lengths)):
+        s, t = offs[e], offs[e + 1]
+        if t == s:
+            continue
+        ro, rdq, rdk, rdv = sdpa_causal(q[s:t], k[s:t], v[s:t], do[s:t])
+        np.testing.assert_allclose(out[s:t], ro, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dq[s:t], rdq, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dk[s:t], rdk, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dv[s:t], rdv, rtol=0, atol=1e-12)
+
+
+def test_window1_is_causal_attention_per_block():
+    """window = 1: the pages' independent blocks, each a causal attention of its own."""
+    rng = np.random.default_rng(8)
+    block = 8
+    lengths = [29, 8, 17]
+    offs, q, k, v, do = rand_case(rng, lengths, 2, 4)
+    out, _ = oracle.fwd(offs, q, k, v, block, 1)
+    dq, dk, dv = oracle.bwd(offs, q, k, v, do, block, 1)
+    for e in range(len(lengths)):
+        for c0 in range(offs[e], offs[e + 1], block):
+            c1 = min(c0 + block, offs[e + 1])
+            ro, rdq, rdk, rdv = sdpa_causal(q[c0:c1], k[c0:c1], v[c0:c1], do[c0:c1])
+            np.testing.assert_allclose(out[c0:c1], ro, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(dq[c0:c1], rdq, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(dk[c0:c1], rdk, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(dv[c0:c1], rdv, rtol=0, atol=1e-12)
+
+
+def test_short_example_needs_one_block():
+    """An example no longer than one block gives the same result for every window."""
+    rng = np.random.default_rng(9)
+    offs, q, k, v, do = rand_case(rng, [16, 5, 1], 2, 4)
+    ref = oracle.fwd(offs, q, k, v, 16, 1)
+    refg = oracle.bwd(offs, q, k, v, do, 16, 1)
+    for window in (2, 3, 7):
+        out, lse = oracle.fwd(offs, q, k, v, 16, window)
+        np.testing.assert_array_equal(out, ref[0])
+        np.testing.assert_array_equal(lse, ref[1])
+        for a, b in zip(oracle.bwd(offs, q, k, v, do, 16, window), refg):
+            np.testing.assert_array_equal(a, b)
+
+
+# ------------------------------------------------------------ closed form ---
+
+def test_first_row_of_each_block_has_one_key():
+    """With window 1 the first query of every block sees only itself: o = v
+    exactly and lse = its own scaled score."""
+    rng = np.random.default_rng(10)
+    block = 5
+    offs, q, k, v, _ = rand_case(rng, [23, 5, 11], 2, 6)
+    out, lse = oracle.fwd(offs, q, k, v, block, 1)
+    for e in range(3):
+        for i in range(0, offs[e + 1] - offs[e], block):
+            r = offs[e] + i
+            np.testing.assert_array_equal(out[r], v[r])
+            for h in range(2):
+                assert lse[h, r] == pytest.approx(q[r, h] @ k[r, h] / math.sqrt(6), abs=1e-14)
+
+
+def test_gradient_sum_identities():
+    """Softmax rows sum to one, so sum_j dv_j = sum_i dO_i; and each row of ds
+    sums to zero, so sum_j dk_j = 0 (per example and head)."""
+    rng = np.random.default_rng(11)
+    offs, q, k, v, do = rand_case(rng, [40, 13, 64], 2, 5)
+    dq, dk, dv = oracle.bwd(offs, q, k, v, do, 8, 2)
+    for e in range(3):
+        s, t = offs[e], offs[e + 1]
+        np.testing.assert_allclose(dv[s:t].sum(0), do[s:t].sum(0), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dk[s:t].sum(0), 0.0, rtol=0, atol=1e-12)
+
+
+def test_finite_differences():
+    rng = np.random.default_rng(12)
+    block, window = 3, 2
+    offs, q, k, v, do = rand_case(rng, [9, 4], 1, 3)
+    dq, dk, dv = oracle.bwd(offs, q, k, v, do, block, window)
+    eps = 1e-6
+
+    def f(q_, k_, v_):
+        return float(np.sum(oracle.fwd(offs, q_, k_, v_, block, window)[0] * do))
+
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            num[idx] = (f(*args_p) - f(*args_m)) / (2 * eps)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8, err_msg=name)
+
+
+# ------------------------------------------------------------- structure ---
+
+def test_jagged_batch_equals_separate_runs_and_permutes():
+    rng = np.random.default_rng(13)
+    lengths = [31, 0, 17, 45]
+    offs, q, k, v, do = rand_case(rng, lengths, 2, 4)
+    out, lse = oracle.fwd(offs, q, k, v, 8, 2)
+    dq, dk, dv = oracle.bwd(offs, q, k, v, do, 8, 2)
+    for e in range(len(lengths)):
+        s, t = offs[e], offs[e + 1]
+        one = np.array([0, t - s], dtype=np.int32)
+        o1, l1 = oracle.fwd(one, q[s:t], k[s:t], v[s:t], 8, 2)
+        np.testing.assert_array_equal(out[s:t], o1)
+        np.testing.assert_array_equal(lse[:, s:t], l1)
+        g1 = oracle.bwd(one, q[s:t], k[s:t], v[s:t], do[s:t], 8, 2)
+        for a, b in zip((dq, dk, dv), g1):
+            np.testing.assert_array_equal(a[s:t], b)
+    perm = [3, 0, 2, 1]
+    idx = np.concatenate([np.arange(offs[e], offs[e + 1]) for e in perm])
+    poffs = np.zeros(5, dtype=np.int32)
+    poffs[1:] = np.cumsum([lengths[e] for e in perm])
+    po, pl = oracle.fwd(poffs, q[idx], k[idx], v[idx], 8, 2)
+    np.testing.assert_array_equal(po, out[idx])
+    np.testing.assert_array_equal(pl, lse[:, idx])
+
+
+def test_skip_passes_values_through():
+    rng = np.random.default_rng(14)
+    offs, q, k, v, do = rand_case(rng, [20, 9, 33], 2, 4)
+    skip = np.array([1, 0, 1], dtype=np.uint8)
+    out, lse = oracle.fwd(offs, q, k, v, 4, 2, skip=skip)
+    dq, dk, dv = oracle.bwd(offs, q, k, v, do, 4, 2, skip=skip)
+    ref_o, ref_l = oracle.fwd(offs, q, k, v, 4, 2)
+    ref_g = oracle.bwd(offs, q, k, v, do, 4, 2)
+    for e in range(3):
+        s, t = offs[e], offs[e + 1]
+        if skip[e]:
+            np.testing.assert_array_equal(out[s:t], v[s:t])
+            np.testing.assert_array_equal(lse[:, s:t], 0.0)
+            np.testing.assert_array_equal(dq[s:t], 0.0)
+            np.testing.assert_array_equal(dk[s:t], 0.0)
+            np.testing.assert_array_equal(dv[s:t], do[s:t])
+        else:
+            np.testing.assert_array_equal(out[s:t], ref_o[s:t])
+            np.testing.assert_array_equal(lse[:, s:t], ref_l[:, s:t])
+            for a, b in zip((dq, dk, dv), ref_g):
+                np.testing.assert_array_equal(a[s:t], b[s:t])
+
+
+def test_sampled_rows_match_full_computation():
+    rng = np.random.default_rng(15)
+    L = 57
+    offs, q, k, v, do = rand_case(rng, [L], 3, 4)
+    out, lse = oracle.fwd(offs, q, k, v, 6, 3)
+    dq, dk, dv = oracle.bwd(offs, q, k, v, do, 6, 3)
+    rows = [0, 5, 6, 17, 56, 30]
+    for h in range(3):
+        r = oracle.rows(q, k, v, h, rows, 6, 3, dout_e=do, want=("out", "lse", "dq", "dk", "dv"))
+        np.testing.assert_allclose(r["out"], out[rows, h], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(r["lse"], lse[h, rows], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(r["dq"], dq[rows, h], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(r["dk"], dk[rows, h], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(r["dv"], dv[rows, h], rtol=0, atol=1e-13)
+
+
+def test_thread_count_does_not_change_bits():
+    rng = np.random.default_rng(16)
+    offs, q, k, v, do = rand_case(rng, [30, 44, 12, 50], 3, 4)
+    a = oracle.fwd(offs, q, k, v, 8, 2, nthreads=1) + oracle.bwd(offs, q, k, v, do, 8, 2, nthreads=1)
+    b = oracle.fwd(offs, q, k, v, 8, 2, nthreads=5) + oracle.bwd(offs, q, k, v, do, 8, 2, nthreads=5)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
