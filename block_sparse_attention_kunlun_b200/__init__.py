@@ -1,0 +1,204 @@
+"""Block attention for NVIDIA B200 (sm_100a).
+
+Python binding over the C ABI in ``include/ba.h`` (``libba.so`` in this
+package directory, built by ``build.py``). The functions named like the C
+entry points (``ba_fwd``, ``ba_bwd``, ...) marshal torch tensors into
+pointers and call the library; every step of the computation runs in the
+library's CUDA kernels. There is no CPU path: if the library is missing or
+the device is not an sm_100 GPU, the calls raise.
+
+Tensors: q, k, v, out, dout, dq, dk, dv are contiguous CUDA tensors of shape
+``[total_tokens, heads, head_dim]`` (bfloat16 or float32); lse is float32
+``[heads, total_tokens]``; seq_offsets is int32 ``[batch + 1]`` on the
+device; skip is uint8 ``[batch]`` on the device or None.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "BAError", "ba_fwd", "ba_bwd", "ba_fwd_workspace_size", "ba_bwd_workspace_size",
+    "ba_device_status", "ba_set_profile_events", "ba_status_string", "ba_version", "block_attention_fwd",
+    "block_attention_bwd", "library_path",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libba.so")
+
+BA_OK, BA_ERR_INVALID_ARG, BA_ERR_UNSUPPORTED, BA_ERR_CUDA, BA_ERR_TIMEOUT = range(5)
+BA_F32, BA_BF16 = 0, 1
+_DTYPES = {torch.float32: BA_F32, torch.bfloat16: BA_BF16}
+
+
+class BAProblem(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("total_tokens", ctypes.c_int32),
+                ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("dtype", ctypes.c_int)]
+
+
+class BAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {ba_status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                          "`python -m block_sparse_attention_kunlun_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, i32 = ctypes.c_void_p, ctypes.c_int32
+    prob = ctypes.POINTER(BAProblem)
+    lib.ba_fwd_workspace_size.argtypes = [prob, i32, i32]
+    lib.ba_fwd_workspace_size.restype = ctypes.c_size_t
+    lib.ba_bwd_workspace_size.argtypes = [prob, i32, i32]
+    lib.ba_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.ba_fwd.argtypes = [prob, P, P, P, P, i32, i32, P, P, P, P, ctypes.c_size_t, P]
+    lib.ba_fwd.restype = ctypes.c_int
+    lib.ba_bwd.argtypes = [prob, P, P, P, P, P, P, P, i32, i32, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.ba_bwd.restype = ctypes.c_int
+    lib.ba_device_status.argtypes = [P, P]
+    lib.ba_device_status.restype = ctypes.c_int
+    lib.ba_status_string.argtypes = [ctypes.c_int]
+    lib.ba_status_string.restype = ctypes.c_char_p
+    lib.ba_set_profile_events.argtypes = [i32, P, P]
+    lib.ba_set_profile_events.restype = ctypes.c_int
+    lib.ba_version.argtypes = []
+    lib.ba_version.restype = ctypes.c_int32
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def make_problem(q: torch.Tensor, seq_offsets: torch.Tensor) -> BAProblem:
+    if q.dim() != 3:
+        raise ValueError("q must be [total_tokens, heads, head_dim]")
+    if q.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    T, H, D = q.shape
+    return BAProblem(int(seq_offsets.numel()) - 1, T, H, D, _DTYPES[q.dtype])
+
+
+def ba_status_string(status: int) -> str:
+    return _load().ba_status_string(int(status)).decode()
+
+
+def ba_version() -> int:
+    return int(_load().ba_version())
+
+
+def ba_fwd_workspace_size(problem: BAProblem, block: int, window: int) -> int:
+    return int(_load().ba_fwd_workspace_size(ctypes.byref(problem), int(block), int(window)))
+
+
+def ba_bwd_workspace_size(problem: BAProblem, block: int, window: int) -> int:
+    return int(_load().ba_bwd_workspace_size(ctypes.byref(problem), int(block), int(window)))
+
+
+def ba_fwd(problem, q, k, v, seq_offsets, block, window, skip, out, lse, workspace,
+           workspace_bytes=None, stream=None) -> int:
+    """Direct call of the C entry point; returns its status code."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(_load().ba_fwd(ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets),
+                              int(block), int(window), _ptr(skip), _ptr(out), _ptr(lse),
+                              _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def ba_bwd(problem, q, k, v, out, lse, dout, seq_offsets, block, window, skip, dq, dk, dv,
+           workspace, workspace_bytes=None, stream=None) -> int:
+    """Direct call of the C entry point; returns its status code."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(_load().ba_bwd(ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                              _ptr(dout), _ptr(seq_offsets), int(block), int(window), _ptr(skip),
+                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), int(workspace_bytes),
+                              _stream(stream)))
+
+
+def ba_set_profile_events(which: int, start=None, stop=None) -> int:
+    """Record torch.cuda.Event ``start``/``stop`` around the attention kernel of
+    every later ba_fwd (which=0) or ba_bwd (which=1) call from this thread."""
+    s = start.cuda_event if start is not None else None
+    e = stop.cuda_event if stop is not None else None
+    return int(_load().ba_set_profile_events(int(which), s, e))
+
+
+def ba_device_status(workspace, stream=None) -> int:
+    return int(_load().ba_device_status(_ptr(workspace), _stream(stream)))
+
+
+def _check_inputs(q, k, v, seq_offsets):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError(f"{name} must match q in shape and dtype")
+    if seq_offsets.dtype != torch.int32 or not seq_offsets.is_cuda:
+        raise ValueError("seq_offsets must be an int32 CUDA tensor")
+
+
+def workspace_for(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte-aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def block_attention_fwd(q, k, v, seq_offsets, block, window, skip=None, out=None, lse=None,
+                        workspace=None, stream=None):
+    """Allocates out/lse (and a workspace) with torch and runs ba_fwd."""
+    _check_inputs(q, k, v, seq_offsets)
+    prob = make_problem(q, seq_offsets)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = workspace_for(ba_fwd_workspace_size(prob, block, window), q.device)
+    st = ba_fwd(prob, q, k, v, seq_offsets, block, window, skip, out, lse, workspace, stream=stream)
+    if st != BA_OK:
+        raise BAError(st, "ba_fwd")
+    return out, lse
+
+
+def block_attention_bwd(q, k, v, out, lse, dout, seq_offsets, block, window, skip=None,
+                        dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Allocates dq/dk/dv (and a workspace) with torch and runs ba_bwd."""
+    _check_inputs(q, k, v, seq_offsets)
+    prob = make_problem(q, seq_offsets)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if workspace is None:
+        workspace = workspace_for(ba_bwd_workspace_size(prob, block, window), q.device)
+    st = ba_bwd(prob, q, k, v, out, lse, dout, seq_offsets, block, window, skip, dq, dk, dv,
+                workspace, stream=stream)
+    if st != BA_OK:
+        raise BAError(st, "ba_bwd")
+    return dq, dk, dv

@@ -1,0 +1,275 @@
+// The library's C ABI (declared in include/ba.h): host-side argument checks,
+// workspace carving, TMA descriptor encoding and the launch sequence.
+//
+//   ba_fwd: worklist -> skip passthrough (if any flags) -> forward kernel
+//           (tcgen05 for bf16, SIMT for fp32)
+//   ba_bwd: worklist -> Delta and dq-accumulator reset -> skip passthrough ->
+//           backward kernel -> dq conversion (bf16) or direct dq (fp32)
+// Nothing here allocates, synchronises or falls back to another device.
+#include "ba.h"
+#include "ba_common.cuh"
+#include "ba_kernels.cuh"
+
+#include <atomic>
+#include <cmath>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+namespace {
+
+using namespace ba;
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_num_sms[kMaxDevices];
+std::atomic<int> g_cc_major[kMaxDevices];
+
+bool device_info(int &num_sms, int &cc_major)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    if (dev < kMaxDevices && g_num_sms[dev].load() > 0) {
+        num_sms = g_num_sms[dev].load();
+        cc_major = g_cc_major[dev].load();
+        return true;
+    }
+    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+    if (cudaDeviceGetAttribute(&cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+    if (dev < kMaxDevices) {
+        g_cc_major[dev].store(cc_major);
+        g_num_sms[dev].store(num_sms);
+    }
+    return true;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static std::atomic<void *> fn{nullptr};
+    void *f = fn.load();
+    if (!f) {
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn.store(f);
+    }
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+}
+
+// 2-D view [total_tokens, heads * head_dim] of a bf16 tensor, boxes of 128
+// rows x 64 columns (128 bytes) with the 128-byte swizzle the MMA
+// descriptors expect; rows past the end read as zeros.
+bool encode_bf16_rows(CUtensorMap *map, const void *base, int64_t T, int64_t H, int64_t D)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cuuint64_t(H * D), cuuint64_t(T)};
+    cuuint64_t strides[1] = {cuuint64_t(H * D * 2)};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool head_dim_supported(const ba_problem &p)
+{
+    if (p.dtype == BA_BF16) return p.head_dim == 64 || p.head_dim == 128;
+    if (p.dtype == BA_F32) return p.head_dim == 32 || p.head_dim == 64;
+    return false;
+}
+
+ba_status check_problem(const ba_problem *p, int32_t block, int32_t window)
+{
+    if (!p) return BA_ERR_INVALID_ARG;
+    if (p->batch < 0 || p->total_tokens < 0 || p->heads < 1 || p->head_dim < 1 || block < 1 || window < 1)
+        return BA_ERR_INVALID_ARG;
+    if (p->dtype != BA_F32 && p->dtype != BA_BF16) return BA_ERR_INVALID_ARG;
+    if (p->batch == 0 && p->total_tokens != 0) return BA_ERR_INVALID_ARG;
+    // element offsets of one tensor must stay below 2^62 and rows below 2^31
+    if (int64_t(p->heads) * p->head_dim > (int64_t(1) << 24)) return BA_ERR_UNSUPPORTED;
+    if (!head_dim_supported(*p)) return BA_ERR_UNSUPPORTED;
+    return BA_OK;
+}
+
+bool tensor_ok(const void *t, int64_t T) { return T == 0 || (t && aligned(t, 16)); }
+
+Problem make_problem(const ba_problem &pp, const int32_t *offs, const uint8_t *skip, int32_t block, int32_t window,
+                     void *workspace, const WorkspaceLayout &lay)
+{
+    Problem p;
+    p.seq_offsets = offs;
+    p.skip = skip;
+    p.tile_prefix = reinterpret_cast<const int32_t *>(static_cast<uint8_t *>(workspace) + lay.tile_prefix);
+    p.status = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + lay.status);
+    p.batch = pp.batch;
+    p.total_tokens = pp.total_tokens;
+    p.heads = pp.heads;
+    p.head_dim = pp.head_dim;
+    p.block = block;
+    p.window = window;
+    p.scale = float(1.0 / std::sqrt(double(pp.head_dim)));
+    return p;
+}
+
+thread_local cudaEvent_t t_prof[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+
+cudaError_t prof_mark(int which, int edge, cudaStream_t stream)
+{
+    cudaEvent_t e = t_prof[which][edge];
+    return e ? cudaEventRecord(e, stream) : cudaSuccess;
+}
+
+#define BA_TRY(expr)                                                                                      \
+    do {                                                                                                  \
+        if ((expr) != cudaSuccess) return BA_ERR_CUDA;                                                    \
+    } while (0)
+
+} // namespace
+
+extern "C" {
+
+size_t ba_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
+{
+    if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
+    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, false, false).total;
+}
+
+size_t ba_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
+{
+    if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
+    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, true, p->dtype == BA_BF16).total;
+}
+
+ba_status ba_fwd(const ba_problem *pp, const void *q, const void *k, const void *v, const int32_t *seq_offsets,
+                 int32_t block, int32_t window, const uint8_t *skip, void *out, float *lse, void *workspace,
+                 size_t workspace_bytes, ba_stream_t stream_)
+{
+    ba_status st = check_problem(pp, block, window);
+    if (st != BA_OK) return st;
+    const ba_problem &P = *pp;
+    const int64_t T = P.total_tokens;
+    if (!seq_offsets || !aligned(seq_offsets, 4) || !tensor_ok(q, T) || !tensor_ok(k, T) || !tensor_ok(v, T) ||
+        !tensor_ok(out, T) || (T > 0 && (!lse || !aligned(lse, 4))))
+        return BA_ERR_INVALID_ARG;
+    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, false, false);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total) return BA_ERR_INVALID_ARG;
+    int num_sms = 0, cc = 0;
+    if (!device_info(num_sms, cc)) return BA_ERR_CUDA;
+    if (P.dtype == BA_BF16 && cc != 10) return BA_ERR_UNSUPPORTED;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+
+    const Problem p = make_problem(P, seq_offsets, skip, block, window, workspace, lay);
+    BA_TRY(launch_worklist(p, stream));
+    if (T == 0) return BA_OK;
+    const size_t esz = P.dtype == BA_BF16 ? 2 : 4;
+    BA_TRY(launch_skip_fwd(p, esz, v, out, lse, stream));
+    if (P.dtype == BA_F32) {
+        BA_TRY(prof_mark(0, 0, stream));
+        BA_TRY(launch_fwd_f32(p, static_cast<const float *>(q), static_cast<const float *>(k),
+                              static_cast<const float *>(v), static_cast<float *>(out), lse, num_sms, stream));
+        BA_TRY(prof_mark(0, 1, stream));
+        return BA_OK;
+    }
+    CUtensorMap tq, tk, tv;
+    if (!encode_bf16_rows(&tq, q, T, P.heads, P.head_dim) || !encode_bf16_rows(&tk, k, T, P.heads, P.head_dim) ||
+        !encode_bf16_rows(&tv, v, T, P.heads, P.head_dim))
+        return BA_ERR_CUDA;
+    BA_TRY(prof_mark(0, 0, stream));
+    if (P.head_dim == 64) BA_TRY(launch_fwd_bf16_sm100<64>(tq, tk, tv, p, out, lse, num_sms, stream));
+    else BA_TRY(launch_fwd_bf16_sm100<128>(tq, tk, tv, p, out, lse, num_sms, stream));
+    BA_TRY(prof_mark(0, 1, stream));
+    return BA_OK;
+}
+
+ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void *v, const void *out,
+                 const float *lse, const void *dout, const int32_t *seq_offsets, int32_t block, int32_t window,
+                 const uint8_t *skip, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                 ba_stream_t stream_)
+{
+    ba_status st = check_problem(pp, block, window);
+    if (st != BA_OK) return st;
+    const ba_problem &P = *pp;
+    const int64_t T = P.total_tokens;
+    if (!seq_offsets || !aligned(seq_offsets, 4) || !tensor_ok(q, T) || !tensor_ok(k, T) || !tensor_ok(v, T) ||
+        !tensor_ok(out, T) || !tensor_ok(dout, T) || !tensor_ok(dq, T) || !tensor_ok(dk, T) || !tensor_ok(dv, T) ||
+        (T > 0 && (!lse || !aligned(lse, 4))))
+        return BA_ERR_INVALID_ARG;
+    const bool bf16 = P.dtype == BA_BF16;
+    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, true, bf16);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total) return BA_ERR_INVALID_ARG;
+    int num_sms = 0, cc = 0;
+    if (!device_info(num_sms, cc)) return BA_ERR_CUDA;
+    if (bf16 && cc != 10) return BA_ERR_UNSUPPORTED;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+
+    const Problem p = make_problem(P, seq_offsets, skip, block, window, workspace, lay);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *delta = reinterpret_cast<float *>(ws + lay.delta);
+    float *dq_acc = bf16 ? reinterpret_cast<float *>(ws + lay.dq_acc) : nullptr;
+    BA_TRY(launch_worklist(p, stream));
+    if (T == 0) return BA_OK;
+    const size_t esz = bf16 ? 2 : 4;
+    if (bf16) BA_TRY(launch_bwd_pre<__nv_bfloat16>(p, out, dout, delta, dq_acc, num_sms, stream));
+    else BA_TRY(launch_bwd_pre<float>(p, out, dout, delta, nullptr, num_sms, stream));
+    BA_TRY(launch_skip_bwd(p, esz, dout, bf16 ? nullptr : dq, dk, dv, stream));
+    if (!bf16) {
+        BA_TRY(prof_mark(1, 0, stream));
+        BA_TRY(launch_bwd_f32(p, static_cast<const float *>(q), static_cast<const float *>(k),
+                              static_cast<const float *>(v), static_cast<const float *>(dout), lse, delta,
+                              static_cast<float *>(dq), static_cast<float *>(dk), static_cast<float *>(dv), num_sms,
+                              stream));
+        BA_TRY(prof_mark(1, 1, stream));
+        return BA_OK;
+    }
+    CUtensorMap tq, tk, tv, tdo;
+    if (!encode_bf16_rows(&tq, q, T, P.heads, P.head_dim) || !encode_bf16_rows(&tk, k, T, P.heads, P.head_dim) ||
+        !encode_bf16_rows(&tv, v, T, P.heads, P.head_dim) || !encode_bf16_rows(&tdo, dout, T, P.heads, P.head_dim))
+        return BA_ERR_CUDA;
+    BA_TRY(prof_mark(1, 0, stream));
+    if (P.head_dim == 64)
+        BA_TRY(launch_bwd_bf16_sm100<64>(tq, tk, tv, tdo, p, lse, delta, dq_acc, dk, dv, num_sms, stream));
+    else
+        BA_TRY(launch_bwd_bf16_sm100<128>(tq, tk, tv, tdo, p, lse, delta, dq_acc, dk, dv, num_sms, stream));
+    BA_TRY(prof_mark(1, 1, stream));
+    BA_TRY(launch_dq_convert<__nv_bfloat16>(p, dq_acc, dq, num_sms, stream));
+    return BA_OK;
+}
+
+ba_status ba_device_status(const void *workspace, ba_stream_t stream_)
+{
+    if (!workspace) return BA_ERR_INVALID_ARG;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int word = 0;
+    if (cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return BA_ERR_CUDA;
+    return (word & kStatusTimeout) ? BA_ERR_TIMEOUT : BA_OK;
+}
+
+ba_status ba_set_profile_events(int32_t which, void *start, void *stop)
+{
+    if (which != 0 && which != 1) return BA_ERR_INVALID_ARG;
+    t_prof[which][0] = static_cast<cudaEvent_t>(start);
+    t_prof[which][1] = static_cast<cudaEvent_t>(stop);
+    return BA_OK;
+}
+
+const char *ba_status_string(ba_status s)
+{
+    switch (s) {
+    case BA_OK: return "ok";
+    case BA_ERR_INVALID_ARG: return "invalid argument";
+    case BA_ERR_UNSUPPORTED: return "unsupported combination";
+    case BA_ERR_CUDA: return "CUDA error";
+    case BA_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+int32_t ba_version(void) { return 100; }
+
+} // extern "C"

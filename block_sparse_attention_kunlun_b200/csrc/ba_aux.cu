@@ -1,0 +1,251 @@
+// Small memory-bound kernels around the attention kernels:
+//   worklist_kernel   per-example count of live 128-row tiles -> exclusive
+//                     prefix sum (the persistent kernels' work list); resets
+//                     the status word
+//   bwd_pre_kernel    Delta = rowsum(dout * out) in fp32; zeroes the fp32 dq
+//                     accumulator
+//   dq_convert_kernel dq = scale * dq_acc, transposed from [H, T, D] to
+//                     [T, H, D] and rounded to the output dtype
+//   skip_*_kernel     component skip: flagged examples pass v through
+//                     ("Meta Scales GEM Ads Model Across Platforms and
+//                     Thousands of GPUs", section "Kunlun changes how GEM
+//                     scales": sequence modules bypassed selectively)
+#include "ba_common.cuh"
+#include "ba_kernels.cuh"
+
+#include <cuda_bf16.h>
+
+namespace ba {
+
+namespace {
+
+__device__ __forceinline__ int32_t live_tiles(const int32_t *offs, const uint8_t *skip, int32_t b)
+{
+    if (skip && skip[b]) return 0;
+    const int32_t L = offs[b + 1] - offs[b];
+    return L > 0 ? (L + kTile - 1) / kTile : 0;
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+} // namespace
+
+__global__ void __launch_bounds__(kWorklistThreads)
+    worklist_kernel(const int32_t *__restrict__ offs, const uint8_t *__restrict__ skip, int32_t batch,
+                    int32_t *__restrict__ tile_prefix, int *__restrict__ status)
+{
+    __shared__ int32_t warp_tot[kWorklistThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int per = (batch + kWorklistThreads - 1) / kWorklistThreads;
+    const int b0 = tid * per;
+    const int b1 = min(batch, b0 + per);
+    int32_t local = 0;
+    for (int b = b0; b < b1; ++b) local += live_tiles(offs, skip, b);
+    // inclusive scan within the warp, then across warp totals
+    int32_t incl = local;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += y;
+    }
+    if (lane == 31) warp_tot[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        int32_t w = warp_tot[lane];
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, w, d);
+            if (lane >= d) w += y;
+        }
+        warp_tot[lane] = w; // inclusive over warps
+    }
+    __syncthreads();
+    int32_t run = incl - local + (wid > 0 ? warp_tot[wid - 1] : 0);
+    for (int b = b0; b < b1; ++b) {
+        tile_prefix[b] = run;
+        run += live_tiles(offs, skip, b);
+    }
+    if (tid == kWorklistThreads - 1) {
+        tile_prefix[batch] = warp_tot[kWorklistThreads / 32 - 1];
+        *status = 0;
+    }
+}
+
+// One warp per (token, head) row.
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+    bwd_pre_kernel(const T *__restrict__ out, const T *__restrict__ dout, int32_t total_tokens,
+                   int32_t heads, float *__restrict__ delta, float *__restrict__ dq_acc)
+{
+    constexpr int PER = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t nrows = int64_t(total_tokens) * heads;
+    const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t rw = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); rw < nrows; rw += wstride) {
+        const int64_t t = rw / heads, h = rw % heads;
+        const T *o = out + rw * D + lane * PER;
+        const T *g = dout + rw * D + lane * PER;
+        float acc = 0.f;
+#pragma unroll
+        for (int x = 0; x < PER; ++x) acc += to_f32(o[x]) * to_f32(g[x]);
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
+        const int64_t hr = h * total_tokens + t;
+        if (lane == 0) delta[hr] = acc;
+        if (dq_acc) {
+            float *z = dq_acc + hr * D + lane * PER;
+#pragma unroll
+            for (int x = 0; x < PER; ++x) z[x] = 0.f;
+        }
+    }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+    dq_convert_kernel(const float *__restrict__ dq_acc, int32_t total_tokens, int32_t heads, float scale,
+                      T *__restrict__ dq)
+{
+    constexpr int PER = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t nrows = int64_t(total_tokens) * heads;
+    const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t rw = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); rw < nrows; rw += wstride) {
+        const int64_t t = rw / heads, h = rw % heads;
+        const float *a = dq_acc + (h * total_tokens + t) * D + lane * PER;
+        T *o = dq + rw * D + lane * PER;
+#pragma unroll
+        for (int x = 0; x < PER; ++x) o[x] = from_f32<T>(a[x] * scale);
+    }
+}
+
+// Forward skip: out = v and lse = 0 for flagged examples. grid.x = example,
+// grid.y splits the example's contiguous rows.
+__global__ void __launch_bounds__(256)
+    skip_fwd_kernel(const int32_t *__restrict__ offs, const uint8_t *__restrict__ skip, int32_t heads,
+                    int32_t total_tokens, int64_t row_bytes, const uint8_t *__restrict__ v,
+                    uint8_t *__restrict__ out, float *__restrict__ lse)
+{
+    const int b = blockIdx.x;
+    if (!skip[b]) return;
+    const int64_t s0 = offs[b], L = offs[b + 1] - s0;
+    if (L <= 0) return;
+    const int64_t nvec = L * row_bytes / 16; // rows are whole multiples of 16 bytes
+    const uint4 *src = reinterpret_cast<const uint4 *>(v + s0 * row_bytes);
+    uint4 *dst = reinterpret_cast<uint4 *>(out + s0 * row_bytes);
+    const int64_t stride = int64_t(gridDim.y) * blockDim.x;
+    for (int64_t x = int64_t(blockIdx.y) * blockDim.x + threadIdx.x; x < nvec; x += stride) dst[x] = src[x];
+    for (int64_t x = int64_t(blockIdx.y) * blockDim.x + threadIdx.x; x < L * heads; x += stride)
+        lse[(x / L) * total_tokens + s0 + x % L] = 0.f;
+}
+
+// Backward skip: dk = 0 and dv = dout for flagged examples; dq = 0 too when
+// `dq` is given (the bf16 path instead gets 0 from its zeroed accumulator,
+// since no tile of a flagged example is scheduled).
+__global__ void __launch_bounds__(256)
+    skip_bwd_kernel(const int32_t *__restrict__ offs, const uint8_t *__restrict__ skip, int64_t row_bytes,
+                    const uint8_t *__restrict__ dout, uint8_t *__restrict__ dq, uint8_t *__restrict__ dk,
+                    uint8_t *__restrict__ dv)
+{
+    const int b = blockIdx.x;
+    if (!skip[b]) return;
+    const int64_t s0 = offs[b], L = offs[b + 1] - s0;
+    if (L <= 0) return;
+    const int64_t nvec = L * row_bytes / 16;
+    const uint4 *src = reinterpret_cast<const uint4 *>(dout + s0 * row_bytes);
+    uint4 *dvv = reinterpret_cast<uint4 *>(dv + s0 * row_bytes);
+    uint4 *dkv = reinterpret_cast<uint4 *>(dk + s0 * row_bytes);
+    const int64_t stride = int64_t(gridDim.y) * blockDim.x;
+    uint4 *dqv = dq ? reinterpret_cast<uint4 *>(dq + s0 * row_bytes) : nullptr;
+    for (int64_t x = int64_t(blockIdx.y) * blockDim.x + threadIdx.x; x < nvec; x += stride) {
+        dvv[x] = src[x];
+        dkv[x] = make_uint4(0, 0, 0, 0);
+        if (dqv) dqv[x] = make_uint4(0, 0, 0, 0);
+    }
+}
+
+// ---------------------------------------------------------------- launchers
+
+cudaError_t launch_worklist(const Problem &p, cudaStream_t stream)
+{
+    worklist_kernel<<<1, kWorklistThreads, 0, stream>>>(p.seq_offsets, p.skip, p.batch,
+                                                        const_cast<int32_t *>(p.tile_prefix), p.status);
+    return cudaGetLastError();
+}
+
+static int grid_for_rows(int64_t nrows, int num_sms)
+{
+    const int64_t warps = 8; // per 256-thread block
+    int64_t g = (nrows + warps - 1) / warps;
+    const int64_t cap = int64_t(num_sms) * 16;
+    if (g > cap) g = cap;
+    return int(g < 1 ? 1 : g);
+}
+
+template <typename T>
+cudaError_t launch_bwd_pre(const Problem &p, const void *out, const void *dout, float *delta, float *dq_acc,
+                           int num_sms, cudaStream_t stream)
+{
+    const int64_t nrows = int64_t(p.total_tokens) * p.heads;
+    if (nrows == 0) return cudaSuccess;
+    const int g = grid_for_rows(nrows, num_sms);
+    const T *o = static_cast<const T *>(out), *d = static_cast<const T *>(dout);
+    switch (p.head_dim) {
+    case 32: bwd_pre_kernel<T, 32><<<g, 256, 0, stream>>>(o, d, p.total_tokens, p.heads, delta, dq_acc); break;
+    case 64: bwd_pre_kernel<T, 64><<<g, 256, 0, stream>>>(o, d, p.total_tokens, p.heads, delta, dq_acc); break;
+    case 128: bwd_pre_kernel<T, 128><<<g, 256, 0, stream>>>(o, d, p.total_tokens, p.heads, delta, dq_acc); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_dq_convert(const Problem &p, const float *dq_acc, void *dq, int num_sms, cudaStream_t stream)
+{
+    const int64_t nrows = int64_t(p.total_tokens) * p.heads;
+    if (nrows == 0) return cudaSuccess;
+    const int g = grid_for_rows(nrows, num_sms);
+    T *o = static_cast<T *>(dq);
+    switch (p.head_dim) {
+    case 32: dq_convert_kernel<T, 32><<<g, 256, 0, stream>>>(dq_acc, p.total_tokens, p.heads, p.scale, o); break;
+    case 64: dq_convert_kernel<T, 64><<<g, 256, 0, stream>>>(dq_acc, p.total_tokens, p.heads, p.scale, o); break;
+    case 128: dq_convert_kernel<T, 128><<<g, 256, 0, stream>>>(dq_acc, p.total_tokens, p.heads, p.scale, o); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_skip_fwd(const Problem &p, size_t elem_bytes, const void *v, void *out, float *lse,
+                            cudaStream_t stream)
+{
+    if (!p.skip || p.batch == 0) return cudaSuccess;
+    const int64_t row_bytes = int64_t(p.heads) * p.head_dim * elem_bytes;
+    skip_fwd_kernel<<<dim3(p.batch, 8), 256, 0, stream>>>(p.seq_offsets, p.skip, p.heads, p.total_tokens,
+                                                         row_bytes, static_cast<const uint8_t *>(v),
+                                                         static_cast<uint8_t *>(out), lse);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_skip_bwd(const Problem &p, size_t elem_bytes, const void *dout, void *dq, void *dk,
+                            void *dv, cudaStream_t stream)
+{
+    if (!p.skip || p.batch == 0) return cudaSuccess;
+    const int64_t row_bytes = int64_t(p.heads) * p.head_dim * elem_bytes;
+    skip_bwd_kernel<<<dim3(p.batch, 8), 256, 0, stream>>>(p.seq_offsets, p.skip, row_bytes,
+                                                         static_cast<const uint8_t *>(dout),
+                                                         static_cast<uint8_t *>(dq), static_cast<uint8_t *>(dk),
+                                                         static_cast<uint8_t *>(dv));
+    return cudaGetLastError();
+}
+
+template cudaError_t launch_bwd_pre<float>(const Problem &, const void *, const void *, float *, float *, int,
+                                           cudaStream_t);
+template cudaError_t launch_bwd_pre<__nv_bfloat16>(const Problem &, const void *, const void *, float *, float *,
+                                                   int, cudaStream_t);
+template cudaError_t launch_dq_convert<float>(const Problem &, const float *, void *, int, cudaStream_t);
+template cudaError_t launch_dq_convert<__nv_bfloat16>(const Problem &, const float *, void *, int, cudaStream_t);
+
+} // namespace ba

@@ -1,0 +1,108 @@
+// Shared definitions for the block-attention kernels: the visibility rule,
+// tile ranges, workspace layout and kernel parameter blocks.
+//
+// Visibility (local 0-based indices within one example, blk(x) = x / block):
+//   query i sees key j  <=>  j <= i  and  blk(j) >= blk(i) - (window - 1)
+// ("Meta Scales GEM Ads Model Across Platforms and Thousands of GPUs",
+// section "Kunlun changes how GEM scales": attention arranged in blocks with
+// cost linear in length for a fixed window; "GEM (Meta)", section "Custom
+// kernels": independent 64-token blocks = window 1, block 64).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+namespace ba {
+
+constexpr int kTile = 128;          // rows per query tile and per key tile
+constexpr int kWorklistThreads = 1024;
+
+// Status bits the kernels OR into the workspace status word.
+constexpr int kStatusTimeout = 1;
+
+// First key visible to query i: the start of block blk(i) - (window - 1),
+// clamped at 0.
+__host__ __device__ __forceinline__ int64_t window_start(int64_t i, int64_t block, int64_t window)
+{
+    const int64_t b = i / block - (window - 1);
+    return b > 0 ? b * block : 0;
+}
+
+// Last query (of an example of length L) that sees key j.
+__host__ __device__ __forceinline__ int64_t last_query_seeing(int64_t j, int64_t L, int64_t block,
+                                                              int64_t window)
+{
+    const int64_t hi = (j / block + window) * block - 1;
+    return hi < L - 1 ? hi : L - 1;
+}
+
+__host__ __device__ __forceinline__ bool visible(int64_t i, int64_t j, int64_t block, int64_t window)
+{
+    return j <= i && j >= window_start(i, block, window);
+}
+
+// Workspace layout (all offsets 256-byte aligned):
+//   [0, 256)            status word (int32) and scheduler counters
+//   tile_prefix         int32[batch + 1]: live 128-row tiles before example b
+//   delta   (bwd only)  float[heads * total_tokens]
+//   dq_acc  (bwd only)  float[heads * total_tokens * head_dim]
+struct WorkspaceLayout {
+    size_t status, tile_prefix, delta, dq_acc, total;
+};
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+__host__ __device__ inline WorkspaceLayout workspace_layout(int64_t batch, int64_t total_tokens,
+                                                            int64_t heads, int64_t head_dim,
+                                                            bool with_delta, bool with_dq_acc)
+{
+    WorkspaceLayout w;
+    w.status = 0;
+    w.tile_prefix = 256;
+    size_t off = align256(w.tile_prefix + sizeof(int32_t) * size_t(batch + 1));
+    w.delta = off;
+    if (with_delta) off = align256(off + sizeof(float) * size_t(heads * total_tokens));
+    w.dq_acc = off;
+    if (with_dq_acc) off = align256(off + sizeof(float) * size_t(heads * total_tokens * head_dim));
+    w.total = off;
+    return w;
+}
+
+// Common problem description handed to every kernel.
+struct Problem {
+    const int32_t *seq_offsets; // [batch + 1], device
+    const uint8_t *skip;        // [batch] or nullptr
+    const int32_t *tile_prefix; // [batch + 1], device (workspace)
+    int *status;                // workspace status word
+    int32_t batch, total_tokens, heads, head_dim, block, window;
+    float scale;                // 1 / sqrt(head_dim)
+};
+
+// One 128-row tile of one (example, head).
+struct TileRef {
+    int32_t e, h, t;   // example, head, tile index within the example
+    int32_t s0, L;     // first global row of the example, its length
+};
+
+// Work item n -> (tile, head); tiles are numbered over live examples in
+// order, heads vary fastest. Returns false past the last item.
+__device__ __forceinline__ bool decode_item(const Problem &p, int64_t n, TileRef &r)
+{
+    const int32_t ntiles = p.tile_prefix[p.batch];
+    if (n >= int64_t(ntiles) * p.heads) return false;
+    const int32_t tile = int32_t(n / p.heads);
+    r.h = int32_t(n % p.heads);
+    int lo = 0, hi = p.batch - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.tile_prefix[mid] <= tile) lo = mid;
+        else hi = mid - 1;
+    }
+    r.e = lo;
+    r.t = tile - p.tile_prefix[lo];
+    r.s0 = p.seq_offsets[lo];
+    r.L = p.seq_offsets[lo + 1] - r.s0;
+    return true;
+}
+
+} // namespace ba

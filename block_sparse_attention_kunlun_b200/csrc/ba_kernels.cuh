@@ -1,0 +1,39 @@
+// Host-side launchers of the library's kernels (internal; the public C ABI is
+// include/ba.h).
+#pragma once
+
+#include "ba_common.cuh"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace ba {
+
+cudaError_t launch_worklist(const Problem &p, cudaStream_t stream);
+
+template <typename T>
+cudaError_t launch_bwd_pre(const Problem &p, const void *out, const void *dout, float *delta, float *dq_acc,
+                           int num_sms, cudaStream_t stream);
+template <typename T>
+cudaError_t launch_dq_convert(const Problem &p, const float *dq_acc, void *dq, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_skip_fwd(const Problem &p, size_t elem_bytes, const void *v, void *out, float *lse,
+                            cudaStream_t stream);
+cudaError_t launch_skip_bwd(const Problem &p, size_t elem_bytes, const void *dout, void *dq, void *dk, void *dv,
+                            cudaStream_t stream);
+
+cudaError_t launch_fwd_f32(const Problem &p, const float *q, const float *k, const float *v, float *out, float *lse,
+                           int num_sms, cudaStream_t stream);
+cudaError_t launch_bwd_f32(const Problem &p, const float *q, const float *k, const float *v, const float *dout,
+                           const float *lse, const float *delta, float *dq, float *dk, float *dv, int num_sms,
+                           cudaStream_t stream);
+
+template <int D>
+cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                  const Problem &p, void *out, float *lse, int num_sms, cudaStream_t stream);
+template <int D>
+cudaError_t launch_bwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                  const CUtensorMap &tdo, const Problem &p, const float *lse, const float *delta,
+                                  float *dq_acc, void *dk, void *dv, int num_sms, cudaStream_t stream);
+
+} // namespace ba

@@ -1,0 +1,150 @@
+/*
+ * ba.h -- block attention on NVIDIA B200 (sm_100a): the library's C ABI.
+ *
+ * Block attention is the sparse self-attention of Kunlun, the architecture
+ * behind Meta's GEM ads model: attention over a long user-engagement history
+ * restricted to blocks, so that cost grows linearly with sequence length for a
+ * fixed window ("Meta Scales GEM Ads Model Across Platforms and Thousands of
+ * GPUs", section "Kunlun changes how GEM scales"; "GEM (Meta)", section
+ * "Custom kernels", BlockAttention; "Scaling Meta's Generative Ads Model (GEM)
+ * for Ads Recommendations", section "Kunlun Architecture Details"). The pages
+ * give no formula; this library fixes one rule and keeps it everywhere:
+ *
+ *   within one example, with 0-based local indices and blk(x) = x / block,
+ *   query i sees key j  <=>  j <= i  and  blk(j) >= blk(i) - (window - 1).
+ *
+ * window = 1 is the pages' "independent 64-token blocks" case (block = 64),
+ * causal inside each block. Blocks start at each example's first token.
+ *
+ * Batches are jagged ("GEM (Meta)", section "Training infrastructure":
+ * histories of hundreds to tens of thousands of events, not padded): example
+ * b owns rows seq_offsets[b] .. seq_offsets[b+1]-1 of every token-major
+ * tensor.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - q, k, v, out, dout, dq, dk, dv: DEVICE pointers to contiguous row-major
+ *    [total_tokens, heads, head_dim] tensors of the problem's dtype, 16-byte
+ *    aligned. out/dq/dk/dv must not alias any input.
+ *  - lse: DEVICE pointer, float32 [heads, total_tokens]: the natural log of
+ *    sum_j exp(q_i . k_j / sqrt(head_dim)) over the visible keys.
+ *  - seq_offsets: DEVICE pointer, int32 [batch + 1], seq_offsets[0] = 0,
+ *    non-decreasing, seq_offsets[batch] = total_tokens (empty examples are
+ *    allowed). This precondition is not checked on the device.
+ *  - skip: DEVICE pointer to uint8 [batch] or NULL. A nonzero flag bypasses
+ *    attention for that example (component skip, "Meta Scales GEM Ads Model
+ *    ...", section "Kunlun changes how GEM scales"): out = v, lse = 0,
+ *    dq = dk = 0, dv = dout, and none of its tiles is scheduled.
+ *  - Scores are scaled by 1/sqrt(head_dim). Accumulation is float32; bf16
+ *    results are rounded to nearest even.
+ *  - workspace: DEVICE scratch owned by the caller, at least the size the
+ *    matching *_workspace_size query returns, 256-byte aligned. Its contents
+ *    need not be initialised. One workspace must not be used by two calls
+ *    that may run at the same time.
+ *  - stream: every launch is asynchronous on this stream; no call
+ *    synchronises the device or allocates memory (ba_device_status is the
+ *    one call that waits, and only on `stream`).
+ *  - Errors: argument checks run on the host before anything is launched and
+ *    return BA_ERR_INVALID_ARG (bad pointer, size or alignment) or
+ *    BA_ERR_UNSUPPORTED (a valid combination this build has no kernel for).
+ *    A launch failure returns BA_ERR_CUDA. Kernel-side waits are bounded;
+ *    one that runs out records BA_ERR_TIMEOUT in the workspace, readable with
+ *    ba_device_status. The library never traps.
+ *  - Thread safety: no global mutable state besides a per-device cache of
+ *    the SM count and the thread-local profiling hook below; calls on
+ *    different streams with different workspaces are independent.
+ */
+#ifndef BA_H
+#define BA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *ba_stream_t; /* same as cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    BA_OK = 0,
+    BA_ERR_INVALID_ARG = 1,
+    BA_ERR_UNSUPPORTED = 2,
+    BA_ERR_CUDA = 3,
+    BA_ERR_TIMEOUT = 4
+} ba_status;
+
+typedef enum {
+    BA_F32 = 0,  /* float32 tensors; SIMT kernels, no TF32 */
+    BA_BF16 = 1  /* bfloat16 tensors; tcgen05 tensor-core kernels */
+} ba_dtype;
+
+/* Host-side description of one jagged batch. */
+typedef struct {
+    int32_t batch;        /* number of examples, >= 0 */
+    int32_t total_tokens; /* seq_offsets[batch], >= 0 */
+    int32_t heads;        /* >= 1; q, k, v share heads */
+    int32_t head_dim;     /* BA_BF16: 64 or 128; BA_F32: 32 or 64 */
+    ba_dtype dtype;
+} ba_problem;
+
+/*
+ * Bytes of workspace ba_fwd / ba_bwd need for this problem (0 on an invalid
+ * problem). The backward's includes a float32 dq accumulator
+ * [heads, total_tokens, head_dim] and a float32 row-dot buffer
+ * [heads, total_tokens].
+ */
+size_t ba_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window);
+size_t ba_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window);
+
+/*
+ * Forward pass: out[i] = sum_j softmax_j(q_i . k_j / sqrt(head_dim)) v_j over
+ * the keys visible to query i under the rule above, and lse as defined above.
+ * block >= 1, window >= 1.
+ */
+ba_status ba_fwd(const ba_problem *p, const void *q, const void *k, const void *v,
+                 const int32_t *seq_offsets, int32_t block, int32_t window,
+                 const uint8_t *skip, void *out, float *lse,
+                 void *workspace, size_t workspace_bytes, ba_stream_t stream);
+
+/*
+ * Backward pass: given the forward's out and lse and the upstream gradient
+ * dout, writes the exact gradients dq, dk, dv of sum(out * dout) with respect
+ * to q, k, v. Probabilities are recomputed from lse (nothing else is saved
+ * by the forward). Same shapes and conventions as ba_fwd.
+ */
+ba_status ba_bwd(const ba_problem *p, const void *q, const void *k, const void *v,
+                 const void *out, const float *lse, const void *dout,
+                 const int32_t *seq_offsets, int32_t block, int32_t window,
+                 const uint8_t *skip, void *dq, void *dk, void *dv,
+                 void *workspace, size_t workspace_bytes, ba_stream_t stream);
+
+/*
+ * Waits for `stream`, then reads the status word a previous ba_fwd/ba_bwd
+ * left in `workspace`: BA_OK, or BA_ERR_TIMEOUT if a kernel gave up waiting
+ * (its outputs are then undefined). BA_ERR_CUDA if the read itself failed.
+ */
+ba_status ba_device_status(const void *workspace, ba_stream_t stream);
+
+/*
+ * Profiling hook. Until changed, every ba_fwd (which = 0) or ba_bwd
+ * (which = 1) call made from THIS host thread records `start` on its stream
+ * right before launching its attention kernel and `stop` right after it, so
+ * that cudaEventElapsedTime(start, stop) is that kernel's own duration. The
+ * events are cudaEvent_t handles owned by the caller; pass NULL, NULL to
+ * stop recording. Returns BA_ERR_INVALID_ARG for another `which`. Only the
+ * hook pointers are stored (thread-local); nothing is synchronised.
+ */
+ba_status ba_set_profile_events(int32_t which, void *start, void *stop);
+
+/* Static, human-readable name of a status code. */
+const char *ba_status_string(ba_status s);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t ba_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BA_H */

@@ -1,0 +1,106 @@
+"""The C ABI without a GPU: the library loads, exports what include/ba.h
+declares, sizes workspaces, and rejects bad arguments on the host before it
+would launch anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_kunlun_b200 as ba
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "ba.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ba_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(ba.library_path())
+    names = declared_functions()
+    assert {"ba_fwd", "ba_bwd", "ba_fwd_workspace_size", "ba_bwd_workspace_size",
+            "ba_device_status", "ba_status_string", "ba_version"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"libba.so does not export {n}"
+
+
+def test_status_strings_and_version():
+    assert ba.ba_status_string(ba.BA_OK) == "ok"
+    assert "timed out" in ba.ba_status_string(ba.BA_ERR_TIMEOUT)
+    assert ba.ba_status_string(99) == "unknown status"
+    assert ba.ba_version() >= 100
+
+
+def prob(batch=2, T=300, H=4, D=64, dt=ba.BA_BF16):
+    return ba.BAProblem(batch, T, H, D, dt)
+
+
+def test_workspace_sizes():
+    p = prob(batch=3, T=1000, H=2, D=128)
+    f = ba.ba_fwd_workspace_size(p, 128, 2)
+    b = ba.ba_bwd_workspace_size(p, 128, 2)
+    assert f >= 256 + 4 * 4 and f % 256 == 0
+    # backward adds Delta (H*T floats) and the fp32 dq accumulator (H*T*D floats)
+    assert b >= f + 4 * 2 * 1000 + 4 * 2 * 1000 * 128
+    pf = prob(batch=3, T=1000, H=2, D=64, dt=ba.BA_F32)
+    assert ba.ba_bwd_workspace_size(pf, 128, 2) < ba.ba_bwd_workspace_size(prob(3, 1000, 2, 64), 128, 2)
+    assert ba.ba_fwd_workspace_size(prob(batch=-1), 128, 2) == 0
+    assert ba.ba_fwd_workspace_size(p, 0, 2) == 0
+    assert ba.ba_fwd_workspace_size(p, 128, 0) == 0
+
+
+FAKE = 1 << 20  # a 256-byte-aligned address that is never dereferenced on invalid arguments
+
+
+def call_fwd(p, block=128, window=2, q=FAKE, k=FAKE, v=FAKE, offs=FAKE, out=FAKE, lse=FAKE,
+             ws=FAKE, ws_bytes=1 << 30):
+    lib = ba._load()
+    return lib.ba_fwd(ctypes.byref(p) if p is not None else None, q, k, v, offs, block, window, None,
+                      out, lse, ws, ws_bytes, None)
+
+
+def call_bwd(p, block=128, window=2, ptrs=None, ws=FAKE, ws_bytes=1 << 30):
+    lib = ba._load()
+    d = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, dout=FAKE, offs=FAKE, dq=FAKE, dk=FAKE, dv=FAKE)
+    d.update(ptrs or {})
+    return lib.ba_bwd(ctypes.byref(p), d["q"], d["k"], d["v"], d["out"], d["lse"], d["dout"], d["offs"],
+                      block, window, None, d["dq"], d["dk"], d["dv"], ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(p=None),
+    dict(block=0), dict(window=0), dict(block=-5),
+    dict(q=0), dict(k=0), dict(v=0), dict(out=0), dict(lse=0), dict(offs=0),
+    dict(q=FAKE + 8), dict(out=FAKE + 4), dict(lse=FAKE + 2), dict(offs=FAKE + 2),
+    dict(ws=0), dict(ws=FAKE + 128), dict(ws_bytes=16),
+])
+def test_fwd_rejects_invalid_arguments(kw):
+    p = kw.pop("p", prob())
+    assert call_fwd(p, **kw) == ba.BA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("p", [prob(batch=-1), prob(T=-1), prob(H=0), prob(D=0), prob(batch=0, T=5),
+                               ba.BAProblem(2, 300, 4, 64, 7)])
+def test_fwd_rejects_invalid_problems(p):
+    assert call_fwd(p) == ba.BA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("p", [prob(D=32), prob(D=96), prob(D=256), prob(D=128, dt=ba.BA_F32),
+                               prob(D=48, dt=ba.BA_F32)])
+def test_unsupported_head_dims(p):
+    assert call_fwd(p) == ba.BA_ERR_UNSUPPORTED
+    assert call_bwd(p) == ba.BA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("name", ["q", "k", "v", "out", "lse", "dout", "offs", "dq", "dk", "dv"])
+def test_bwd_rejects_null_pointers(name):
+    assert call_bwd(prob(), ptrs={name: 0}) == ba.BA_ERR_INVALID_ARG
+
+
+def test_bwd_rejects_small_workspace():
+    p = prob(batch=2, T=300, H=4, D=64)
+    need = ba.ba_bwd_workspace_size(p, 128, 2)
+    assert call_bwd(p, ws_bytes=need - 1) == ba.BA_ERR_INVALID_ARG
