@@ -145,9 +145,13 @@ def ba_bwd(problem, q, k, v, out, lse, dout, seq_offsets, block, window, skip, d
 
 def ba_set_profile_events(which: int, start=None, stop=None) -> int:
     """Record torch.cuda.Event ``start``/``stop`` around the attention kernel of
-    every later ba_fwd (which=0) or ba_bwd (which=1) call from this thread."""
+    every later ba_fwd (which=0) or ba_bwd (which=1) call from this thread.
+    The events must already exist on the device (torch creates an event on
+    its first ``record``)."""
     s = start.cuda_event if start is not None else None
     e = stop.cuda_event if stop is not None else None
+    if (start is not None and not s) or (stop is not None and not e):
+        raise ValueError("record each event once before handing it to the library")
     return int(_load().ba_set_profile_events(int(which), s, e))
 
 
