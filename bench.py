@@ -361,7 +361,7 @@ def main():
             traffic = tr[key]["bytes_per_launch"]
     except (OSError, ValueError):
         pass
-    roofline = {"kernel": "bwd_bf16_sm100_kernel", "bound": "tensor", "achieved": bwd_achieved,
+    roofline = {"kernel": "bwd_d128_sm100_kernel" if D == 128 else "bwd_bf16_sm100_kernel", "bound": "tensor", "achieved": bwd_achieved,
                 "peak": tensor_peak, "unit": "TFLOP/s", "frac": bwd_achieved / tensor_peak,
                 "traffic": traffic, "peak_source": f"{peaks_src} bf16_tflops_sustained",
                 "algorithmic_flops_per_launch": fl["bwd"], "ms_per_launch": ms_bwd_k,
@@ -396,7 +396,7 @@ def main():
 def kernel_sha() -> str:
     """Hash of the backward kernel source, to tell whether stored counters are current."""
     import hashlib
-    p = os.path.join(ROOT, "block_sparse_attention_kunlun_b200", "csrc", "ba_bwd_sm100.cu")
+    p = os.path.join(ROOT, "block_sparse_attention_kunlun_b200", "csrc", "ba_bwd_d128_sm100.cu")
     with open(p, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 

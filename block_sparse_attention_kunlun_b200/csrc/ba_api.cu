@@ -104,6 +104,7 @@ Problem make_problem(const ba_problem &pp, const int32_t *offs, const uint8_t *s
     p.seq_offsets = offs;
     p.skip = skip;
     p.tile_prefix = reinterpret_cast<const int32_t *>(static_cast<uint8_t *>(workspace) + lay.tile_prefix);
+    p.tile_info = reinterpret_cast<const int4 *>(static_cast<uint8_t *>(workspace) + lay.tile_info);
     p.status = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + lay.status);
     p.batch = pp.batch;
     p.total_tokens = pp.total_tokens;
@@ -233,7 +234,7 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
     if (P.head_dim == 64)
         BA_TRY(launch_bwd_bf16_sm100<64>(tq, tk, tv, tdo, p, lse, delta, dq_acc, dk, dv, num_sms, stream));
     else
-        BA_TRY(launch_bwd_bf16_sm100<128>(tq, tk, tv, tdo, p, lse, delta, dq_acc, dk, dv, num_sms, stream));
+        BA_TRY(launch_bwd_d128_sm100(tq, tk, tv, tdo, p, lse, delta, dq_acc, dk, dv, num_sms, stream));
     BA_TRY(prof_mark(1, 1, stream));
     BA_TRY(launch_dq_convert<__nv_bfloat16>(p, dq_acc, dq, num_sms, stream));
     return BA_OK;

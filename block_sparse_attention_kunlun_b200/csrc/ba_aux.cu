@@ -36,7 +36,7 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 
 __global__ void __launch_bounds__(kWorklistThreads)
     worklist_kernel(const int32_t *__restrict__ offs, const uint8_t *__restrict__ skip, int32_t batch,
-                    int32_t *__restrict__ tile_prefix, int *__restrict__ status)
+                    int32_t *__restrict__ tile_prefix, int4 *__restrict__ tile_info, int *__restrict__ status)
 {
     __shared__ int32_t warp_tot[kWorklistThreads / 32];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -67,7 +67,10 @@ __global__ void __launch_bounds__(kWorklistThreads)
     int32_t run = incl - local + (wid > 0 ? warp_tot[wid - 1] : 0);
     for (int b = b0; b < b1; ++b) {
         tile_prefix[b] = run;
-        run += live_tiles(offs, skip, b);
+        const int32_t nt = live_tiles(offs, skip, b);
+        const int32_t s0 = offs[b], L = offs[b + 1] - s0;
+        for (int32_t t = 0; t < nt; ++t) tile_info[run + t] = make_int4(s0, L, t, b);
+        run += nt;
     }
     if (tid == kWorklistThreads - 1) {
         tile_prefix[batch] = warp_tot[kWorklistThreads / 32 - 1];
@@ -172,7 +175,8 @@ __global__ void __launch_bounds__(256)
 cudaError_t launch_worklist(const Problem &p, cudaStream_t stream)
 {
     worklist_kernel<<<1, kWorklistThreads, 0, stream>>>(p.seq_offsets, p.skip, p.batch,
-                                                        const_cast<int32_t *>(p.tile_prefix), p.status);
+                                                        const_cast<int32_t *>(p.tile_prefix),
+                                                        const_cast<int4 *>(p.tile_info), p.status);
     return cudaGetLastError();
 }
 

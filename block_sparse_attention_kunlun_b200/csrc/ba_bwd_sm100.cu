@@ -1,4 +1,5 @@
-// Block attention backward on sm_100a, key-tile stationary.
+// Block attention backward on sm_100a, key-tile stationary (head_dim 64;
+// head_dim 128 has its own kernel in ba_bwd_d128_sm100.cu).
 //
 // Gradients of out = softmax(q k^T / sqrt(D)) v over the visible keys
 // (visibility rule in ba_common.cuh), with the probabilities recomputed from
@@ -130,8 +131,9 @@ __global__ void __launch_bounds__(320, 1)
         // ------------------------------------------------ TMA producer ---
         uint32_t it = 0, item_cnt = 0;
         TileRef r;
+        const int32_t ntiles = live_tile_count(p);
         bool ok = true;
-        for (int64_t n = blockIdx.x; ok && decode_item(p, n, r); n += gridDim.x, ++item_cnt) {
+        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
             int ilo, ihi;
             last_q_tile(r, B, W, ilo, ihi);
             if (!mbar_wait(&sb.kv_empty, (item_cnt & 1) ^ 1, abort)) break;
@@ -172,8 +174,9 @@ __global__ void __launch_bounds__(320, 1)
         constexpr uint32_t idesc_dq = idesc_bf16(128, 64, true, true);      // dQ halves (A, B MN-major)
         uint32_t it = 0, item_cnt = 0;
         TileRef r;
+        const int32_t ntiles = live_tile_count(p);
         bool ok = true;
-        for (int64_t n = blockIdx.x; ok && decode_item(p, n, r); n += gridDim.x, ++item_cnt) {
+        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
             int ilo, ihi;
             last_q_tile(r, B, W, ilo, ihi);
             if (!mbar_wait(&sb.kv_full, item_cnt & 1, abort)) break;
@@ -258,8 +261,9 @@ __global__ void __launch_bounds__(320, 1)
         const float scale_log2 = p.scale * 1.4426950408889634f;
         uint32_t it = 0, item_cnt = 0;
         TileRef r;
+        const int32_t ntiles = live_tile_count(p);
         bool ok = true;
-        for (int64_t n = blockIdx.x; ok && decode_item(p, n, r); n += gridDim.x, ++item_cnt) {
+        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
             int ilo, ihi;
             last_q_tile(r, B, W, ilo, ihi);
             const int64_t k = int64_t(r.t) * kTile + row; // local key index
@@ -371,8 +375,9 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
         uint32_t it = 0;
         TileRef r;
+        const int32_t ntiles = live_tile_count(p);
         bool ok = true;
-        for (int64_t n = blockIdx.x; ok && decode_item(p, n, r); n += gridDim.x) {
+        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x) {
             int ilo, ihi;
             last_q_tile(r, B, W, ilo, ihi);
             for (int i = ilo; i <= ihi; ++i, ++it) {
@@ -432,8 +437,5 @@ cudaError_t launch_bwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
 template cudaError_t launch_bwd_bf16_sm100<64>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
                                                const CUtensorMap &, const Problem &, const float *,
                                                const float *, float *, void *, void *, int, cudaStream_t);
-template cudaError_t launch_bwd_bf16_sm100<128>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                                                const CUtensorMap &, const Problem &, const float *,
-                                                const float *, float *, void *, void *, int, cudaStream_t);
 
 } // namespace ba

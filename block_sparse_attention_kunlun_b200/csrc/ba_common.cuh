@@ -42,15 +42,23 @@ __host__ __device__ __forceinline__ bool visible(int64_t i, int64_t j, int64_t b
 }
 
 // Workspace layout (all offsets 256-byte aligned):
-//   [0, 256)            status word (int32) and scheduler counters
+//   [0, 256)            status word (int32)
 //   tile_prefix         int32[batch + 1]: live 128-row tiles before example b
+//   tile_info           int4[max_tiles]: per live tile {first row of its
+//                       example, example length, tile index in the example,
+//                       example index}, max_tiles = ceil(T / 128) + batch
 //   delta   (bwd only)  float[heads * total_tokens]
 //   dq_acc  (bwd only)  float[heads * total_tokens * head_dim]
 struct WorkspaceLayout {
-    size_t status, tile_prefix, delta, dq_acc, total;
+    size_t status, tile_prefix, tile_info, delta, dq_acc, total;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+__host__ __device__ inline int64_t max_tiles(int64_t batch, int64_t total_tokens)
+{
+    return (total_tokens + kTile - 1) / kTile + batch;
+}
 
 __host__ __device__ inline WorkspaceLayout workspace_layout(int64_t batch, int64_t total_tokens,
                                                             int64_t heads, int64_t head_dim,
@@ -60,6 +68,8 @@ __host__ __device__ inline WorkspaceLayout workspace_layout(int64_t batch, int64
     w.status = 0;
     w.tile_prefix = 256;
     size_t off = align256(w.tile_prefix + sizeof(int32_t) * size_t(batch + 1));
+    w.tile_info = off;
+    off = align256(off + 16 * size_t(max_tiles(batch, total_tokens)));
     w.delta = off;
     if (with_delta) off = align256(off + sizeof(float) * size_t(heads * total_tokens));
     w.dq_acc = off;
@@ -73,6 +83,7 @@ struct Problem {
     const int32_t *seq_offsets; // [batch + 1], device
     const uint8_t *skip;        // [batch] or nullptr
     const int32_t *tile_prefix; // [batch + 1], device (workspace)
+    const int4 *tile_info;      // [max_tiles], device (workspace)
     int *status;                // workspace status word
     int32_t batch, total_tokens, heads, head_dim, block, window;
     float scale;                // 1 / sqrt(head_dim)
@@ -80,28 +91,24 @@ struct Problem {
 
 // One 128-row tile of one (example, head).
 struct TileRef {
-    int32_t e, h, t;   // example, head, tile index within the example
+    int32_t h, t;      // head, tile index within the example
     int32_t s0, L;     // first global row of the example, its length
 };
 
+// Number of live tiles (read once per kernel role).
+__device__ __forceinline__ int32_t live_tile_count(const Problem &p) { return p.tile_prefix[p.batch]; }
+
 // Work item n -> (tile, head); tiles are numbered over live examples in
 // order, heads vary fastest. Returns false past the last item.
-__device__ __forceinline__ bool decode_item(const Problem &p, int64_t n, TileRef &r)
+__device__ __forceinline__ bool decode_item(const Problem &p, int32_t ntiles, int64_t n, TileRef &r)
 {
-    const int32_t ntiles = p.tile_prefix[p.batch];
     if (n >= int64_t(ntiles) * p.heads) return false;
     const int32_t tile = int32_t(n / p.heads);
     r.h = int32_t(n % p.heads);
-    int lo = 0, hi = p.batch - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (p.tile_prefix[mid] <= tile) lo = mid;
-        else hi = mid - 1;
-    }
-    r.e = lo;
-    r.t = tile - p.tile_prefix[lo];
-    r.s0 = p.seq_offsets[lo];
-    r.L = p.seq_offsets[lo + 1] - r.s0;
+    const int4 info = p.tile_info[tile];
+    r.s0 = info.x;
+    r.L = info.y;
+    r.t = info.z;
     return true;
 }
 

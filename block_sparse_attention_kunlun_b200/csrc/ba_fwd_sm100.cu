@@ -16,7 +16,8 @@
 //              reads S, masks, keeps the running max/sum, writes P (bf16) back
 //              into TMEM over S, rescales O when the max grows by > 2^8, and
 //              stores out and lse at the end of the item;
-//   warp 4     TMA producer: Q once per item, K and V per key tile into a ring;
+//   warp 4     TMA producer: Q once per item (two buffers, so the next item's
+//              Q arrives while this one runs), K and V per key tile into a ring;
 //   warp 5     MMA issuer: S = Q K^T into one of two TMEM S buffers, then
 //              O += P V with P read straight from TMEM (no shared-memory trip).
 // TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D).
@@ -37,9 +38,9 @@ struct FwdLayout {
     static constexpr int kChunks = D / 64;               // 128-byte column chunks per row
     static constexpr int kChunkBytes = kTile * 128;      // one chunk of a 128-row tile
     static constexpr int kTileBytes = kTile * D * 2;     // one 128 x D bf16 tile
-    static constexpr int kQ = 0;
-    static constexpr int kK0 = kTileBytes;               // stage s: K at kK0 + 2 s tile, V after it
-    static constexpr int kBytes = kTileBytes * (1 + 2 * kStages);
+    static constexpr int kQ = 0;                         // two Q buffers (consecutive items)
+    static constexpr int kK0 = 2 * kTileBytes;           // stage s: K at kK0 + 2 s tile, V after it
+    static constexpr int kBytes = kTileBytes * (2 + 2 * kStages);
     static constexpr int kAlloc = kBytes + 1024;         // slack to align the base to 1024 B
     static constexpr int kThreads = 192;
     static constexpr uint32_t kTmemCols = 512;
@@ -47,7 +48,7 @@ struct FwdLayout {
 };
 
 struct FwdBarriers {
-    uint64_t q_full, q_empty, o_done, o_free;
+    uint64_t q_full[2], q_empty[2], o_done, o_free;
     uint64_t s_full[2], p_full[2];
     uint64_t kv_full[4], kv_empty[4];
     uint32_t tmem_base;
@@ -73,8 +74,10 @@ __global__ void __launch_bounds__(192, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sb.q_full, 1);
-        mbar_init(&sb.q_empty, 1);
+        mbar_init(&sb.q_full[0], 1);
+        mbar_init(&sb.q_full[1], 1);
+        mbar_init(&sb.q_empty[0], 1);
+        mbar_init(&sb.q_empty[1], 1);
         mbar_init(&sb.o_done, 1);
         mbar_init(&sb.o_free, 4);
         for (int i = 0; i < 2; ++i) {
@@ -108,14 +111,16 @@ __global__ void __launch_bounds__(192, 1)
         // ------------------------------------------------ TMA producer ---
         uint32_t kv_cnt = 0, item_cnt = 0;
         TileRef r;
-        for (int64_t n = blockIdx.x; decode_item(p, n, r); n += gridDim.x, ++item_cnt) {
+        const int32_t ntiles = live_tile_count(p);
+        for (int64_t n = blockIdx.x; decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
             const int jlo = int(window_start(int64_t(r.t) * kTile, B, W) / kTile);
-            if (!mbar_wait(&sb.q_empty, (item_cnt & 1) ^ 1, abort)) break;
+            const int qb = item_cnt & 1;
+            if (!mbar_wait(&sb.q_empty[qb], ((item_cnt >> 1) & 1) ^ 1, abort)) break;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&sb.q_full, Lay::kTileBytes);
+                mbar_arrive_expect_tx(&sb.q_full[qb], Lay::kTileBytes);
                 for (int c = 0; c < Lay::kChunks; ++c)
-                    tma_load_2d(smem + Lay::kQ + c * Lay::kChunkBytes, &tm_q, &sb.q_full,
-                                r.h * D + c * 64, r.s0 + r.t * kTile);
+                    tma_load_2d(smem + Lay::kQ + qb * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_q,
+                                &sb.q_full[qb], r.h * D + c * 64, r.s0 + r.t * kTile);
             }
             __syncwarp();
             bool ok = true;
@@ -146,11 +151,13 @@ __global__ void __launch_bounds__(192, 1)
         constexpr uint32_t idesc_o = idesc_bf16(128, D, false, true);
         uint32_t kv_cnt = 0, s_cnt = 0, item_cnt = 0;
         TileRef r;
+        const int32_t ntiles = live_tile_count(p);
         bool ok = true;
-        for (int64_t n = blockIdx.x; ok && decode_item(p, n, r); n += gridDim.x, ++item_cnt) {
+        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
             const int jlo = int(window_start(int64_t(r.t) * kTile, B, W) / kTile);
             const int nkv = r.t - jlo + 1;
-            if (!mbar_wait(&sb.q_full, item_cnt & 1, abort)) break;
+            const int qb = item_cnt & 1;
+            if (!mbar_wait(&sb.q_full[qb], (item_cnt >> 1) & 1, abort)) break;
             tc_fence_after();
             // O += P_m V_m for the key tile issued m-th in this item.
             auto issue_pv = [&](int m, uint32_t s_idx, uint32_t kv_idx) -> bool {
@@ -181,7 +188,7 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t q_addr = smem_base + Lay::kQ;
+                    const uint32_t q_addr = smem_base + Lay::kQ + qb * Lay::kTileBytes;
                     const uint32_t k_addr = smem_base + Lay::kK0 + 2 * st * Lay::kTileBytes;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
@@ -190,7 +197,7 @@ __global__ void __launch_bounds__(192, 1)
                                sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
                     }
                     tc_commit(&sb.s_full[s_cnt & 1]);
-                    if (m == nkv - 1) tc_commit(&sb.q_empty);
+                    if (m == nkv - 1) tc_commit(&sb.q_empty[qb]);
                 }
                 __syncwarp();
                 if (m > 0 && !issue_pv(m - 1, s_cnt - 1, kv_cnt - 1)) {
@@ -207,8 +214,9 @@ __global__ void __launch_bounds__(192, 1)
         const float scale_log2 = p.scale * 1.4426950408889634f;
         uint32_t s_cnt = 0, pv_cnt = 0;
         TileRef r;
+        const int32_t ntiles = live_tile_count(p);
         bool ok = true;
-        for (int64_t n = blockIdx.x; ok && decode_item(p, n, r); n += gridDim.x) {
+        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x) {
             const int64_t i = int64_t(r.t) * kTile + row;
             const bool valid = i < r.L;
             const int64_t ws = window_start(i, B, W);

@@ -36,4 +36,8 @@ cudaError_t launch_bwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
                                   const CUtensorMap &tdo, const Problem &p, const float *lse, const float *delta,
                                   float *dq_acc, void *dk, void *dv, int num_sms, cudaStream_t stream);
 
+cudaError_t launch_bwd_d128_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                  const CUtensorMap &tdo, const Problem &p, const float *lse, const float *delta,
+                                  float *dq_acc, void *dk, void *dv, int num_sms, cudaStream_t stream);
+
 } // namespace ba

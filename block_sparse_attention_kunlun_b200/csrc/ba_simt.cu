@@ -20,7 +20,8 @@ __global__ void __launch_bounds__(128)
     __shared__ float ks[kChunk][D], vs[kChunk][D];
     const int64_t B = p.block, W = p.window, H = p.heads;
     TileRef r;
-    for (int64_t n = blockIdx.x; decode_item(p, n, r); n += gridDim.x) {
+    const int32_t ntiles = live_tile_count(p);
+    for (int64_t n = blockIdx.x; decode_item(p, ntiles, n, r); n += gridDim.x) {
         const int64_t i = int64_t(r.t) * kTile + threadIdx.x;
         const bool valid = i < r.L;
         const int64_t ws = window_start(i, B, W);
@@ -84,7 +85,8 @@ __global__ void __launch_bounds__(128)
     __shared__ float ks[kChunk][D], vs[kChunk][D];
     const int64_t B = p.block, W = p.window, H = p.heads, T = p.total_tokens;
     TileRef r;
-    for (int64_t n = blockIdx.x; decode_item(p, n, r); n += gridDim.x) {
+    const int32_t ntiles = live_tile_count(p);
+    for (int64_t n = blockIdx.x; decode_item(p, ntiles, n, r); n += gridDim.x) {
         const int64_t i = int64_t(r.t) * kTile + threadIdx.x;
         const bool valid = i < r.L;
         const int64_t ws = window_start(i, B, W);
@@ -143,7 +145,8 @@ __global__ void __launch_bounds__(128)
     __shared__ float qs[kChunk][D], gs[kChunk][D], ls[kChunk], dls[kChunk];
     const int64_t B = p.block, W = p.window, H = p.heads, T = p.total_tokens;
     TileRef r;
-    for (int64_t n = blockIdx.x; decode_item(p, n, r); n += gridDim.x) {
+    const int32_t ntiles = live_tile_count(p);
+    for (int64_t n = blockIdx.x; decode_item(p, ntiles, n, r); n += gridDim.x) {
         const int64_t j = int64_t(r.t) * kTile + threadIdx.x;
         const bool valid = j < r.L;
         const int64_t jmax = (int64_t(r.t) * kTile + kTile < r.L ? int64_t(r.t) * kTile + kTile : r.L) - 1;
