@@ -20,7 +20,7 @@ import os
 import torch
 
 __all__ = [
-    "BAError", "ba_fwd", "ba_bwd", "ba_fwd_workspace_size", "ba_bwd_workspace_size",
+    "BAError", "ba_fwd", "ba_fwd_noalloc", "ba_bwd", "ba_fwd_workspace_size", "ba_bwd_workspace_size",
     "ba_device_status", "ba_set_profile_events", "ba_status_string", "ba_version", "block_attention_fwd",
     "block_attention_bwd", "library_path",
 ]
@@ -73,6 +73,8 @@ def _load():
     lib.ba_device_status.restype = ctypes.c_int
     lib.ba_status_string.argtypes = [ctypes.c_int]
     lib.ba_status_string.restype = ctypes.c_char_p
+    lib.ba_fwd_noalloc.argtypes = [prob, P, P, P, P, i32, i32, P, P, P, P]
+    lib.ba_fwd_noalloc.restype = ctypes.c_int
     lib.ba_set_profile_events.argtypes = [i32, P, P]
     lib.ba_set_profile_events.restype = ctypes.c_int
     lib.ba_version.argtypes = []
@@ -130,6 +132,13 @@ def ba_fwd(problem, q, k, v, seq_offsets, block, window, skip, out, lse, workspa
     return int(_load().ba_fwd(ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets),
                               int(block), int(window), _ptr(skip), _ptr(out), _ptr(lse),
                               _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def ba_fwd_noalloc(problem, q, k, v, seq_offsets, block, window, skip, out, lse, stream=None) -> int:
+    """Direct call of the no-allocation forward (scratch inside the library)."""
+    return int(_load().ba_fwd_noalloc(ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets),
+                                      int(block), int(window), _ptr(skip), _ptr(out), _ptr(lse),
+                                      _stream(stream)))
 
 
 def ba_bwd(problem, q, k, v, out, lse, dout, seq_offsets, block, window, skip, dq, dk, dv,

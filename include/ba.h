@@ -120,6 +120,28 @@ ba_status ba_bwd(const ba_problem *p, const void *q, const void *k, const void *
                  void *workspace, size_t workspace_bytes, ba_stream_t stream);
 
 /*
+ * Forward pass that allocates nothing and takes no workspace (the pages have
+ * no counterpart; this is a convenience of this library). For callers that
+ * cannot allocate device memory: a serving loop that records its forward into
+ * a CUDA graph (allocation is not allowed during stream capture), or a host
+ * framework that owns all device memory and hands kernels only their inputs
+ * and outputs. Same arguments and results as ba_fwd minus the workspace.
+ *  - Scratch: a fixed 1 MiB array inside the library, held by every GPU that
+ *    loads it until the process exits. Problems whose ba_fwd_workspace_size
+ *    exceeds 1 MiB are rejected with BA_ERR_INVALID_ARG before anything runs
+ *    (roughly: ceil(total_tokens / 128) + batch must stay below ~65,000).
+ *  - The first call on each device looks up the array's device address;
+ *    make that first call before any stream capture.
+ *  - All calls share the array: calls that may overlap on the GPU race and
+ *    must be ordered by the caller (one stream, or events). Nothing a call
+ *    reads from the array is left over from an earlier call.
+ *  - ba_device_status cannot be used with this entry point (no workspace).
+ */
+ba_status ba_fwd_noalloc(const ba_problem *p, const void *q, const void *k, const void *v,
+                         const int32_t *seq_offsets, int32_t block, int32_t window,
+                         const uint8_t *skip, void *out, float *lse, ba_stream_t stream);
+
+/*
  * Waits for `stream`, then reads the status word a previous ba_fwd/ba_bwd
  * left in `workspace`: BA_OK, or BA_ERR_TIMEOUT if a kernel gave up waiting
  * (its outputs are then undefined). BA_ERR_CUDA if the read itself failed.
