@@ -256,7 +256,8 @@ def main():
         if dist is not None:
             dist.barrier()
 
-    launches_per_step = (2 + (skip is not None)) + (4 + (skip is not None))
+    # ba_fwd: work list, (skip), attention; ba_bwd: work list, (skip), dQ, dK/dV
+    launches_per_step = (2 + (skip is not None)) + (3 + (skip is not None))
 
     for _ in range(args.warmup):
         step()
@@ -267,8 +268,9 @@ def main():
     K = args.steps
     ev = lambda: torch.cuda.Event(enable_timing=True)
     kf = [(ev(), ev()) for _ in range(K)]
+    kq = [(ev(), ev()) for _ in range(K)]
     kb = [(ev(), ev()) for _ in range(K)]
-    for pair in kf + kb:  # torch creates the CUDA event on its first record
+    for pair in kf + kq + kb:  # torch creates the CUDA event on its first record
         for e in pair:
             e.record(stream)
     t_start, t_stop = ev(), ev()
@@ -279,17 +281,19 @@ def main():
     t_start.record(stream)
     for i in range(K):
         ba.ba_set_profile_events(0, *kf[i])
-        ba.ba_set_profile_events(1, *kb[i])
+        ba.ba_set_profile_events(1, *kq[i])
+        ba.ba_set_profile_events(2, *kb[i])
         step()
     t_stop.record(stream)
-    ba.ba_set_profile_events(0)
-    ba.ba_set_profile_events(1)
+    for which in range(3):
+        ba.ba_set_profile_events(which)
     barrier()
     clocks.mark("t1")
     clk = clocks.stop()
     ms_total = t_start.elapsed_time(t_stop)
     ms_fwd_k = statistics.mean(a.elapsed_time(b) for a, b in kf)
-    ms_bwd_k = statistics.mean(a.elapsed_time(b) for a, b in kb)
+    ms_dq_k = statistics.mean(a.elapsed_time(b) for a, b in kq)
+    ms_dkv_k = statistics.mean(a.elapsed_time(b) for a, b in kb)
     if ba.ba_device_status(ws_f) != ba.BA_OK or ba.ba_device_status(ws_b) != ba.BA_OK:
         raise RuntimeError("a kernel timed out during the timed steps")
 
@@ -350,22 +354,28 @@ def main():
     peaks, peaks_src = load_peaks()
     tensor_peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     burst_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    bwd_achieved = fl["bwd"] / (ms_bwd_k / 1e3) / 1e12
-    fwd_achieved = fl["fwd"] / (ms_fwd_k / 1e3) / 1e12
+    # Per kernel, the FLOPs its own tensor-core work does on visible pairs: forward 4 D (S, PV),
+    # dQ pass 6 D (S, dP, dQ), dK/dV pass 8 D (S, dP, dV, dK); per visible pair and head.
+    unit = pairs * H * D
+    kern = {"fwd": (4 * unit, ms_fwd_k), "bwd_dq": (6 * unit, ms_dq_k), "bwd_dkdv": (8 * unit, ms_dkv_k)}
+    kstats = {n: {"ms": ms, "tflops": f / (ms / 1e3) / 1e12, "flops_per_launch": f} for n, (f, ms) in kern.items()}
+    dom = max(kstats, key=lambda n: kstats[n]["ms"])
+    names = {"fwd": "fwd_bf16_sm100_kernel", "bwd_dq": "bwd_dq_sm100_kernel", "bwd_dkdv": "bwd_dkdv_sm100_kernel"}
     traffic = None
     try:
         with open(args.traffic_file) as f:
             tr = json.load(f)
-        key = f"bwd_bf16_sm100:config{args.config}"
-        if key in tr and tr[key].get("kernel_sha") == kernel_sha():
+        key = f"{names[dom]}:config{args.config}"
+        if key in tr and tr[key].get("kernel_sha") == kernel_sha(dom):
             traffic = tr[key]["bytes_per_launch"]
     except (OSError, ValueError):
         pass
-    roofline = {"kernel": "bwd_d128_sm100_kernel" if D == 128 else "bwd_bf16_sm100_kernel", "bound": "tensor", "achieved": bwd_achieved,
-                "peak": tensor_peak, "unit": "TFLOP/s", "frac": bwd_achieved / tensor_peak,
-                "traffic": traffic, "peak_source": f"{peaks_src} bf16_tflops_sustained",
-                "algorithmic_flops_per_launch": fl["bwd"], "ms_per_launch": ms_bwd_k,
-                "share_of_step": ms_bwd_k * K / ms_total}
+    achieved = kstats[dom]["tflops"]
+    roofline = {"kernel": names[dom], "bound": "tensor", "achieved": achieved, "peak": tensor_peak,
+                "unit": "TFLOP/s", "frac": achieved / tensor_peak, "traffic": traffic,
+                "peak_source": f"{peaks_src} bf16_tflops_sustained",
+                "algorithmic_flops_per_launch": kstats[dom]["flops_per_launch"],
+                "ms_per_launch": kstats[dom]["ms"], "share_of_step": kstats[dom]["ms"] * K / ms_total}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
@@ -379,8 +389,7 @@ def main():
         "tokens_per_s": job_tokens / (ms_max / 1e3),
         "pct_of_bf16_peak": {"sustained": value / tensor_peak, "burst": value / burst_peak,
                              "source": peaks_src},
-        "kernels": {"fwd": {"ms": ms_fwd_k, "tflops": fwd_achieved},
-                    "bwd": {"ms": ms_bwd_k, "tflops": bwd_achieved}},
+        "kernels": kstats,
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": launches_per_step * K,
@@ -393,10 +402,11 @@ def main():
         dist.destroy_process_group()
 
 
-def kernel_sha() -> str:
-    """Hash of the backward kernel source, to tell whether stored counters are current."""
+def kernel_sha(which: str) -> str:
+    """Hash of a kernel's source file, to tell whether stored counters are current."""
     import hashlib
-    p = os.path.join(ROOT, "block_sparse_attention_kunlun_b200", "csrc", "ba_bwd_d128_sm100.cu")
+    src = {"fwd": "ba_fwd_sm100.cu", "bwd_dq": "ba_bwd_dq_sm100.cu", "bwd_dkdv": "ba_bwd_dkdv_sm100.cu"}[which]
+    p = os.path.join(ROOT, "block_sparse_attention_kunlun_b200", "csrc", src)
     with open(p, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 

@@ -153,8 +153,9 @@ def ba_bwd(problem, q, k, v, out, lse, dout, seq_offsets, block, window, skip, d
 
 
 def ba_set_profile_events(which: int, start=None, stop=None) -> int:
-    """Record torch.cuda.Event ``start``/``stop`` around the attention kernel of
-    every later ba_fwd (which=0) or ba_bwd (which=1) call from this thread.
+    """Record torch.cuda.Event ``start``/``stop`` around one kernel of every
+    later call from this thread: 0 the forward attention kernel, 1 the
+    backward dQ kernel, 2 the backward dK/dV kernel.
     The events must already exist on the device (torch creates an event on
     its first ``record``)."""
     s = start.cuda_event if start is not None else None

@@ -18,8 +18,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libba.so")
 OBJDIR = os.path.join(HERE, "_build")
 
-SOURCES = ["ba_api.cu", "ba_aux.cu", "ba_simt.cu", "ba_fwd_sm100.cu", "ba_bwd_sm100.cu",
-           "ba_bwd_d128_sm100.cu", "ba_noalloc.cu"]
+SOURCES = ["ba_api.cu", "ba_aux.cu", "ba_simt.cu", "ba_fwd_sm100.cu", "ba_bwd_dq_sm100.cu",
+           "ba_bwd_dkdv_sm100.cu", "ba_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

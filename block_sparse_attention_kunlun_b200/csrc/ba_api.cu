@@ -3,8 +3,9 @@
 //
 //   ba_fwd: worklist -> skip passthrough (if any flags) -> forward kernel
 //           (tcgen05 for bf16, SIMT for fp32)
-//   ba_bwd: worklist -> Delta and dq-accumulator reset -> skip passthrough ->
-//           backward kernel -> dq conversion (bf16) or direct dq (fp32)
+//   ba_bwd: worklist -> skip passthrough -> bf16: dQ kernel (also writes
+//           Delta) -> dK/dV kernel; fp32: Delta pre-pass -> dQ and dK/dV
+//           SIMT kernels
 // Nothing here allocates, synchronises or falls back to another device.
 #include "ba.h"
 #include "ba_common.cuh"
@@ -116,7 +117,7 @@ Problem make_problem(const ba_problem &pp, const int32_t *offs, const uint8_t *s
     return p;
 }
 
-thread_local cudaEvent_t t_prof[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+thread_local cudaEvent_t t_prof[3][2] = {{nullptr, nullptr}, {nullptr, nullptr}, {nullptr, nullptr}};
 
 cudaError_t prof_mark(int which, int edge, cudaStream_t stream)
 {
@@ -142,7 +143,7 @@ size_t ba_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
 size_t ba_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
 {
     if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
-    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, true, p->dtype == BA_BF16).total;
+    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, true, false).total;
 }
 
 ba_status ba_fwd(const ba_problem *pp, const void *q, const void *k, const void *v, const int32_t *seq_offsets,
@@ -200,7 +201,7 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
         (T > 0 && (!lse || !aligned(lse, 4))))
         return BA_ERR_INVALID_ARG;
     const bool bf16 = P.dtype == BA_BF16;
-    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, true, bf16);
+    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, true, false);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total) return BA_ERR_INVALID_ARG;
     int num_sms = 0, cc = 0;
     if (!device_info(num_sms, cc)) return BA_ERR_CUDA;
@@ -210,33 +211,37 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
     const Problem p = make_problem(P, seq_offsets, skip, block, window, workspace, lay);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     float *delta = reinterpret_cast<float *>(ws + lay.delta);
-    float *dq_acc = bf16 ? reinterpret_cast<float *>(ws + lay.dq_acc) : nullptr;
     BA_TRY(launch_worklist(p, stream));
     if (T == 0) return BA_OK;
     const size_t esz = bf16 ? 2 : 4;
-    if (bf16) BA_TRY(launch_bwd_pre<__nv_bfloat16>(p, out, dout, delta, dq_acc, num_sms, stream));
-    else BA_TRY(launch_bwd_pre<float>(p, out, dout, delta, nullptr, num_sms, stream));
-    BA_TRY(launch_skip_bwd(p, esz, dout, bf16 ? nullptr : dq, dk, dv, stream));
+    BA_TRY(launch_skip_bwd(p, esz, dout, dq, dk, dv, stream));
     if (!bf16) {
+        BA_TRY(launch_bwd_pre<float>(p, out, dout, delta, nullptr, num_sms, stream));
         BA_TRY(prof_mark(1, 0, stream));
         BA_TRY(launch_bwd_f32(p, static_cast<const float *>(q), static_cast<const float *>(k),
                               static_cast<const float *>(v), static_cast<const float *>(dout), lse, delta,
                               static_cast<float *>(dq), static_cast<float *>(dk), static_cast<float *>(dv), num_sms,
                               stream));
-        BA_TRY(prof_mark(1, 1, stream));
+        BA_TRY(prof_mark(2, 1, stream));
         return BA_OK;
     }
-    CUtensorMap tq, tk, tv, tdo;
+    CUtensorMap tq, tk, tv, tdo, to;
     if (!encode_bf16_rows(&tq, q, T, P.heads, P.head_dim) || !encode_bf16_rows(&tk, k, T, P.heads, P.head_dim) ||
-        !encode_bf16_rows(&tv, v, T, P.heads, P.head_dim) || !encode_bf16_rows(&tdo, dout, T, P.heads, P.head_dim))
+        !encode_bf16_rows(&tv, v, T, P.heads, P.head_dim) || !encode_bf16_rows(&tdo, dout, T, P.heads, P.head_dim) ||
+        !encode_bf16_rows(&to, out, T, P.heads, P.head_dim))
         return BA_ERR_CUDA;
     BA_TRY(prof_mark(1, 0, stream));
     if (P.head_dim == 64)
-        BA_TRY(launch_bwd_bf16_sm100<64>(tq, tk, tv, tdo, p, lse, delta, dq_acc, dk, dv, num_sms, stream));
+        BA_TRY(launch_bwd_dq_sm100<64>(tq, tk, tv, tdo, to, p, lse, delta, dq, num_sms, stream));
     else
-        BA_TRY(launch_bwd_d128_sm100(tq, tk, tv, tdo, p, lse, delta, dq_acc, dk, dv, num_sms, stream));
+        BA_TRY(launch_bwd_dq_sm100<128>(tq, tk, tv, tdo, to, p, lse, delta, dq, num_sms, stream));
     BA_TRY(prof_mark(1, 1, stream));
-    BA_TRY(launch_dq_convert<__nv_bfloat16>(p, dq_acc, dq, num_sms, stream));
+    BA_TRY(prof_mark(2, 0, stream));
+    if (P.head_dim == 64)
+        BA_TRY(launch_bwd_dkdv_sm100<64>(tq, tk, tv, tdo, p, lse, delta, dk, dv, num_sms, stream));
+    else
+        BA_TRY(launch_bwd_dkdv_sm100<128>(tq, tk, tv, tdo, p, lse, delta, dk, dv, num_sms, stream));
+    BA_TRY(prof_mark(2, 1, stream));
     return BA_OK;
 }
 
@@ -253,7 +258,7 @@ ba_status ba_device_status(const void *workspace, ba_stream_t stream_)
 
 ba_status ba_set_profile_events(int32_t which, void *start, void *stop)
 {
-    if (which != 0 && which != 1) return BA_ERR_INVALID_ARG;
+    if (which < 0 || which > 2) return BA_ERR_INVALID_ARG;
     t_prof[which][0] = static_cast<cudaEvent_t>(start);
     t_prof[which][1] = static_cast<cudaEvent_t>(stop);
     return BA_OK;

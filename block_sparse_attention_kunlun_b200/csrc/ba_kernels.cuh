@@ -31,13 +31,14 @@ cudaError_t launch_bwd_f32(const Problem &p, const float *q, const float *k, con
 template <int D>
 cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const Problem &p, void *out, float *lse, int num_sms, cudaStream_t stream);
-template <int D>
-cudaError_t launch_bwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                  const CUtensorMap &tdo, const Problem &p, const float *lse, const float *delta,
-                                  float *dq_acc, void *dk, void *dv, int num_sms, cudaStream_t stream);
 
-cudaError_t launch_bwd_d128_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+template <int D>
+cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                const CUtensorMap &tdo, const CUtensorMap &to, const Problem &p, const float *lse,
+                                float *delta, void *dq, int num_sms, cudaStream_t stream);
+template <int D>
+cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &tdo, const Problem &p, const float *lse, const float *delta,
-                                  float *dq_acc, void *dk, void *dv, int num_sms, cudaStream_t stream);
+                                  void *dk, void *dv, int num_sms, cudaStream_t stream);
 
 } // namespace ba

@@ -90,8 +90,8 @@ typedef struct {
 
 /*
  * Bytes of workspace ba_fwd / ba_bwd need for this problem (0 on an invalid
- * problem). The backward's includes a float32 dq accumulator
- * [heads, total_tokens, head_dim] and a float32 row-dot buffer
+ * problem): a status word and a work table of about 16 bytes per 128-row
+ * tile, plus, for the backward, a float32 row-dot buffer Delta
  * [heads, total_tokens].
  */
 size_t ba_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window);
@@ -149,13 +149,14 @@ ba_status ba_fwd_noalloc(const ba_problem *p, const void *q, const void *k, cons
 ba_status ba_device_status(const void *workspace, ba_stream_t stream);
 
 /*
- * Profiling hook. Until changed, every ba_fwd (which = 0) or ba_bwd
- * (which = 1) call made from THIS host thread records `start` on its stream
- * right before launching its attention kernel and `stop` right after it, so
- * that cudaEventElapsedTime(start, stop) is that kernel's own duration. The
- * events are cudaEvent_t handles owned by the caller; pass NULL, NULL to
- * stop recording. Returns BA_ERR_INVALID_ARG for another `which`. Only the
- * hook pointers are stored (thread-local); nothing is synchronised.
+ * Profiling hook. Until changed, calls made from THIS host thread record
+ * `start` on their stream right before one kernel and `stop` right after it,
+ * so that cudaEventElapsedTime(start, stop) is that kernel's own duration:
+ * which = 0 the forward attention kernel of ba_fwd, 1 the dQ kernel of
+ * ba_bwd, 2 its dK/dV kernel. The events are cudaEvent_t handles owned by
+ * the caller; pass NULL, NULL to stop recording. Returns BA_ERR_INVALID_ARG
+ * for another `which`. Only the hook pointers are stored (thread-local);
+ * nothing is synchronised.
  */
 ba_status ba_set_profile_events(int32_t which, void *start, void *stop);
 

@@ -43,10 +43,10 @@ def test_workspace_sizes():
     f = ba.ba_fwd_workspace_size(p, 128, 2)
     b = ba.ba_bwd_workspace_size(p, 128, 2)
     assert f >= 256 + 4 * 4 and f % 256 == 0
-    # backward adds Delta (H*T floats) and the fp32 dq accumulator (H*T*D floats)
-    assert b >= f + 4 * 2 * 1000 + 4 * 2 * 1000 * 128
-    pf = prob(batch=3, T=1000, H=2, D=64, dt=ba.BA_F32)
-    assert ba.ba_bwd_workspace_size(pf, 128, 2) < ba.ba_bwd_workspace_size(prob(3, 1000, 2, 64), 128, 2)
+    # backward adds Delta (H*T floats)
+    assert f + 4 * 2 * 1000 <= b <= f + 4 * 2 * 1000 + 256
+    # the work table grows with the number of 128-row tiles
+    assert ba.ba_fwd_workspace_size(prob(batch=3, T=100000, H=2, D=128), 128, 2) >= 16 * (100000 // 128)
     assert ba.ba_fwd_workspace_size(prob(batch=-1), 128, 2) == 0
     assert ba.ba_fwd_workspace_size(p, 0, 2) == 0
     assert ba.ba_fwd_workspace_size(p, 128, 0) == 0
