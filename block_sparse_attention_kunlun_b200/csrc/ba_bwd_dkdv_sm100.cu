@@ -20,15 +20,16 @@
 //              lane t), group g the queries [64g, 64g+64) of each query tile.
 //              They read S^T (then release it, so the next tile's S^T can be
 //              issued while they work), form P^T, read dP^T, form dS^T and
-//              write P^T and dS^T as bf16 over their dP^T columns; at the end
-//              of the item group 0 stores dV and group 1 stores dK.
-//   warp 8     TMA producer: K, V per item (with an L2 prefetch of the next
+//              write P^T and dS^T as bf16 over their dP^T columns.
+//   warps 8-11 epilogue: at the end of an item, move dV and dK from TMEM to
+//              global memory while the compute warps start the next item.
+//   warp 12    TMA producer: K, V per item (with an L2 prefetch of the next
 //              item's); Q, dO per query tile into a ring.
-//   warp 9     MMA issuer.
+//   warp 13    MMA issuer.
 // TMEM columns: S^T [0,128), dP^T [128,256), dV [256, 256+D), dK [256+D,
 // 256+2D). After the compute warps have read group g's dP^T columns
-// [128+64g, 192+64g), each 32-query half h2 of the group holds P^T (bf16) in
-// [128+64g+32h2, +16) and dS^T in the next 16 columns.
+// [128+64g, 192+64g), each 16-query block b of the group holds P^T (bf16) in
+// [128+64g+16b, +8) and dS^T in the next 8 columns.
 #include "ba_common.cuh"
 #include "ba_kernels.cuh"
 #include "ba_ptx.cuh"
@@ -51,7 +52,7 @@ struct DkvLayout {
     static constexpr int kQ0 = 2 * kTileBytes;           // stage s: Q at kQ0 + 2 s tile, dO after it
     static constexpr int kBytes = kQ0 + 2 * kStages * kTileBytes;
     static constexpr int kAlloc = kBytes + 1024;
-    static constexpr int kThreads = 320;
+    static constexpr int kThreads = 448;
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
     static constexpr uint32_t kTmemCols = 512;
 };
@@ -62,8 +63,8 @@ struct DkvBarriers {
     uint64_t s_full, s_free, dp_full, ds_full[2];
     uint32_t tmem_base;
     int abort;
-    float lse2[2][kTile];
-    float delta[2][kTile];
+    __align__(16) float lse2[2][kTile];
+    __align__(16) float delta[2][kTile];
 };
 
 __device__ __forceinline__ void query_tile_range(const TileRef &r, int64_t B, int64_t W, int &ilo, int &ihi)
@@ -76,7 +77,7 @@ __device__ __forceinline__ void query_tile_range(const TileRef &r, int64_t B, in
 } // namespace
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                           const Problem p, const float *__restrict__ lse, const float *__restrict__ delta,
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(320, 1)
         mbar_init(&sb.kv_full, 1);
         mbar_init(&sb.kv_empty, 1);
         mbar_init(&sb.dkv_full, 1);
-        mbar_init(&sb.dkv_free, 8);
+        mbar_init(&sb.dkv_free, 4);
         for (int i = 0; i < S; ++i) {
             mbar_init(&sb.qo_full[i], 1);
             mbar_init(&sb.qo_empty[i], 1);
@@ -108,13 +109,13 @@ __global__ void __launch_bounds__(320, 1)
         sb.abort = 0;
         fence_mbar_init();
     }
-    if (warp == 8 && lane == 0) {
+    if (warp == 12 && lane == 0) {
         tma_prefetch_map(&tm_q);
         tma_prefetch_map(&tm_k);
         tma_prefetch_map(&tm_v);
         tma_prefetch_map(&tm_do);
     }
-    if (warp == 9) {
+    if (warp == 13) {
         tmem_alloc(&sb.tmem_base, Lay::kTmemCols);
         tmem_relinquish();
     }
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(320, 1)
     const int64_t T = p.total_tokens;
     const int32_t ntiles = live_tile_count(p);
 
-    if (warp == 8) {
+    if (warp == 12) {
         // ------------------------------------------------ TMA producer ---
         uint32_t it = 0, item_cnt = 0;
         TileRef r;
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(320, 1)
                 __syncwarp();
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == 13) {
         // -------------------------------------------------- MMA issuer ---
         constexpr uint32_t idesc_sp = idesc_bf16(128, 128, false, false); // S^T, dP^T
         constexpr uint32_t idesc_kv = idesc_bf16(128, D, false, true);    // dV, dK (B MN-major)
@@ -194,11 +195,11 @@ __global__ void __launch_bounds__(320, 1)
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t boff = (4 * g + kk) * 2048; // query rows 64g + 16kk ..
                         const uint32_t acc = (m > 0 || g > 0 || kk > 0) ? 1u : 0u;
-                        // P^T of queries 16kk.. at column 32(kk/2) + 8(kk%2), dS^T 16 columns later
-                        const uint32_t acol = pcol + 32 * (kk >> 1) + 8 * (kk & 1);
+                        // P^T of queries 64g + 16kk .. at column 16kk of the group, dS^T 8 columns later
+                        const uint32_t acol = pcol + 16 * kk;
                         mma_ts(tmem + Lay::kColDV, acol, sdesc_sw128(o_addr + boff, Lay::kChunkBytes, 1024),
                                idesc_kv, acc);
-                        mma_ts(tmem + Lay::kColDK, acol + 16, sdesc_sw128(q_addr + boff, Lay::kChunkBytes, 1024),
+                        mma_ts(tmem + Lay::kColDK, acol + 8, sdesc_sw128(q_addr + boff, Lay::kChunkBytes, 1024),
                                idesc_kv, acc);
                     }
                     if (g == 1) tc_commit(&sb.qo_empty[st]);
@@ -257,13 +258,13 @@ __global__ void __launch_bounds__(320, 1)
             if (lane == 0) tc_commit(&sb.dkv_full);
             __syncwarp();
         }
-    } else {
+    } else if (warp < 8) {
         // ----------------------------------------------------- compute ---
         const int g = warp >> 2;              // column group: queries [64g, 64g+64)
         const int row = threadIdx.x & 127;    // key row within the tile, TMEM lane
         const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
         const float scale_log2 = p.scale * 1.4426950408889634f;
-        uint32_t it = 0, item_cnt = 0;
+        uint32_t it = 0;
         TileRef r;
         bool ok = true;
         // lse (log2 units, group 0) or Delta (group 1) of query row `row` of tile i
@@ -273,7 +274,7 @@ __global__ void __launch_bounds__(320, 1)
             const int64_t gi = int64_t(rr.h) * T + rr.s0 + q;
             return g == 0 ? lse[gi] * 1.4426950408889634f : delta[gi];
         };
-        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
+        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x) {
             int ilo, ihi;
             query_tile_range(r, B, W, ilo, ihi);
             const int64_t k = int64_t(r.t) * kTile + row; // local key index
@@ -291,8 +292,8 @@ __global__ void __launch_bounds__(320, 1)
                 const int lo_c = int(lo64 < -1 ? -1 : (lo64 > 64 ? 64 : lo64));
                 const int hi_c = int(hi64 < -1 ? -1 : (hi64 > 64 ? 64 : hi64));
                 const bool full = __all_sync(0xffffffffu, lo_c <= 0 && hi_c >= 63);
-                const float *l2s = sb.lse2[buf] + 64 * g;
-                const float *dls = sb.delta[buf] + 64 * g;
+                const float4 *l2v = reinterpret_cast<const float4 *>(sb.lse2[buf] + 64 * g);
+                const float4 *dlv = reinterpret_cast<const float4 *>(sb.delta[buf] + 64 * g);
                 // phase A: P^T from S^T
                 if (!mbar_wait(&sb.s_full, it & 1, abort)) { ok = false; break; }
                 tc_fence_after();
@@ -303,79 +304,105 @@ __global__ void __launch_bounds__(320, 1)
                     tmem_ld32(tmem + lane_base + Lay::kColS + 64 * g + 32 * h2, sr);
                     tmem_wait_ld();
                     reg_fence(sr);
-                    if (h2 == 1) { // both halves read: the next tile's S may overwrite them
+                    if (h2 == 1) { // both halves read: the next tile's S^T may overwrite them
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&sb.s_free);
                     }
-                    if (full) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            pr[32 * h2 + c] = ex2_approx(fmaf(__uint_as_float(sr[c]), scale_log2, -l2s[32 * h2 + c]));
-                    } else {
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 l4 = l2v[8 * h2 + c4];
+                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            const int cc = 32 * h2 + c;
-                            const float e = ex2_approx(fmaf(__uint_as_float(sr[c]), scale_log2, -l2s[32 * h2 + c]));
-                            pr[cc] = (cc >= lo_c && cc <= hi_c) ? e : 0.f;
+                        for (int e = 0; e < 4; ++e) {
+                            const int cc = 32 * h2 + 4 * c4 + e;
+                            const float x = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + e]), scale_log2, -lv[e]));
+                            pr[cc] = (full || (cc >= lo_c && cc <= hi_c)) ? x : 0.f;
                         }
                     }
                 }
-                // phase B: dS^T = P^T (dP^T - Delta); P^T and dS^T (bf16) over this group's dP^T columns
+                // phase B: dS^T = P^T (dP^T - Delta); 16 queries at a time, P^T and dS^T (bf16)
+                // written over exactly the 16 dP^T columns just read
                 if (!mbar_wait(&sb.dp_full, it & 1, abort)) { ok = false; break; }
                 tc_fence_after();
-                // 32 queries at a time; chunk h2 writes P^T to [64g+32h2, +16) and dS^T to
-                // [64g+32h2+16, +16), both inside the columns it has just read.
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t dr[32];
-                    tmem_ld32(tmem + lane_base + Lay::kColDP + 64 * g + 32 * h2, dr);
+                for (int b = 0; b < 4; ++b) {
+                    uint32_t dr[16];
+                    tmem_ld16(tmem + lane_base + Lay::kColDP + 64 * g + 16 * b, dr);
                     tmem_wait_ld();
                     reg_fence(dr);
-                    uint32_t pk[16], dk16[16];
+                    uint32_t pk[8], dk8[8];
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const int q0c = 32 * h2 + 2 * c;
-                        pk[c] = pack_bf16x2(pr[q0c], pr[q0c + 1]);
-                        dk16[c] = pack_bf16x2(pr[q0c] * (__uint_as_float(dr[2 * c]) - dls[q0c]),
-                                              pr[q0c + 1] * (__uint_as_float(dr[2 * c + 1]) - dls[q0c + 1]));
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const float4 d4 = dlv[4 * b + c4];
+                        const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int q = 16 * b + 4 * c4 + 2 * e;
+                            const int j = 4 * c4 + 2 * e;
+                            pk[2 * c4 + e] = pack_bf16x2(pr[q], pr[q + 1]);
+                            dk8[2 * c4 + e] = pack_bf16x2(pr[q] * (__uint_as_float(dr[j]) - dv4[2 * e]),
+                                                          pr[q + 1] * (__uint_as_float(dr[j + 1]) - dv4[2 * e + 1]));
+                        }
                     }
-                    tmem_st16(tmem + lane_base + Lay::kColDP + 64 * g + 32 * h2, pk);
-                    tmem_st16(tmem + lane_base + Lay::kColDP + 64 * g + 32 * h2 + 16, dk16);
+                    tmem_st8(tmem + lane_base + Lay::kColDP + 64 * g + 16 * b, pk);
+                    tmem_st8(tmem + lane_base + Lay::kColDP + 64 * g + 16 * b + 8, dk8);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sb.ds_full[g]);
             }
-            if (!ok) break;
-            // epilogue: group 0 stores dV, group 1 stores dK
+        }
+    } else if (warp < 12) {
+        // ---------------------------------------------------- epilogue ---
+        const int row = threadIdx.x & 127;    // key row within the tile, TMEM lane
+        const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+        uint32_t item_cnt = 0;
+        TileRef r;
+        for (int64_t n = blockIdx.x; decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
+            const int64_t k = int64_t(r.t) * kTile + row;
+            const bool valid_k = k < r.L;
+            const int64_t grow = (int64_t(r.s0) + k) * p.heads + r.h;
             if (!mbar_wait(&sb.dkv_full, item_cnt & 1, abort)) break;
             tc_fence_after();
-            {
-                const uint32_t col0 = g == 0 ? Lay::kColDV : Lay::kColDK;
-                const float mul = g == 0 ? 1.f : p.scale;
-                __nv_bfloat16 *dst_row = (g == 0 ? dv : dk) + ((int64_t(r.s0) + k) * p.heads + r.h) * D;
+            // dV: load and store chunk by chunk
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t rr[32];
-                    tmem_ld32(tmem + lane_base + col0 + c * 32, rr);
-                    tmem_wait_ld();
-                    reg_fence(rr);
-                    if (valid_k) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(dst_row + c * 32);
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t rr[32];
+                tmem_ld32(tmem + lane_base + Lay::kColDV + c * 32, rr);
+                tmem_wait_ld();
+                reg_fence(rr);
+                if (valid_k) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(dv + grow * D + c * 32);
 #pragma unroll
-                        for (int x = 0; x < 4; ++x)
-                            dst[x] = make_uint4(
-                                pack_bf16x2(__uint_as_float(rr[8 * x + 0]) * mul, __uint_as_float(rr[8 * x + 1]) * mul),
-                                pack_bf16x2(__uint_as_float(rr[8 * x + 2]) * mul, __uint_as_float(rr[8 * x + 3]) * mul),
-                                pack_bf16x2(__uint_as_float(rr[8 * x + 4]) * mul, __uint_as_float(rr[8 * x + 5]) * mul),
-                                pack_bf16x2(__uint_as_float(rr[8 * x + 6]) * mul, __uint_as_float(rr[8 * x + 7]) * mul));
-                    }
+                    for (int x = 0; x < 4; ++x)
+                        dst[x] = make_uint4(pack_bf16x2(__uint_as_float(rr[8 * x + 0]), __uint_as_float(rr[8 * x + 1])),
+                                            pack_bf16x2(__uint_as_float(rr[8 * x + 2]), __uint_as_float(rr[8 * x + 3])),
+                                            pack_bf16x2(__uint_as_float(rr[8 * x + 4]), __uint_as_float(rr[8 * x + 5])),
+                                            pack_bf16x2(__uint_as_float(rr[8 * x + 6]), __uint_as_float(rr[8 * x + 7])));
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sb.dkv_free);
+            }
+            // dK: take it all out of TMEM, release the accumulators, then store
+            uint32_t kp[D / 2];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t rr[32];
+                tmem_ld32(tmem + lane_base + Lay::kColDK + c * 32, rr);
+                tmem_wait_ld();
+                reg_fence(rr);
+#pragma unroll
+                for (int x = 0; x < 16; ++x)
+                    kp[16 * c + x] = pack_bf16x2(__uint_as_float(rr[2 * x]) * p.scale,
+                                                 __uint_as_float(rr[2 * x + 1]) * p.scale);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sb.dkv_free);
+            if (valid_k) {
+                uint4 *dst = reinterpret_cast<uint4 *>(dk + grow * D);
+#pragma unroll
+                for (int x = 0; x < D / 8; ++x) dst[x] = make_uint4(kp[4 * x], kp[4 * x + 1], kp[4 * x + 2], kp[4 * x + 3]);
             }
         }
     }
@@ -383,7 +410,7 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 9) tmem_dealloc(tmem, Lay::kTmemCols);
+    if (warp == 13) tmem_dealloc(tmem, Lay::kTmemCols);
     if (threadIdx.x == 0 && sb.abort) atomicOr(p.status, kStatusTimeout);
 }
 
