@@ -106,6 +106,8 @@ Problem make_problem(const ba_problem &pp, const int32_t *offs, const uint8_t *s
     p.skip = skip;
     p.tile_prefix = reinterpret_cast<const int32_t *>(static_cast<uint8_t *>(workspace) + lay.tile_prefix);
     p.tile_info = reinterpret_cast<const int4 *>(static_cast<uint8_t *>(workspace) + lay.tile_info);
+    p.pair_prefix = reinterpret_cast<const int32_t *>(static_cast<uint8_t *>(workspace) + lay.pair_prefix);
+    p.pair_info = reinterpret_cast<const int4 *>(static_cast<uint8_t *>(workspace) + lay.pair_info);
     p.status = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + lay.status);
     p.batch = pp.batch;
     p.total_tokens = pp.total_tokens;

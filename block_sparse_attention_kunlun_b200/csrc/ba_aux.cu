@@ -34,24 +34,18 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 
 } // namespace
 
-__global__ void __launch_bounds__(kWorklistThreads)
-    worklist_kernel(const int32_t *__restrict__ offs, const uint8_t *__restrict__ skip, int32_t batch,
-                    int32_t *__restrict__ tile_prefix, int4 *__restrict__ tile_info, int *__restrict__ status)
+// Exclusive block-wide scan of one value per thread; returns the prefix and
+// stores the total in *total (read after the call's final barrier).
+__device__ __forceinline__ int32_t block_exclusive_scan(int32_t local, int32_t *warp_tot, int32_t &total)
 {
-    __shared__ int32_t warp_tot[kWorklistThreads / 32];
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int per = (batch + kWorklistThreads - 1) / kWorklistThreads;
-    const int b0 = tid * per;
-    const int b1 = min(batch, b0 + per);
-    int32_t local = 0;
-    for (int b = b0; b < b1; ++b) local += live_tiles(offs, skip, b);
-    // inclusive scan within the warp, then across warp totals
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     int32_t incl = local;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
         const int32_t y = __shfl_up_sync(0xffffffffu, incl, d);
         if (lane >= d) incl += y;
     }
+    __syncthreads();
     if (lane == 31) warp_tot[wid] = incl;
     __syncthreads();
     if (wid == 0) {
@@ -64,16 +58,44 @@ __global__ void __launch_bounds__(kWorklistThreads)
         warp_tot[lane] = w; // inclusive over warps
     }
     __syncthreads();
-    int32_t run = incl - local + (wid > 0 ? warp_tot[wid - 1] : 0);
+    total = warp_tot[kWorklistThreads / 32 - 1];
+    return incl - local + (wid > 0 ? warp_tot[wid - 1] : 0);
+}
+
+// Per live example: its 128-row tiles, and pairs of consecutive tiles (the
+// forward processes two query tiles of one example together).
+__global__ void __launch_bounds__(kWorklistThreads)
+    worklist_kernel(const int32_t *__restrict__ offs, const uint8_t *__restrict__ skip, int32_t batch,
+                    int32_t *__restrict__ tile_prefix, int4 *__restrict__ tile_info,
+                    int32_t *__restrict__ pair_prefix, int4 *__restrict__ pair_info, int *__restrict__ status)
+{
+    __shared__ int32_t warp_tot[kWorklistThreads / 32];
+    const int tid = threadIdx.x;
+    const int per = (batch + kWorklistThreads - 1) / kWorklistThreads;
+    const int b0 = tid * per;
+    const int b1 = min(batch, b0 + per);
+    int32_t ltiles = 0, lpairs = 0;
     for (int b = b0; b < b1; ++b) {
-        tile_prefix[b] = run;
+        const int32_t nt = live_tiles(offs, skip, b);
+        ltiles += nt;
+        lpairs += (nt + 1) / 2;
+    }
+    int32_t ttot, ptot;
+    int32_t trun = block_exclusive_scan(ltiles, warp_tot, ttot);
+    int32_t prun = block_exclusive_scan(lpairs, warp_tot, ptot);
+    for (int b = b0; b < b1; ++b) {
+        tile_prefix[b] = trun;
+        pair_prefix[b] = prun;
         const int32_t nt = live_tiles(offs, skip, b);
         const int32_t s0 = offs[b], L = offs[b + 1] - s0;
-        for (int32_t t = 0; t < nt; ++t) tile_info[run + t] = make_int4(s0, L, t, b);
-        run += nt;
+        for (int32_t t = 0; t < nt; ++t) tile_info[trun + t] = make_int4(s0, L, t, b);
+        for (int32_t t = 0; t < nt; t += 2) pair_info[prun + t / 2] = make_int4(s0, L, t, b);
+        trun += nt;
+        prun += (nt + 1) / 2;
     }
     if (tid == kWorklistThreads - 1) {
-        tile_prefix[batch] = warp_tot[kWorklistThreads / 32 - 1];
+        tile_prefix[batch] = ttot;
+        pair_prefix[batch] = ptot;
         *status = 0;
     }
 }
@@ -174,9 +196,9 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_worklist(const Problem &p, cudaStream_t stream)
 {
-    worklist_kernel<<<1, kWorklistThreads, 0, stream>>>(p.seq_offsets, p.skip, p.batch,
-                                                        const_cast<int32_t *>(p.tile_prefix),
-                                                        const_cast<int4 *>(p.tile_info), p.status);
+    worklist_kernel<<<1, kWorklistThreads, 0, stream>>>(
+        p.seq_offsets, p.skip, p.batch, const_cast<int32_t *>(p.tile_prefix), const_cast<int4 *>(p.tile_info),
+        const_cast<int32_t *>(p.pair_prefix), const_cast<int4 *>(p.pair_info), p.status);
     return cudaGetLastError();
 }
 

@@ -267,12 +267,12 @@ __global__ void __launch_bounds__(448, 1)
         uint32_t it = 0;
         TileRef r;
         bool ok = true;
-        // lse (log2 units, group 0) or Delta (group 1) of query row `row` of tile i
+        // -lse (log2 units, group 0) or -Delta (group 1) of query row `row` of tile i
         auto load_row = [&](const TileRef &rr, int i) -> float {
             const int64_t q = int64_t(i) * kTile + row;
-            if (q >= rr.L) return g == 0 ? INFINITY : 0.f;
+            if (q >= rr.L) return g == 0 ? -INFINITY : 0.f;
             const int64_t gi = int64_t(rr.h) * T + rr.s0 + q;
-            return g == 0 ? lse[gi] * 1.4426950408889634f : delta[gi];
+            return g == 0 ? -lse[gi] * 1.4426950408889634f : -delta[gi];
         };
         for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x) {
             int ilo, ihi;
@@ -292,6 +292,7 @@ __global__ void __launch_bounds__(448, 1)
                 const int lo_c = int(lo64 < -1 ? -1 : (lo64 > 64 ? 64 : lo64));
                 const int hi_c = int(hi64 < -1 ? -1 : (hi64 > 64 ? 64 : hi64));
                 const bool full = __all_sync(0xffffffffu, lo_c <= 0 && hi_c >= 63);
+                // shared copies hold -lse (log2 units) and -Delta, so each use is one packed FMA/add
                 const float4 *l2v = reinterpret_cast<const float4 *>(sb.lse2[buf] + 64 * g);
                 const float4 *dlv = reinterpret_cast<const float4 *>(sb.delta[buf] + 64 * g);
                 // phase A: P^T from S^T
@@ -309,14 +310,19 @@ __global__ void __launch_bounds__(448, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&sb.s_free);
                     }
+                    const float2 sc2 = make_float2(scale_log2, scale_log2);
 #pragma unroll
                     for (int c4 = 0; c4 < 8; ++c4) {
-                        const float4 l4 = l2v[8 * h2 + c4];
-                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                        const float4 l4 = l2v[8 * h2 + c4]; // -lse of 4 queries
+                        const float2 x01 = ffma2(make_float2(__uint_as_float(sr[4 * c4]), __uint_as_float(sr[4 * c4 + 1])),
+                                                 sc2, make_float2(l4.x, l4.y));
+                        const float2 x23 = ffma2(make_float2(__uint_as_float(sr[4 * c4 + 2]), __uint_as_float(sr[4 * c4 + 3])),
+                                                 sc2, make_float2(l4.z, l4.w));
+                        const float xv[4] = {x01.x, x01.y, x23.x, x23.y};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int cc = 32 * h2 + 4 * c4 + e;
-                            const float x = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + e]), scale_log2, -lv[e]));
+                            const float x = ex2_approx(xv[e]);
                             pr[cc] = (full || (cc >= lo_c && cc <= hi_c)) ? x : 0.f;
                         }
                     }
@@ -334,16 +340,18 @@ __global__ void __launch_bounds__(448, 1)
                     uint32_t pk[8], dk8[8];
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
-                        const float4 d4 = dlv[4 * b + c4];
-                        const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int q = 16 * b + 4 * c4 + 2 * e;
-                            const int j = 4 * c4 + 2 * e;
-                            pk[2 * c4 + e] = pack_bf16x2(pr[q], pr[q + 1]);
-                            dk8[2 * c4 + e] = pack_bf16x2(pr[q] * (__uint_as_float(dr[j]) - dv4[2 * e]),
-                                                          pr[q + 1] * (__uint_as_float(dr[j + 1]) - dv4[2 * e + 1]));
-                        }
+                        const float4 d4 = dlv[4 * b + c4]; // -Delta of 4 queries
+                        const int q = 16 * b + 4 * c4, j = 4 * c4;
+                        const float2 ds01 = fmul2(make_float2(pr[q], pr[q + 1]),
+                                                  fadd2(make_float2(__uint_as_float(dr[j]), __uint_as_float(dr[j + 1])),
+                                                        make_float2(d4.x, d4.y)));
+                        const float2 ds23 = fmul2(make_float2(pr[q + 2], pr[q + 3]),
+                                                  fadd2(make_float2(__uint_as_float(dr[j + 2]), __uint_as_float(dr[j + 3])),
+                                                        make_float2(d4.z, d4.w)));
+                        pk[2 * c4] = pack_bf16x2(pr[q], pr[q + 1]);
+                        pk[2 * c4 + 1] = pack_bf16x2(pr[q + 2], pr[q + 3]);
+                        dk8[2 * c4] = pack_bf16x2(ds01.x, ds01.y);
+                        dk8[2 * c4 + 1] = pack_bf16x2(ds23.x, ds23.y);
                     }
                     tmem_st8(tmem + lane_base + Lay::kColDP + 64 * g + 16 * b, pk);
                     tmem_st8(tmem + lane_base + Lay::kColDP + 64 * g + 16 * b + 8, dk8);

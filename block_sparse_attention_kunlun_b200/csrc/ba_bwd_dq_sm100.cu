@@ -340,17 +340,14 @@ __global__ void __launch_bounds__(320, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&sb.s_free);
                     }
-                    if (full) {
+                    const float2 sc2 = make_float2(scale_log2, scale_log2), nl2 = make_float2(-l2, -l2);
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            pr[32 * h2 + c] = ex2_approx(fmaf(__uint_as_float(sr[c]), scale_log2, -l2));
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            const int cc = 32 * h2 + c;
-                            const float e = ex2_approx(fmaf(__uint_as_float(sr[c]), scale_log2, -l2));
-                            pr[cc] = (cc >= lo_c && cc <= hi_c) ? e : 0.f;
-                        }
+                    for (int c = 0; c < 32; c += 2) {
+                        const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nl2);
+                        const int cc = 32 * h2 + c;
+                        const float e0 = ex2_approx(x.x), e1 = ex2_approx(x.y);
+                        pr[cc] = (full || (cc >= lo_c && cc <= hi_c)) ? e0 : 0.f;
+                        pr[cc + 1] = (full || (cc + 1 >= lo_c && cc + 1 <= hi_c)) ? e1 : 0.f;
                     }
                 }
                 // phase B: dS = P (dP - Delta), written as bf16 over this group's dP columns
@@ -365,11 +362,13 @@ __global__ void __launch_bounds__(320, 1)
                     tmem_wait_ld();
                     reg_fence(dr);
                     uint32_t pk[16];
+                    const float2 ndl = make_float2(-dl, -dl);
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
                         const int k0c = 32 * h2 + 2 * c;
-                        pk[c] = pack_bf16x2(pr[k0c] * (__uint_as_float(dr[2 * c]) - dl),
-                                            pr[k0c + 1] * (__uint_as_float(dr[2 * c + 1]) - dl));
+                        const float2 ds = fmul2(make_float2(pr[k0c], pr[k0c + 1]),
+                                                fadd2(make_float2(__uint_as_float(dr[2 * c]), __uint_as_float(dr[2 * c + 1])), ndl));
+                        pk[c] = pack_bf16x2(ds.x, ds.y);
                     }
                     tmem_st16(tmem + lane_base + Lay::kColDP + 64 * g + 16 * h2, pk);
                 }

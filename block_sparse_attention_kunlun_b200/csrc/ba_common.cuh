@@ -21,18 +21,20 @@ constexpr int kWorklistThreads = 1024;
 constexpr int kStatusTimeout = 1;
 
 // First key visible to query i: the start of block blk(i) - (window - 1),
-// clamped at 0.
+// clamped at 0. Indices are local to an example and fit in 32 bits; the
+// product below never exceeds i, so the 32-bit division is exact and cheap.
 __host__ __device__ __forceinline__ int64_t window_start(int64_t i, int64_t block, int64_t window)
 {
-    const int64_t b = i / block - (window - 1);
-    return b > 0 ? b * block : 0;
+    const int32_t b = int32_t(i) / int32_t(block);
+    return b >= int32_t(window) ? int64_t(b - int32_t(window) + 1) * block : 0;
 }
 
 // Last query (of an example of length L) that sees key j.
 __host__ __device__ __forceinline__ int64_t last_query_seeing(int64_t j, int64_t L, int64_t block,
                                                               int64_t window)
 {
-    const int64_t hi = (j / block + window) * block - 1;
+    const int32_t b = int32_t(j) / int32_t(block);
+    const int64_t hi = (int64_t(b) + window) * block - 1;
     return hi < L - 1 ? hi : L - 1;
 }
 
@@ -47,10 +49,13 @@ __host__ __device__ __forceinline__ bool visible(int64_t i, int64_t j, int64_t b
 //   tile_info           int4[max_tiles]: per live tile {first row of its
 //                       example, example length, tile index in the example,
 //                       example index}, max_tiles = ceil(T / 128) + batch
+//   pair_prefix         int32[batch + 1]: live pairs of consecutive tiles
+//   pair_info           int4[max_pairs]: per pair {row0, length, first tile,
+//                       example}, max_pairs = ceil(T / 256) + batch
 //   delta   (bwd only)  float[heads * total_tokens]
 //   dq_acc  (bwd only)  float[heads * total_tokens * head_dim]
 struct WorkspaceLayout {
-    size_t status, tile_prefix, tile_info, delta, dq_acc, total;
+    size_t status, tile_prefix, tile_info, pair_prefix, pair_info, delta, dq_acc, total;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -58,6 +63,11 @@ __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_
 __host__ __device__ inline int64_t max_tiles(int64_t batch, int64_t total_tokens)
 {
     return (total_tokens + kTile - 1) / kTile + batch;
+}
+
+__host__ __device__ inline int64_t max_pairs(int64_t batch, int64_t total_tokens)
+{
+    return (total_tokens + 2 * kTile - 1) / (2 * kTile) + batch;
 }
 
 __host__ __device__ inline WorkspaceLayout workspace_layout(int64_t batch, int64_t total_tokens,
@@ -70,6 +80,10 @@ __host__ __device__ inline WorkspaceLayout workspace_layout(int64_t batch, int64
     size_t off = align256(w.tile_prefix + sizeof(int32_t) * size_t(batch + 1));
     w.tile_info = off;
     off = align256(off + 16 * size_t(max_tiles(batch, total_tokens)));
+    w.pair_prefix = off;
+    off = align256(off + sizeof(int32_t) * size_t(batch + 1));
+    w.pair_info = off;
+    off = align256(off + 16 * size_t(max_pairs(batch, total_tokens)));
     w.delta = off;
     if (with_delta) off = align256(off + sizeof(float) * size_t(heads * total_tokens));
     w.dq_acc = off;
@@ -84,6 +98,8 @@ struct Problem {
     const uint8_t *skip;        // [batch] or nullptr
     const int32_t *tile_prefix; // [batch + 1], device (workspace)
     const int4 *tile_info;      // [max_tiles], device (workspace)
+    const int32_t *pair_prefix; // [batch + 1], device (workspace)
+    const int4 *pair_info;      // [max_pairs], device (workspace)
     int *status;                // workspace status word
     int32_t batch, total_tokens, heads, head_dim, block, window;
     float scale;                // 1 / sqrt(head_dim)
@@ -109,6 +125,24 @@ __device__ __forceinline__ bool decode_item(const Problem &p, int32_t ntiles, in
     r.s0 = info.x;
     r.L = info.y;
     r.t = info.z;
+    return true;
+}
+
+// Number of live tile pairs (read once per kernel role).
+__device__ __forceinline__ int32_t live_pair_count(const Problem &p) { return p.pair_prefix[p.batch]; }
+
+// Work item n -> (pair of query tiles 2k and 2k+1 of one example, head).
+// r.t is the first tile; `second` tells whether tile r.t + 1 exists.
+__device__ __forceinline__ bool decode_pair(const Problem &p, int32_t npairs, int64_t n, TileRef &r, bool &second)
+{
+    if (n >= int64_t(npairs) * p.heads) return false;
+    const int32_t pair = int32_t(n / p.heads);
+    r.h = int32_t(n % p.heads);
+    const int4 info = p.pair_info[pair];
+    r.s0 = info.x;
+    r.L = info.y;
+    r.t = info.z;
+    second = int64_t(r.t + 1) * kTile < r.L;
     return true;
 }
 

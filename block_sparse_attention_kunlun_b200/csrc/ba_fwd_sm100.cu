@@ -5,27 +5,34 @@
 // of GPUs", section "Kunlun changes how GEM scales"; "GEM (Meta)", section
 // "Custom kernels", BlockAttention): for each query row i of each example and
 // head, out_i = softmax over the visible keys j of (q_i . k_j / sqrt(D))
-// applied to v_j, and lse_i = log of that softmax's normaliser. The work is
-// tiled 128 queries x 128 keys; a query tile only visits the key tiles from
-// its first row's window start up to the diagonal (block skipping), so the
-// cost is linear in the example length for a fixed window.
+// applied to v_j, and lse_i = log of that softmax's normaliser. Work is tiled
+// 128 queries x 128 keys; a query tile only visits the key tiles from its
+// first row's window start up to the diagonal (block skipping), so the cost
+// is linear in the example length for a fixed window.
 //
-// CTA roles (persistent: one CTA per SM, static round-robin over the
-// (query tile, head) items):
-//   warps 0-3  softmax: thread t owns TMEM lane t = query row t of the tile;
-//              reads S, masks, keeps the running max/sum, writes P (bf16) back
-//              into TMEM over S, rescales O when the max grows by > 2^8, and
-//              stores out and lse at the end of the item;
-//   warp 4     TMA producer: Q once per item (two buffers, so the next item's
-//              Q arrives while this one runs), K and V per key tile into a ring;
-//   warp 5     MMA issuer: S = Q K^T into one of two TMEM S buffers, then
-//              O += P V with P read straight from TMEM (no shared-memory trip).
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D).
+// One item = two consecutive query tiles (t, t+1) of one (example, head).
+// Their key-tile ranges overlap almost entirely, so each K/V tile is loaded
+// once and used by both. Two softmax warpgroups own one query tile each; the
+// MMA warp interleaves their work as
+//   ... PV0(j-1) S0(j) | PV1(j-1) S1(j) | PV0(j) S0(j+1) | ...
+// so that one group's softmax runs while the tensor core serves the other.
+//
+// CTA roles (persistent, round-robin over items):
+//   warps 0-3 / 4-7  softmax group w: thread t owns TMEM lane t = query row t
+//              of tile t+w. Reads S, masks, keeps the running max/sum (O is
+//              rescaled only when the max grows by more than 2^8), writes P
+//              (bf16) back over S for the P V MMA, stores out and lse.
+//   warp 8     TMA producer: both Q tiles per item, K and V per key tile
+//              into a ring shared by the two groups.
+//   warp 9     MMA issuer.
+// TMEM columns: S of group w at [128w, 128w+128) (P bf16 in its first 64),
+// O of group w at [256 + D w, 256 + D w + D).
 #include "ba_common.cuh"
 #include "ba_kernels.cuh"
 #include "ba_ptx.cuh"
 
 #include <cuda_bf16.h>
+#include <type_traits>
 
 namespace ba {
 
@@ -38,29 +45,48 @@ struct FwdLayout {
     static constexpr int kChunks = D / 64;               // 128-byte column chunks per row
     static constexpr int kChunkBytes = kTile * 128;      // one chunk of a 128-row tile
     static constexpr int kTileBytes = kTile * D * 2;     // one 128 x D bf16 tile
-    static constexpr int kQ = 0;                         // two Q buffers (consecutive items)
+    static constexpr int kQ = 0;                         // Q tile of group w at kQ + w tile
     static constexpr int kK0 = 2 * kTileBytes;           // stage s: K at kK0 + 2 s tile, V after it
     static constexpr int kBytes = kTileBytes * (2 + 2 * kStages);
     static constexpr int kAlloc = kBytes + 1024;         // slack to align the base to 1024 B
-    static constexpr int kThreads = 192;
+    static constexpr int kThreads = 320;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColO = 256;
 };
 
 struct FwdBarriers {
-    uint64_t q_full[2], q_empty[2], o_done, o_free;
-    uint64_t s_full[2], p_full[2];
+    uint64_t q_full, q_empty;
+    uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
     uint64_t kv_full[4], kv_empty[4];
     uint32_t tmem_base;
     int abort;
 };
 
+// 2^x on the FMA pipe for x <= 8 (values below 2^-125 come out as 2^-125 or
+// smaller, far below what a bf16 P can hold next to the row maximum). Round x
+// to the nearest integer n with the 1.5 * 2^23 trick, evaluate 2^(x-n) on
+// [-0.5, 0.5] with a cubic fitted to 2^f (relative error < 8e-5, measured on a
+// dense grid), and add n to the exponent field.
+__device__ __forceinline__ float exp2_fma(float x)
+{
+    x = fmaxf(x, -125.f);
+    const float t = x + 12582912.f;
+    const float f = x - (t - 12582912.f);
+    const float p = fmaf(fmaf(fmaf(0.055171654f, f, 0.24261115f), f, 0.69326097f), f, 0.99992806f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Key-tile range of query tile t: [first_key_tile, t].
+__device__ __forceinline__ int first_key_tile(int t, int64_t B, int64_t W)
+{
+    return int(window_start(int64_t(t) * kTile, B, W) / kTile);
+}
+
 } // namespace
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
-    fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
-                          const __grid_constant__ CUtensorMap tm_k,
+__global__ void __launch_bounds__(320, 1)
+    fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const Problem p,
                           __nv_bfloat16 *__restrict__ out, float *__restrict__ lse)
 {
@@ -74,15 +100,13 @@ __global__ void __launch_bounds__(192, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sb.q_full[0], 1);
-        mbar_init(&sb.q_full[1], 1);
-        mbar_init(&sb.q_empty[0], 1);
-        mbar_init(&sb.q_empty[1], 1);
-        mbar_init(&sb.o_done, 1);
-        mbar_init(&sb.o_free, 4);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&sb.s_full[i], 1);
-            mbar_init(&sb.p_full[i], 4);
+        mbar_init(&sb.q_full, 1);
+        mbar_init(&sb.q_empty, 1);
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(&sb.s_full[w], 1);
+            mbar_init(&sb.p_full[w], 4);
+            mbar_init(&sb.o_final[w], 1);
+            mbar_init(&sb.o_free[w], 4);
         }
         for (int i = 0; i < S; ++i) {
             mbar_init(&sb.kv_full[i], 1);
@@ -91,12 +115,12 @@ __global__ void __launch_bounds__(192, 1)
         sb.abort = 0;
         fence_mbar_init();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == 8 && lane == 0) {
         tma_prefetch_map(&tm_q);
         tma_prefetch_map(&tm_k);
         tma_prefetch_map(&tm_v);
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(&sb.tmem_base, Lay::kTmemCols);
         tmem_relinquish();
     }
@@ -106,25 +130,34 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tmem = sb.tmem_base;
     volatile int *abort = &sb.abort;
     const int64_t B = p.block, W = p.window;
+    const int32_t npairs = live_pair_count(p);
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------ TMA producer ---
         uint32_t kv_cnt = 0, item_cnt = 0;
         TileRef r;
-        const int32_t ntiles = live_tile_count(p);
-        for (int64_t n = blockIdx.x; decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
-            const int jlo = int(window_start(int64_t(r.t) * kTile, B, W) / kTile);
-            const int qb = item_cnt & 1;
-            if (!mbar_wait(&sb.q_empty[qb], ((item_cnt >> 1) & 1) ^ 1, abort)) break;
+        bool second;
+        bool ok = true;
+        for (int64_t n = blockIdx.x; ok && decode_pair(p, npairs, n, r, second); n += gridDim.x, ++item_cnt) {
+            const int jlo = first_key_tile(r.t, B, W);
+            const int jhi = r.t + (second ? 1 : 0);
+            if (!mbar_wait(&sb.q_empty, (item_cnt & 1) ^ 1, abort)) break;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&sb.q_full[qb], Lay::kTileBytes);
-                for (int c = 0; c < Lay::kChunks; ++c)
-                    tma_load_2d(smem + Lay::kQ + qb * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_q,
-                                &sb.q_full[qb], r.h * D + c * 64, r.s0 + r.t * kTile);
+                mbar_arrive_expect_tx(&sb.q_full, (second ? 2 : 1) * Lay::kTileBytes);
+                for (int w = 0; w < (second ? 2 : 1); ++w)
+                    for (int c = 0; c < Lay::kChunks; ++c)
+                        tma_load_2d(smem + Lay::kQ + w * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_q, &sb.q_full,
+                                    r.h * D + c * 64, r.s0 + (r.t + w) * kTile);
+                // warm L2 with the next item's query tiles
+                TileRef rn;
+                bool sn;
+                if (decode_pair(p, npairs, n + gridDim.x, rn, sn))
+                    for (int w = 0; w < (sn ? 2 : 1); ++w)
+                        for (int c = 0; c < Lay::kChunks; ++c)
+                            tma_prefetch_l2_2d(&tm_q, rn.h * D + c * 64, rn.s0 + (rn.t + w) * kTile);
             }
             __syncwarp();
-            bool ok = true;
-            for (int j = jlo; j <= r.t; ++j, ++kv_cnt) {
+            for (int j = jlo; j <= jhi; ++j, ++kv_cnt) {
                 const int st = kv_cnt % S;
                 if (!mbar_wait(&sb.kv_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
                     ok = false;
@@ -132,104 +165,122 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 if (lane == 0) {
                     uint8_t *kdst = smem + Lay::kK0 + 2 * st * Lay::kTileBytes;
-                    uint8_t *vdst = kdst + Lay::kTileBytes;
                     mbar_arrive_expect_tx(&sb.kv_full[st], 2 * Lay::kTileBytes);
                     for (int c = 0; c < Lay::kChunks; ++c) {
-                        tma_load_2d(kdst + c * Lay::kChunkBytes, &tm_k, &sb.kv_full[st],
-                                    r.h * D + c * 64, r.s0 + j * kTile);
-                        tma_load_2d(vdst + c * Lay::kChunkBytes, &tm_v, &sb.kv_full[st],
+                        tma_load_2d(kdst + c * Lay::kChunkBytes, &tm_k, &sb.kv_full[st], r.h * D + c * 64,
+                                    r.s0 + j * kTile);
+                        tma_load_2d(kdst + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_v, &sb.kv_full[st],
                                     r.h * D + c * 64, r.s0 + j * kTile);
                     }
                 }
                 __syncwarp();
             }
-            if (!ok) break;
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // -------------------------------------------------- MMA issuer ---
         constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
         constexpr uint32_t idesc_o = idesc_bf16(128, D, false, true);
-        uint32_t kv_cnt = 0, s_cnt = 0, item_cnt = 0;
+        uint32_t kv_cnt = 0, item_cnt = 0;
+        uint32_t pcnt[2] = {0, 0}; // P tiles consumed so far by each group
+        uint32_t icnt[2] = {0, 0}; // items each group has finished (group 1 skips single-tile items)
         TileRef r;
-        const int32_t ntiles = live_tile_count(p);
+        bool second;
         bool ok = true;
-        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
-            const int jlo = int(window_start(int64_t(r.t) * kTile, B, W) / kTile);
-            const int nkv = r.t - jlo + 1;
-            const int qb = item_cnt & 1;
-            if (!mbar_wait(&sb.q_full[qb], (item_cnt >> 1) & 1, abort)) break;
+        for (int64_t n = blockIdx.x; ok && decode_pair(p, npairs, n, r, second); n += gridDim.x, ++item_cnt) {
+            const int lo[2] = {first_key_tile(r.t, B, W), second ? first_key_tile(r.t + 1, B, W) : 1};
+            const int hi[2] = {r.t, second ? r.t + 1 : 0};
+            const int jlo = lo[0], jhi = second ? hi[1] : hi[0];
+            if (!mbar_wait(&sb.q_full, item_cnt & 1, abort)) break;
             tc_fence_after();
-            // O += P_m V_m for the key tile issued m-th in this item.
-            auto issue_pv = [&](int m, uint32_t s_idx, uint32_t kv_idx) -> bool {
-                if (!mbar_wait(&sb.p_full[s_idx & 1], (s_idx >> 1) & 1, abort)) return false;
-                if (m == 0 && !mbar_wait(&sb.o_free, (item_cnt & 1) ^ 1, abort)) return false;
+            // O_w += P_w V for key tile j of group w (V from ring stage st)
+            auto issue_pv = [&](int w, int j, int st) -> bool {
+                if (!mbar_wait(&sb.p_full[w], pcnt[w] & 1, abort)) return false;
+                const bool first = (j == lo[w]);
+                if (first && !mbar_wait(&sb.o_free[w], (icnt[w] & 1) ^ 1, abort)) return false;
                 tc_fence_after();
                 if (lane == 0) {
-                    const int st = kv_idx % S;
                     const uint32_t v_addr = smem_base + Lay::kK0 + (2 * st + 1) * Lay::kTileBytes;
-                    const uint32_t a_tmem = tmem + (s_idx & 1) * 128;
 #pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk) {
-                        const uint64_t bdesc = sdesc_sw128(v_addr + kk * 2048, Lay::kChunkBytes, 1024);
-                        mma_ts(tmem + Lay::kColO, a_tmem + kk * 8, bdesc, idesc_o,
-                               (m > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    tc_commit(&sb.kv_empty[st]);
-                    tc_commit(&sb.o_done);
+                    for (int kk = 0; kk < kTile / 16; ++kk)
+                        mma_ts(tmem + Lay::kColO + D * w, tmem + 128 * w + kk * 8,
+                               sdesc_sw128(v_addr + kk * 2048, Lay::kChunkBytes, 1024), idesc_o,
+                               (!first || kk > 0) ? 1u : 0u);
+                    if (j == hi[w]) tc_commit(&sb.o_final[w]);
                 }
                 __syncwarp();
+                ++pcnt[w];
                 return true;
             };
-            for (int m = 0; m < nkv; ++m, ++s_cnt, ++kv_cnt) {
+            auto issue_s = [&](int w, int st) {
+                if (lane == 0) {
+                    const uint32_t q_addr = smem_base + Lay::kQ + w * Lay::kTileBytes;
+                    const uint32_t k_addr = smem_base + Lay::kK0 + 2 * st * Lay::kTileBytes;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk / 4) * Lay::kChunkBytes + (kk % 4) * 32;
+                        mma_ss(tmem + 128 * w, sdesc_sw128(q_addr + off, 16, 1024),
+                               sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&sb.s_full[w]);
+                }
+                __syncwarp();
+            };
+            for (int j = jlo; j <= jhi && ok; ++j, ++kv_cnt) {
                 const int st = kv_cnt % S;
                 if (!mbar_wait(&sb.kv_full[st], (kv_cnt / S) & 1, abort)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                for (int w = 0; w < 2 && ok; ++w) {
+                    // the previous tile's P V of this group reads P from the S buffer: issue it first
+                    if (j - 1 >= lo[w] && j - 1 <= hi[w] && !issue_pv(w, j - 1, (kv_cnt - 1) % S)) ok = false;
+                    if (ok && j >= lo[w] && j <= hi[w]) issue_s(w, st);
+                }
+                if (!ok) break;
                 if (lane == 0) {
-                    const uint32_t q_addr = smem_base + Lay::kQ + qb * Lay::kTileBytes;
-                    const uint32_t k_addr = smem_base + Lay::kK0 + 2 * st * Lay::kTileBytes;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk / 4) * Lay::kChunkBytes + (kk % 4) * 32;
-                        mma_ss(tmem + (s_cnt & 1) * 128, sdesc_sw128(q_addr + off, 16, 1024),
-                               sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-                    }
-                    tc_commit(&sb.s_full[s_cnt & 1]);
-                    if (m == nkv - 1) tc_commit(&sb.q_empty[qb]);
+                    if (j == jhi) tc_commit(&sb.q_empty);
+                    if (j > jlo) tc_commit(&sb.kv_empty[(kv_cnt - 1) % S]); // tile j-1 has no reader left
                 }
                 __syncwarp();
-                if (m > 0 && !issue_pv(m - 1, s_cnt - 1, kv_cnt - 1)) {
-                    ok = false;
-                    break;
-                }
             }
-            if (ok && !issue_pv(nkv - 1, s_cnt - 1, kv_cnt - 1)) ok = false;
+            if (!ok) break;
+            for (int w = 0; w < 2 && ok; ++w)
+                if (jhi >= lo[w] && jhi <= hi[w] && !issue_pv(w, jhi, (kv_cnt - 1) % S)) ok = false;
+            if (!ok) break;
+            if (lane == 0) tc_commit(&sb.kv_empty[(kv_cnt - 1) % S]);
+            __syncwarp();
+            ++icnt[0];
+            if (second) ++icnt[1];
         }
     } else {
         // ----------------------------------------------------- softmax ---
-        const int row = threadIdx.x; // 0..127
-        const uint32_t lane_base = uint32_t(warp * 32) << 16;
+        const int w = warp >> 2;              // group: query tile t + w
+        const int row = threadIdx.x & 127;    // query row within the tile, TMEM lane
+        const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+        const uint32_t s_addr = tmem + lane_base + 128 * w;
+        const uint32_t o_addr = tmem + lane_base + Lay::kColO + D * w;
         const float scale_log2 = p.scale * 1.4426950408889634f;
-        uint32_t s_cnt = 0, pv_cnt = 0;
+        uint32_t cnt = 0, my_items = 0; // tiles and items this group has processed
         TileRef r;
-        const int32_t ntiles = live_tile_count(p);
+        bool second;
         bool ok = true;
-        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x) {
-            const int64_t i = int64_t(r.t) * kTile + row;
+        for (int64_t n = blockIdx.x; ok && decode_pair(p, npairs, n, r, second); n += gridDim.x) {
+            if (w == 1 && !second) continue;
+            const int t = r.t + w;
+            const int jlo = first_key_tile(t, B, W);
+            const int64_t i = int64_t(t) * kTile + row;
             const bool valid = i < r.L;
             const int64_t ws = window_start(i, B, W);
-            const int jlo = int(window_start(int64_t(r.t) * kTile, B, W) / kTile);
-            const int nkv = r.t - jlo + 1;
             float m_ref = -INFINITY, l = 0.f;
-            for (int m = 0; m < nkv; ++m, ++s_cnt) {
-                const int64_t key0 = int64_t(jlo + m) * kTile;
-                const uint32_t s_addr = tmem + lane_base + (s_cnt & 1) * 128;
-                if (!mbar_wait(&sb.s_full[s_cnt & 1], (s_cnt >> 1) & 1, abort)) {
-                    ok = false;
-                    break;
-                }
+            for (int j = jlo; j <= t; ++j, ++cnt) {
+                const int64_t key0 = int64_t(j) * kTile;
+                int64_t lo64 = ws - key0, hi64 = i - key0;
+                if (!valid) { lo64 = 1; hi64 = 0; }
+                const int lo_c = int(lo64 < -1 ? -1 : (lo64 > 128 ? 128 : lo64));
+                const int hi_c = int(hi64 < -1 ? -1 : (hi64 > 128 ? 128 : hi64));
+                const bool full = __all_sync(0xffffffffu, lo_c <= 0 && hi_c >= 127);
+                if (!mbar_wait(&sb.s_full[w], cnt & 1, abort)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t sr[4][32];
 #pragma unroll
@@ -237,74 +288,87 @@ __global__ void __launch_bounds__(192, 1)
                 tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
-                // visible columns of this row: lo_c <= c <= hi_c
-                int64_t lo64 = ws - key0, hi64 = i - key0;
-                if (!valid) { lo64 = 1; hi64 = 0; }
-                const int lo_c = int(lo64 < -1 ? -1 : (lo64 > 128 ? 128 : lo64));
-                const int hi_c = int(hi64 < -1 ? -1 : (hi64 > 128 ? 128 : hi64));
-                float x[128];
-                float mx = -INFINITY;
+                // One pass for the row maximum of the visible raw scores (the scale is
+                // positive), one for P; a tile visible to the whole warp skips masking.
+                float alpha = 1.f, rs = 0.f;
+                bool grow = false;
+                auto softmax_tile = [&](auto full_t) {
+                    constexpr bool FULL = decltype(full_t)::value;
+                    float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    const bool vis = c >= lo_c && c <= hi_c;
-                    x[c] = vis ? __uint_as_float(sr[c / 32][c % 32]) * scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, x[c]);
-                }
-                const float m_new = fmaxf(m_ref, mx);
-                const bool grow = m_new > m_ref + 8.0f;
-                float alpha = 1.f;
-                if (grow) {
-                    alpha = ex2_approx(m_ref - m_new);
-                    m_ref = m_new;
-                }
-                const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-                float rs = 0.f;
-                uint32_t pk[4][16];
-#pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const float p0 = ex2_approx(x[2 * c] - m_use);
-                    const float p1 = ex2_approx(x[2 * c + 1] - m_use);
-                    rs += p0 + p1;
-                    pk[c / 16][c % 16] = pack_bf16x2(p0, p1);
-                }
-                l = l * alpha + rs;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_st16(s_addr + c * 16, pk[c]);
-                tmem_wait_st();
-                if (m > 0) {
-                    // O must hold P_{m-1} V_{m-1} before it is rescaled.
-                    if (!mbar_wait(&sb.o_done, pv_cnt & 1, abort)) {
-                        ok = false;
-                        break;
-                    }
-                    ++pv_cnt;
-                    tc_fence_after();
-                    if (__any_sync(0xffffffffu, grow)) {
-                        const uint32_t o_addr = tmem + lane_base + Lay::kColO;
-#pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t orr[32];
-                            tmem_ld32(o_addr + c * 32, orr);
-                            tmem_wait_ld();
-                            reg_fence(orr);
-#pragma unroll
-                            for (int k = 0; k < 32; ++k)
-                                orr[k] = __float_as_uint(__uint_as_float(orr[k]) * alpha);
-                            tmem_st32(o_addr + c * 32, orr);
+                    for (int c = 0; c < 128; c += 2) {
+                        float a = __uint_as_float(sr[c / 32][c % 32]), b = __uint_as_float(sr[c / 32][c % 32 + 1]);
+                        if (!FULL) {
+                            a = (c >= lo_c && c <= hi_c) ? a : -INFINITY;
+                            b = (c + 1 >= lo_c && c + 1 <= hi_c) ? b : -INFINITY;
+                            sr[c / 32][c % 32] = __float_as_uint(a);
+                            sr[c / 32][c % 32 + 1] = __float_as_uint(b);
                         }
-                        tmem_wait_st();
+                        mp[(c / 2) % 4] = fmax3(mp[(c / 2) % 4], a, b);
                     }
+                    const float mx = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+                    const float m_new = mx * scale_log2;
+                    grow = m_new > m_ref + 8.0f;
+                    if (grow) {
+                        alpha = ex2_approx(m_ref - m_new);
+                        m_ref = m_new;
+                    }
+                    const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
+                    const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(neg_m, neg_m);
+                    float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+                    // P in two 64-column halves, each stored (packed bf16) over S columns
+                    // this thread has already read
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const int c0 = 64 * hh + 2 * c;
+                            const float2 x = ffma2(make_float2(__uint_as_float(sr[c0 / 32][c0 % 32]),
+                                                               __uint_as_float(sr[c0 / 32][c0 % 32 + 1])),
+                                                   sc2, nm2);
+                            // one pair in eight goes through the FMA pipe to offload the MUFU unit
+                            float p0 = (c % 8 == 7) ? exp2_fma(x.x) : ex2_approx(x.x);
+                            float p1 = (c % 8 == 7) ? exp2_fma(x.y) : ex2_approx(x.y);
+                            if (!FULL) {
+                                p0 = x.x > -INFINITY ? p0 : 0.f;
+                                p1 = x.y > -INFINITY ? p1 : 0.f;
+                            }
+                            acc[c % 4] = fadd2(acc[c % 4], make_float2(p0, p1));
+                            pk[c] = pack_bf16x2(p0, p1);
+                        }
+                        tmem_st32(s_addr + 32 * hh, pk);
+                    }
+                    const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+                    const float2 a = fadd2(a01, a23);
+                    rs = a.x + a.y;
+                };
+                if (full) softmax_tile(std::true_type{});
+                else softmax_tile(std::false_type{});
+                l = l * alpha + rs;
+                tmem_wait_st();
+                // O holds the earlier tiles' P V (complete: this S was issued after it).
+                if (j > jlo && __any_sync(0xffffffffu, grow)) {
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t orr[32];
+                        tmem_ld32(o_addr + c * 32, orr);
+                        tmem_wait_ld();
+                        reg_fence(orr);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) orr[k] = __float_as_uint(__uint_as_float(orr[k]) * alpha);
+                        tmem_st32(o_addr + c * 32, orr);
+                    }
+                    tmem_wait_st();
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sb.p_full[s_cnt & 1]);
+                if (lane == 0) mbar_arrive(&sb.p_full[w]);
             }
             if (!ok) break;
-            // epilogue: wait for the last P V, normalise, store.
-            if (!mbar_wait(&sb.o_done, pv_cnt & 1, abort)) break;
-            ++pv_cnt;
+            // epilogue: wait for this group's last P V, normalise, store
+            if (!mbar_wait(&sb.o_final[w], my_items & 1, abort)) break;
             tc_fence_after();
-            const uint32_t o_addr = tmem + lane_base + Lay::kColO;
             const float inv_l = valid ? 1.f / l : 0.f;
             __nv_bfloat16 *orow = out + ((int64_t(r.s0) + i) * p.heads + r.h) * D;
 #pragma unroll
@@ -316,55 +380,48 @@ __global__ void __launch_bounds__(192, 1)
                 if (valid) {
                     uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        uint4 v4;
-                        v4.x = pack_bf16x2(__uint_as_float(orr[8 * k + 0]) * inv_l,
-                                           __uint_as_float(orr[8 * k + 1]) * inv_l);
-                        v4.y = pack_bf16x2(__uint_as_float(orr[8 * k + 2]) * inv_l,
-                                           __uint_as_float(orr[8 * k + 3]) * inv_l);
-                        v4.z = pack_bf16x2(__uint_as_float(orr[8 * k + 4]) * inv_l,
-                                           __uint_as_float(orr[8 * k + 5]) * inv_l);
-                        v4.w = pack_bf16x2(__uint_as_float(orr[8 * k + 6]) * inv_l,
-                                           __uint_as_float(orr[8 * k + 7]) * inv_l);
-                        dst[k] = v4;
-                    }
+                    for (int k = 0; k < 4; ++k)
+                        dst[k] = make_uint4(pack_bf16x2(__uint_as_float(orr[8 * k + 0]) * inv_l,
+                                                        __uint_as_float(orr[8 * k + 1]) * inv_l),
+                                            pack_bf16x2(__uint_as_float(orr[8 * k + 2]) * inv_l,
+                                                        __uint_as_float(orr[8 * k + 3]) * inv_l),
+                                            pack_bf16x2(__uint_as_float(orr[8 * k + 4]) * inv_l,
+                                                        __uint_as_float(orr[8 * k + 5]) * inv_l),
+                                            pack_bf16x2(__uint_as_float(orr[8 * k + 6]) * inv_l,
+                                                        __uint_as_float(orr[8 * k + 7]) * inv_l));
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sb.o_free);
+            if (lane == 0) mbar_arrive(&sb.o_free[w]);
             if (valid)
-                lse[int64_t(r.h) * p.total_tokens + r.s0 + i] =
-                    (m_ref + log2f(l)) * 0.6931471805599453f;
+                lse[int64_t(r.h) * p.total_tokens + r.s0 + i] = (m_ref + log2f(l)) * 0.6931471805599453f;
+            ++my_items;
         }
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5) tmem_dealloc(tmem, Lay::kTmemCols);
+    if (warp == 9) tmem_dealloc(tmem, Lay::kTmemCols);
     if (threadIdx.x == 0 && sb.abort) atomicOr(p.status, kStatusTimeout);
 }
 
 template <int D>
-cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk,
-                                  const CUtensorMap &tv, const Problem &p, void *out, float *lse,
-                                  int num_sms, cudaStream_t stream)
+cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                  const Problem &p, void *out, float *lse, int num_sms, cudaStream_t stream)
 {
     using Lay = FwdLayout<D>;
     auto kern = fwd_bf16_sm100_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, p,
-                                                          static_cast<__nv_bfloat16 *>(out), lse);
+    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, p, static_cast<__nv_bfloat16 *>(out), lse);
     return cudaGetLastError();
 }
 
-template cudaError_t launch_fwd_bf16_sm100<64>(const CUtensorMap &, const CUtensorMap &,
-                                               const CUtensorMap &, const Problem &, void *,
-                                               float *, int, cudaStream_t);
-template cudaError_t launch_fwd_bf16_sm100<128>(const CUtensorMap &, const CUtensorMap &,
-                                                const CUtensorMap &, const Problem &, void *,
-                                                float *, int, cudaStream_t);
+template cudaError_t launch_fwd_bf16_sm100<64>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
+                                               const Problem &, void *, float *, int, cudaStream_t);
+template cudaError_t launch_fwd_bf16_sm100<128>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
+                                                const Problem &, void *, float *, int, cudaStream_t);
 
 } // namespace ba

@@ -271,6 +271,41 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 // --------------------------------------------------------------- scalar ---
 
+// Two fp32 lanes per instruction (sm_100 packed f32x2 arithmetic).
+union F2Bits {
+    float2 f;
+    unsigned long long u;
+};
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    F2Bits A{a}, B{b}, C{c}, R;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(R.u) : "l"(A.u), "l"(B.u), "l"(C.u));
+    return R.f;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b)
+{
+    F2Bits A{a}, B{b}, R;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(R.u) : "l"(A.u), "l"(B.u));
+    return R.f;
+}
+
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b)
+{
+    F2Bits A{a}, B{b}, R;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(R.u) : "l"(A.u), "l"(B.u));
+    return R.f;
+}
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 __device__ __forceinline__ float ex2_approx(float x)
 {
     float y;
