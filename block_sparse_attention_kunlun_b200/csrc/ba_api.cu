@@ -227,10 +227,11 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
         BA_TRY(prof_mark(2, 1, stream));
         return BA_OK;
     }
-    CUtensorMap tq, tk, tv, tdo, to;
+    CUtensorMap tq, tk, tv, tdo, to, tdk, tdv;
     if (!encode_bf16_rows(&tq, q, T, P.heads, P.head_dim) || !encode_bf16_rows(&tk, k, T, P.heads, P.head_dim) ||
         !encode_bf16_rows(&tv, v, T, P.heads, P.head_dim) || !encode_bf16_rows(&tdo, dout, T, P.heads, P.head_dim) ||
-        !encode_bf16_rows(&to, out, T, P.heads, P.head_dim))
+        !encode_bf16_rows(&to, out, T, P.heads, P.head_dim) || !encode_bf16_rows(&tdk, dk, T, P.heads, P.head_dim) ||
+        !encode_bf16_rows(&tdv, dv, T, P.heads, P.head_dim))
         return BA_ERR_CUDA;
     BA_TRY(prof_mark(1, 0, stream));
     if (P.head_dim == 64)
@@ -240,9 +241,9 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
     BA_TRY(prof_mark(1, 1, stream));
     BA_TRY(prof_mark(2, 0, stream));
     if (P.head_dim == 64)
-        BA_TRY(launch_bwd_dkdv_sm100<64>(tq, tk, tv, tdo, p, lse, delta, dk, dv, num_sms, stream));
+        BA_TRY(launch_bwd_dkdv_sm100<64>(tq, tk, tv, tdo, tdk, tdv, p, lse, delta, dk, dv, num_sms, stream));
     else
-        BA_TRY(launch_bwd_dkdv_sm100<128>(tq, tk, tv, tdo, p, lse, delta, dk, dv, num_sms, stream));
+        BA_TRY(launch_bwd_dkdv_sm100<128>(tq, tk, tv, tdo, tdk, tdv, p, lse, delta, dk, dv, num_sms, stream));
     BA_TRY(prof_mark(2, 1, stream));
     return BA_OK;
 }

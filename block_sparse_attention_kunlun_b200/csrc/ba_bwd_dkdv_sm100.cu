@@ -15,21 +15,30 @@
 //   dV  += P^T dO_i   A = P^T from TMEM (bf16), B = dO_i smem (MN-major)
 //   dK  += dS^T Q_i   A = dS^T from TMEM (bf16), B = Q_i smem (MN-major)
 //
+// MMA order per query tile m (one issuing thread, so the tensor pipe runs
+// them in this order):
+//   ... dV(m-1) | S^T(m) | dK(m-1) | dP^T(m) | dV(m) | S^T(m+1) | dK(m) ...
+// dV(m) needs only P^T(m), so it is issued as soon as the compute warps have
+// turned S^T(m) into P^T(m); S^T(m+1) then reuses those columns. dK(m) waits
+// for dS^T(m) and dP^T(m+1) reuses its columns. The compute warps alternate
+// P (phase A) and dS (phase B) while the tensor core runs the products of the
+// other phase, so the per-tile time is the larger of the two, not their sum.
+// Q and dO sit in separate rings: dO(m) is free after dV(m), Q(m) after dK(m).
+//
 // CTA roles (persistent, round-robin over (key tile, head) items):
 //   warps 0-3 / 4-7  two compute warpgroups; thread t owns key row t (TMEM
 //              lane t), group g the queries [64g, 64g+64) of each query tile.
-//              They read S^T (then release it, so the next tile's S^T can be
-//              issued while they work), form P^T, read dP^T, form dS^T and
-//              write P^T and dS^T as bf16 over their dP^T columns.
+//              Phase A: read S^T, write P^T (bf16) over the first 32 of the
+//              group's S^T columns. Phase B: read dP^T, write dS^T (bf16) over
+//              the first 32 of the group's dP^T columns.
 //   warps 8-11 epilogue: at the end of an item, move dV and dK from TMEM to
 //              global memory while the compute warps start the next item.
 //   warp 12    TMA producer: K, V per item (with an L2 prefetch of the next
-//              item's); Q, dO per query tile into a ring.
+//              item's); Q and dO per query tile into their rings, with an L2
+//              prefetch two tiles ahead.
 //   warp 13    MMA issuer.
-// TMEM columns: S^T [0,128), dP^T [128,256), dV [256, 256+D), dK [256+D,
-// 256+2D). After the compute warps have read group g's dP^T columns
-// [128+64g, 192+64g), each 16-query block b of the group holds P^T (bf16) in
-// [128+64g+16b, +8) and dS^T in the next 8 columns.
+// TMEM columns: S^T / P^T [0,128), dP^T / dS^T [128,256), dV [256, 256+D),
+// dK [256+D, 256+2D).
 #include "ba_common.cuh"
 #include "ba_kernels.cuh"
 #include "ba_ptx.cuh"
@@ -46,11 +55,14 @@ struct DkvLayout {
     static constexpr int kChunks = D / 64;
     static constexpr int kChunkBytes = kTile * 128;
     static constexpr int kTileBytes = kTile * D * 2;
-    static constexpr int kStages = D == 64 ? 3 : 2;      // Q / dO ring
+    static constexpr int kQSlots = D == 64 ? 4 : 2;      // Q ring
+    static constexpr int kOSlots = D == 64 ? 4 : 2;      // dO ring
     static constexpr int kK = 0;
     static constexpr int kV = kTileBytes;
-    static constexpr int kQ0 = 2 * kTileBytes;           // stage s: Q at kQ0 + 2 s tile, dO after it
-    static constexpr int kBytes = kQ0 + 2 * kStages * kTileBytes;
+    static constexpr int kQ0 = 2 * kTileBytes;           // Q slot s at kQ0 + s tile
+    static constexpr int kO0 = kQ0 + kQSlots * kTileBytes; // dO slot s at kO0 + s tile
+    static constexpr int kStage = kO0 + kOSlots * kTileBytes; // epilogue staging: 128 rows x 64 columns
+    static constexpr int kBytes = kStage + kChunkBytes;
     static constexpr int kAlloc = kBytes + 1024;
     static constexpr int kThreads = 448;
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
@@ -59,8 +71,9 @@ struct DkvLayout {
 
 struct DkvBarriers {
     uint64_t kv_full, kv_empty, dkv_full, dkv_free;
-    uint64_t qo_full[3], qo_empty[3];
-    uint64_t s_full, s_free, dp_full, ds_full[2];
+    uint64_t q_full[4], q_empty[4], o_full[4], o_empty[4];
+    uint64_t s_full, dp_full, pa_done[2], pb_done[2];
+    uint64_t cmp_sync, epi_sync; // group barriers of the compute and epilogue warps
     uint32_t tmem_base;
     int abort;
     __align__(16) float lse2[2][kTile];
@@ -80,11 +93,12 @@ template <int D>
 __global__ void __launch_bounds__(448, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                          const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                           const Problem p, const float *__restrict__ lse, const float *__restrict__ delta,
                           __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv)
 {
     using Lay = DkvLayout<D>;
-    constexpr int S = Lay::kStages;
+    constexpr int QS = Lay::kQSlots, OS = Lay::kOSlots;
     extern __shared__ uint8_t smem_raw[];
     __shared__ DkvBarriers sb;
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -97,15 +111,20 @@ __global__ void __launch_bounds__(448, 1)
         mbar_init(&sb.kv_empty, 1);
         mbar_init(&sb.dkv_full, 1);
         mbar_init(&sb.dkv_free, 4);
-        for (int i = 0; i < S; ++i) {
-            mbar_init(&sb.qo_full[i], 1);
-            mbar_init(&sb.qo_empty[i], 1);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&sb.q_full[i], 1);
+            mbar_init(&sb.q_empty[i], 1);
+            mbar_init(&sb.o_full[i], 1);
+            mbar_init(&sb.o_empty[i], 1);
         }
         mbar_init(&sb.s_full, 1);
-        mbar_init(&sb.s_free, 8);
         mbar_init(&sb.dp_full, 1);
-        mbar_init(&sb.ds_full[0], 4);
-        mbar_init(&sb.ds_full[1], 4);
+        mbar_init(&sb.cmp_sync, 256);
+        mbar_init(&sb.epi_sync, 128);
+        for (int g = 0; g < 2; ++g) {
+            mbar_init(&sb.pa_done[g], 4);
+            mbar_init(&sb.pb_done[g], 4);
+        }
         sb.abort = 0;
         fence_mbar_init();
     }
@@ -147,28 +166,48 @@ __global__ void __launch_bounds__(448, 1)
                 }
                 // warm L2 with the next item's K and V
                 TileRef rn;
-                if (decode_item(p, ntiles, n + gridDim.x, rn))
+                if (decode_item(p, ntiles, n + gridDim.x, rn)) {
+                    int nlo, nhi;
+                    query_tile_range(rn, B, W, nlo, nhi);
                     for (int c = 0; c < Lay::kChunks; ++c) {
                         tma_prefetch_l2_2d(&tm_k, rn.h * D + c * 64, rn.s0 + rn.t * kTile);
                         tma_prefetch_l2_2d(&tm_v, rn.h * D + c * 64, rn.s0 + rn.t * kTile);
+                        for (int i = nlo; i <= nhi && i < nlo + 2; ++i) {
+                            tma_prefetch_l2_2d(&tm_q, rn.h * D + c * 64, rn.s0 + i * kTile);
+                            tma_prefetch_l2_2d(&tm_do, rn.h * D + c * 64, rn.s0 + i * kTile);
+                        }
                     }
+                }
             }
             __syncwarp();
             for (int i = ilo; i <= ihi; ++i, ++it) {
-                const int st = it % S;
-                if (!mbar_wait(&sb.qo_empty[st], ((it / S) & 1) ^ 1, abort)) {
+                const int qs = it % QS, os = it % OS;
+                if (!mbar_wait(&sb.q_empty[qs], ((it / QS) & 1) ^ 1, abort)) {
                     ok = false;
                     break;
                 }
                 if (lane == 0) {
-                    uint8_t *qdst = smem + Lay::kQ0 + 2 * st * Lay::kTileBytes;
-                    mbar_arrive_expect_tx(&sb.qo_full[st], 2 * Lay::kTileBytes);
-                    for (int c = 0; c < Lay::kChunks; ++c) {
-                        tma_load_2d(qdst + c * Lay::kChunkBytes, &tm_q, &sb.qo_full[st], r.h * D + c * 64,
-                                    r.s0 + i * kTile);
-                        tma_load_2d(qdst + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_do, &sb.qo_full[st],
-                                    r.h * D + c * 64, r.s0 + i * kTile);
-                    }
+                    mbar_arrive_expect_tx(&sb.q_full[qs], Lay::kTileBytes);
+                    for (int c = 0; c < Lay::kChunks; ++c)
+                        tma_load_2d(smem + Lay::kQ0 + qs * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_q,
+                                    &sb.q_full[qs], r.h * D + c * 64, r.s0 + i * kTile);
+                }
+                __syncwarp();
+                if (!mbar_wait(&sb.o_empty[os], ((it / OS) & 1) ^ 1, abort)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sb.o_full[os], Lay::kTileBytes);
+                    for (int c = 0; c < Lay::kChunks; ++c)
+                        tma_load_2d(smem + Lay::kO0 + os * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_do,
+                                    &sb.o_full[os], r.h * D + c * 64, r.s0 + i * kTile);
+                    // warm L2 two query tiles ahead
+                    if (i + 2 <= ihi)
+                        for (int c = 0; c < Lay::kChunks; ++c) {
+                            tma_prefetch_l2_2d(&tm_q, r.h * D + c * 64, r.s0 + (i + 2) * kTile);
+                            tma_prefetch_l2_2d(&tm_do, r.h * D + c * 64, r.s0 + (i + 2) * kTile);
+                        }
                 }
                 __syncwarp();
             }
@@ -177,55 +216,23 @@ __global__ void __launch_bounds__(448, 1)
         // -------------------------------------------------- MMA issuer ---
         constexpr uint32_t idesc_sp = idesc_bf16(128, 128, false, false); // S^T, dP^T
         constexpr uint32_t idesc_kv = idesc_bf16(128, D, false, true);    // dV, dK (B MN-major)
-        uint32_t it = 0, s_cnt = 0, d_cnt = 0, item_cnt = 0;
+        uint32_t it0 = 0, item_cnt = 0;
         TileRef r;
         bool ok = true;
         const uint32_t k_addr = smem_base + Lay::kK, v_addr = smem_base + Lay::kV;
-        // dV += P^T dO and dK += dS^T Q of the query tile in ring stage st (m = its index in the item)
-        auto issue_dkv = [&](int m, int st) -> bool {
-            const uint32_t q_addr = smem_base + Lay::kQ0 + 2 * st * Lay::kTileBytes;
-            const uint32_t o_addr = q_addr + Lay::kTileBytes;
-            for (int g = 0; g < 2; ++g) {
-                if (!mbar_wait(&sb.ds_full[g], d_cnt & 1, abort)) return false;
-                if (m == 0 && g == 0 && !mbar_wait(&sb.dkv_free, (item_cnt & 1) ^ 1, abort)) return false;
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t pcol = tmem + Lay::kColDP + 64 * g;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t boff = (4 * g + kk) * 2048; // query rows 64g + 16kk ..
-                        const uint32_t acc = (m > 0 || g > 0 || kk > 0) ? 1u : 0u;
-                        // P^T of queries 64g + 16kk .. at column 16kk of the group, dS^T 8 columns later
-                        const uint32_t acol = pcol + 16 * kk;
-                        mma_ts(tmem + Lay::kColDV, acol, sdesc_sw128(o_addr + boff, Lay::kChunkBytes, 1024),
-                               idesc_kv, acc);
-                        mma_ts(tmem + Lay::kColDK, acol + 8, sdesc_sw128(q_addr + boff, Lay::kChunkBytes, 1024),
-                               idesc_kv, acc);
-                    }
-                    if (g == 1) tc_commit(&sb.qo_empty[st]);
-                }
-                __syncwarp();
-            }
-            ++d_cnt;
-            return true;
-        };
         for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
             int ilo, ihi;
             query_tile_range(r, B, W, ilo, ihi);
-            if (!mbar_wait(&sb.kv_full, item_cnt & 1, abort)) break;
-            tc_fence_after();
             const int nq = ihi - ilo + 1;
-            for (int m = 0; m < nq; ++m, ++it, ++s_cnt) {
-                const int st = it % S;
-                const uint32_t q_addr = smem_base + Lay::kQ0 + 2 * st * Lay::kTileBytes;
-                const uint32_t o_addr = q_addr + Lay::kTileBytes;
-                if (!mbar_wait(&sb.qo_full[st], (it / S) & 1, abort) ||
-                    !mbar_wait(&sb.s_free, (s_cnt & 1) ^ 1, abort)) {
-                    ok = false;
-                    break;
-                }
+            if (!mbar_wait_warp(&sb.kv_full, item_cnt & 1, abort)) break;
+            tc_fence_after();
+            // S^T = K Q^T of query tile m of this item
+            auto issue_s = [&](int m) -> bool {
+                const uint32_t it = it0 + m, qs = it % QS;
+                if (!mbar_wait_warp(&sb.q_full[qs], (it / QS) & 1, abort)) return false;
                 tc_fence_after();
-                if (lane == 0) {
+                {
+                    const uint32_t q_addr = smem_base + Lay::kQ0 + qs * Lay::kTileBytes;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t off = (kk / 4) * Lay::kChunkBytes + (kk % 4) * 32;
@@ -235,13 +242,15 @@ __global__ void __launch_bounds__(448, 1)
                     tc_commit(&sb.s_full);
                 }
                 __syncwarp();
-                // dV / dK of the previous query tile read P^T / dS^T from the dP^T
-                // columns, so they go before this tile's dP^T.
-                if (m > 0 && !issue_dkv(m - 1, (it - 1) % S)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) {
+                return true;
+            };
+            // dP^T = V dO^T of query tile m; after the item's last one K and V are not read again
+            auto issue_dp = [&](int m) -> bool {
+                const uint32_t it = it0 + m, os = it % OS;
+                if (!mbar_wait_warp(&sb.o_full[os], (it / OS) & 1, abort)) return false;
+                tc_fence_after();
+                {
+                    const uint32_t o_addr = smem_base + Lay::kO0 + os * Lay::kTileBytes;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t off = (kk / 4) * Lay::kChunkBytes + (kk % 4) * 32;
@@ -249,14 +258,46 @@ __global__ void __launch_bounds__(448, 1)
                                sdesc_sw128(o_addr + off, 16, 1024), idesc_sp, kk > 0 ? 1u : 0u);
                     }
                     tc_commit(&sb.dp_full);
-                    if (m == nq - 1) tc_commit(&sb.kv_empty); // K and V are not read again
+                    if (m == nq - 1) tc_commit(&sb.kv_empty);
                 }
                 __syncwarp();
+                return true;
+            };
+            // dV += P^T dO (phase == 0) or dK += dS^T Q (phase == 1) of query tile m,
+            // group by group as the compute warps finish; then release the operand's slot
+            auto issue_acc = [&](int m, int phase) -> bool {
+                const uint32_t it = it0 + m;
+                const uint32_t slot = phase == 0 ? it % OS : it % QS;
+                const uint32_t b_addr = smem_base + (phase == 0 ? Lay::kO0 + slot * Lay::kTileBytes
+                                                                : Lay::kQ0 + slot * Lay::kTileBytes);
+                for (int g = 0; g < 2; ++g) {
+                    if (!mbar_wait_warp(phase == 0 ? &sb.pa_done[g] : &sb.pb_done[g], it & 1, abort)) return false;
+                    if (phase == 0 && m == 0 && g == 0 && !mbar_wait_warp(&sb.dkv_free, (item_cnt & 1) ^ 1, abort))
+                        return false;
+                    tc_fence_after();
+                    {
+                        const uint32_t acol = tmem + (phase == 0 ? Lay::kColS : Lay::kColDP) + 64 * g;
+                        const uint32_t dcol = tmem + (phase == 0 ? Lay::kColDV : Lay::kColDK);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) // queries 64g + 16kk .. of the tile
+                            mma_ts(dcol, acol + 8 * kk,
+                                   sdesc_sw128(b_addr + (4 * g + kk) * 2048, Lay::kChunkBytes, 1024), idesc_kv,
+                                   (m > 0 || g > 0 || kk > 0) ? 1u : 0u);
+                        if (g == 1) tc_commit(phase == 0 ? &sb.o_empty[slot] : &sb.q_empty[slot]);
+                    }
+                    __syncwarp();
+                }
+                return true;
+            };
+            ok = issue_s(0) && issue_dp(0);
+            for (int m = 0; ok && m < nq; ++m) {
+                ok = issue_acc(m, 0) && (m + 1 >= nq || issue_s(m + 1)) && issue_acc(m, 1) &&
+                     (m + 1 >= nq || issue_dp(m + 1));
             }
             if (!ok) break;
-            if (!issue_dkv(nq - 1, (it - 1) % S)) break;
-            if (lane == 0) tc_commit(&sb.dkv_full);
+            tc_commit(&sb.dkv_full);
             __syncwarp();
+            it0 += nq;
         }
     } else if (warp < 8) {
         // ----------------------------------------------------- compute ---
@@ -264,7 +305,7 @@ __global__ void __launch_bounds__(448, 1)
         const int row = threadIdx.x & 127;    // key row within the tile, TMEM lane
         const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
         const float scale_log2 = p.scale * 1.4426950408889634f;
-        uint32_t it = 0;
+        uint32_t it = 0, sync_phase = 0;
         TileRef r;
         bool ok = true;
         // -lse (log2 units, group 0) or -Delta (group 1) of query row `row` of tile i
@@ -284,7 +325,7 @@ __global__ void __launch_bounds__(448, 1)
             for (int i = ilo; i <= ihi && ok; ++i, ++it) {
                 const int buf = it & 1;
                 (g == 0 ? sb.lse2[buf] : sb.delta[buf])[row] = nxt;
-                named_bar_sync(1, 256);
+                if (!group_sync(&sb.cmp_sync, sync_phase, abort)) { ok = false; break; }
                 if (i < ihi) nxt = load_row(r, i + 1);
                 const int64_t q0 = int64_t(i) * kTile + 64 * g;
                 int64_t lo64 = k - q0, hi64 = qmax - q0;
@@ -294,125 +335,141 @@ __global__ void __launch_bounds__(448, 1)
                 const bool full = __all_sync(0xffffffffu, lo_c <= 0 && hi_c >= 63);
                 // shared copies hold -lse (log2 units) and -Delta, so each use is one packed FMA/add
                 const float4 *l2v = reinterpret_cast<const float4 *>(sb.lse2[buf] + 64 * g);
-                const float4 *dlv = reinterpret_cast<const float4 *>(sb.delta[buf] + 64 * g);
-                // phase A: P^T from S^T
+                const float2 *dlv2 = reinterpret_cast<const float2 *>(sb.delta[buf] + 64 * g);
+                // phase A: P^T from S^T, written (bf16) over the group's first 32 S^T columns
                 if (!mbar_wait(&sb.s_full, it & 1, abort)) { ok = false; break; }
                 tc_fence_after();
-                float pr[64];
+                // P^T of the group's 64 queries as bf16 pairs: the dV product reads the same
+                // rounded values from TMEM, and phase B forms dS from them
+                uint32_t pp[4][8];
+                const float2 sc2 = make_float2(scale_log2, scale_log2);
+                uint32_t sr[2][16];
+                tmem_ld16(tmem + lane_base + Lay::kColS + 64 * g, sr[0]);
+                tmem_wait_ld();
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t sr[32];
-                    tmem_ld32(tmem + lane_base + Lay::kColS + 64 * g + 32 * h2, sr);
-                    tmem_wait_ld();
-                    reg_fence(sr);
-                    if (h2 == 1) { // both halves read: the next tile's S^T may overwrite them
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sb.s_free);
-                    }
-                    const float2 sc2 = make_float2(scale_log2, scale_log2);
-#pragma unroll
-                    for (int c4 = 0; c4 < 8; ++c4) {
-                        const float4 l4 = l2v[8 * h2 + c4]; // -lse of 4 queries
-                        const float2 x01 = ffma2(make_float2(__uint_as_float(sr[4 * c4]), __uint_as_float(sr[4 * c4 + 1])),
-                                                 sc2, make_float2(l4.x, l4.y));
-                        const float2 x23 = ffma2(make_float2(__uint_as_float(sr[4 * c4 + 2]), __uint_as_float(sr[4 * c4 + 3])),
-                                                 sc2, make_float2(l4.z, l4.w));
-                        const float xv[4] = {x01.x, x01.y, x23.x, x23.y};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int cc = 32 * h2 + 4 * c4 + e;
-                            const float x = ex2_approx(xv[e]);
-                            pr[cc] = (full || (cc >= lo_c && cc <= hi_c)) ? x : 0.f;
-                        }
-                    }
-                }
-                // phase B: dS^T = P^T (dP^T - Delta); 16 queries at a time, P^T and dS^T (bf16)
-                // written over exactly the 16 dP^T columns just read
-                if (!mbar_wait(&sb.dp_full, it & 1, abort)) { ok = false; break; }
-                tc_fence_after();
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    uint32_t dr[16];
-                    tmem_ld16(tmem + lane_base + Lay::kColDP + 64 * g + 16 * b, dr);
-                    tmem_wait_ld();
-                    reg_fence(dr);
-                    uint32_t pk[8], dk8[8];
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    // 16 queries at a time, the next 16 in flight; their P^T lands in 8
+                    // columns this thread has already read
+                    uint32_t(&cur)[16] = sr[q4 & 1];
+                    reg_fence(cur);
+                    if (q4 < 3) tmem_ld16(tmem + lane_base + Lay::kColS + 64 * g + 16 * (q4 + 1), sr[(q4 + 1) & 1]);
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
-                        const float4 d4 = dlv[4 * b + c4]; // -Delta of 4 queries
-                        const int q = 16 * b + 4 * c4, j = 4 * c4;
-                        const float2 ds01 = fmul2(make_float2(pr[q], pr[q + 1]),
-                                                  fadd2(make_float2(__uint_as_float(dr[j]), __uint_as_float(dr[j + 1])),
-                                                        make_float2(d4.x, d4.y)));
-                        const float2 ds23 = fmul2(make_float2(pr[q + 2], pr[q + 3]),
-                                                  fadd2(make_float2(__uint_as_float(dr[j + 2]), __uint_as_float(dr[j + 3])),
-                                                        make_float2(d4.z, d4.w)));
-                        pk[2 * c4] = pack_bf16x2(pr[q], pr[q + 1]);
-                        pk[2 * c4 + 1] = pack_bf16x2(pr[q + 2], pr[q + 3]);
-                        dk8[2 * c4] = pack_bf16x2(ds01.x, ds01.y);
-                        dk8[2 * c4 + 1] = pack_bf16x2(ds23.x, ds23.y);
+                        const float4 l4 = l2v[4 * q4 + c4]; // -lse of 4 queries
+                        const float2 x01 = ffma2(make_float2(__uint_as_float(cur[4 * c4]), __uint_as_float(cur[4 * c4 + 1])),
+                                                 sc2, make_float2(l4.x, l4.y));
+                        const float2 x23 = ffma2(make_float2(__uint_as_float(cur[4 * c4 + 2]), __uint_as_float(cur[4 * c4 + 3])),
+                                                 sc2, make_float2(l4.z, l4.w));
+                        // one value in four goes through the FMA pipe to offload the MUFU unit
+                        float ev[4] = {ex2_approx(x01.x), ex2_approx(x01.y), ex2_approx(x23.x), exp2_fma(x23.y)};
+                        if (!full) {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int cc = 16 * q4 + 4 * c4 + e;
+                                ev[e] = (cc >= lo_c && cc <= hi_c) ? ev[e] : 0.f;
+                            }
+                        }
+                        pp[q4][2 * c4] = pack_bf16x2(ev[0], ev[1]);
+                        pp[q4][2 * c4 + 1] = pack_bf16x2(ev[2], ev[3]);
                     }
-                    tmem_st8(tmem + lane_base + Lay::kColDP + 64 * g + 16 * b, pk);
-                    tmem_st8(tmem + lane_base + Lay::kColDP + 64 * g + 16 * b + 8, dk8);
+                    tmem_st8(tmem + lane_base + Lay::kColS + 64 * g + 8 * q4, pp[q4]);
+                    if (q4 < 3) tmem_wait_ld();
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sb.ds_full[g]);
+                if (lane == 0) mbar_arrive(&sb.pa_done[g]);
+                // phase B: dS^T = P^T (dP^T - Delta), written (bf16) over the group's first 32 dP^T columns
+                if (!mbar_wait(&sb.dp_full, it & 1, abort)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    // 32 queries at a time; their dS^T lands in 16 columns this thread has read
+                    uint32_t dr[32];
+                    tmem_ld32(tmem + lane_base + Lay::kColDP + 64 * g + 32 * h2, dr);
+                    tmem_wait_ld();
+                    reg_fence(dr);
+                    uint32_t dk16[16];
+#pragma unroll
+                    for (int c2 = 0; c2 < 16; ++c2) {
+                        const float2 d2 = dlv2[16 * h2 + c2]; // -Delta of 2 queries
+                        const uint32_t pw = pp[2 * h2 + c2 / 8][c2 % 8];
+                        const float2 p2 = make_float2(__uint_as_float(pw << 16), __uint_as_float(pw & 0xffff0000u));
+                        const float2 ds = fmul2(p2, fadd2(make_float2(__uint_as_float(dr[2 * c2]),
+                                                                      __uint_as_float(dr[2 * c2 + 1])), d2));
+                        dk16[c2] = pack_bf16x2(ds.x, ds.y);
+                    }
+                    tmem_st16(tmem + lane_base + Lay::kColDP + 64 * g + 16 * h2, dk16);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sb.pb_done[g]);
             }
         }
     } else if (warp < 12) {
         // ---------------------------------------------------- epilogue ---
+        // A full tile leaves through a 128-row x 64-column shared staging buffer and
+        // TMA stores, so the rows are written as whole lines; the last tile of an
+        // example (rows past its end belong to the next example) is stored row by row.
         const int row = threadIdx.x & 127;    // key row within the tile, TMEM lane
         const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
-        uint32_t item_cnt = 0;
+        const bool leader = threadIdx.x == 256;
+        uint8_t *stage = smem + Lay::kStage;
+        uint32_t item_cnt = 0, sync_phase = 0;
+        bool ok = true;
         TileRef r;
-        for (int64_t n = blockIdx.x; decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
+        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
             const int64_t k = int64_t(r.t) * kTile + row;
             const bool valid_k = k < r.L;
+            const bool full_tile = int64_t(r.t) * kTile + kTile <= r.L;
             const int64_t grow = (int64_t(r.s0) + k) * p.heads + r.h;
             if (!mbar_wait(&sb.dkv_full, item_cnt & 1, abort)) break;
             tc_fence_after();
-            // dV: load and store chunk by chunk
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t rr[32];
-                tmem_ld32(tmem + lane_base + Lay::kColDV + c * 32, rr);
+            // 64 columns at a time: dV chunks, then dK chunks (scaled by 1/sqrt(D))
+#pragma unroll 1
+            for (int part = 0; part < 2 * Lay::kChunks; ++part) {
+                const bool is_k = part >= Lay::kChunks;
+                const int c = is_k ? part - Lay::kChunks : part;
+                const float sc = is_k ? p.scale : 1.f;
+                uint32_t rr[2][32];
+                tmem_ld32(tmem + lane_base + (is_k ? Lay::kColDK : Lay::kColDV) + 64 * c, rr[0]);
+                tmem_ld32(tmem + lane_base + (is_k ? Lay::kColDK : Lay::kColDV) + 64 * c + 32, rr[1]);
                 tmem_wait_ld();
-                reg_fence(rr);
-                if (valid_k) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(dv + grow * D + c * 32);
+                reg_fence(rr[0]);
+                reg_fence(rr[1]);
+                if (part == 2 * Lay::kChunks - 1) { // every accumulator column read: the next item may start
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sb.dkv_free);
+                }
+                uint32_t pk[32];
 #pragma unroll
-                    for (int x = 0; x < 4; ++x)
-                        dst[x] = make_uint4(pack_bf16x2(__uint_as_float(rr[8 * x + 0]), __uint_as_float(rr[8 * x + 1])),
-                                            pack_bf16x2(__uint_as_float(rr[8 * x + 2]), __uint_as_float(rr[8 * x + 3])),
-                                            pack_bf16x2(__uint_as_float(rr[8 * x + 4]), __uint_as_float(rr[8 * x + 5])),
-                                            pack_bf16x2(__uint_as_float(rr[8 * x + 6]), __uint_as_float(rr[8 * x + 7])));
+                for (int x = 0; x < 32; ++x)
+                    pk[x] = pack_bf16x2(__uint_as_float(rr[x / 16][2 * (x % 16)]) * sc,
+                                        __uint_as_float(rr[x / 16][2 * (x % 16) + 1]) * sc);
+                if (full_tile) {
+                    if (leader) bulk_wait_group_read<0>(); // the previous store has left the buffer
+                    if (!group_sync(&sb.epi_sync, sync_phase, abort)) { ok = false; break; }
+                    uint8_t *srow = stage + row * 128;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        *reinterpret_cast<uint4 *>(srow + ((u ^ (row & 7)) << 4)) =
+                            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                    fence_proxy_async_smem();
+                    if (!group_sync(&sb.epi_sync, sync_phase, abort)) { ok = false; break; }
+                    if (leader) {
+                        tma_store_2d(is_k ? &tm_dk : &tm_dv, stage, r.h * D + 64 * c, r.s0 + r.t * kTile);
+                        bulk_commit_group();
+                    }
+                } else if (valid_k) {
+                    uint4 *dst = reinterpret_cast<uint4 *>((is_k ? dk : dv) + grow * D + 64 * c);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
                 }
             }
-            // dK: take it all out of TMEM, release the accumulators, then store
-            uint32_t kp[D / 2];
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t rr[32];
-                tmem_ld32(tmem + lane_base + Lay::kColDK + c * 32, rr);
-                tmem_wait_ld();
-                reg_fence(rr);
-#pragma unroll
-                for (int x = 0; x < 16; ++x)
-                    kp[16 * c + x] = pack_bf16x2(__uint_as_float(rr[2 * x]) * p.scale,
-                                                 __uint_as_float(rr[2 * x + 1]) * p.scale);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sb.dkv_free);
-            if (valid_k) {
-                uint4 *dst = reinterpret_cast<uint4 *>(dk + grow * D);
-#pragma unroll
-                for (int x = 0; x < D / 8; ++x) dst[x] = make_uint4(kp[4 * x], kp[4 * x + 1], kp[4 * x + 2], kp[4 * x + 3]);
-            }
         }
+        if (leader) bulk_wait_group<0>();
     }
 
     tc_fence_before();
@@ -424,24 +481,27 @@ __global__ void __launch_bounds__(448, 1)
 
 template <int D>
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                  const CUtensorMap &tdo, const Problem &p, const float *lse, const float *delta,
-                                  void *dk, void *dv, int num_sms, cudaStream_t stream)
+                                  const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
+                                  const Problem &p, const float *lse, const float *delta, void *dk, void *dv,
+                                  int num_sms, cudaStream_t stream)
 {
     using Lay = DkvLayout<D>;
     auto kern = bwd_dkdv_sm100_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, p, lse, delta,
+    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, tdk, tdv, p, lse, delta,
                                                           static_cast<__nv_bfloat16 *>(dk),
                                                           static_cast<__nv_bfloat16 *>(dv));
     return cudaGetLastError();
 }
 
 template cudaError_t launch_bwd_dkdv_sm100<64>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                                               const CUtensorMap &, const Problem &, const float *, const float *,
-                                               void *, void *, int, cudaStream_t);
+                                               const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
+                                               const Problem &, const float *, const float *, void *, void *, int,
+                                               cudaStream_t);
 template cudaError_t launch_bwd_dkdv_sm100<128>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                                                const CUtensorMap &, const Problem &, const float *, const float *,
-                                                void *, void *, int, cudaStream_t);
+                                                const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
+                                                const Problem &, const float *, const float *, void *, void *, int,
+                                                cudaStream_t);
 
 } // namespace ba

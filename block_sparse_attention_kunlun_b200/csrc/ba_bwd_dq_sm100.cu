@@ -52,7 +52,9 @@ struct DqLayout {
     static constexpr int kStaging = 2 * kStages * kTileBytes; // Q, dO, out tiles of the next item
     static constexpr int kBytes = kStaging + 3 * kTileBytes;
     static constexpr int kAlloc = kBytes + 1024;
-    static constexpr int kThreads = 320;
+    static constexpr int kThreads = 384;                 // three warpgroups
+    // register budgets after the split; 2 * 128 * 216 + 128 * 72 = 384 * 168
+    static constexpr uint32_t kRegsCompute = 216, kRegsOther = 72;
     static constexpr uint32_t kColQ = 0, kColDO = D / 2, kColS = D, kColDP = D + 128, kColDQ = D + 256;
     static constexpr uint32_t kTmemCols = 512;
 };
@@ -74,7 +76,7 @@ __device__ __forceinline__ int first_key_tile(const TileRef &r, int64_t B, int64
 } // namespace
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_o, const Problem p, const float *__restrict__ lse,
@@ -127,124 +129,129 @@ __global__ void __launch_bounds__(320, 1)
     const int64_t T = p.total_tokens;
     const int32_t ntiles = live_tile_count(p);
 
-    if (warp == 8) {
-        // ------------------------------------------------ TMA producer ---
-        uint32_t kv_cnt = 0, item_cnt = 0;
-        TileRef r;
-        bool ok = true;
-        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
-            const int jlo = first_key_tile(r, B, W);
-            if (!mbar_wait(&sb.st_empty, (item_cnt & 1) ^ 1, abort)) break;
-            if (lane == 0) {
-                uint8_t *st = smem + Lay::kStaging;
-                mbar_arrive_expect_tx(&sb.st_full, 3 * Lay::kTileBytes);
-                for (int c = 0; c < Lay::kChunks; ++c) {
-                    const int x = r.h * D + c * 64, y = r.s0 + r.t * kTile;
-                    tma_load_2d(st + c * Lay::kChunkBytes, &tm_q, &sb.st_full, x, y);
-                    tma_load_2d(st + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_do, &sb.st_full, x, y);
-                    tma_load_2d(st + 2 * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_o, &sb.st_full, x, y);
-                }
-            }
-            __syncwarp();
-            for (int j = jlo; j <= r.t; ++j, ++kv_cnt) {
-                const int st = kv_cnt % S;
-                if (!mbar_wait(&sb.kv_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
-                    ok = false;
-                    break;
-                }
+    if (warp >= 8) {
+        // warps 8-11 (one warpgroup: TMA, MMA, two idle) hand registers to the compute warpgroups
+        warpgroup_regs_dec<Lay::kRegsOther>();
+        if (warp == 8) {
+            // ------------------------------------------------ TMA producer ---
+            uint32_t kv_cnt = 0, item_cnt = 0;
+            TileRef r;
+            bool ok = true;
+            for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
+                const int jlo = first_key_tile(r, B, W);
+                if (!mbar_wait(&sb.st_empty, (item_cnt & 1) ^ 1, abort)) break;
                 if (lane == 0) {
-                    uint8_t *kdst = smem + Lay::kKV0 + 2 * st * Lay::kTileBytes;
-                    mbar_arrive_expect_tx(&sb.kv_full[st], 2 * Lay::kTileBytes);
+                    uint8_t *st = smem + Lay::kStaging;
+                    mbar_arrive_expect_tx(&sb.st_full, 3 * Lay::kTileBytes);
                     for (int c = 0; c < Lay::kChunks; ++c) {
-                        tma_load_2d(kdst + c * Lay::kChunkBytes, &tm_k, &sb.kv_full[st], r.h * D + c * 64,
-                                    r.s0 + j * kTile);
-                        tma_load_2d(kdst + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_v, &sb.kv_full[st],
-                                    r.h * D + c * 64, r.s0 + j * kTile);
+                        const int x = r.h * D + c * 64, y = r.s0 + r.t * kTile;
+                        tma_load_2d(st + c * Lay::kChunkBytes, &tm_q, &sb.st_full, x, y);
+                        tma_load_2d(st + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_do, &sb.st_full, x, y);
+                        tma_load_2d(st + 2 * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_o, &sb.st_full, x, y);
                     }
                 }
                 __syncwarp();
-            }
-        }
-    } else if (warp == 9) {
-        // -------------------------------------------------- MMA issuer ---
-        constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false); // S, dP
-        constexpr uint32_t idesc_q = idesc_bf16(128, D, false, true);    // dQ (B = K, MN-major)
-        uint32_t kv_cnt = 0, s_cnt = 0, d_cnt = 0, item_cnt = 0;
-        TileRef r;
-        bool ok = true;
-        // dQ += dS K for the key tile in ring stage `st` (m = its index in the item)
-        auto issue_dq = [&](int m, int st) -> bool {
-            if (!mbar_wait(&sb.ds_full[0], d_cnt & 1, abort)) return false;
-            if (m == 0 && !mbar_wait(&sb.dq_free, (item_cnt & 1) ^ 1, abort)) return false;
-            tc_fence_after();
-            const uint32_t k_addr = smem_base + Lay::kKV0 + 2 * st * Lay::kTileBytes;
-            if (lane == 0) {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + Lay::kColDQ, tmem + Lay::kColDP + kk * 8,
-                           sdesc_sw128(k_addr + kk * 2048, Lay::kChunkBytes, 1024), idesc_q,
-                           (m > 0 || kk > 0) ? 1u : 0u);
-            }
-            __syncwarp();
-            if (!mbar_wait(&sb.ds_full[1], d_cnt & 1, abort)) return false;
-            tc_fence_after();
-            if (lane == 0) {
-#pragma unroll
-                for (int kk = 4; kk < 8; ++kk)
-                    mma_ts(tmem + Lay::kColDQ, tmem + Lay::kColDP + 64 + (kk - 4) * 8,
-                           sdesc_sw128(k_addr + kk * 2048, Lay::kChunkBytes, 1024), idesc_q, 1u);
-                tc_commit(&sb.kv_empty[st]);
-            }
-            __syncwarp();
-            ++d_cnt;
-            return true;
-        };
-        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
-            const int jlo = first_key_tile(r, B, W);
-            const int nkv = r.t - jlo + 1;
-            if (!mbar_wait(&sb.qt_ready, item_cnt & 1, abort)) break;
-            tc_fence_after();
-            for (int m = 0; m < nkv; ++m, ++kv_cnt, ++s_cnt) {
-                const int st = kv_cnt % S;
-                if (!mbar_wait(&sb.kv_full[st], (kv_cnt / S) & 1, abort) ||
-                    !mbar_wait(&sb.s_free, (s_cnt & 1) ^ 1, abort)) {
-                    ok = false;
-                    break;
+                for (int j = jlo; j <= r.t; ++j, ++kv_cnt) {
+                    const int st = kv_cnt % S;
+                    if (!mbar_wait(&sb.kv_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        uint8_t *kdst = smem + Lay::kKV0 + 2 * st * Lay::kTileBytes;
+                        mbar_arrive_expect_tx(&sb.kv_full[st], 2 * Lay::kTileBytes);
+                        for (int c = 0; c < Lay::kChunks; ++c) {
+                            tma_load_2d(kdst + c * Lay::kChunkBytes, &tm_k, &sb.kv_full[st], r.h * D + c * 64,
+                                        r.s0 + j * kTile);
+                            tma_load_2d(kdst + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_v, &sb.kv_full[st],
+                                        r.h * D + c * 64, r.s0 + j * kTile);
+                        }
+                    }
+                    __syncwarp();
                 }
+            }
+        } else if (warp == 9) {
+            // -------------------------------------------------- MMA issuer ---
+            constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false); // S, dP
+            constexpr uint32_t idesc_q = idesc_bf16(128, D, false, true);    // dQ (B = K, MN-major)
+            uint32_t kv_cnt = 0, s_cnt = 0, d_cnt = 0, item_cnt = 0;
+            TileRef r;
+            bool ok = true;
+            // dQ += dS K for the key tile in ring stage `st` (m = its index in the item)
+            auto issue_dq = [&](int m, int st) -> bool {
+                if (!mbar_wait_warp(&sb.ds_full[0], d_cnt & 1, abort)) return false;
+                if (m == 0 && !mbar_wait_warp(&sb.dq_free, (item_cnt & 1) ^ 1, abort)) return false;
                 tc_fence_after();
                 const uint32_t k_addr = smem_base + Lay::kKV0 + 2 * st * Lay::kTileBytes;
-                const uint32_t v_addr = k_addr + Lay::kTileBytes;
-                if (lane == 0) {
+                {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ts(tmem + Lay::kColS, tmem + Lay::kColQ + kk * 8,
-                               sdesc_sw128(k_addr + (kk / 4) * Lay::kChunkBytes + (kk % 4) * 32, 16, 1024),
-                               idesc_s, kk > 0 ? 1u : 0u);
-                    tc_commit(&sb.s_full);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tmem + Lay::kColDQ, tmem + Lay::kColDP + kk * 8,
+                               sdesc_sw128(k_addr + kk * 2048, Lay::kChunkBytes, 1024), idesc_q,
+                               (m > 0 || kk > 0) ? 1u : 0u);
                 }
                 __syncwarp();
-                // dQ of the previous key tile: it reads dS from the dP columns,
-                // so it must be issued before this tile's dP overwrites them.
-                if (m > 0 && !issue_dq(m - 1, (kv_cnt - 1) % S)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) {
+                if (!mbar_wait_warp(&sb.ds_full[1], d_cnt & 1, abort)) return false;
+                tc_fence_after();
+                {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ts(tmem + Lay::kColDP, tmem + Lay::kColDO + kk * 8,
-                               sdesc_sw128(v_addr + (kk / 4) * Lay::kChunkBytes + (kk % 4) * 32, 16, 1024),
-                               idesc_s, kk > 0 ? 1u : 0u);
-                    tc_commit(&sb.dp_full);
+                    for (int kk = 4; kk < 8; ++kk)
+                        mma_ts(tmem + Lay::kColDQ, tmem + Lay::kColDP + 64 + (kk - 4) * 8,
+                               sdesc_sw128(k_addr + kk * 2048, Lay::kChunkBytes, 1024), idesc_q, 1u);
+                    tc_commit(&sb.kv_empty[st]);
                 }
+                __syncwarp();
+                ++d_cnt;
+                return true;
+            };
+            for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
+                const int jlo = first_key_tile(r, B, W);
+                const int nkv = r.t - jlo + 1;
+                if (!mbar_wait_warp(&sb.qt_ready, item_cnt & 1, abort)) break;
+                tc_fence_after();
+                for (int m = 0; m < nkv; ++m, ++kv_cnt, ++s_cnt) {
+                    const int st = kv_cnt % S;
+                    if (!mbar_wait_warp(&sb.kv_full[st], (kv_cnt / S) & 1, abort) ||
+                        !mbar_wait_warp(&sb.s_free, (s_cnt & 1) ^ 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_base + Lay::kKV0 + 2 * st * Lay::kTileBytes;
+                    const uint32_t v_addr = k_addr + Lay::kTileBytes;
+                    {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            mma_ts(tmem + Lay::kColS, tmem + Lay::kColQ + kk * 8,
+                                   sdesc_sw128(k_addr + (kk / 4) * Lay::kChunkBytes + (kk % 4) * 32, 16, 1024),
+                                   idesc_s, kk > 0 ? 1u : 0u);
+                        tc_commit(&sb.s_full);
+                    }
+                    __syncwarp();
+                    // dQ of the previous key tile: it reads dS from the dP columns,
+                    // so it must be issued before this tile's dP overwrites them.
+                    if (m > 0 && !issue_dq(m - 1, (kv_cnt - 1) % S)) {
+                        ok = false;
+                        break;
+                    }
+                    {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            mma_ts(tmem + Lay::kColDP, tmem + Lay::kColDO + kk * 8,
+                                   sdesc_sw128(v_addr + (kk / 4) * Lay::kChunkBytes + (kk % 4) * 32, 16, 1024),
+                                   idesc_s, kk > 0 ? 1u : 0u);
+                        tc_commit(&sb.dp_full);
+                    }
+                    __syncwarp();
+                }
+                if (!ok) break;
+                if (!issue_dq(nkv - 1, (kv_cnt - 1) % S)) break;
+                tc_commit(&sb.dq_done);
                 __syncwarp();
             }
-            if (!ok) break;
-            if (!issue_dq(nkv - 1, (kv_cnt - 1) % S)) break;
-            if (lane == 0) tc_commit(&sb.dq_done);
-            __syncwarp();
         }
     } else {
+        warpgroup_regs_inc<Lay::kRegsCompute>();
         // ----------------------------------------------------- compute ---
         const int g = warp >> 2;              // column group: keys [64g, 64g+64)
         const int row = threadIdx.x & 127;    // query row within the tile, TMEM lane
@@ -328,46 +335,60 @@ __global__ void __launch_bounds__(320, 1)
                 // phase A: P from S
                 if (!mbar_wait(&sb.s_full, s_cnt & 1, abort)) { ok = false; break; }
                 tc_fence_after();
-                float pr[64];
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t sr[32];
-                    tmem_ld32(tmem + lane_base + Lay::kColS + 64 * g + 32 * h2, sr);
+                // P of this group's 64 keys as bf16 pairs (phase B only needs it to form dS)
+                uint32_t pp[4][8];
+                const float2 sc2 = make_float2(scale_log2, scale_log2), nl2 = make_float2(-l2, -l2);
+                {
+                    uint32_t sr[2][16];
+                    tmem_ld16(tmem + lane_base + Lay::kColS + 64 * g, sr[0]);
                     tmem_wait_ld();
-                    reg_fence(sr);
-                    if (h2 == 1) { // both halves read: the next tile's S may overwrite them
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sb.s_free);
-                    }
-                    const float2 sc2 = make_float2(scale_log2, scale_log2), nl2 = make_float2(-l2, -l2);
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2) {
-                        const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nl2);
-                        const int cc = 32 * h2 + c;
-                        const float e0 = ex2_approx(x.x), e1 = ex2_approx(x.y);
-                        pr[cc] = (full || (cc >= lo_c && cc <= hi_c)) ? e0 : 0.f;
-                        pr[cc + 1] = (full || (cc + 1 >= lo_c && cc + 1 <= hi_c)) ? e1 : 0.f;
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        // 16 keys at a time, the next 16 in flight
+                        uint32_t(&cur)[16] = sr[q4 & 1];
+                        reg_fence(cur);
+                        if (q4 < 3) tmem_ld16(tmem + lane_base + Lay::kColS + 64 * g + 16 * (q4 + 1), sr[(q4 + 1) & 1]);
+                        else {
+                            // all of S read: the next tile's S may overwrite it
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&sb.s_free);
+                        }
+#pragma unroll
+                        for (int c2 = 0; c2 < 8; ++c2) {
+                            const float2 x = ffma2(make_float2(__uint_as_float(cur[2 * c2]), __uint_as_float(cur[2 * c2 + 1])),
+                                                   sc2, nl2);
+                            // one value in four goes through the FMA pipe to offload the MUFU unit
+                            float e0 = ex2_approx(x.x), e1 = (c2 & 1) ? exp2_fma(x.y) : ex2_approx(x.y);
+                            if (!full) {
+                                const int cc = 16 * q4 + 2 * c2;
+                                e0 = (cc >= lo_c && cc <= hi_c) ? e0 : 0.f;
+                                e1 = (cc + 1 >= lo_c && cc + 1 <= hi_c) ? e1 : 0.f;
+                            }
+                            pp[q4][c2] = pack_bf16x2(e0, e1);
+                        }
+                        if (q4 < 3) tmem_wait_ld();
                     }
                 }
                 // phase B: dS = P (dP - Delta), written as bf16 over this group's dP columns
                 if (!mbar_wait(&sb.dp_full, s_cnt & 1, abort)) { ok = false; break; }
                 tc_fence_after();
-                // 32 keys at a time; chunk h2's dS (16 columns) lands in [64g+16h2, +16),
-                // inside the dP columns this thread has already read.
+                const float2 ndl = make_float2(-dl, -dl);
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
+                    // 32 keys at a time; their dS (16 columns) lands in [64g+16h2, +16),
+                    // inside the dP columns this thread has already read
                     uint32_t dr[32];
                     tmem_ld32(tmem + lane_base + Lay::kColDP + 64 * g + 32 * h2, dr);
                     tmem_wait_ld();
                     reg_fence(dr);
                     uint32_t pk[16];
-                    const float2 ndl = make_float2(-dl, -dl);
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        const int k0c = 32 * h2 + 2 * c;
-                        const float2 ds = fmul2(make_float2(pr[k0c], pr[k0c + 1]),
-                                                fadd2(make_float2(__uint_as_float(dr[2 * c]), __uint_as_float(dr[2 * c + 1])), ndl));
+                        const uint32_t pw = pp[2 * h2 + c / 8][c % 8];
+                        const float2 p2 = make_float2(__uint_as_float(pw << 16), __uint_as_float(pw & 0xffff0000u));
+                        const float2 ds = fmul2(p2, fadd2(make_float2(__uint_as_float(dr[2 * c]),
+                                                                      __uint_as_float(dr[2 * c + 1])), ndl));
                         pk[c] = pack_bf16x2(ds.x, ds.y);
                     }
                     tmem_st16(tmem + lane_base + Lay::kColDP + 64 * g + 16 * h2, pk);
@@ -388,7 +409,7 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_after();
             {
                 __nv_bfloat16 *qrow = dq + ((int64_t(r.s0) + i) * p.heads + r.h) * D + (D / 2) * g;
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < D / 64; ++c) {
                     uint32_t a[32];
                     tmem_ld32(tmem + lane_base + Lay::kColDQ + (D / 2) * g + 32 * c, a);
@@ -433,6 +454,12 @@ cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, co
     auto kern = bwd_dq_sm100_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
+    // the register split only works if the CTA is launched with at least the budgets' sum
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * Lay::kThreads < int(256 * Lay::kRegsCompute + 128 * Lay::kRegsOther))
+        return cudaErrorInvalidConfiguration;
     kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, to, p, lse, delta,
                                                           static_cast<__nv_bfloat16 *>(dq));
     return cudaGetLastError();

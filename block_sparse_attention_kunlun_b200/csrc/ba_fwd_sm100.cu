@@ -49,7 +49,9 @@ struct FwdLayout {
     static constexpr int kK0 = 2 * kTileBytes;           // stage s: K at kK0 + 2 s tile, V after it
     static constexpr int kBytes = kTileBytes * (2 + 2 * kStages);
     static constexpr int kAlloc = kBytes + 1024;         // slack to align the base to 1024 B
-    static constexpr int kThreads = 320;
+    static constexpr int kThreads = 384;                 // three warpgroups
+    // register budgets after the split; 2 * 128 * 200 + 128 * 104 = 384 * 168
+    static constexpr uint32_t kRegsCompute = 200, kRegsOther = 104;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColO = 256;
 };
@@ -57,24 +59,10 @@ struct FwdLayout {
 struct FwdBarriers {
     uint64_t q_full, q_empty;
     uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
-    uint64_t kv_full[4], kv_empty[4];
+    uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
     uint32_t tmem_base;
     int abort;
 };
-
-// 2^x on the FMA pipe for x <= 8 (values below 2^-125 come out as 2^-125 or
-// smaller, far below what a bf16 P can hold next to the row maximum). Round x
-// to the nearest integer n with the 1.5 * 2^23 trick, evaluate 2^(x-n) on
-// [-0.5, 0.5] with a cubic fitted to 2^f (relative error < 8e-5, measured on a
-// dense grid), and add n to the exponent field.
-__device__ __forceinline__ float exp2_fma(float x)
-{
-    x = fmaxf(x, -125.f);
-    const float t = x + 12582912.f;
-    const float f = x - (t - 12582912.f);
-    const float p = fmaf(fmaf(fmaf(0.055171654f, f, 0.24261115f), f, 0.69326097f), f, 0.99992806f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
 
 // Key-tile range of query tile t: [first_key_tile, t].
 __device__ __forceinline__ int first_key_tile(int t, int64_t B, int64_t W)
@@ -85,7 +73,7 @@ __device__ __forceinline__ int first_key_tile(int t, int64_t B, int64_t W)
 } // namespace
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const Problem p,
                           __nv_bfloat16 *__restrict__ out, float *__restrict__ lse)
@@ -109,8 +97,10 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(&sb.o_free[w], 4);
         }
         for (int i = 0; i < S; ++i) {
-            mbar_init(&sb.kv_full[i], 1);
-            mbar_init(&sb.kv_empty[i], 1);
+            mbar_init(&sb.k_full[i], 1);
+            mbar_init(&sb.k_empty[i], 1);
+            mbar_init(&sb.v_full[i], 1);
+            mbar_init(&sb.v_empty[i], 1);
         }
         sb.abort = 0;
         fence_mbar_init();
@@ -132,128 +122,152 @@ __global__ void __launch_bounds__(320, 1)
     const int64_t B = p.block, W = p.window;
     const int32_t npairs = live_pair_count(p);
 
-    if (warp == 8) {
-        // ------------------------------------------------ TMA producer ---
-        uint32_t kv_cnt = 0, item_cnt = 0;
-        TileRef r;
-        bool second;
-        bool ok = true;
-        for (int64_t n = blockIdx.x; ok && decode_pair(p, npairs, n, r, second); n += gridDim.x, ++item_cnt) {
-            const int jlo = first_key_tile(r.t, B, W);
-            const int jhi = r.t + (second ? 1 : 0);
-            if (!mbar_wait(&sb.q_empty, (item_cnt & 1) ^ 1, abort)) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&sb.q_full, (second ? 2 : 1) * Lay::kTileBytes);
-                for (int w = 0; w < (second ? 2 : 1); ++w)
-                    for (int c = 0; c < Lay::kChunks; ++c)
-                        tma_load_2d(smem + Lay::kQ + w * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_q, &sb.q_full,
-                                    r.h * D + c * 64, r.s0 + (r.t + w) * kTile);
-                // warm L2 with the next item's query tiles
-                TileRef rn;
-                bool sn;
-                if (decode_pair(p, npairs, n + gridDim.x, rn, sn))
-                    for (int w = 0; w < (sn ? 2 : 1); ++w)
+    if (warp >= 8) {
+        // warps 8-11 (one warpgroup: TMA, MMA, two idle) hand registers to the compute warpgroups
+        warpgroup_regs_dec<Lay::kRegsOther>();
+        if (warp == 8) {
+            // ------------------------------------------------ TMA producer ---
+            uint32_t kv_cnt = 0, item_cnt = 0;
+            TileRef r;
+            bool second;
+            bool ok = true;
+            for (int64_t n = blockIdx.x; ok && decode_pair(p, npairs, n, r, second); n += gridDim.x, ++item_cnt) {
+                const int jlo = first_key_tile(r.t, B, W);
+                const int jhi = r.t + (second ? 1 : 0);
+                if (!mbar_wait(&sb.q_empty, (item_cnt & 1) ^ 1, abort)) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sb.q_full, (second ? 2 : 1) * Lay::kTileBytes);
+                    for (int w = 0; w < (second ? 2 : 1); ++w)
                         for (int c = 0; c < Lay::kChunks; ++c)
-                            tma_prefetch_l2_2d(&tm_q, rn.h * D + c * 64, rn.s0 + (rn.t + w) * kTile);
-            }
-            __syncwarp();
-            for (int j = jlo; j <= jhi; ++j, ++kv_cnt) {
-                const int st = kv_cnt % S;
-                if (!mbar_wait(&sb.kv_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
-                    ok = false;
-                    break;
+                            tma_load_2d(smem + Lay::kQ + w * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_q, &sb.q_full,
+                                        r.h * D + c * 64, r.s0 + (r.t + w) * kTile);
+                    // warm L2 with the next item's query tiles
+                    TileRef rn;
+                    bool sn;
+                    if (decode_pair(p, npairs, n + gridDim.x, rn, sn))
+                        for (int w = 0; w < (sn ? 2 : 1); ++w)
+                            for (int c = 0; c < Lay::kChunks; ++c)
+                                tma_prefetch_l2_2d(&tm_q, rn.h * D + c * 64, rn.s0 + (rn.t + w) * kTile);
                 }
-                if (lane == 0) {
+                __syncwarp();
+                for (int j = jlo; j <= jhi; ++j, ++kv_cnt) {
+                    const int st = kv_cnt % S;
                     uint8_t *kdst = smem + Lay::kK0 + 2 * st * Lay::kTileBytes;
-                    mbar_arrive_expect_tx(&sb.kv_full[st], 2 * Lay::kTileBytes);
-                    for (int c = 0; c < Lay::kChunks; ++c) {
-                        tma_load_2d(kdst + c * Lay::kChunkBytes, &tm_k, &sb.kv_full[st], r.h * D + c * 64,
-                                    r.s0 + j * kTile);
-                        tma_load_2d(kdst + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_v, &sb.kv_full[st],
-                                    r.h * D + c * 64, r.s0 + j * kTile);
+                    // K and V of a stage are released separately (K after the tile's S products,
+                    // V after its P V products), so each is refilled as soon as it is free
+                    if (!mbar_wait(&sb.k_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
+                        ok = false;
+                        break;
                     }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&sb.k_full[st], Lay::kTileBytes);
+                        for (int c = 0; c < Lay::kChunks; ++c)
+                            tma_load_2d(kdst + c * Lay::kChunkBytes, &tm_k, &sb.k_full[st], r.h * D + c * 64,
+                                        r.s0 + j * kTile);
+                    }
+                    __syncwarp();
+                    if (!mbar_wait(&sb.v_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&sb.v_full[st], Lay::kTileBytes);
+                        for (int c = 0; c < Lay::kChunks; ++c)
+                            tma_load_2d(kdst + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_v, &sb.v_full[st],
+                                        r.h * D + c * 64, r.s0 + j * kTile);
+                    }
+                    __syncwarp();
                 }
-                __syncwarp();
             }
-        }
-    } else if (warp == 9) {
-        // -------------------------------------------------- MMA issuer ---
-        constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
-        constexpr uint32_t idesc_o = idesc_bf16(128, D, false, true);
-        uint32_t kv_cnt = 0, item_cnt = 0;
-        uint32_t pcnt[2] = {0, 0}; // P tiles consumed so far by each group
-        uint32_t icnt[2] = {0, 0}; // items each group has finished (group 1 skips single-tile items)
-        TileRef r;
-        bool second;
-        bool ok = true;
-        for (int64_t n = blockIdx.x; ok && decode_pair(p, npairs, n, r, second); n += gridDim.x, ++item_cnt) {
-            const int lo[2] = {first_key_tile(r.t, B, W), second ? first_key_tile(r.t + 1, B, W) : 1};
-            const int hi[2] = {r.t, second ? r.t + 1 : 0};
-            const int jlo = lo[0], jhi = second ? hi[1] : hi[0];
-            if (!mbar_wait(&sb.q_full, item_cnt & 1, abort)) break;
-            tc_fence_after();
-            // O_w += P_w V for key tile j of group w (V from ring stage st)
-            auto issue_pv = [&](int w, int j, int st) -> bool {
-                if (!mbar_wait(&sb.p_full[w], pcnt[w] & 1, abort)) return false;
-                const bool first = (j == lo[w]);
-                if (first && !mbar_wait(&sb.o_free[w], (icnt[w] & 1) ^ 1, abort)) return false;
+        } else if (warp == 9) {
+            // -------------------------------------------------- MMA issuer ---
+            constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t idesc_o = idesc_bf16(128, D, false, true);
+            uint32_t kv_cnt = 0, item_cnt = 0;
+            uint32_t pcnt[2] = {0, 0}; // P tiles consumed so far by each group
+            uint32_t icnt[2] = {0, 0}; // items each group has finished (group 1 skips single-tile items)
+            TileRef r;
+            bool second;
+            bool ok = true;
+            for (int64_t n = blockIdx.x; ok && decode_pair(p, npairs, n, r, second); n += gridDim.x, ++item_cnt) {
+                const int lo[2] = {first_key_tile(r.t, B, W), second ? first_key_tile(r.t + 1, B, W) : 1};
+                const int hi[2] = {r.t, second ? r.t + 1 : 0};
+                const int jlo = lo[0], jhi = second ? hi[1] : hi[0];
+                if (!mbar_wait_warp(&sb.q_full, item_cnt & 1, abort)) break;
                 tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t v_addr = smem_base + Lay::kK0 + (2 * st + 1) * Lay::kTileBytes;
+                // O_w += P_w V for key tile j of group w (V from ring stage st)
+                auto issue_pv = [&](int w, int j, int st) -> bool {
+                    if (!mbar_wait_warp(&sb.p_full[w], pcnt[w] & 1, abort)) return false;
+                    const bool first = (j == lo[w]);
+                    if (first && !mbar_wait_warp(&sb.o_free[w], (icnt[w] & 1) ^ 1, abort)) return false;
+                    tc_fence_after();
+                    {
+                        const uint32_t v_addr = smem_base + Lay::kK0 + (2 * st + 1) * Lay::kTileBytes;
 #pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk)
-                        mma_ts(tmem + Lay::kColO + D * w, tmem + 128 * w + kk * 8,
-                               sdesc_sw128(v_addr + kk * 2048, Lay::kChunkBytes, 1024), idesc_o,
-                               (!first || kk > 0) ? 1u : 0u);
-                    if (j == hi[w]) tc_commit(&sb.o_final[w]);
-                }
-                __syncwarp();
-                ++pcnt[w];
-                return true;
-            };
-            auto issue_s = [&](int w, int st) {
-                if (lane == 0) {
-                    const uint32_t q_addr = smem_base + Lay::kQ + w * Lay::kTileBytes;
-                    const uint32_t k_addr = smem_base + Lay::kK0 + 2 * st * Lay::kTileBytes;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk / 4) * Lay::kChunkBytes + (kk % 4) * 32;
-                        mma_ss(tmem + 128 * w, sdesc_sw128(q_addr + off, 16, 1024),
-                               sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < kTile / 16; ++kk)
+                            mma_ts(tmem + Lay::kColO + D * w, tmem + 128 * w + kk * 8,
+                                   sdesc_sw128(v_addr + kk * 2048, Lay::kChunkBytes, 1024), idesc_o,
+                                   (!first || kk > 0) ? 1u : 0u);
+                        if (j == hi[w]) tc_commit(&sb.o_final[w]);
                     }
-                    tc_commit(&sb.s_full[w]);
-                }
-                __syncwarp();
-            };
-            for (int j = jlo; j <= jhi && ok; ++j, ++kv_cnt) {
-                const int st = kv_cnt % S;
-                if (!mbar_wait(&sb.kv_full[st], (kv_cnt / S) & 1, abort)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                for (int w = 0; w < 2 && ok; ++w) {
-                    // the previous tile's P V of this group reads P from the S buffer: issue it first
-                    if (j - 1 >= lo[w] && j - 1 <= hi[w] && !issue_pv(w, j - 1, (kv_cnt - 1) % S)) ok = false;
-                    if (ok && j >= lo[w] && j <= hi[w]) issue_s(w, st);
+                    __syncwarp();
+                    ++pcnt[w];
+                    return true;
+                };
+                auto issue_s = [&](int w, int st) {
+                    {
+                        const uint32_t q_addr = smem_base + Lay::kQ + w * Lay::kTileBytes;
+                        const uint32_t k_addr = smem_base + Lay::kK0 + 2 * st * Lay::kTileBytes;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off = (kk / 4) * Lay::kChunkBytes + (kk % 4) * 32;
+                            mma_ss(tmem + 128 * w, sdesc_sw128(q_addr + off, 16, 1024),
+                                   sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                        }
+                        tc_commit(&sb.s_full[w]);
+                    }
+                    __syncwarp();
+                };
+                // V of the previous key tile (ring position kv_cnt - 1) before its first P V
+                auto wait_v_prev = [&]() -> bool {
+                    const uint32_t pc = kv_cnt - 1;
+                    if (!mbar_wait_warp(&sb.v_full[pc % S], (pc / S) & 1, abort)) return false;
+                    tc_fence_after();
+                    return true;
+                };
+                for (int j = jlo; j <= jhi && ok; ++j, ++kv_cnt) {
+                    const int st = kv_cnt % S;
+                    if (!mbar_wait_warp(&sb.k_full[st], (kv_cnt / S) & 1, abort) || (j > jlo && !wait_v_prev())) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    for (int w = 0; w < 2 && ok; ++w) {
+                        // the previous tile's P V of this group reads P from the S buffer: issue it first
+                        if (j - 1 >= lo[w] && j - 1 <= hi[w] && !issue_pv(w, j - 1, (kv_cnt - 1) % S)) ok = false;
+                        if (ok && j >= lo[w] && j <= hi[w]) issue_s(w, st);
+                    }
+                    if (!ok) break;
+                    {
+                        if (j == jhi) tc_commit(&sb.q_empty);
+                        tc_commit(&sb.k_empty[st]);                            // K of tile j: S products issued
+                        if (j > jlo) tc_commit(&sb.v_empty[(kv_cnt - 1) % S]); // V of tile j-1: P V issued
+                    }
+                    __syncwarp();
                 }
                 if (!ok) break;
-                if (lane == 0) {
-                    if (j == jhi) tc_commit(&sb.q_empty);
-                    if (j > jlo) tc_commit(&sb.kv_empty[(kv_cnt - 1) % S]); // tile j-1 has no reader left
-                }
+                if (!wait_v_prev()) break;
+                for (int w = 0; w < 2 && ok; ++w)
+                    if (jhi >= lo[w] && jhi <= hi[w] && !issue_pv(w, jhi, (kv_cnt - 1) % S)) ok = false;
+                if (!ok) break;
+                tc_commit(&sb.v_empty[(kv_cnt - 1) % S]);
                 __syncwarp();
+                ++icnt[0];
+                if (second) ++icnt[1];
             }
-            if (!ok) break;
-            for (int w = 0; w < 2 && ok; ++w)
-                if (jhi >= lo[w] && jhi <= hi[w] && !issue_pv(w, jhi, (kv_cnt - 1) % S)) ok = false;
-            if (!ok) break;
-            if (lane == 0) tc_commit(&sb.kv_empty[(kv_cnt - 1) % S]);
-            __syncwarp();
-            ++icnt[0];
-            if (second) ++icnt[1];
         }
     } else {
+        warpgroup_regs_inc<Lay::kRegsCompute>();
         // ----------------------------------------------------- softmax ---
         const int w = warp >> 2;              // group: query tile t + w
         const int row = threadIdx.x & 127;    // query row within the tile, TMEM lane
@@ -349,7 +363,7 @@ __global__ void __launch_bounds__(320, 1)
                 tmem_wait_st();
                 // O holds the earlier tiles' P V (complete: this S was issued after it).
                 if (j > jlo && __any_sync(0xffffffffu, grow)) {
-#pragma unroll
+#pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t orr[32];
                         tmem_ld32(o_addr + c * 32, orr);
@@ -371,7 +385,7 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_after();
             const float inv_l = valid ? 1.f / l : 0.f;
             __nv_bfloat16 *orow = out + ((int64_t(r.s0) + i) * p.heads + r.h) * D;
-#pragma unroll
+#pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t orr[32];
                 tmem_ld32(o_addr + c * 32, orr);
@@ -415,6 +429,12 @@ cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
     auto kern = fwd_bf16_sm100_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
+    // the register split only works if the CTA is launched with at least the budgets' sum
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * Lay::kThreads < int(256 * Lay::kRegsCompute + 128 * Lay::kRegsOther))
+        return cudaErrorInvalidConfiguration;
     kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, p, static_cast<__nv_bfloat16 *>(out), lse);
     return cudaGetLastError();
 }

@@ -38,7 +38,8 @@ cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, co
                                 float *delta, void *dq, int num_sms, cudaStream_t stream);
 template <int D>
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                  const CUtensorMap &tdo, const Problem &p, const float *lse, const float *delta,
-                                  void *dk, void *dv, int num_sms, cudaStream_t stream);
+                                  const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
+                                  const Problem &p, const float *lse, const float *delta, void *dk, void *dv,
+                                  int num_sms, cudaStream_t stream);
 
 } // namespace ba

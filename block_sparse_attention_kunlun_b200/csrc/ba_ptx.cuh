@@ -70,6 +70,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
+#pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
@@ -78,6 +79,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
             return false;
         }
     }
+}
+
+// mbar_wait for a warp that issues warp-collective instructions next: every
+// lane waits, and the result is made uniform so that on a timeout all lanes
+// leave together instead of some of them waiting in elect.sync.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+
+// Barrier over a group of threads, on an mbarrier initialised with the group's
+// thread count: every thread arrives, then waits (bounded) for the phase to
+// complete, so a thread that has given up cannot leave the others waiting
+// forever. `phase` is the caller's parity, flipped on each use. Arrival and
+// wait order the group's shared-memory writes before its later reads.
+__device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t &phase, volatile int *abort)
+{
+    mbar_arrive(bar);
+    const bool ok = mbar_wait(bar, phase, abort);
+    phase ^= 1;
+    return ok;
 }
 
 // ------------------------------------------------------------------ TMA ---
@@ -105,6 +127,36 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int32
 {
     asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
                  : "memory");
+}
+
+// 2-D tiled store of one box from shared memory to global memory, tracked by
+// the issuing thread's bulk async-groups. x (innermost, elements) must be a
+// multiple of 16 bytes and neither coordinate may be negative; rows past the
+// tensor's end are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t x, int32_t y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group()
+{
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Waits until at most N of this thread's bulk groups are incomplete.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group()
+{
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // Makes generic-proxy shared-memory writes visible to the async proxy
@@ -148,31 +200,41 @@ __device__ __forceinline__ void tc_fence_after()
 
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far
 // has completed.
+// Called by all 32 lanes of the issuing warp; the elected lane (the lowest
+// active one, the same lane that issues the MMAs below) commits, so the
+// barrier tracks that lane's MMAs.
 __device__ __forceinline__ void tc_commit(uint64_t *bar)
 {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(
                      smem_u32(bar))
                  : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T   (bf16 in, fp32 accumulate)
+// D[tmem] (+)= A[smem] * B[smem]^T   (bf16 in, fp32 accumulate). Called by all 32
+// lanes of one warp with the same operands; one elected lane issues. Issuing from
+// a converged warp keeps the operands in uniform registers, which makes the
+// issue several times faster than from a single-lane branch.
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accumulate)
 {
-    asm volatile("{\n\t.reg .pred p;\n\t"
+    asm volatile("{\n\t.reg .pred p, e;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
                  "setp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
                  "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
                  : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T   (A K-major in TMEM, two bf16 per column)
+// D[tmem] (+)= A[tmem] * B[smem]^T   (A K-major in TMEM, two bf16 per column).
+// Warp-collective like mma_ss.
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accumulate)
 {
-    asm volatile("{\n\t.reg .pred p;\n\t"
+    asm volatile("{\n\t.reg .pred p, e;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
                  "setp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
                  "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
                  : "memory");
 }
@@ -271,6 +333,20 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 // --------------------------------------------------------------- scalar ---
 
+// Per-warpgroup register budget (all four warps of the warpgroup execute it).
+// The budgets of a CTA's warpgroups must add up to no more than it was
+// launched with, or the increase waits for registers that never come free.
+template <uint32_t N>
+__device__ __forceinline__ void warpgroup_regs_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void warpgroup_regs_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Two fp32 lanes per instruction (sm_100 packed f32x2 arithmetic).
 union F2Bits {
     float2 f;
@@ -311,6 +387,20 @@ __device__ __forceinline__ float ex2_approx(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x on the FMA pipe for x <= 8 (values below 2^-125 come out as 2^-125 or
+// smaller, far below what a bf16 P can hold next to the row maximum). Round x
+// to the nearest integer n with the 1.5 * 2^23 trick, evaluate 2^(x-n) on
+// [-0.5, 0.5] with a cubic fitted to 2^f (relative error < 8e-5, measured on a
+// dense grid), and add n to the exponent field.
+__device__ __forceinline__ float exp2_fma(float x)
+{
+    x = fmaxf(x, -125.f);
+    const float t = x + 12582912.f;
+    const float f = x - (t - 12582912.f);
+    const float p = fmaf(fmaf(fmaf(0.055171654f, f, 0.24261115f), f, 0.69326097f), f, 0.99992806f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
