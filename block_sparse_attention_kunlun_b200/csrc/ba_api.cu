@@ -92,6 +92,8 @@ ba_status check_problem(const ba_problem *p, int32_t block, int32_t window)
     if (p->batch == 0 && p->total_tokens != 0) return BA_ERR_INVALID_ARG;
     // element offsets of one tensor must stay below 2^62 and rows below 2^31
     if (int64_t(p->heads) * p->head_dim > (int64_t(1) << 24)) return BA_ERR_UNSUPPORTED;
+    // work items (128-row tiles x heads) are numbered in 31 bits
+    if (max_tiles(p->batch, p->total_tokens) * p->heads > INT32_MAX) return BA_ERR_UNSUPPORTED;
     if (!head_dim_supported(*p)) return BA_ERR_UNSUPPORTED;
     return BA_OK;
 }
@@ -178,13 +180,13 @@ ba_status ba_fwd(const ba_problem *pp, const void *q, const void *k, const void 
         BA_TRY(prof_mark(0, 1, stream));
         return BA_OK;
     }
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!encode_bf16_rows(&tq, q, T, P.heads, P.head_dim) || !encode_bf16_rows(&tk, k, T, P.heads, P.head_dim) ||
-        !encode_bf16_rows(&tv, v, T, P.heads, P.head_dim))
+        !encode_bf16_rows(&tv, v, T, P.heads, P.head_dim) || !encode_bf16_rows(&to, out, T, P.heads, P.head_dim))
         return BA_ERR_CUDA;
     BA_TRY(prof_mark(0, 0, stream));
-    if (P.head_dim == 64) BA_TRY(launch_fwd_bf16_sm100<64>(tq, tk, tv, p, out, lse, num_sms, stream));
-    else BA_TRY(launch_fwd_bf16_sm100<128>(tq, tk, tv, p, out, lse, num_sms, stream));
+    if (P.head_dim == 64) BA_TRY(launch_fwd_bf16_sm100<64>(tq, tk, tv, to, p, out, lse, num_sms, stream));
+    else BA_TRY(launch_fwd_bf16_sm100<128>(tq, tk, tv, to, p, out, lse, num_sms, stream));
     BA_TRY(prof_mark(0, 1, stream));
     return BA_OK;
 }
@@ -213,6 +215,7 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
     const Problem p = make_problem(P, seq_offsets, skip, block, window, workspace, lay);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     float *delta = reinterpret_cast<float *>(ws + lay.delta);
+    float *nlse2 = reinterpret_cast<float *>(ws + lay.nlse2);
     BA_TRY(launch_worklist(p, stream));
     if (T == 0) return BA_OK;
     const size_t esz = bf16 ? 2 : 4;
@@ -235,15 +238,15 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
         return BA_ERR_CUDA;
     BA_TRY(prof_mark(1, 0, stream));
     if (P.head_dim == 64)
-        BA_TRY(launch_bwd_dq_sm100<64>(tq, tk, tv, tdo, to, p, lse, delta, dq, num_sms, stream));
+        BA_TRY(launch_bwd_dq_sm100<64>(tq, tk, tv, tdo, to, p, lse, delta, nlse2, dq, num_sms, stream));
     else
-        BA_TRY(launch_bwd_dq_sm100<128>(tq, tk, tv, tdo, to, p, lse, delta, dq, num_sms, stream));
+        BA_TRY(launch_bwd_dq_sm100<128>(tq, tk, tv, tdo, to, p, lse, delta, nlse2, dq, num_sms, stream));
     BA_TRY(prof_mark(1, 1, stream));
     BA_TRY(prof_mark(2, 0, stream));
     if (P.head_dim == 64)
-        BA_TRY(launch_bwd_dkdv_sm100<64>(tq, tk, tv, tdo, tdk, tdv, p, lse, delta, dk, dv, num_sms, stream));
+        BA_TRY(launch_bwd_dkdv_sm100<64>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, delta, dk, dv, num_sms, stream));
     else
-        BA_TRY(launch_bwd_dkdv_sm100<128>(tq, tk, tv, tdo, tdk, tdv, p, lse, delta, dk, dv, num_sms, stream));
+        BA_TRY(launch_bwd_dkdv_sm100<128>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, delta, dk, dv, num_sms, stream));
     BA_TRY(prof_mark(2, 1, stream));
     return BA_OK;
 }

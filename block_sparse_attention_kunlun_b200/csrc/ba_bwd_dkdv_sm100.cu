@@ -55,8 +55,11 @@ struct DkvLayout {
     static constexpr int kChunks = D / 64;
     static constexpr int kChunkBytes = kTile * 128;
     static constexpr int kTileBytes = kTile * D * 2;
-    static constexpr int kQSlots = D == 64 ? 4 : 2;      // Q ring
-    static constexpr int kOSlots = D == 64 ? 4 : 2;      // dO ring
+    // Q ring and dO ring. Q(m) is read until dK(m), late in tile m's step, and
+    // S^T(m+1) needs Q(m+1): three Q slots keep its load well ahead. dO(m) is free
+    // after dV(m), early in the step, so at D = 128 one dO slot is enough.
+    static constexpr int kQSlots = D == 64 ? 4 : 3;
+    static constexpr int kOSlots = D == 64 ? 4 : 1;
     static constexpr int kK = 0;
     static constexpr int kV = kTileBytes;
     static constexpr int kQ0 = 2 * kTileBytes;           // Q slot s at kQ0 + s tile
@@ -73,11 +76,12 @@ struct DkvBarriers {
     uint64_t kv_full, kv_empty, dkv_full, dkv_free;
     uint64_t q_full[4], q_empty[4], o_full[4], o_empty[4];
     uint64_t s_full, dp_full, pa_done[2], pb_done[2];
-    uint64_t cmp_sync, epi_sync; // group barriers of the compute and epilogue warps
+    uint64_t epi_sync; // group barrier of the epilogue warps
     uint32_t tmem_base;
     int abort;
-    __align__(16) float lse2[2][kTile];
-    __align__(16) float delta[2][kTile];
+    // per Q slot: -lse in log2 units and -Delta of the tile's 128 queries
+    // (-inf and 0 past the example's end), filled with the Q tile
+    __align__(16) float stat[4][2][kTile];
 };
 
 __device__ __forceinline__ void query_tile_range(const TileRef &r, int64_t B, int64_t W, int &ilo, int &ihi)
@@ -94,7 +98,7 @@ __global__ void __launch_bounds__(448, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                           const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-                          const Problem p, const float *__restrict__ lse, const float *__restrict__ delta,
+                          const Problem p, const float *__restrict__ nlse2, const float *__restrict__ neg_delta,
                           __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv)
 {
     using Lay = DkvLayout<D>;
@@ -112,14 +116,13 @@ __global__ void __launch_bounds__(448, 1)
         mbar_init(&sb.dkv_full, 1);
         mbar_init(&sb.dkv_free, 4);
         for (int i = 0; i < 4; ++i) {
-            mbar_init(&sb.q_full[i], 1);
+            mbar_init(&sb.q_full[i], 1 + 32); // the Q tile's expect_tx arrival + one per lane's copies
             mbar_init(&sb.q_empty[i], 1);
             mbar_init(&sb.o_full[i], 1);
             mbar_init(&sb.o_empty[i], 1);
         }
         mbar_init(&sb.s_full, 1);
         mbar_init(&sb.dp_full, 1);
-        mbar_init(&sb.cmp_sync, 256);
         mbar_init(&sb.epi_sync, 128);
         for (int g = 0; g < 2; ++g) {
             mbar_init(&sb.pa_done[g], 4);
@@ -152,7 +155,8 @@ __global__ void __launch_bounds__(448, 1)
         uint32_t it = 0, item_cnt = 0;
         TileRef r;
         bool ok = true;
-        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
+        ItemWalker items(p.tile_info, ntiles, p.heads);
+        for (; ok && items.advance(r); ++item_cnt) {
             int ilo, ihi;
             query_tile_range(r, B, W, ilo, ihi);
             if (!mbar_wait(&sb.kv_empty, (item_cnt & 1) ^ 1, abort)) break;
@@ -166,7 +170,7 @@ __global__ void __launch_bounds__(448, 1)
                 }
                 // warm L2 with the next item's K and V
                 TileRef rn;
-                if (decode_item(p, ntiles, n + gridDim.x, rn)) {
+                if (items.peek(rn)) {
                     int nlo, nhi;
                     query_tile_range(rn, B, W, nlo, nhi);
                     for (int c = 0; c < Lay::kChunks; ++c) {
@@ -192,6 +196,18 @@ __global__ void __launch_bounds__(448, 1)
                         tma_load_2d(smem + Lay::kQ0 + qs * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_q,
                                     &sb.q_full[qs], r.h * D + c * 64, r.s0 + i * kTile);
                 }
+                // the tile's -lse (log2 units) and -Delta, four queries per lane, copied
+                // asynchronously; each lane's copies arrive on q_full when they land. Rows past
+                // the example's end copy its last row (those queries are masked out).
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int qr = 4 * lane + e;
+                    const int64_t q = int64_t(i) * kTile + qr;
+                    const int64_t gi = int64_t(r.h) * T + r.s0 + (q < r.L ? q : r.L - 1);
+                    cp_async_4(&sb.stat[qs][0][qr], nlse2 + gi);
+                    cp_async_4(&sb.stat[qs][1][qr], neg_delta + gi);
+                }
+                cp_async_arrive_noinc(&sb.q_full[qs]);
                 __syncwarp();
                 if (!mbar_wait(&sb.o_empty[os], ((it / OS) & 1) ^ 1, abort)) {
                     ok = false;
@@ -220,16 +236,17 @@ __global__ void __launch_bounds__(448, 1)
         TileRef r;
         bool ok = true;
         const uint32_t k_addr = smem_base + Lay::kK, v_addr = smem_base + Lay::kV;
-        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
+        ItemWalker items(p.tile_info, ntiles, p.heads);
+        for (; ok && items.advance(r); ++item_cnt) {
             int ilo, ihi;
             query_tile_range(r, B, W, ilo, ihi);
             const int nq = ihi - ilo + 1;
-            if (!mbar_wait_warp(&sb.kv_full, item_cnt & 1, abort)) break;
+            if (!mbar_wait(&sb.kv_full, item_cnt & 1, abort)) break;
             tc_fence_after();
             // S^T = K Q^T of query tile m of this item
             auto issue_s = [&](int m) -> bool {
                 const uint32_t it = it0 + m, qs = it % QS;
-                if (!mbar_wait_warp(&sb.q_full[qs], (it / QS) & 1, abort)) return false;
+                if (!mbar_wait(&sb.q_full[qs], (it / QS) & 1, abort)) return false;
                 tc_fence_after();
                 {
                     const uint32_t q_addr = smem_base + Lay::kQ0 + qs * Lay::kTileBytes;
@@ -247,7 +264,7 @@ __global__ void __launch_bounds__(448, 1)
             // dP^T = V dO^T of query tile m; after the item's last one K and V are not read again
             auto issue_dp = [&](int m) -> bool {
                 const uint32_t it = it0 + m, os = it % OS;
-                if (!mbar_wait_warp(&sb.o_full[os], (it / OS) & 1, abort)) return false;
+                if (!mbar_wait(&sb.o_full[os], (it / OS) & 1, abort)) return false;
                 tc_fence_after();
                 {
                     const uint32_t o_addr = smem_base + Lay::kO0 + os * Lay::kTileBytes;
@@ -271,8 +288,8 @@ __global__ void __launch_bounds__(448, 1)
                 const uint32_t b_addr = smem_base + (phase == 0 ? Lay::kO0 + slot * Lay::kTileBytes
                                                                 : Lay::kQ0 + slot * Lay::kTileBytes);
                 for (int g = 0; g < 2; ++g) {
-                    if (!mbar_wait_warp(phase == 0 ? &sb.pa_done[g] : &sb.pb_done[g], it & 1, abort)) return false;
-                    if (phase == 0 && m == 0 && g == 0 && !mbar_wait_warp(&sb.dkv_free, (item_cnt & 1) ^ 1, abort))
+                    if (!mbar_wait(phase == 0 ? &sb.pa_done[g] : &sb.pb_done[g], it & 1, abort)) return false;
+                    if (phase == 0 && m == 0 && g == 0 && !mbar_wait(&sb.dkv_free, (item_cnt & 1) ^ 1, abort))
                         return false;
                     tc_fence_after();
                     {
@@ -305,37 +322,29 @@ __global__ void __launch_bounds__(448, 1)
         const int row = threadIdx.x & 127;    // key row within the tile, TMEM lane
         const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
         const float scale_log2 = p.scale * 1.4426950408889634f;
-        uint32_t it = 0, sync_phase = 0;
+        uint32_t it = 0;
         TileRef r;
         bool ok = true;
-        // -lse (log2 units, group 0) or -Delta (group 1) of query row `row` of tile i
-        auto load_row = [&](const TileRef &rr, int i) -> float {
-            const int64_t q = int64_t(i) * kTile + row;
-            if (q >= rr.L) return g == 0 ? -INFINITY : 0.f;
-            const int64_t gi = int64_t(rr.h) * T + rr.s0 + q;
-            return g == 0 ? -lse[gi] * 1.4426950408889634f : -delta[gi];
-        };
-        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x) {
+        ItemWalker items(p.tile_info, ntiles, p.heads);
+        while (ok && items.advance(r)) {
             int ilo, ihi;
             query_tile_range(r, B, W, ilo, ihi);
             const int64_t k = int64_t(r.t) * kTile + row; // local key index
             const bool valid_k = k < r.L;
             const int64_t qmax = valid_k ? last_query_seeing(k, r.L, B, W) : -1;
-            float nxt = load_row(r, ilo);
             for (int i = ilo; i <= ihi && ok; ++i, ++it) {
-                const int buf = it & 1;
-                (g == 0 ? sb.lse2[buf] : sb.delta[buf])[row] = nxt;
-                if (!group_sync(&sb.cmp_sync, sync_phase, abort)) { ok = false; break; }
-                if (i < ihi) nxt = load_row(r, i + 1);
+                const int qs = it % QS;
                 const int64_t q0 = int64_t(i) * kTile + 64 * g;
                 int64_t lo64 = k - q0, hi64 = qmax - q0;
                 if (!valid_k) { lo64 = 1; hi64 = 0; }
                 const int lo_c = int(lo64 < -1 ? -1 : (lo64 > 64 ? 64 : lo64));
                 const int hi_c = int(hi64 < -1 ? -1 : (hi64 > 64 ? 64 : hi64));
                 const bool full = __all_sync(0xffffffffu, lo_c <= 0 && hi_c >= 63);
-                // shared copies hold -lse (log2 units) and -Delta, so each use is one packed FMA/add
-                const float4 *l2v = reinterpret_cast<const float4 *>(sb.lse2[buf] + 64 * g);
-                const float2 *dlv2 = reinterpret_cast<const float2 *>(sb.delta[buf] + 64 * g);
+                // -lse (log2 units) and -Delta of this group's queries, staged with the Q tile
+                // (complete once S^T is: the S^T product waited for the same barrier phase)
+                if (!mbar_wait(&sb.q_full[qs], (it / QS) & 1, abort)) { ok = false; break; }
+                const float4 *l2v = reinterpret_cast<const float4 *>(sb.stat[qs][0] + 64 * g);
+                const float2 *dlv2 = reinterpret_cast<const float2 *>(sb.stat[qs][1] + 64 * g);
                 // phase A: P^T from S^T, written (bf16) over the group's first 32 S^T columns
                 if (!mbar_wait(&sb.s_full, it & 1, abort)) { ok = false; break; }
                 tc_fence_after();
@@ -419,7 +428,8 @@ __global__ void __launch_bounds__(448, 1)
         uint32_t item_cnt = 0, sync_phase = 0;
         bool ok = true;
         TileRef r;
-        for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
+        ItemWalker items(p.tile_info, ntiles, p.heads);
+        for (; ok && items.advance(r); ++item_cnt) {
             const int64_t k = int64_t(r.t) * kTile + row;
             const bool valid_k = k < r.L;
             const bool full_tile = int64_t(r.t) * kTile + kTile <= r.L;
@@ -482,14 +492,14 @@ __global__ void __launch_bounds__(448, 1)
 template <int D>
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
-                                  const Problem &p, const float *lse, const float *delta, void *dk, void *dv,
+                                  const Problem &p, const float *nlse2, const float *neg_delta, void *dk, void *dv,
                                   int num_sms, cudaStream_t stream)
 {
     using Lay = DkvLayout<D>;
     auto kern = bwd_dkdv_sm100_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, tdk, tdv, p, lse, delta,
+    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, neg_delta,
                                                           static_cast<__nv_bfloat16 *>(dk),
                                                           static_cast<__nv_bfloat16 *>(dv));
     return cudaGetLastError();

@@ -60,7 +60,7 @@ struct DqLayout {
 };
 
 struct DqBarriers {
-    uint64_t kv_full[3], kv_empty[3];
+    uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
     uint64_t st_full, st_empty, qt_ready;
     uint64_t s_full, s_free, dp_full, ds_full[2], dq_done, dq_free;
     uint32_t tmem_base;
@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(384, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_o, const Problem p, const float *__restrict__ lse,
-                        float *__restrict__ delta, __nv_bfloat16 *__restrict__ dq)
+                        float *__restrict__ neg_delta, float *__restrict__ nlse2, __nv_bfloat16 *__restrict__ dq)
 {
     using Lay = DqLayout<D>;
     constexpr int S = Lay::kStages;
@@ -93,8 +93,10 @@ __global__ void __launch_bounds__(384, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
-            mbar_init(&sb.kv_full[i], 1);
-            mbar_init(&sb.kv_empty[i], 1);
+            mbar_init(&sb.k_full[i], 1);
+            mbar_init(&sb.k_empty[i], 1);
+            mbar_init(&sb.v_full[i], 1);
+            mbar_init(&sb.v_empty[i], 1);
         }
         mbar_init(&sb.st_full, 1);
         mbar_init(&sb.st_empty, 8);
@@ -137,7 +139,8 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t kv_cnt = 0, item_cnt = 0;
             TileRef r;
             bool ok = true;
-            for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
+            ItemWalker items(p.tile_info, ntiles, p.heads);
+            for (; ok && items.advance(r); ++item_cnt) {
                 const int jlo = first_key_tile(r, B, W);
                 if (!mbar_wait(&sb.st_empty, (item_cnt & 1) ^ 1, abort)) break;
                 if (lane == 0) {
@@ -153,19 +156,28 @@ __global__ void __launch_bounds__(384, 1)
                 __syncwarp();
                 for (int j = jlo; j <= r.t; ++j, ++kv_cnt) {
                     const int st = kv_cnt % S;
-                    if (!mbar_wait(&sb.kv_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
+                    uint8_t *kdst = smem + Lay::kKV0 + 2 * st * Lay::kTileBytes;
+                    // K is read until dQ, V only by dP: they are released and refilled separately
+                    if (!mbar_wait(&sb.k_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
                         ok = false;
                         break;
                     }
                     if (lane == 0) {
-                        uint8_t *kdst = smem + Lay::kKV0 + 2 * st * Lay::kTileBytes;
-                        mbar_arrive_expect_tx(&sb.kv_full[st], 2 * Lay::kTileBytes);
-                        for (int c = 0; c < Lay::kChunks; ++c) {
-                            tma_load_2d(kdst + c * Lay::kChunkBytes, &tm_k, &sb.kv_full[st], r.h * D + c * 64,
+                        mbar_arrive_expect_tx(&sb.k_full[st], Lay::kTileBytes);
+                        for (int c = 0; c < Lay::kChunks; ++c)
+                            tma_load_2d(kdst + c * Lay::kChunkBytes, &tm_k, &sb.k_full[st], r.h * D + c * 64,
                                         r.s0 + j * kTile);
-                            tma_load_2d(kdst + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_v, &sb.kv_full[st],
+                    }
+                    __syncwarp();
+                    if (!mbar_wait(&sb.v_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&sb.v_full[st], Lay::kTileBytes);
+                        for (int c = 0; c < Lay::kChunks; ++c)
+                            tma_load_2d(kdst + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_v, &sb.v_full[st],
                                         r.h * D + c * 64, r.s0 + j * kTile);
-                        }
                     }
                     __syncwarp();
                 }
@@ -179,8 +191,8 @@ __global__ void __launch_bounds__(384, 1)
             bool ok = true;
             // dQ += dS K for the key tile in ring stage `st` (m = its index in the item)
             auto issue_dq = [&](int m, int st) -> bool {
-                if (!mbar_wait_warp(&sb.ds_full[0], d_cnt & 1, abort)) return false;
-                if (m == 0 && !mbar_wait_warp(&sb.dq_free, (item_cnt & 1) ^ 1, abort)) return false;
+                if (!mbar_wait(&sb.ds_full[0], d_cnt & 1, abort)) return false;
+                if (m == 0 && !mbar_wait(&sb.dq_free, (item_cnt & 1) ^ 1, abort)) return false;
                 tc_fence_after();
                 const uint32_t k_addr = smem_base + Lay::kKV0 + 2 * st * Lay::kTileBytes;
                 {
@@ -191,28 +203,29 @@ __global__ void __launch_bounds__(384, 1)
                                (m > 0 || kk > 0) ? 1u : 0u);
                 }
                 __syncwarp();
-                if (!mbar_wait_warp(&sb.ds_full[1], d_cnt & 1, abort)) return false;
+                if (!mbar_wait(&sb.ds_full[1], d_cnt & 1, abort)) return false;
                 tc_fence_after();
                 {
 #pragma unroll
                     for (int kk = 4; kk < 8; ++kk)
                         mma_ts(tmem + Lay::kColDQ, tmem + Lay::kColDP + 64 + (kk - 4) * 8,
                                sdesc_sw128(k_addr + kk * 2048, Lay::kChunkBytes, 1024), idesc_q, 1u);
-                    tc_commit(&sb.kv_empty[st]);
+                    tc_commit(&sb.k_empty[st]);
                 }
                 __syncwarp();
                 ++d_cnt;
                 return true;
             };
-            for (int64_t n = blockIdx.x; ok && decode_item(p, ntiles, n, r); n += gridDim.x, ++item_cnt) {
+            ItemWalker items(p.tile_info, ntiles, p.heads);
+            for (; ok && items.advance(r); ++item_cnt) {
                 const int jlo = first_key_tile(r, B, W);
                 const int nkv = r.t - jlo + 1;
-                if (!mbar_wait_warp(&sb.qt_ready, item_cnt & 1, abort)) break;
+                if (!mbar_wait(&sb.qt_ready, item_cnt & 1, abort)) break;
                 tc_fence_after();
                 for (int m = 0; m < nkv; ++m, ++kv_cnt, ++s_cnt) {
                     const int st = kv_cnt % S;
-                    if (!mbar_wait_warp(&sb.kv_full[st], (kv_cnt / S) & 1, abort) ||
-                        !mbar_wait_warp(&sb.s_free, (s_cnt & 1) ^ 1, abort)) {
+                    if (!mbar_wait(&sb.k_full[st], (kv_cnt / S) & 1, abort) ||
+                        !mbar_wait(&sb.s_free, (s_cnt & 1) ^ 1, abort)) {
                         ok = false;
                         break;
                     }
@@ -234,6 +247,11 @@ __global__ void __launch_bounds__(384, 1)
                         ok = false;
                         break;
                     }
+                    if (!mbar_wait(&sb.v_full[st], (kv_cnt / S) & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
                     {
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk)
@@ -241,6 +259,7 @@ __global__ void __launch_bounds__(384, 1)
                                    sdesc_sw128(v_addr + (kk / 4) * Lay::kChunkBytes + (kk % 4) * 32, 16, 1024),
                                    idesc_s, kk > 0 ? 1u : 0u);
                         tc_commit(&sb.dp_full);
+                        tc_commit(&sb.v_empty[st]); // V of this tile has no other reader
                     }
                     __syncwarp();
                 }
@@ -263,7 +282,7 @@ __global__ void __launch_bounds__(384, 1)
 
         // Copy this item's Q (group 0) or dO (group 1) row into TMEM and
         // compute Delta from the staged dO and out rows.
-        auto fill = [&](const TileRef &rr, uint32_t cnt, float &delta_row) -> bool {
+        auto fill = [&](const TileRef &rr, uint32_t cnt, float &delta_row, float lse_val) -> bool {
             if (!mbar_wait(&sb.st_full, cnt & 1, abort)) return false;
             const uint8_t *qsrc = staging;
             const uint8_t *dsrc = staging + Lay::kTileBytes;
@@ -308,22 +327,32 @@ __global__ void __launch_bounds__(384, 1)
             }
             delta_row = dl;
             const int64_t i = int64_t(rr.t) * kTile + row;
-            if (g == 0 && i < rr.L) delta[int64_t(rr.h) * T + rr.s0 + i] = dl;
+            // for the dK/dV pass: -Delta (group 0) and -lse in log2 units (group 1)
+            if (i < rr.L) {
+                if (g == 0) neg_delta[int64_t(rr.h) * T + rr.s0 + i] = -dl;
+                else nlse2[int64_t(rr.h) * T + rr.s0 + i] = -lse_val * 1.4426950408889634f;
+            }
             return true;
         };
 
         TileRef r;
-        int64_t n = blockIdx.x;
-        bool have = decode_item(p, ntiles, n, r);
+        ItemWalker items(p.tile_info, ntiles, p.heads);
+        bool have = items.advance(r);
         float delta_row = 0.f;
-        if (have) ok = fill(r, 0, delta_row);
+        // lse of this thread's query row (log2 units), loaded an item ahead
+        auto load_l2 = [&](const TileRef &rr) -> float {
+            const int64_t q = int64_t(rr.t) * kTile + row;
+            return q < rr.L ? lse[int64_t(rr.h) * T + rr.s0 + q] : INFINITY;
+        };
+        float lse_row = have ? load_l2(r) : 0.f;
+        if (have) ok = fill(r, 0, delta_row, lse_row);
         while (have && ok) {
             const int jlo = first_key_tile(r, B, W);
             const int nkv = r.t - jlo + 1;
             const int64_t i = int64_t(r.t) * kTile + row;
             const bool valid = i < r.L;
             const int64_t ws = window_start(i, B, W);
-            const float l2 = valid ? lse[int64_t(r.h) * T + r.s0 + i] * 1.4426950408889634f : INFINITY;
+            const float l2 = lse_row * 1.4426950408889634f;
             const float dl = delta_row;
             for (int m = 0; m < nkv; ++m, ++s_cnt) {
                 const int64_t key0 = int64_t(jlo + m) * kTile + 64 * g;
@@ -401,9 +430,10 @@ __global__ void __launch_bounds__(384, 1)
             if (!ok) break;
             // the next item's Q / dO go into TMEM now: this item's last S and dP have completed
             TileRef rn;
-            const bool have_next = decode_item(p, ntiles, n + gridDim.x, rn);
+            const bool have_next = items.advance(rn);
             float delta_next = 0.f;
-            if (have_next && !fill(rn, item_cnt + 1, delta_next)) break;
+            const float lse_next = have_next ? load_l2(rn) : 0.f;
+            if (have_next && !fill(rn, item_cnt + 1, delta_next, lse_next)) break;
             // epilogue: dq of this item
             if (!mbar_wait(&sb.dq_done, item_cnt & 1, abort)) break;
             tc_fence_after();
@@ -431,10 +461,10 @@ __global__ void __launch_bounds__(384, 1)
                 if (lane == 0) mbar_arrive(&sb.dq_free);
             }
             ++item_cnt;
-            n += gridDim.x;
             r = rn;
             have = have_next;
             delta_row = delta_next;
+            lse_row = lse_next;
         }
     }
 
@@ -448,7 +478,7 @@ __global__ void __launch_bounds__(384, 1)
 template <int D>
 cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const CUtensorMap &tdo, const CUtensorMap &to, const Problem &p, const float *lse,
-                                float *delta, void *dq, int num_sms, cudaStream_t stream)
+                                float *neg_delta, float *nlse2, void *dq, int num_sms, cudaStream_t stream)
 {
     using Lay = DqLayout<D>;
     auto kern = bwd_dq_sm100_kernel<D>;
@@ -460,16 +490,16 @@ cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, co
     if (e != cudaSuccess) return e;
     if (fa.numRegs * Lay::kThreads < int(256 * Lay::kRegsCompute + 128 * Lay::kRegsOther))
         return cudaErrorInvalidConfiguration;
-    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, to, p, lse, delta,
+    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, to, p, lse, neg_delta, nlse2,
                                                           static_cast<__nv_bfloat16 *>(dq));
     return cudaGetLastError();
 }
 
 template cudaError_t launch_bwd_dq_sm100<64>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
                                              const CUtensorMap &, const CUtensorMap &, const Problem &, const float *,
-                                             float *, void *, int, cudaStream_t);
+                                             float *, float *, void *, int, cudaStream_t);
 template cudaError_t launch_bwd_dq_sm100<128>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
                                               const CUtensorMap &, const CUtensorMap &, const Problem &, const float *,
-                                              float *, void *, int, cudaStream_t);
+                                              float *, float *, void *, int, cudaStream_t);
 
 } // namespace ba

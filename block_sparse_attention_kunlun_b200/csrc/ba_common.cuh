@@ -55,7 +55,7 @@ __host__ __device__ __forceinline__ bool visible(int64_t i, int64_t j, int64_t b
 //   delta   (bwd only)  float[heads * total_tokens]
 //   dq_acc  (bwd only)  float[heads * total_tokens * head_dim]
 struct WorkspaceLayout {
-    size_t status, tile_prefix, tile_info, pair_prefix, pair_info, delta, dq_acc, total;
+    size_t status, tile_prefix, tile_info, pair_prefix, pair_info, delta, nlse2, dq_acc, total;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -84,7 +84,10 @@ __host__ __device__ inline WorkspaceLayout workspace_layout(int64_t batch, int64
     off = align256(off + sizeof(int32_t) * size_t(batch + 1));
     w.pair_info = off;
     off = align256(off + 16 * size_t(max_pairs(batch, total_tokens)));
+    // backward only: per-row Delta, and (bf16 path) -lse in log2 units, both [heads, total_tokens]
     w.delta = off;
+    if (with_delta) off = align256(off + sizeof(float) * size_t(heads * total_tokens));
+    w.nlse2 = off;
     if (with_delta) off = align256(off + sizeof(float) * size_t(heads * total_tokens));
     w.dq_acc = off;
     if (with_dq_acc) off = align256(off + sizeof(float) * size_t(heads * total_tokens * head_dim));
@@ -145,5 +148,42 @@ __device__ __forceinline__ bool decode_pair(const Problem &p, int32_t npairs, in
     second = int64_t(r.t + 1) * kTile < r.L;
     return true;
 }
+
+// Walks one CTA's work items n = blockIdx.x, blockIdx.x + gridDim.x, ...
+// (item n is entry n / heads of a tile or pair table, head n % heads; the
+// host checks that entries * heads fits in 31 bits). Each item's table entry
+// is loaded one item ahead, so its global-memory latency overlaps the
+// previous item's work, and the index arithmetic is 32-bit.
+struct ItemWalker {
+    const int4 *table;
+    uint32_t total, heads, n;
+    int4 next;
+    __device__ __forceinline__ ItemWalker(const int4 *t, int32_t entries, int32_t h)
+        : table(t), total(uint32_t(entries) * uint32_t(h)), heads(uint32_t(h)), n(blockIdx.x), next()
+    {
+        if (n < total) next = table[n / heads];
+    }
+    // The next item into r; false once the CTA's items are done.
+    __device__ __forceinline__ bool advance(TileRef &r)
+    {
+        if (!peek(r)) return false;
+        n += gridDim.x;
+        if (n < total) next = table[n / heads];
+        return true;
+    }
+    // The item advance() would return next, without moving on.
+    __device__ __forceinline__ bool peek(TileRef &r) const
+    {
+        if (n >= total) return false;
+        r.h = int32_t(n % heads);
+        r.s0 = next.x;
+        r.L = next.y;
+        r.t = next.z;
+        return true;
+    }
+};
+
+// Whether a pair item (first tile r.t) has its second tile.
+__device__ __forceinline__ bool pair_has_second(const TileRef &r) { return int64_t(r.t + 1) * kTile < r.L; }
 
 } // namespace ba

@@ -47,11 +47,13 @@ struct FwdLayout {
     static constexpr int kTileBytes = kTile * D * 2;     // one 128 x D bf16 tile
     static constexpr int kQ = 0;                         // Q tile of group w at kQ + w tile
     static constexpr int kK0 = 2 * kTileBytes;           // stage s: K at kK0 + 2 s tile, V after it
-    static constexpr int kBytes = kTileBytes * (2 + 2 * kStages);
+    static constexpr int kStage = kTileBytes * (2 + 2 * kStages); // epilogue staging of group w at
+                                                                  // kStage + w chunk (128 x 64 bf16)
+    static constexpr int kBytes = kStage + 2 * kChunkBytes;
     static constexpr int kAlloc = kBytes + 1024;         // slack to align the base to 1024 B
     static constexpr int kThreads = 384;                 // three warpgroups
-    // register budgets after the split; 2 * 128 * 200 + 128 * 104 = 384 * 168
-    static constexpr uint32_t kRegsCompute = 200, kRegsOther = 104;
+    // register budgets after the split; 2 * 128 * 192 + 128 * 120 = 384 * 168
+    static constexpr uint32_t kRegsCompute = 192, kRegsOther = 120;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColO = 256;
 };
@@ -60,6 +62,7 @@ struct FwdBarriers {
     uint64_t q_full, q_empty;
     uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
     uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+    uint64_t o_sync[2]; // group barrier of each softmax warpgroup (epilogue staging)
     uint32_t tmem_base;
     int abort;
 };
@@ -75,7 +78,8 @@ __device__ __forceinline__ int first_key_tile(int t, int64_t B, int64_t W)
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, const Problem p,
+                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                          const Problem p,
                           __nv_bfloat16 *__restrict__ out, float *__restrict__ lse)
 {
     using Lay = FwdLayout<D>;
@@ -95,6 +99,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&sb.p_full[w], 4);
             mbar_init(&sb.o_final[w], 1);
             mbar_init(&sb.o_free[w], 4);
+            mbar_init(&sb.o_sync[w], 128);
         }
         for (int i = 0; i < S; ++i) {
             mbar_init(&sb.k_full[i], 1);
@@ -131,7 +136,9 @@ __global__ void __launch_bounds__(384, 1)
             TileRef r;
             bool second;
             bool ok = true;
-            for (int64_t n = blockIdx.x; ok && decode_pair(p, npairs, n, r, second); n += gridDim.x, ++item_cnt) {
+            ItemWalker items(p.pair_info, npairs, p.heads);
+            for (; ok && items.advance(r); ++item_cnt) {
+                second = pair_has_second(r);
                 const int jlo = first_key_tile(r.t, B, W);
                 const int jhi = r.t + (second ? 1 : 0);
                 if (!mbar_wait(&sb.q_empty, (item_cnt & 1) ^ 1, abort)) break;
@@ -143,11 +150,12 @@ __global__ void __launch_bounds__(384, 1)
                                         r.h * D + c * 64, r.s0 + (r.t + w) * kTile);
                     // warm L2 with the next item's query tiles
                     TileRef rn;
-                    bool sn;
-                    if (decode_pair(p, npairs, n + gridDim.x, rn, sn))
+                    if (items.peek(rn)) {
+                        const bool sn = pair_has_second(rn);
                         for (int w = 0; w < (sn ? 2 : 1); ++w)
                             for (int c = 0; c < Lay::kChunks; ++c)
                                 tma_prefetch_l2_2d(&tm_q, rn.h * D + c * 64, rn.s0 + (rn.t + w) * kTile);
+                    }
                 }
                 __syncwarp();
                 for (int j = jlo; j <= jhi; ++j, ++kv_cnt) {
@@ -189,17 +197,19 @@ __global__ void __launch_bounds__(384, 1)
             TileRef r;
             bool second;
             bool ok = true;
-            for (int64_t n = blockIdx.x; ok && decode_pair(p, npairs, n, r, second); n += gridDim.x, ++item_cnt) {
+            ItemWalker items(p.pair_info, npairs, p.heads);
+            for (; ok && items.advance(r); ++item_cnt) {
+                second = pair_has_second(r);
                 const int lo[2] = {first_key_tile(r.t, B, W), second ? first_key_tile(r.t + 1, B, W) : 1};
                 const int hi[2] = {r.t, second ? r.t + 1 : 0};
                 const int jlo = lo[0], jhi = second ? hi[1] : hi[0];
-                if (!mbar_wait_warp(&sb.q_full, item_cnt & 1, abort)) break;
+                if (!mbar_wait(&sb.q_full, item_cnt & 1, abort)) break;
                 tc_fence_after();
                 // O_w += P_w V for key tile j of group w (V from ring stage st)
                 auto issue_pv = [&](int w, int j, int st) -> bool {
-                    if (!mbar_wait_warp(&sb.p_full[w], pcnt[w] & 1, abort)) return false;
+                    if (!mbar_wait(&sb.p_full[w], pcnt[w] & 1, abort)) return false;
                     const bool first = (j == lo[w]);
-                    if (first && !mbar_wait_warp(&sb.o_free[w], (icnt[w] & 1) ^ 1, abort)) return false;
+                    if (first && !mbar_wait(&sb.o_free[w], (icnt[w] & 1) ^ 1, abort)) return false;
                     tc_fence_after();
                     {
                         const uint32_t v_addr = smem_base + Lay::kK0 + (2 * st + 1) * Lay::kTileBytes;
@@ -231,13 +241,13 @@ __global__ void __launch_bounds__(384, 1)
                 // V of the previous key tile (ring position kv_cnt - 1) before its first P V
                 auto wait_v_prev = [&]() -> bool {
                     const uint32_t pc = kv_cnt - 1;
-                    if (!mbar_wait_warp(&sb.v_full[pc % S], (pc / S) & 1, abort)) return false;
+                    if (!mbar_wait(&sb.v_full[pc % S], (pc / S) & 1, abort)) return false;
                     tc_fence_after();
                     return true;
                 };
                 for (int j = jlo; j <= jhi && ok; ++j, ++kv_cnt) {
                     const int st = kv_cnt % S;
-                    if (!mbar_wait_warp(&sb.k_full[st], (kv_cnt / S) & 1, abort) || (j > jlo && !wait_v_prev())) {
+                    if (!mbar_wait(&sb.k_full[st], (kv_cnt / S) & 1, abort) || (j > jlo && !wait_v_prev())) {
                         ok = false;
                         break;
                     }
@@ -276,10 +286,15 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t o_addr = tmem + lane_base + Lay::kColO + D * w;
         const float scale_log2 = p.scale * 1.4426950408889634f;
         uint32_t cnt = 0, my_items = 0; // tiles and items this group has processed
+        uint32_t sync_phase = 0;
+        const bool leader = row == 0;
+        uint8_t *stage = smem + Lay::kStage + w * Lay::kChunkBytes;
         TileRef r;
         bool second;
         bool ok = true;
-        for (int64_t n = blockIdx.x; ok && decode_pair(p, npairs, n, r, second); n += gridDim.x) {
+        ItemWalker items(p.pair_info, npairs, p.heads);
+        while (ok && items.advance(r)) {
+            second = pair_has_second(r);
             if (w == 1 && !second) continue;
             const int t = r.t + w;
             const int jlo = first_key_tile(t, B, W);
@@ -380,38 +395,58 @@ __global__ void __launch_bounds__(384, 1)
                 if (lane == 0) mbar_arrive(&sb.p_full[w]);
             }
             if (!ok) break;
-            // epilogue: wait for this group's last P V, normalise, store
+            // epilogue: wait for this group's last P V, normalise, store. A tile whose
+            // rows all belong to the example leaves through this group's staging
+            // buffer and TMA stores (whole lines); the example's last tile row by row.
             if (!mbar_wait(&sb.o_final[w], my_items & 1, abort)) break;
             tc_fence_after();
             const float inv_l = valid ? 1.f / l : 0.f;
+            const bool full_tile = int64_t(t) * kTile + kTile <= r.L;
             __nv_bfloat16 *orow = out + ((int64_t(r.s0) + i) * p.heads + r.h) * D;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t orr[32];
-                tmem_ld32(o_addr + c * 32, orr);
+            for (int c = 0; c < D / 64; ++c) {
+                uint32_t orr[2][32];
+                tmem_ld32(o_addr + 64 * c, orr[0]);
+                tmem_ld32(o_addr + 64 * c + 32, orr[1]);
                 tmem_wait_ld();
-                reg_fence(orr);
-                if (valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+                reg_fence(orr[0]);
+                reg_fence(orr[1]);
+                if (c == D / 64 - 1) { // all of O read: the next item's P V may overwrite it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sb.o_free[w]);
+                }
+                uint32_t pk[32];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        dst[k] = make_uint4(pack_bf16x2(__uint_as_float(orr[8 * k + 0]) * inv_l,
-                                                        __uint_as_float(orr[8 * k + 1]) * inv_l),
-                                            pack_bf16x2(__uint_as_float(orr[8 * k + 2]) * inv_l,
-                                                        __uint_as_float(orr[8 * k + 3]) * inv_l),
-                                            pack_bf16x2(__uint_as_float(orr[8 * k + 4]) * inv_l,
-                                                        __uint_as_float(orr[8 * k + 5]) * inv_l),
-                                            pack_bf16x2(__uint_as_float(orr[8 * k + 6]) * inv_l,
-                                                        __uint_as_float(orr[8 * k + 7]) * inv_l));
+                for (int x = 0; x < 32; ++x)
+                    pk[x] = pack_bf16x2(__uint_as_float(orr[x / 16][2 * (x % 16)]) * inv_l,
+                                        __uint_as_float(orr[x / 16][2 * (x % 16) + 1]) * inv_l);
+                if (full_tile) {
+                    if (leader) bulk_wait_group_read<0>(); // the previous store has left the buffer
+                    if (!group_sync(&sb.o_sync[w], sync_phase, abort)) { ok = false; break; }
+                    uint8_t *srow = stage + row * 128;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        *reinterpret_cast<uint4 *>(srow + ((u ^ (row & 7)) << 4)) =
+                            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                    fence_proxy_async_smem();
+                    if (!group_sync(&sb.o_sync[w], sync_phase, abort)) { ok = false; break; }
+                    if (leader) {
+                        tma_store_2d(&tm_o, stage, r.h * D + 64 * c, r.s0 + t * kTile);
+                        bulk_commit_group();
+                    }
+                } else if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 64 * c);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sb.o_free[w]);
+            if (!ok) break;
             if (valid)
                 lse[int64_t(r.h) * p.total_tokens + r.s0 + i] = (m_ref + log2f(l)) * 0.6931471805599453f;
             ++my_items;
         }
+        if (leader) bulk_wait_group<0>();
     }
 
     tc_fence_before();
@@ -423,7 +458,8 @@ __global__ void __launch_bounds__(384, 1)
 
 template <int D>
 cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                  const Problem &p, void *out, float *lse, int num_sms, cudaStream_t stream)
+                                  const CUtensorMap &to, const Problem &p, void *out, float *lse, int num_sms,
+                                  cudaStream_t stream)
 {
     using Lay = FwdLayout<D>;
     auto kern = fwd_bf16_sm100_kernel<D>;
@@ -435,13 +471,16 @@ cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
     if (e != cudaSuccess) return e;
     if (fa.numRegs * Lay::kThreads < int(256 * Lay::kRegsCompute + 128 * Lay::kRegsOther))
         return cudaErrorInvalidConfiguration;
-    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, p, static_cast<__nv_bfloat16 *>(out), lse);
+    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, to, p, static_cast<__nv_bfloat16 *>(out),
+                                                          lse);
     return cudaGetLastError();
 }
 
 template cudaError_t launch_fwd_bf16_sm100<64>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                                               const Problem &, void *, float *, int, cudaStream_t);
+                                               const CUtensorMap &, const Problem &, void *, float *, int,
+                                               cudaStream_t);
 template cudaError_t launch_fwd_bf16_sm100<128>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                                                const Problem &, void *, float *, int, cudaStream_t);
+                                                const CUtensorMap &, const Problem &, void *, float *, int,
+                                                cudaStream_t);
 
 } // namespace ba

@@ -30,16 +30,17 @@ cudaError_t launch_bwd_f32(const Problem &p, const float *q, const float *k, con
 
 template <int D>
 cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                  const Problem &p, void *out, float *lse, int num_sms, cudaStream_t stream);
+                                  const CUtensorMap &to, const Problem &p, void *out, float *lse, int num_sms,
+                                  cudaStream_t stream);
 
 template <int D>
 cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const CUtensorMap &tdo, const CUtensorMap &to, const Problem &p, const float *lse,
-                                float *delta, void *dq, int num_sms, cudaStream_t stream);
+                                float *neg_delta, float *nlse2, void *dq, int num_sms, cudaStream_t stream);
 template <int D>
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
-                                  const Problem &p, const float *lse, const float *delta, void *dk, void *dv,
+                                  const Problem &p, const float *nlse2, const float *neg_delta, void *dk, void *dv,
                                   int num_sms, cudaStream_t stream);
 
 } // namespace ba

@@ -62,10 +62,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
-// Waits for the phase of `bar` with the given parity to complete. Returns
-// false (after setting *abort) if the wait ran past kWaitLimitNs or another
-// thread of the CTA already gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
+// One lane's wait for the phase of `bar` with the given parity to complete.
+// Returns false (after setting *abort) if the wait ran past kWaitLimitNs or
+// another thread of the CTA already gave up.
+__device__ __forceinline__ bool mbar_wait_lane(uint64_t *bar, uint32_t parity, volatile int *abort)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
@@ -81,12 +81,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
-// mbar_wait for a warp that issues warp-collective instructions next: every
-// lane waits, and the result is made uniform so that on a timeout all lanes
-// leave together instead of some of them waiting in elect.sync.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort)
+// Waits for the phase of `bar` with the given parity to complete. Called by
+// all 32 lanes of a warp: every lane waits and the result is made uniform, so
+// that after a timeout no lane is left behind at a warp-collective
+// instruction (elect.sync, tcgen05.ld, shuffles) that the others never reach.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
 {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+    return __all_sync(0xffffffffu, mbar_wait_lane(bar, parity, abort));
 }
 
 // Barrier over a group of threads, on an mbarrier initialised with the group's
@@ -157,6 +158,19 @@ template <int N>
 __device__ __forceinline__ void bulk_wait_group()
 {
     asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// 4-byte asynchronous copy global -> shared (no register staging).
+__device__ __forceinline__ void cp_async_4(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+// Arrives on `bar` once all of this thread's earlier cp.async copies have
+// landed; the arrival is counted in the barrier's expected count.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Makes generic-proxy shared-memory writes visible to the async proxy

@@ -91,8 +91,9 @@ typedef struct {
 /*
  * Bytes of workspace ba_fwd / ba_bwd need for this problem (0 on an invalid
  * problem): a status word and a work table of about 16 bytes per 128-row
- * tile, plus, for the backward, a float32 row-dot buffer Delta
- * [heads, total_tokens].
+ * tile, plus, for the backward, two float32 per-row buffers [heads,
+ * total_tokens]: the row dot product Delta = dO . out and (bf16) the
+ * forward's lse in the form the dK/dV pass reads.
  */
 size_t ba_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window);
 size_t ba_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window);
