@@ -73,7 +73,7 @@ struct DkvLayout {
 };
 
 struct DkvBarriers {
-    uint64_t kv_full, kv_empty, dkv_full, dkv_free;
+    uint64_t k_full, k_empty, v_full, v_empty, dkv_full, dkv_free;
     uint64_t q_full[4], q_empty[4], o_full[4], o_empty[4];
     uint64_t s_full, dp_full, pa_done[2], pb_done[2];
     uint64_t epi_sync; // group barrier of the epilogue warps
@@ -111,8 +111,10 @@ __global__ void __launch_bounds__(448, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sb.kv_full, 1);
-        mbar_init(&sb.kv_empty, 1);
+        mbar_init(&sb.k_full, 1);
+        mbar_init(&sb.k_empty, 1);
+        mbar_init(&sb.v_full, 1);
+        mbar_init(&sb.v_empty, 1);
         mbar_init(&sb.dkv_full, 1);
         mbar_init(&sb.dkv_free, 4);
         for (int i = 0; i < 4; ++i) {
@@ -159,31 +161,6 @@ __global__ void __launch_bounds__(448, 1)
         for (; ok && items.advance(r); ++item_cnt) {
             int ilo, ihi;
             query_tile_range(r, B, W, ilo, ihi);
-            if (!mbar_wait(&sb.kv_empty, (item_cnt & 1) ^ 1, abort)) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&sb.kv_full, 2 * Lay::kTileBytes);
-                for (int c = 0; c < Lay::kChunks; ++c) {
-                    tma_load_2d(smem + Lay::kK + c * Lay::kChunkBytes, &tm_k, &sb.kv_full, r.h * D + c * 64,
-                                r.s0 + r.t * kTile);
-                    tma_load_2d(smem + Lay::kV + c * Lay::kChunkBytes, &tm_v, &sb.kv_full, r.h * D + c * 64,
-                                r.s0 + r.t * kTile);
-                }
-                // warm L2 with the next item's K and V
-                TileRef rn;
-                if (items.peek(rn)) {
-                    int nlo, nhi;
-                    query_tile_range(rn, B, W, nlo, nhi);
-                    for (int c = 0; c < Lay::kChunks; ++c) {
-                        tma_prefetch_l2_2d(&tm_k, rn.h * D + c * 64, rn.s0 + rn.t * kTile);
-                        tma_prefetch_l2_2d(&tm_v, rn.h * D + c * 64, rn.s0 + rn.t * kTile);
-                        for (int i = nlo; i <= nhi && i < nlo + 2; ++i) {
-                            tma_prefetch_l2_2d(&tm_q, rn.h * D + c * 64, rn.s0 + i * kTile);
-                            tma_prefetch_l2_2d(&tm_do, rn.h * D + c * 64, rn.s0 + i * kTile);
-                        }
-                    }
-                }
-            }
-            __syncwarp();
             for (int i = ilo; i <= ihi; ++i, ++it) {
                 const int qs = it % QS, os = it % OS;
                 if (!mbar_wait(&sb.q_empty[qs], ((it / QS) & 1) ^ 1, abort)) {
@@ -209,6 +186,32 @@ __global__ void __launch_bounds__(448, 1)
                 }
                 cp_async_arrive_noinc(&sb.q_full[qs]);
                 __syncwarp();
+                if (i == ilo) {
+                    // the item's K and V, once the previous item's last S^T (K) and dP^T (V)
+                    // are done; the first Q tile went out first, since its slot frees earlier
+                    if (!mbar_wait(&sb.k_empty, (item_cnt & 1) ^ 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&sb.k_full, Lay::kTileBytes);
+                        for (int c = 0; c < Lay::kChunks; ++c)
+                            tma_load_2d(smem + Lay::kK + c * Lay::kChunkBytes, &tm_k, &sb.k_full, r.h * D + c * 64,
+                                        r.s0 + r.t * kTile);
+                    }
+                    __syncwarp();
+                    if (!mbar_wait(&sb.v_empty, (item_cnt & 1) ^ 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&sb.v_full, Lay::kTileBytes);
+                        for (int c = 0; c < Lay::kChunks; ++c)
+                            tma_load_2d(smem + Lay::kV + c * Lay::kChunkBytes, &tm_v, &sb.v_full, r.h * D + c * 64,
+                                        r.s0 + r.t * kTile);
+                    }
+                    __syncwarp();
+                }
                 if (!mbar_wait(&sb.o_empty[os], ((it / OS) & 1) ^ 1, abort)) {
                     ok = false;
                     break;
@@ -218,12 +221,25 @@ __global__ void __launch_bounds__(448, 1)
                     for (int c = 0; c < Lay::kChunks; ++c)
                         tma_load_2d(smem + Lay::kO0 + os * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_do,
                                     &sb.o_full[os], r.h * D + c * 64, r.s0 + i * kTile);
-                    // warm L2 two query tiles ahead
+                    // warm L2 two query tiles ahead, and with the next item's K, V and first tiles
                     if (i + 2 <= ihi)
                         for (int c = 0; c < Lay::kChunks; ++c) {
                             tma_prefetch_l2_2d(&tm_q, r.h * D + c * 64, r.s0 + (i + 2) * kTile);
                             tma_prefetch_l2_2d(&tm_do, r.h * D + c * 64, r.s0 + (i + 2) * kTile);
                         }
+                    TileRef rn;
+                    if (i == ilo && items.peek(rn)) {
+                        int nlo, nhi;
+                        query_tile_range(rn, B, W, nlo, nhi);
+                        for (int c = 0; c < Lay::kChunks; ++c) {
+                            tma_prefetch_l2_2d(&tm_k, rn.h * D + c * 64, rn.s0 + rn.t * kTile);
+                            tma_prefetch_l2_2d(&tm_v, rn.h * D + c * 64, rn.s0 + rn.t * kTile);
+                            for (int i2 = nlo; i2 <= nhi && i2 < nlo + 2; ++i2) {
+                                tma_prefetch_l2_2d(&tm_q, rn.h * D + c * 64, rn.s0 + i2 * kTile);
+                                tma_prefetch_l2_2d(&tm_do, rn.h * D + c * 64, rn.s0 + i2 * kTile);
+                            }
+                        }
+                    }
                 }
                 __syncwarp();
             }
@@ -241,9 +257,7 @@ __global__ void __launch_bounds__(448, 1)
             int ilo, ihi;
             query_tile_range(r, B, W, ilo, ihi);
             const int nq = ihi - ilo + 1;
-            if (!mbar_wait(&sb.kv_full, item_cnt & 1, abort)) break;
-            tc_fence_after();
-            // S^T = K Q^T of query tile m of this item
+            // S^T = K Q^T of query tile m of this item; after the item's last one K is not read again
             auto issue_s = [&](int m) -> bool {
                 const uint32_t it = it0 + m, qs = it % QS;
                 if (!mbar_wait(&sb.q_full[qs], (it / QS) & 1, abort)) return false;
@@ -257,11 +271,12 @@ __global__ void __launch_bounds__(448, 1)
                                sdesc_sw128(q_addr + off, 16, 1024), idesc_sp, kk > 0 ? 1u : 0u);
                     }
                     tc_commit(&sb.s_full);
+                    if (m == nq - 1) tc_commit(&sb.k_empty);
                 }
                 __syncwarp();
                 return true;
             };
-            // dP^T = V dO^T of query tile m; after the item's last one K and V are not read again
+            // dP^T = V dO^T of query tile m; after the item's last one V is not read again
             auto issue_dp = [&](int m) -> bool {
                 const uint32_t it = it0 + m, os = it % OS;
                 if (!mbar_wait(&sb.o_full[os], (it / OS) & 1, abort)) return false;
@@ -275,7 +290,7 @@ __global__ void __launch_bounds__(448, 1)
                                sdesc_sw128(o_addr + off, 16, 1024), idesc_sp, kk > 0 ? 1u : 0u);
                     }
                     tc_commit(&sb.dp_full);
-                    if (m == nq - 1) tc_commit(&sb.kv_empty);
+                    if (m == nq - 1) tc_commit(&sb.v_empty);
                 }
                 __syncwarp();
                 return true;
@@ -306,7 +321,11 @@ __global__ void __launch_bounds__(448, 1)
                 }
                 return true;
             };
-            ok = issue_s(0) && issue_dp(0);
+            ok = mbar_wait(&sb.k_full, item_cnt & 1, abort);
+            if (ok) tc_fence_after();
+            ok = ok && issue_s(0) && mbar_wait(&sb.v_full, item_cnt & 1, abort);
+            if (ok) tc_fence_after();
+            ok = ok && issue_dp(0);
             for (int m = 0; ok && m < nq; ++m) {
                 ok = issue_acc(m, 0) && (m + 1 >= nq || issue_s(m + 1)) && issue_acc(m, 1) &&
                      (m + 1 >= nq || issue_dp(m + 1));
