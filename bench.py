@@ -403,12 +403,15 @@ def main():
 
 
 def kernel_sha(which: str) -> str:
-    """Hash of a kernel's source file, to tell whether stored counters are current."""
+    """Hash of a kernel's source file and the device headers it includes, to tell
+    whether stored counters are current."""
     import hashlib
     src = {"fwd": "ba_fwd_sm100.cu", "bwd_dq": "ba_bwd_dq_sm100.cu", "bwd_dkdv": "ba_bwd_dkdv_sm100.cu"}[which]
-    p = os.path.join(ROOT, "block_sparse_attention_kunlun_b200", "csrc", src)
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for name in (src, "ba_common.cuh", "ba_ptx.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_attention_kunlun_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 if __name__ == "__main__":
