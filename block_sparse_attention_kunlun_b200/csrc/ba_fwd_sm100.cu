@@ -51,18 +51,21 @@ struct FwdLayout {
                                                                   // kStage + w chunk (128 x 64 bf16)
     static constexpr int kBytes = kStage + 2 * kChunkBytes;
     static constexpr int kAlloc = kBytes + 1024;         // slack to align the base to 1024 B
-    static constexpr int kThreads = 384;                 // three warpgroups
-    // register budgets after the split; 2 * 128 * 192 + 128 * 120 = 384 * 168
-    static constexpr uint32_t kRegsCompute = 192, kRegsOther = 120;
+    static constexpr int kThreads = 512;                 // four warpgroups
+    // register budgets after the split: softmax warpgroups, epilogue warpgroup,
+    // TMA / MMA warpgroup; 2 * 128 * compute + 128 * epi + 128 * other = 512 * 128
+    static constexpr uint32_t kRegsCompute = D == 64 ? 168 : 184, kRegsEpi = 64, kRegsOther = D == 64 ? 112 : 80;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColO = 256;
 };
 
 struct FwdBarriers {
-    uint64_t q_full, q_empty;
+    uint64_t q_full[2], q_empty[2]; // query tile of group w, released after its last S
     uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
     uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-    uint64_t o_sync[2]; // group barrier of each softmax warpgroup (epilogue staging)
+    uint64_t o_ready[2]; // group w's softmax is done with its item: inv_l[w] holds 1 / l
+    uint64_t epi_sync;   // group barrier of the epilogue warpgroup
+    float inv_l[2][kTile];
     uint32_t tmem_base;
     int abort;
 };
@@ -76,7 +79,7 @@ __device__ __forceinline__ int first_key_tile(int t, int64_t B, int64_t W)
 } // namespace
 
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                           const Problem p,
@@ -92,14 +95,16 @@ __global__ void __launch_bounds__(384, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sb.q_full, 1);
-        mbar_init(&sb.q_empty, 1);
+        mbar_init(&sb.q_full[0], 1);
+        mbar_init(&sb.q_empty[0], 1);
+        mbar_init(&sb.q_full[1], 1);
+        mbar_init(&sb.q_empty[1], 1);
         for (int w = 0; w < 2; ++w) {
             mbar_init(&sb.s_full[w], 1);
             mbar_init(&sb.p_full[w], 4);
             mbar_init(&sb.o_final[w], 1);
             mbar_init(&sb.o_free[w], 4);
-            mbar_init(&sb.o_sync[w], 128);
+            mbar_init(&sb.o_ready[w], 4);
         }
         for (int i = 0; i < S; ++i) {
             mbar_init(&sb.k_full[i], 1);
@@ -107,6 +112,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&sb.v_full[i], 1);
             mbar_init(&sb.v_empty[i], 1);
         }
+        mbar_init(&sb.epi_sync, 128);
         sb.abort = 0;
         fence_mbar_init();
     }
@@ -127,12 +133,13 @@ __global__ void __launch_bounds__(384, 1)
     const int64_t B = p.block, W = p.window;
     const int32_t npairs = live_pair_count(p);
 
-    if (warp >= 8) {
-        // warps 8-11 (one warpgroup: TMA, MMA, two idle) hand registers to the compute warpgroups
+    if (warp >= 8 && warp < 12) {
+        // warps 8-11 (one warpgroup: TMA, MMA, two idle) hand registers to the softmax warpgroups
         warpgroup_regs_dec<Lay::kRegsOther>();
         if (warp == 8) {
             // ------------------------------------------------ TMA producer ---
             uint32_t kv_cnt = 0, item_cnt = 0;
+            uint32_t qcnt[2] = {0, 0}; // query tiles loaded per group
             TileRef r;
             bool second;
             bool ok = true;
@@ -141,13 +148,23 @@ __global__ void __launch_bounds__(384, 1)
                 second = pair_has_second(r);
                 const int jlo = first_key_tile(r.t, B, W);
                 const int jhi = r.t + (second ? 1 : 0);
-                if (!mbar_wait(&sb.q_empty, (item_cnt & 1) ^ 1, abort)) break;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&sb.q_full, (second ? 2 : 1) * Lay::kTileBytes);
-                    for (int w = 0; w < (second ? 2 : 1); ++w)
+                // each group's query tile as soon as that group's previous one is done with
+                for (int w = 0; w < (second ? 2 : 1) && ok; ++w) {
+                    if (!mbar_wait(&sb.q_empty[w], (qcnt[w] & 1) ^ 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&sb.q_full[w], Lay::kTileBytes);
                         for (int c = 0; c < Lay::kChunks; ++c)
-                            tma_load_2d(smem + Lay::kQ + w * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_q, &sb.q_full,
-                                        r.h * D + c * 64, r.s0 + (r.t + w) * kTile);
+                            tma_load_2d(smem + Lay::kQ + w * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_q,
+                                        &sb.q_full[w], r.h * D + c * 64, r.s0 + (r.t + w) * kTile);
+                    }
+                    __syncwarp();
+                    ++qcnt[w];
+                }
+                if (!ok) break;
+                if (lane == 0) {
                     // warm L2 with the next item's query tiles
                     TileRef rn;
                     if (items.peek(rn)) {
@@ -193,6 +210,7 @@ __global__ void __launch_bounds__(384, 1)
             constexpr uint32_t idesc_o = idesc_bf16(128, D, false, true);
             uint32_t kv_cnt = 0, item_cnt = 0;
             uint32_t pcnt[2] = {0, 0}; // P tiles consumed so far by each group
+            uint32_t qf[2] = {0, 0};   // query tiles used up so far by each group
             uint32_t icnt[2] = {0, 0}; // items each group has finished (group 1 skips single-tile items)
             TileRef r;
             bool second;
@@ -203,8 +221,6 @@ __global__ void __launch_bounds__(384, 1)
                 const int lo[2] = {first_key_tile(r.t, B, W), second ? first_key_tile(r.t + 1, B, W) : 1};
                 const int hi[2] = {r.t, second ? r.t + 1 : 0};
                 const int jlo = lo[0], jhi = second ? hi[1] : hi[0];
-                if (!mbar_wait(&sb.q_full, item_cnt & 1, abort)) break;
-                tc_fence_after();
                 // O_w += P_w V for key tile j of group w (V from ring stage st)
                 auto issue_pv = [&](int w, int j, int st) -> bool {
                     if (!mbar_wait(&sb.p_full[w], pcnt[w] & 1, abort)) return false;
@@ -224,7 +240,11 @@ __global__ void __launch_bounds__(384, 1)
                     ++pcnt[w];
                     return true;
                 };
-                auto issue_s = [&](int w, int st) {
+                auto issue_s = [&](int w, int j, int st) -> bool {
+                    if (j == lo[w]) { // this group's query tile of the item
+                        if (!mbar_wait(&sb.q_full[w], qf[w] & 1, abort)) return false;
+                        tc_fence_after();
+                    }
                     {
                         const uint32_t q_addr = smem_base + Lay::kQ + w * Lay::kTileBytes;
                         const uint32_t k_addr = smem_base + Lay::kK0 + 2 * st * Lay::kTileBytes;
@@ -235,8 +255,11 @@ __global__ void __launch_bounds__(384, 1)
                                    sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
                         }
                         tc_commit(&sb.s_full[w]);
+                        if (j == hi[w]) tc_commit(&sb.q_empty[w]); // its last S: the tile may be replaced
                     }
                     __syncwarp();
+                    if (j == hi[w]) ++qf[w];
+                    return true;
                 };
                 // V of the previous key tile (ring position kv_cnt - 1) before its first P V
                 auto wait_v_prev = [&]() -> bool {
@@ -255,11 +278,10 @@ __global__ void __launch_bounds__(384, 1)
                     for (int w = 0; w < 2 && ok; ++w) {
                         // the previous tile's P V of this group reads P from the S buffer: issue it first
                         if (j - 1 >= lo[w] && j - 1 <= hi[w] && !issue_pv(w, j - 1, (kv_cnt - 1) % S)) ok = false;
-                        if (ok && j >= lo[w] && j <= hi[w]) issue_s(w, st);
+                        if (ok && j >= lo[w] && j <= hi[w] && !issue_s(w, j, st)) ok = false;
                     }
                     if (!ok) break;
                     {
-                        if (j == jhi) tc_commit(&sb.q_empty);
                         tc_commit(&sb.k_empty[st]);                            // K of tile j: S products issued
                         if (j > jlo) tc_commit(&sb.v_empty[(kv_cnt - 1) % S]); // V of tile j-1: P V issued
                     }
@@ -276,7 +298,7 @@ __global__ void __launch_bounds__(384, 1)
                 if (second) ++icnt[1];
             }
         }
-    } else {
+    } else if (warp < 8) {
         warpgroup_regs_inc<Lay::kRegsCompute>();
         // ----------------------------------------------------- softmax ---
         const int w = warp >> 2;              // group: query tile t + w
@@ -285,10 +307,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t s_addr = tmem + lane_base + 128 * w;
         const uint32_t o_addr = tmem + lane_base + Lay::kColO + D * w;
         const float scale_log2 = p.scale * 1.4426950408889634f;
-        uint32_t cnt = 0, my_items = 0; // tiles and items this group has processed
-        uint32_t sync_phase = 0;
-        const bool leader = row == 0;
-        uint8_t *stage = smem + Lay::kStage + w * Lay::kChunkBytes;
+        uint32_t cnt = 0; // tiles this group has processed
         TileRef r;
         bool second;
         bool ok = true;
@@ -395,56 +414,93 @@ __global__ void __launch_bounds__(384, 1)
                 if (lane == 0) mbar_arrive(&sb.p_full[w]);
             }
             if (!ok) break;
-            // epilogue: wait for this group's last P V, normalise, store. A tile whose
-            // rows all belong to the example leaves through this group's staging
-            // buffer and TMA stores (whole lines); the example's last tile row by row.
-            if (!mbar_wait(&sb.o_final[w], my_items & 1, abort)) break;
-            tc_fence_after();
-            const float inv_l = valid ? 1.f / l : 0.f;
-            const bool full_tile = int64_t(t) * kTile + kTile <= r.L;
-            __nv_bfloat16 *orow = out + ((int64_t(r.s0) + i) * p.heads + r.h) * D;
-#pragma unroll 1
-            for (int c = 0; c < D / 64; ++c) {
-                uint32_t orr[2][32];
-                tmem_ld32(o_addr + 64 * c, orr[0]);
-                tmem_ld32(o_addr + 64 * c + 32, orr[1]);
-                tmem_wait_ld();
-                reg_fence(orr[0]);
-                reg_fence(orr[1]);
-                if (c == D / 64 - 1) { // all of O read: the next item's P V may overwrite it
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sb.o_free[w]);
-                }
-                uint32_t pk[32];
-#pragma unroll
-                for (int x = 0; x < 32; ++x)
-                    pk[x] = pack_bf16x2(__uint_as_float(orr[x / 16][2 * (x % 16)]) * inv_l,
-                                        __uint_as_float(orr[x / 16][2 * (x % 16) + 1]) * inv_l);
-                if (full_tile) {
-                    if (leader) bulk_wait_group_read<0>(); // the previous store has left the buffer
-                    if (!group_sync(&sb.o_sync[w], sync_phase, abort)) { ok = false; break; }
-                    uint8_t *srow = stage + row * 128;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        *reinterpret_cast<uint4 *>(srow + ((u ^ (row & 7)) << 4)) =
-                            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-                    fence_proxy_async_smem();
-                    if (!group_sync(&sb.o_sync[w], sync_phase, abort)) { ok = false; break; }
-                    if (leader) {
-                        tma_store_2d(&tm_o, stage, r.h * D + 64 * c, r.s0 + t * kTile);
-                        bulk_commit_group();
-                    }
-                } else if (valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 64 * c);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-                }
-            }
-            if (!ok) break;
+            // hand 1 / l to the epilogue warps, write lse, and go on with the next item
+            sb.inv_l[w][row] = valid ? 1.f / l : 0.f;
             if (valid)
                 lse[int64_t(r.h) * p.total_tokens + r.s0 + i] = (m_ref + log2f(l)) * 0.6931471805599453f;
-            ++my_items;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sb.o_ready[w]);
+        }
+    } else {
+        warpgroup_regs_dec<Lay::kRegsEpi>();
+        // ---------------------------------------------------- epilogue ---
+        // Per item and group: wait for the softmax (1 / l) and the last P V, then
+        // normalise O and store it. A tile whose rows all belong to the example
+        // leaves through the two staging buffers (alternating) and TMA stores; the
+        // example's last tile is stored row by row.
+        const int row = threadIdx.x & 127;    // query row within the tile, TMEM lane
+        const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+        const bool leader = threadIdx.x == 384;
+        uint32_t done[2] = {0, 0}, sync_phase = 0, nstored = 0;
+        TileRef r;
+        bool ok = true;
+        ItemWalker items(p.pair_info, npairs, p.heads);
+        while (ok && items.advance(r)) {
+            const bool second = pair_has_second(r);
+            for (int w = 0; w < (second ? 2 : 1) && ok; ++w) {
+                if (!mbar_wait(&sb.o_ready[w], done[w] & 1, abort) ||
+                    !mbar_wait(&sb.o_final[w], done[w] & 1, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                ++done[w];
+                const float inv_l = sb.inv_l[w][row];
+                const int t = r.t + w;
+                const int64_t i = int64_t(t) * kTile + row;
+                const bool valid = i < r.L;
+                const bool full_tile = int64_t(t) * kTile + kTile <= r.L;
+                const uint32_t o_addr = tmem + lane_base + Lay::kColO + D * w;
+                __nv_bfloat16 *orow = out + ((int64_t(r.s0) + i) * p.heads + r.h) * D;
+#pragma unroll 1
+                for (int c = 0; c < D / 64; ++c) {
+                    uint8_t *stage = smem + Lay::kStage + (nstored & 1) * Lay::kChunkBytes;
+                    if (full_tile) {
+                        if (leader) bulk_wait_group_read<1>(); // this buffer's previous store has left it
+                        if (!group_sync(&sb.epi_sync, sync_phase, abort)) { ok = false; break; }
+                    }
+                    // 32 columns at a time: normalise, pack, and put them in the staging row
+                    // (or straight into the output row for the example's last tile)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t orr[32];
+                        tmem_ld32(o_addr + 64 * c + 32 * hh, orr);
+                        tmem_wait_ld();
+                        reg_fence(orr);
+                        if (c == D / 64 - 1 && hh == 1) { // all of O read: the next item's P V may overwrite it
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&sb.o_free[w]);
+                        }
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int x = 0; x < 16; ++x)
+                            pk[x] = pack_bf16x2(__uint_as_float(orr[2 * x]) * inv_l,
+                                                __uint_as_float(orr[2 * x + 1]) * inv_l);
+                        if (full_tile) {
+                            uint8_t *srow = stage + row * 128;
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                *reinterpret_cast<uint4 *>(srow + (((4 * hh + u) ^ (row & 7)) << 4)) =
+                                    make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                        } else if (valid) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(orow + 64 * c + 32 * hh);
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                        }
+                    }
+                    if (full_tile) {
+                        fence_proxy_async_smem();
+                        if (!group_sync(&sb.epi_sync, sync_phase, abort)) { ok = false; break; }
+                        if (leader) {
+                            tma_store_2d(&tm_o, stage, r.h * D + 64 * c, r.s0 + t * kTile);
+                            bulk_commit_group();
+                        }
+                        ++nstored;
+                    }
+                }
+            }
         }
         if (leader) bulk_wait_group<0>();
     }
@@ -469,7 +525,7 @@ cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, kern);
     if (e != cudaSuccess) return e;
-    if (fa.numRegs * Lay::kThreads < int(256 * Lay::kRegsCompute + 128 * Lay::kRegsOther))
+    if (fa.numRegs * Lay::kThreads < int(256 * Lay::kRegsCompute + 128 * Lay::kRegsEpi + 128 * Lay::kRegsOther))
         return cudaErrorInvalidConfiguration;
     kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, to, p, static_cast<__nv_bfloat16 *>(out),
                                                           lse);
