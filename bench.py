@@ -49,6 +49,11 @@ def parse():
     ap.add_argument("--config", type=int, default=3, choices=sorted(CONFIGS))
     ap.add_argument("--examples", type=int, default=0,
                     help="keep only the first N examples (small cases for profiling)")
+    ap.add_argument("--block", type=int, default=0, help="override the config's block size")
+    ap.add_argument("--window", type=int, default=0, help="override the config's window (in blocks)")
+    ap.add_argument("--swa", type=int, default=0, metavar="W",
+                    help="time sliding-window attention (each query sees its last W tokens; block 1, "
+                         "window W) on the config's shapes instead of block attention")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic-file", default=os.path.join(ROOT, "profiles", "traffic.json"),
@@ -66,8 +71,21 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload(args, rank=0):
+def config_workload(args):
+    """The config's workload, or its sliding-window variant under --swa."""
+    import re
     w = CONFIGS[args.config]
+    if args.swa:
+        return w.replace(block=1, window=args.swa,
+                         name=re.sub(r"block \d+, window \d+", f"sliding window {args.swa} tokens", w.name))
+    if args.block or args.window:
+        b, win = args.block or w.block, args.window or w.window
+        w = w.replace(block=b, window=win, name=re.sub(r"block \d+, window \d+", f"block {b}, window {win}", w.name))
+    return w
+
+
+def workload(args, rank=0):
+    w = config_workload(args)
     inp = make_inputs(w, seed=w.seed + 7919 * rank)
     if args.examples:
         n = min(args.examples, w.batch)
@@ -166,7 +184,7 @@ def run_reference(args):
     if rank != 0:
         return
     import oracle
-    w = CONFIGS[args.config]
+    w = config_workload(args)
     inp = make_inputs(w)
     offs = inp["seq_offsets"].numpy()
     lens = np.diff(offs)
@@ -365,7 +383,8 @@ def main():
     try:
         with open(args.traffic_file) as f:
             tr = json.load(f)
-        key = f"{names[dom]}:config{args.config}"
+        key = f"{names[dom]}:config{args.config}" + (f":block{w.block}:window{w.window}"
+                                                       if (args.swa or args.block or args.window) else "")
         if key in tr and tr[key].get("kernel_sha") == kernel_sha(dom):
             traffic = tr[key]["bytes_per_launch"]
     except (OSError, ValueError):

@@ -79,6 +79,14 @@ def _load():
     lib.ba_set_profile_events.restype = ctypes.c_int
     lib.ba_version.argtypes = []
     lib.ba_version.restype = ctypes.c_int32
+    lib.ba_swa_fwd_workspace_size.argtypes = [prob, i32]
+    lib.ba_swa_fwd_workspace_size.restype = ctypes.c_size_t
+    lib.ba_swa_bwd_workspace_size.argtypes = [prob, i32]
+    lib.ba_swa_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.ba_swa_fwd.argtypes = [prob, P, P, P, P, i32, P, P, P, P, ctypes.c_size_t, P]
+    lib.ba_swa_fwd.restype = ctypes.c_int
+    lib.ba_swa_bwd.argtypes = [prob, P, P, P, P, P, P, P, i32, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.ba_swa_bwd.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -152,6 +160,35 @@ def ba_bwd(problem, q, k, v, out, lse, dout, seq_offsets, block, window, skip, d
                               _stream(stream)))
 
 
+def ba_swa_fwd_workspace_size(problem: BAProblem, window_tokens: int) -> int:
+    return int(_load().ba_swa_fwd_workspace_size(ctypes.byref(problem), int(window_tokens)))
+
+
+def ba_swa_bwd_workspace_size(problem: BAProblem, window_tokens: int) -> int:
+    return int(_load().ba_swa_bwd_workspace_size(ctypes.byref(problem), int(window_tokens)))
+
+
+def ba_swa_fwd(problem, q, k, v, seq_offsets, window_tokens, skip, out, lse, workspace,
+               workspace_bytes=None, stream=None) -> int:
+    """Direct call of the sliding-window forward; returns its status code."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(_load().ba_swa_fwd(ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets),
+                                  int(window_tokens), _ptr(skip), _ptr(out), _ptr(lse), _ptr(workspace),
+                                  int(workspace_bytes), _stream(stream)))
+
+
+def ba_swa_bwd(problem, q, k, v, out, lse, dout, seq_offsets, window_tokens, skip, dq, dk, dv,
+               workspace, workspace_bytes=None, stream=None) -> int:
+    """Direct call of the sliding-window backward; returns its status code."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(_load().ba_swa_bwd(ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                  _ptr(dout), _ptr(seq_offsets), int(window_tokens), _ptr(skip),
+                                  _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), int(workspace_bytes),
+                                  _stream(stream)))
+
+
 def ba_set_profile_events(which: int, start=None, stop=None) -> int:
     """Record torch.cuda.Event ``start``/``stop`` around one kernel of every
     later call from this thread: 0 the forward attention kernel, 1 the
@@ -215,4 +252,39 @@ def block_attention_bwd(q, k, v, out, lse, dout, seq_offsets, block, window, ski
                 workspace, stream=stream)
     if st != BA_OK:
         raise BAError(st, "ba_bwd")
+    return dq, dk, dv
+
+
+def sliding_window_attention_fwd(q, k, v, seq_offsets, window_tokens, skip=None, out=None, lse=None,
+                                 workspace=None, stream=None):
+    """Allocates out/lse (and a workspace) with torch and runs ba_swa_fwd:
+    query i sees keys i - window_tokens < j <= i of its example."""
+    _check_inputs(q, k, v, seq_offsets)
+    prob = make_problem(q, seq_offsets)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = workspace_for(ba_swa_fwd_workspace_size(prob, window_tokens), q.device)
+    st = ba_swa_fwd(prob, q, k, v, seq_offsets, window_tokens, skip, out, lse, workspace, stream=stream)
+    if st != BA_OK:
+        raise BAError(st, "ba_swa_fwd")
+    return out, lse
+
+
+def sliding_window_attention_bwd(q, k, v, out, lse, dout, seq_offsets, window_tokens, skip=None,
+                                 dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Allocates dq/dk/dv (and a workspace) with torch and runs ba_swa_bwd."""
+    _check_inputs(q, k, v, seq_offsets)
+    prob = make_problem(q, seq_offsets)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if workspace is None:
+        workspace = workspace_for(ba_swa_bwd_workspace_size(prob, window_tokens), q.device)
+    st = ba_swa_bwd(prob, q, k, v, out, lse, dout, seq_offsets, window_tokens, skip, dq, dk, dv,
+                    workspace, stream=stream)
+    if st != BA_OK:
+        raise BAError(st, "ba_swa_bwd")
     return dq, dk, dv

@@ -251,6 +251,34 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
     return BA_OK;
 }
 
+// Sliding-window attention: the block rule with block = 1 (one token per block),
+// so window counts tokens.
+size_t ba_swa_fwd_workspace_size(const ba_problem *p, int32_t window_tokens)
+{
+    return ba_fwd_workspace_size(p, 1, window_tokens);
+}
+
+size_t ba_swa_bwd_workspace_size(const ba_problem *p, int32_t window_tokens)
+{
+    return ba_bwd_workspace_size(p, 1, window_tokens);
+}
+
+ba_status ba_swa_fwd(const ba_problem *p, const void *q, const void *k, const void *v, const int32_t *seq_offsets,
+                     int32_t window_tokens, const uint8_t *skip, void *out, float *lse, void *workspace,
+                     size_t workspace_bytes, ba_stream_t stream)
+{
+    return ba_fwd(p, q, k, v, seq_offsets, 1, window_tokens, skip, out, lse, workspace, workspace_bytes, stream);
+}
+
+ba_status ba_swa_bwd(const ba_problem *p, const void *q, const void *k, const void *v, const void *out,
+                     const float *lse, const void *dout, const int32_t *seq_offsets, int32_t window_tokens,
+                     const uint8_t *skip, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                     ba_stream_t stream)
+{
+    return ba_bwd(p, q, k, v, out, lse, dout, seq_offsets, 1, window_tokens, skip, dq, dk, dv, workspace,
+                  workspace_bytes, stream);
+}
+
 ba_status ba_device_status(const void *workspace, ba_stream_t stream_)
 {
     if (!workspace) return BA_ERR_INVALID_ARG;

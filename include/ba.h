@@ -121,6 +121,29 @@ ba_status ba_bwd(const ba_problem *p, const void *q, const void *k, const void *
                  void *workspace, size_t workspace_bytes, ba_stream_t stream);
 
 /*
+ * Token-granular sliding-window attention, the predecessor that block
+ * attention replaced ("GEM (Meta)", section "Custom kernels": long
+ * user-history self-attention first moved to a sliding window, then to
+ * independent blocks; the pages compare the two by self-attention layer
+ * MFU). Query i of an example sees key j <=> i - window_tokens < j <= i
+ * (local indices, causal, window_tokens >= 1). This is the block rule above
+ * with block = 1 and window = window_tokens, and these entry points run
+ * exactly that: same kernels, arguments, layouts, workspace, ownership and
+ * errors as ba_fwd / ba_bwd / ba_*_workspace_size.
+ */
+size_t ba_swa_fwd_workspace_size(const ba_problem *p, int32_t window_tokens);
+size_t ba_swa_bwd_workspace_size(const ba_problem *p, int32_t window_tokens);
+ba_status ba_swa_fwd(const ba_problem *p, const void *q, const void *k, const void *v,
+                     const int32_t *seq_offsets, int32_t window_tokens, const uint8_t *skip,
+                     void *out, float *lse, void *workspace, size_t workspace_bytes,
+                     ba_stream_t stream);
+ba_status ba_swa_bwd(const ba_problem *p, const void *q, const void *k, const void *v,
+                     const void *out, const float *lse, const void *dout,
+                     const int32_t *seq_offsets, int32_t window_tokens, const uint8_t *skip,
+                     void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                     ba_stream_t stream);
+
+/*
  * Forward pass that allocates nothing and takes no workspace (the pages have
  * no counterpart; this is a convenience of this library). For callers that
  * cannot allocate device memory: a serving loop that records its forward into

@@ -301,3 +301,54 @@ def test_thread_count_does_not_change_bits():
     b = oracle.fwd(offs, q, k, v, 8, 2, nthreads=5) + oracle.bwd(offs, q, k, v, do, 8, 2, nthreads=5)
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
+
+
+# --------------------------------------------- sliding-window attention ---
+# Token-granular sliding window ("GEM (Meta)", "Custom kernels": the
+# predecessor of block attention): query i sees keys i - w < j <= i. The
+# library runs it as the block rule with block = 1; these pins check that
+# reading against the window rule written out directly.
+
+def _swa_brute_fwd(offsets, q, k, v, w):
+    T, H, D = q.shape
+    out = np.zeros((T, H, D))
+    lse = np.zeros((H, T))
+    scale = 1.0 / math.sqrt(D)
+    for e in range(len(offsets) - 1):
+        s0, s1 = int(offsets[e]), int(offsets[e + 1])
+        for h in range(H):
+            for i in range(s1 - s0):
+                keys = [j for j in range(s1 - s0) if i - w < j <= i]
+                wts = [math.exp(math.fsum(q[s0 + i, h, d] * k[s0 + j, h, d] for d in range(D)) * scale)
+                       for j in keys]
+                z = math.fsum(wts)
+                for d in range(D):
+                    out[s0 + i, h, d] = math.fsum(a * v[s0 + j, h, d] for a, j in zip(wts, keys)) / z
+                lse[h, s0 + i] = math.log(z)
+    return out, lse
+
+
+@pytest.mark.parametrize("w", [1, 2, 5, 17])
+def test_sliding_window_is_block_rule_with_block_1(w):
+    rng = np.random.default_rng(300 + w)
+    offs, q, k, v, _ = rand_case(rng, [23, 0, 9, 31], 2, 3)
+    out, lse = oracle.fwd(offs, q, k, v, 1, w)
+    bout, blse = _swa_brute_fwd(offs, q, k, v, w)
+    np.testing.assert_allclose(out, bout, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, blse, rtol=0, atol=1e-12)
+
+
+def test_sliding_window_gradients_match_masked_sdpa():
+    """Backward against PyTorch attention with an explicit band mask (fp64)."""
+    rng = np.random.default_rng(41)
+    L, H, D, w = 40, 2, 8, 7
+    offs, q, k, v, do = rand_case(rng, [L], H, D)
+    dq, dk, dv = oracle.bwd(offs, q, k, v, do, 1, w)
+    i = torch.arange(L)[:, None]
+    j = torch.arange(L)[None, :]
+    band = (j <= i) & (j > i - w)
+    tq, tk, tv = (torch.tensor(x.transpose(1, 0, 2), dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=band)
+    o.backward(torch.tensor(do.transpose(1, 0, 2)))
+    for name, got, ref in (("dq", dq, tq.grad), ("dk", dk, tk.grad), ("dv", dv, tv.grad)):
+        np.testing.assert_allclose(got, ref.numpy().transpose(1, 0, 2), rtol=0, atol=1e-11, err_msg=name)

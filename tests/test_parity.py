@@ -205,3 +205,61 @@ def test_full_size_sampled(cfg):
         assert torch.equal(got["out"][sl], inp["v"][sl])
         assert torch.equal(got["dv"][sl], inp["dout"][sl])
         assert not got["dq"][sl].any() and not got["dk"][sl].any()
+
+
+# ------------------------------------------- sliding-window attention ---
+# ba_swa_fwd / ba_swa_bwd (query i sees keys i - w < j <= i) against the
+# oracle's block rule with block = 1 (pinned to the window rule on the CPU).
+
+def run_gpu_swa(inp, wt):
+    q, k, v, dout = (inp[n].to(DEV) for n in ("q", "k", "v", "dout"))
+    offs = inp["seq_offsets"].to(DEV)
+    out, lse = ba.sliding_window_attention_fwd(q, k, v, offs, wt)
+    dq, dk, dv = ba.sliding_window_attention_bwd(q, k, v, out, lse, dout, offs, wt)
+    torch.cuda.synchronize()
+    return {n: t.cpu() for n, t in dict(out=out, lse=lse, dq=dq, dk=dk, dv=dv).items()}
+
+
+SWA_CASES = [
+    # (head_dim, window in tokens, lengths)
+    (128, 512, [1500, 513, 1, 128, 0, 900]),
+    (64, 100, [250, 99, 101, 640]),
+    (128, 64, [2000, 65, 63, 129]),
+    (128, 1000000, [700, 300]),          # window covers everything: full causal
+]
+
+
+@pytest.mark.parametrize("head_dim,wt,lengths", SWA_CASES)
+@pytest.mark.parametrize("peaked", [False, True], ids=["config", "peaked"])
+def test_sliding_window(head_dim, wt, lengths, peaked):
+    w = CONFIGS[3].replace(head_dim=head_dim, heads=2, batch=len(lengths))
+    q_gain = 1.0
+    if peaked:
+        w = w.replace(qkv_scale=1.0)
+        q_gain = 3.0
+    inp = make_inputs(w, q_gain=q_gain, lengths=lengths, seed=500 + wt % 997 + head_dim)
+    got = run_gpu_swa(inp, wt)
+    ref = run_oracle(inp, 1, wt)
+    compare(got, ref, peaked=peaked)
+
+
+def test_sliding_window_full_size_sampled():
+    """Config 3 shapes (256 jagged histories, H8 D128) with a 512-token window, sampled rows."""
+    w = CONFIGS[3]
+    wt = 512
+    inp = make_inputs(w)
+    got = run_gpu_swa(inp, wt)
+    offs = inp["seq_offsets"].numpy()
+    lens = np.diff(offs)
+    rng = np.random.default_rng(512)
+    picks = sorted({0, w.batch - 1, *rng.choice(w.batch, size=2, replace=False)})
+    for e in picks:
+        s0, L = int(offs[e]), int(lens[e])
+        sl = slice(s0, s0 + L)
+        qe, ke, ve, de = (f64(inp[n][sl]) for n in ("q", "k", "v", "dout"))
+        for h in (0, w.heads - 1):
+            rows = sample_rows(L, wt, rng)
+            ref = oracle.rows(qe, ke, ve, h, rows, 1, wt, dout_e=de, want=("out", "lse", "dq", "dk", "dv"))
+            for n in ("out", "dq", "dk", "dv"):
+                check_bf16(f"swa e{e} h{h} {n}", f64(got[n][sl][rows, h]), ref[n])
+            check_abs(f"swa e{e} h{h} lse", f64(got["lse"][h, s0:s0 + L][rows]), ref["lse"], 2e-3)
