@@ -223,6 +223,19 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def job_totals(flops, tokens, ms, dist=None, device="cpu"):
+    """Whole-job aggregate over ranks: useful FLOPs and tokens are summed, the
+    time is the slowest rank's (each rank runs its own batch; nothing else is
+    exchanged)."""
+    totals = torch.tensor([flops, tokens, ms], dtype=torch.float64, device=device)
+    if dist is not None:
+        mx = totals[2:].clone()
+        dist.all_reduce(totals, op=dist.ReduceOp.SUM)
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        totals[2] = mx[0]
+    return tuple(float(x) for x in totals.tolist())
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -315,14 +328,7 @@ def main():
     if ba.ba_device_status(ws_f) != ba.BA_OK or ba.ba_device_status(ws_b) != ba.BA_OK:
         raise RuntimeError("a kernel timed out during the timed steps")
 
-    # whole job: useful FLOPs summed over ranks, time = max over ranks
-    totals = torch.tensor([fl["step"] * K, T * K, ms_total], dtype=torch.float64, device=dev)
-    if dist is not None:
-        mx = totals[2:].clone()
-        dist.all_reduce(totals, op=dist.ReduceOp.SUM)
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        totals[2] = mx[0]
-    job_flops, job_tokens, ms_max = (float(x) for x in totals.tolist())
+    job_flops, job_tokens, ms_max = job_totals(fl["step"] * K, T * K, ms_total, dist, dev)
     value = job_flops / (ms_max / 1e3) / 1e12
 
     # end to end through the same API: pinned host in, results out
