@@ -73,7 +73,7 @@ struct DkvLayout {
 };
 
 struct DkvBarriers {
-    uint64_t k_full, k_empty, v_full, v_empty, dkv_full, dkv_free;
+    uint64_t k_full, k_empty, v_full, v_empty, dkv_full, dv_free, dk_free;
     uint64_t q_full[4], q_empty[4], o_full[4], o_empty[4];
     uint64_t s_full, dp_full, pa_done[2], pb_done[2];
     uint64_t epi_sync; // group barrier of the epilogue warps
@@ -116,7 +116,8 @@ __global__ void __launch_bounds__(448, 1)
         mbar_init(&sb.v_full, 1);
         mbar_init(&sb.v_empty, 1);
         mbar_init(&sb.dkv_full, 1);
-        mbar_init(&sb.dkv_free, 4);
+        mbar_init(&sb.dv_free, 4);
+        mbar_init(&sb.dk_free, 4);
         for (int i = 0; i < 4; ++i) {
             mbar_init(&sb.q_full[i], 1 + 32); // the Q tile's expect_tx arrival + one per lane's copies
             mbar_init(&sb.q_empty[i], 1);
@@ -304,7 +305,10 @@ __global__ void __launch_bounds__(448, 1)
                                                                 : Lay::kQ0 + slot * Lay::kTileBytes);
                 for (int g = 0; g < 2; ++g) {
                     if (!mbar_wait(phase == 0 ? &sb.pa_done[g] : &sb.pb_done[g], it & 1, abort)) return false;
-                    if (phase == 0 && m == 0 && g == 0 && !mbar_wait(&sb.dkv_free, (item_cnt & 1) ^ 1, abort))
+                    // the first product of an item overwrites the accumulator: the epilogue
+                    // must have read the previous item's (dV and dK are released separately)
+                    if (m == 0 && g == 0 &&
+                        !mbar_wait(phase == 0 ? &sb.dv_free : &sb.dk_free, (item_cnt & 1) ^ 1, abort))
                         return false;
                     tc_fence_after();
                     {
@@ -467,10 +471,10 @@ __global__ void __launch_bounds__(448, 1)
                 tmem_wait_ld();
                 reg_fence(rr[0]);
                 reg_fence(rr[1]);
-                if (part == 2 * Lay::kChunks - 1) { // every accumulator column read: the next item may start
+                if (c == Lay::kChunks - 1) { // all of dV (or dK) read: the next item may accumulate into it
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sb.dkv_free);
+                    if (lane == 0) mbar_arrive(is_k ? &sb.dk_free : &sb.dv_free);
                 }
                 uint32_t pk[32];
 #pragma unroll
