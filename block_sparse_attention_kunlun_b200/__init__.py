@@ -79,6 +79,8 @@ def _load():
     lib.ba_set_profile_events.restype = ctypes.c_int
     lib.ba_version.argtypes = []
     lib.ba_version.restype = ctypes.c_int32
+    lib.ba_selftest_wait_timeout.argtypes = [P, ctypes.c_size_t, i32, P]
+    lib.ba_selftest_wait_timeout.restype = ctypes.c_int
     lib.ba_swa_fwd_workspace_size.argtypes = [prob, i32]
     lib.ba_swa_fwd_workspace_size.restype = ctypes.c_size_t
     lib.ba_swa_bwd_workspace_size.argtypes = [prob, i32]
@@ -200,6 +202,14 @@ def ba_set_profile_events(which: int, start=None, stop=None) -> int:
     if (start is not None and not s) or (stop is not None and not e):
         raise ValueError("record each event once before handing it to the library")
     return int(_load().ba_set_profile_events(int(which), s, e))
+
+
+def ba_selftest_wait_timeout(workspace, limit_us: int, workspace_bytes=None, stream=None) -> int:
+    """Launch the bounded-wait self-test (a wait that must time out); returns its status code."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(_load().ba_selftest_wait_timeout(_ptr(workspace), int(workspace_bytes), int(limit_us),
+                                                _stream(stream)))
 
 
 def ba_device_status(workspace, stream=None) -> int:

@@ -290,6 +290,17 @@ ba_status ba_device_status(const void *workspace, ba_stream_t stream_)
     return (word & kStatusTimeout) ? BA_ERR_TIMEOUT : BA_OK;
 }
 
+ba_status ba_selftest_wait_timeout(void *workspace, size_t workspace_bytes, int32_t limit_us, ba_stream_t stream_)
+{
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < 256 || limit_us < 1 || limit_us > 1000000)
+        return BA_ERR_INVALID_ARG;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int *status = static_cast<int *>(workspace);
+    if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return BA_ERR_CUDA;
+    BA_TRY(launch_wait_selftest(status, uint64_t(limit_us) * 1000, stream));
+    return BA_OK;
+}
+
 ba_status ba_set_profile_events(int32_t which, void *start, void *stop)
 {
     if (which < 0 || which > 2) return BA_ERR_INVALID_ARG;

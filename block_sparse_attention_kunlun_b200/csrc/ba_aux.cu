@@ -6,12 +6,16 @@
 //                     accumulator
 //   dq_convert_kernel dq = scale * dq_acc, transposed from [H, T, D] to
 //                     [T, H, D] and rounded to the output dtype
+//   wait_selftest_kernel  one warp waits on a barrier nothing completes, with a
+//                     short limit, through the same bounded wait the attention
+//                     kernels use, and reports the timeout in the status word
 //   skip_*_kernel     component skip: flagged examples pass v through
 //                     ("Meta Scales GEM Ads Model Across Platforms and
 //                     Thousands of GPUs", section "Kunlun changes how GEM
 //                     scales": sequence modules bypassed selectively)
 #include "ba_common.cuh"
 #include "ba_kernels.cuh"
+#include "ba_ptx.cuh"
 
 #include <cuda_bf16.h>
 
@@ -264,6 +268,26 @@ cudaError_t launch_skip_bwd(const Problem &p, size_t elem_bytes, const void *dou
                                                          static_cast<const uint8_t *>(dout),
                                                          static_cast<uint8_t *>(dq), static_cast<uint8_t *>(dk),
                                                          static_cast<uint8_t *>(dv));
+    return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(32) wait_selftest_kernel(int *status, uint64_t limit_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort = 0;
+        fence_mbar_init();
+    }
+    __syncwarp();
+    // nothing ever arrives on `bar`
+    if (!mbar_wait(&bar, 0, &abort, limit_ns) && threadIdx.x == 0) atomicOr(status, kStatusTimeout);
+}
+
+cudaError_t launch_wait_selftest(int *status, uint64_t limit_ns, cudaStream_t stream)
+{
+    wait_selftest_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
     return cudaGetLastError();
 }
 

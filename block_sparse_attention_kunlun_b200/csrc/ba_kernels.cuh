@@ -10,6 +10,7 @@
 namespace ba {
 
 cudaError_t launch_worklist(const Problem &p, cudaStream_t stream);
+cudaError_t launch_wait_selftest(int *status, uint64_t limit_ns, cudaStream_t stream);
 
 template <typename T>
 cudaError_t launch_bwd_pre(const Problem &p, const void *out, const void *dout, float *delta, float *dq_acc,

@@ -63,9 +63,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 }
 
 // One lane's wait for the phase of `bar` with the given parity to complete.
-// Returns false (after setting *abort) if the wait ran past kWaitLimitNs or
+// Returns false (after setting *abort) if the wait ran past limit_ns or
 // another thread of the CTA already gave up.
-__device__ __forceinline__ bool mbar_wait_lane(uint64_t *bar, uint32_t parity, volatile int *abort)
+__device__ __forceinline__ bool mbar_wait_lane(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                               uint64_t limit_ns = kWaitLimitNs)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
@@ -74,7 +75,7 @@ __device__ __forceinline__ bool mbar_wait_lane(uint64_t *bar, uint32_t parity, v
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             *abort = 1;
             return false;
         }
@@ -85,9 +86,10 @@ __device__ __forceinline__ bool mbar_wait_lane(uint64_t *bar, uint32_t parity, v
 // all 32 lanes of a warp: every lane waits and the result is made uniform, so
 // that after a timeout no lane is left behind at a warp-collective
 // instruction (elect.sync, tcgen05.ld, shuffles) that the others never reach.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          uint64_t limit_ns = kWaitLimitNs)
 {
-    return __all_sync(0xffffffffu, mbar_wait_lane(bar, parity, abort));
+    return __all_sync(0xffffffffu, mbar_wait_lane(bar, parity, abort, limit_ns));
 }
 
 // Barrier over a group of threads, on an mbarrier initialised with the group's

@@ -173,6 +173,21 @@ ba_status ba_fwd_noalloc(const ba_problem *p, const void *q, const void *k, cons
 ba_status ba_device_status(const void *workspace, ba_stream_t stream);
 
 /*
+ * Self-test of the bounded waits (the pages have no counterpart; this checks
+ * the library's own failure detection without faulting anything). Every
+ * wait in the attention kernels gives up after 2 s, makes the kernel return,
+ * and sets the workspace status word that ba_device_status reports as
+ * BA_ERR_TIMEOUT. This launches one warp that waits, through that same code,
+ * on a barrier nothing ever completes, with a limit of limit_us microseconds
+ * (1 .. 1,000,000). Afterwards ba_device_status(workspace) returns
+ * BA_ERR_TIMEOUT and the device stays usable. workspace: at least 256 bytes,
+ * 256-byte aligned; its status word is overwritten. Returns
+ * BA_ERR_INVALID_ARG for bad arguments (nothing launched).
+ */
+ba_status ba_selftest_wait_timeout(void *workspace, size_t workspace_bytes, int32_t limit_us,
+                                   ba_stream_t stream);
+
+/*
  * Profiling hook. Until changed, calls made from THIS host thread record
  * `start` on their stream right before one kernel and `stop` right after it,
  * so that cudaEventElapsedTime(start, stop) is that kernel's own duration:
