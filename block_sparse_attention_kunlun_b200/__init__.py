@@ -21,8 +21,10 @@ import torch
 
 __all__ = [
     "BAError", "ba_fwd", "ba_fwd_noalloc", "ba_bwd", "ba_fwd_workspace_size", "ba_bwd_workspace_size",
-    "ba_device_status", "ba_set_profile_events", "ba_status_string", "ba_version", "block_attention_fwd",
-    "block_attention_bwd", "library_path",
+    "ba_swa_fwd", "ba_swa_bwd", "ba_swa_fwd_workspace_size", "ba_swa_bwd_workspace_size",
+    "ba_device_status", "ba_selftest_wait_timeout", "ba_set_profile_events", "ba_status_string", "ba_version",
+    "block_attention_fwd", "block_attention_bwd", "sliding_window_attention_fwd", "sliding_window_attention_bwd",
+    "library_path",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
