@@ -141,13 +141,13 @@ extern "C" {
 size_t ba_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
 {
     if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
-    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, false, false).total;
+    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, false).total;
 }
 
 size_t ba_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
 {
     if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
-    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, true, false).total;
+    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, true).total;
 }
 
 ba_status ba_fwd(const ba_problem *pp, const void *q, const void *k, const void *v, const int32_t *seq_offsets,
@@ -161,7 +161,7 @@ ba_status ba_fwd(const ba_problem *pp, const void *q, const void *k, const void 
     if (!seq_offsets || !aligned(seq_offsets, 4) || !tensor_ok(q, T) || !tensor_ok(k, T) || !tensor_ok(v, T) ||
         !tensor_ok(out, T) || (T > 0 && (!lse || !aligned(lse, 4))))
         return BA_ERR_INVALID_ARG;
-    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, false, false);
+    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, false);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total) return BA_ERR_INVALID_ARG;
     int num_sms = 0, cc = 0;
     if (!device_info(num_sms, cc)) return BA_ERR_CUDA;
@@ -205,7 +205,7 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
         (T > 0 && (!lse || !aligned(lse, 4))))
         return BA_ERR_INVALID_ARG;
     const bool bf16 = P.dtype == BA_BF16;
-    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, true, false);
+    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, true);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total) return BA_ERR_INVALID_ARG;
     int num_sms = 0, cc = 0;
     if (!device_info(num_sms, cc)) return BA_ERR_CUDA;
@@ -221,7 +221,7 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
     const size_t esz = bf16 ? 2 : 4;
     BA_TRY(launch_skip_bwd(p, esz, dout, dq, dk, dv, stream));
     if (!bf16) {
-        BA_TRY(launch_bwd_pre<float>(p, out, dout, delta, nullptr, num_sms, stream));
+        BA_TRY(launch_bwd_pre<float>(p, out, dout, delta, num_sms, stream));
         BA_TRY(prof_mark(1, 0, stream));
         BA_TRY(launch_bwd_f32(p, static_cast<const float *>(q), static_cast<const float *>(k),
                               static_cast<const float *>(v), static_cast<const float *>(dout), lse, delta,

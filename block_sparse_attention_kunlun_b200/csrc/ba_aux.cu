@@ -2,10 +2,8 @@
 //   worklist_kernel   per-example count of live 128-row tiles -> exclusive
 //                     prefix sum (the persistent kernels' work list); resets
 //                     the status word
-//   bwd_pre_kernel    Delta = rowsum(dout * out) in fp32; zeroes the fp32 dq
-//                     accumulator
-//   dq_convert_kernel dq = scale * dq_acc, transposed from [H, T, D] to
-//                     [T, H, D] and rounded to the output dtype
+//   bwd_pre_kernel    Delta = rowsum(dout * out) in fp32 (the fp32 path; the
+//                     bf16 dQ pass computes Delta itself)
 //   wait_selftest_kernel  one warp waits on a barrier nothing completes, with a
 //                     short limit, through the same bounded wait the attention
 //                     kernels use, and reports the timeout in the status word
@@ -32,9 +30,6 @@ __device__ __forceinline__ int32_t live_tiles(const int32_t *offs, const uint8_t
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
-template <typename T> __device__ __forceinline__ T from_f32(float x);
-template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
-template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
 } // namespace
 
@@ -108,7 +103,7 @@ __global__ void __launch_bounds__(kWorklistThreads)
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
     bwd_pre_kernel(const T *__restrict__ out, const T *__restrict__ dout, int32_t total_tokens,
-                   int32_t heads, float *__restrict__ delta, float *__restrict__ dq_acc)
+                   int32_t heads, float *__restrict__ delta)
 {
     constexpr int PER = D / 32;
     const int lane = threadIdx.x & 31;
@@ -125,29 +120,6 @@ __global__ void __launch_bounds__(256)
         for (int d = 16; d > 0; d >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
         const int64_t hr = h * total_tokens + t;
         if (lane == 0) delta[hr] = acc;
-        if (dq_acc) {
-            float *z = dq_acc + hr * D + lane * PER;
-#pragma unroll
-            for (int x = 0; x < PER; ++x) z[x] = 0.f;
-        }
-    }
-}
-
-template <typename T, int D>
-__global__ void __launch_bounds__(256)
-    dq_convert_kernel(const float *__restrict__ dq_acc, int32_t total_tokens, int32_t heads, float scale,
-                      T *__restrict__ dq)
-{
-    constexpr int PER = D / 32;
-    const int lane = threadIdx.x & 31;
-    const int64_t nrows = int64_t(total_tokens) * heads;
-    const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
-    for (int64_t rw = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); rw < nrows; rw += wstride) {
-        const int64_t t = rw / heads, h = rw % heads;
-        const float *a = dq_acc + (h * total_tokens + t) * D + lane * PER;
-        T *o = dq + rw * D + lane * PER;
-#pragma unroll
-        for (int x = 0; x < PER; ++x) o[x] = from_f32<T>(a[x] * scale);
     }
 }
 
@@ -216,33 +188,17 @@ static int grid_for_rows(int64_t nrows, int num_sms)
 }
 
 template <typename T>
-cudaError_t launch_bwd_pre(const Problem &p, const void *out, const void *dout, float *delta, float *dq_acc,
-                           int num_sms, cudaStream_t stream)
+cudaError_t launch_bwd_pre(const Problem &p, const void *out, const void *dout, float *delta, int num_sms,
+                           cudaStream_t stream)
 {
     const int64_t nrows = int64_t(p.total_tokens) * p.heads;
     if (nrows == 0) return cudaSuccess;
     const int g = grid_for_rows(nrows, num_sms);
     const T *o = static_cast<const T *>(out), *d = static_cast<const T *>(dout);
     switch (p.head_dim) {
-    case 32: bwd_pre_kernel<T, 32><<<g, 256, 0, stream>>>(o, d, p.total_tokens, p.heads, delta, dq_acc); break;
-    case 64: bwd_pre_kernel<T, 64><<<g, 256, 0, stream>>>(o, d, p.total_tokens, p.heads, delta, dq_acc); break;
-    case 128: bwd_pre_kernel<T, 128><<<g, 256, 0, stream>>>(o, d, p.total_tokens, p.heads, delta, dq_acc); break;
-    default: return cudaErrorInvalidValue;
-    }
-    return cudaGetLastError();
-}
-
-template <typename T>
-cudaError_t launch_dq_convert(const Problem &p, const float *dq_acc, void *dq, int num_sms, cudaStream_t stream)
-{
-    const int64_t nrows = int64_t(p.total_tokens) * p.heads;
-    if (nrows == 0) return cudaSuccess;
-    const int g = grid_for_rows(nrows, num_sms);
-    T *o = static_cast<T *>(dq);
-    switch (p.head_dim) {
-    case 32: dq_convert_kernel<T, 32><<<g, 256, 0, stream>>>(dq_acc, p.total_tokens, p.heads, p.scale, o); break;
-    case 64: dq_convert_kernel<T, 64><<<g, 256, 0, stream>>>(dq_acc, p.total_tokens, p.heads, p.scale, o); break;
-    case 128: dq_convert_kernel<T, 128><<<g, 256, 0, stream>>>(dq_acc, p.total_tokens, p.heads, p.scale, o); break;
+    case 32: bwd_pre_kernel<T, 32><<<g, 256, 0, stream>>>(o, d, p.total_tokens, p.heads, delta); break;
+    case 64: bwd_pre_kernel<T, 64><<<g, 256, 0, stream>>>(o, d, p.total_tokens, p.heads, delta); break;
+    case 128: bwd_pre_kernel<T, 128><<<g, 256, 0, stream>>>(o, d, p.total_tokens, p.heads, delta); break;
     default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
@@ -291,11 +247,8 @@ cudaError_t launch_wait_selftest(int *status, uint64_t limit_ns, cudaStream_t st
     return cudaGetLastError();
 }
 
-template cudaError_t launch_bwd_pre<float>(const Problem &, const void *, const void *, float *, float *, int,
-                                           cudaStream_t);
-template cudaError_t launch_bwd_pre<__nv_bfloat16>(const Problem &, const void *, const void *, float *, float *,
-                                                   int, cudaStream_t);
-template cudaError_t launch_dq_convert<float>(const Problem &, const float *, void *, int, cudaStream_t);
-template cudaError_t launch_dq_convert<__nv_bfloat16>(const Problem &, const float *, void *, int, cudaStream_t);
+template cudaError_t launch_bwd_pre<float>(const Problem &, const void *, const void *, float *, int, cudaStream_t);
+template cudaError_t launch_bwd_pre<__nv_bfloat16>(const Problem &, const void *, const void *, float *, int,
+                                                   cudaStream_t);
 
 } // namespace ba

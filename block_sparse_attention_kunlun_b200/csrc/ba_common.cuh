@@ -52,10 +52,11 @@ __host__ __device__ __forceinline__ bool visible(int64_t i, int64_t j, int64_t b
 //   pair_prefix         int32[batch + 1]: live pairs of consecutive tiles
 //   pair_info           int4[max_pairs]: per pair {row0, length, first tile,
 //                       example}, max_pairs = ceil(T / 256) + batch
-//   delta   (bwd only)  float[heads * total_tokens]
-//   dq_acc  (bwd only)  float[heads * total_tokens * head_dim]
+//   delta   (bwd only)  float[heads * total_tokens]: Delta (fp32 path) or -Delta
+//                       (bf16 path, written by the dQ pass for the dK/dV pass)
+//   nlse2   (bwd only)  float[heads * total_tokens]: -lse in log2 units (bf16 path)
 struct WorkspaceLayout {
-    size_t status, tile_prefix, tile_info, pair_prefix, pair_info, delta, nlse2, dq_acc, total;
+    size_t status, tile_prefix, tile_info, pair_prefix, pair_info, delta, nlse2, total;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -72,7 +73,7 @@ __host__ __device__ inline int64_t max_pairs(int64_t batch, int64_t total_tokens
 
 __host__ __device__ inline WorkspaceLayout workspace_layout(int64_t batch, int64_t total_tokens,
                                                             int64_t heads, int64_t head_dim,
-                                                            bool with_delta, bool with_dq_acc)
+                                                            bool with_delta)
 {
     WorkspaceLayout w;
     w.status = 0;
@@ -89,8 +90,6 @@ __host__ __device__ inline WorkspaceLayout workspace_layout(int64_t batch, int64
     if (with_delta) off = align256(off + sizeof(float) * size_t(heads * total_tokens));
     w.nlse2 = off;
     if (with_delta) off = align256(off + sizeof(float) * size_t(heads * total_tokens));
-    w.dq_acc = off;
-    if (with_dq_acc) off = align256(off + sizeof(float) * size_t(heads * total_tokens * head_dim));
     w.total = off;
     return w;
 }

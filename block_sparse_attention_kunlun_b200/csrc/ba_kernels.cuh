@@ -13,10 +13,8 @@ cudaError_t launch_worklist(const Problem &p, cudaStream_t stream);
 cudaError_t launch_wait_selftest(int *status, uint64_t limit_ns, cudaStream_t stream);
 
 template <typename T>
-cudaError_t launch_bwd_pre(const Problem &p, const void *out, const void *dout, float *delta, float *dq_acc,
-                           int num_sms, cudaStream_t stream);
-template <typename T>
-cudaError_t launch_dq_convert(const Problem &p, const float *dq_acc, void *dq, int num_sms, cudaStream_t stream);
+cudaError_t launch_bwd_pre(const Problem &p, const void *out, const void *dout, float *delta, int num_sms,
+                           cudaStream_t stream);
 
 cudaError_t launch_skip_fwd(const Problem &p, size_t elem_bytes, const void *v, void *out, float *lse,
                             cudaStream_t stream);
