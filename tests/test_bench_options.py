@@ -1,0 +1,47 @@
+"""bench.py's workload selection: --swa W runs the sliding window (block 1, window W) and
+--block/--window override the block rule, on the config's own shapes and seeds."""
+import importlib.util
+import os
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+class Args:
+    config, examples, swa, block, window = 3, 0, 0, 0, 0
+
+
+def test_default_is_the_configured_workload():
+    b = _bench()
+    w = b.config_workload(Args())
+    assert (w.block, w.window) == (256, 2) and "block 256, window 2" in w.name
+
+
+def test_sliding_window_option():
+    b = _bench()
+    a = Args()
+    a.swa = 512
+    w = b.config_workload(a)
+    assert (w.block, w.window) == (1, 512)
+    assert "sliding window 512 tokens" in w.name and "block 256" not in w.name
+    base = b.config_workload(Args())
+    assert (w.batch, w.heads, w.head_dim, w.seed) == (base.batch, base.heads, base.head_dim, base.seed)
+
+
+def test_block_window_overrides():
+    b = _bench()
+    a = Args()
+    a.block, a.window = 64, 1
+    w = b.config_workload(a)
+    assert (w.block, w.window) == (64, 1) and "block 64, window 1" in w.name
+
+
+def test_job_totals_single_rank_is_identity():
+    b = _bench()
+    assert b.job_totals(5.0, 7.0, 3.0) == (5.0, 7.0, 3.0)
