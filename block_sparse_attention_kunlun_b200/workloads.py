@@ -1,7 +1,8 @@
 """Seeded synthetic inputs for block attention.
 
-This module only draws random numbers; it holds none of the attention
-arithmetic, so both the CUDA path and the CPU oracle can be fed from it.
+This module only draws random numbers and builds the rotary tables a
+caller supplies; it holds none of the attention arithmetic, so both the CUDA
+path and the CPU oracle can be fed from it.
 
 The pages describe the workload only in words: user-engagement histories
 whose lengths run from hundreds to tens of thousands of events, batched as
@@ -107,3 +108,14 @@ def make_inputs(w: Workload, seed: int | None = None, q_gain: float = 1.0,
     if want_dout if want_dout is not None else not w.fwd_only:
         out["dout"] = normal(1.0)
     return out
+
+
+def rope_tables(rows: int, head_dim: int, base: float = 10000.0):
+    """cos and sin tables, float32 [rows, head_dim / 2], for rotary position
+    embeddings with RoFormer's frequencies: entry [p, k] is the cosine (sine)
+    of p * base ** (-2k / head_dim). Angles are formed in float64 and the
+    results rounded to float32 (the tables the library reads)."""
+    p = torch.arange(rows, dtype=torch.float64)[:, None]
+    inv_freq = base ** (-2.0 * torch.arange(head_dim // 2, dtype=torch.float64) / head_dim)
+    ang = p * inv_freq[None, :]
+    return torch.cos(ang).to(torch.float32), torch.sin(ang).to(torch.float32)

@@ -16,6 +16,16 @@ infrastructure").
 Every function takes numpy arrays: q, k, v, dout as float64 [T, H, D]
 (C-contiguous), seq_offsets as int32 [batch + 1], skip as uint8 [batch] or
 None. Pins: tests/test_oracle.py.
+
+Rotary position embedding (``rope_*``; "GEM (Meta)", section "Custom
+kernels": the production block-attention kernel fuses the backward pass of
+the rotary position embedding; the pages say nothing more about it). The
+reading used here and in the library is RoFormer's rotation applied to q and
+k (not v) before the scores: the adjacent pair (x[2k], x[2k+1]) of a row at
+position p is turned by the angle whose cosine and sine the caller's tables
+hold at [p, k]; p is the row's index within its example, the origin the
+blocks use. The gradient with respect to the unrotated q (k) is the
+transposed rotation of the gradient with respect to the rotated q (k).
 """
 from __future__ import annotations
 
@@ -24,6 +34,7 @@ import os
 import subprocess
 
 import numpy as np
+import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
@@ -144,4 +155,90 @@ def rows(q_e, k_e, v_e, head, rows_idx, block, window, dout_e=None,
                              int(nthreads or default_threads()))
     if rc != 0:
         raise RuntimeError(f"oracle_rows failed ({rc})")
+    return res
+
+
+# ------------------------------------------------------------ rotary ---
+
+def positions(seq_offsets):
+    """Local position of every row: its index within its own example."""
+    offs = np.asarray(seq_offsets, dtype=np.int64)
+    lens = np.diff(offs)
+    return np.arange(int(offs[-1]), dtype=np.int64) - np.repeat(offs[:-1], lens)
+
+
+def _rotate_at(x, pos, cos, sin, transpose):
+    """Rotate the adjacent pairs of rows x[n, ..., D] sitting at positions pos[n]:
+    y[2k] = x[2k] c - x[2k+1] s, y[2k+1] = x[2k] s + x[2k+1] c with c, s the
+    tables' entries at [pos, k]. transpose=True applies the transposed 2 x 2
+    map instead (c, s) -> (c, -s), which takes a gradient with respect to y
+    to the gradient with respect to x; it is also the inverse when the
+    tables hold exact cosines and sines."""
+    x = _f64(x)
+    cos = np.asarray(cos, dtype=np.float64)
+    sin = np.asarray(sin, dtype=np.float64)
+    D = x.shape[-1]
+    if D % 2 or cos.ndim != 2 or cos.shape[1] != D // 2 or sin.shape != cos.shape:
+        raise ValueError("rotary tables must be [rows, head_dim / 2] with an even head_dim")
+    pos = np.asarray(pos, dtype=np.int64)
+    if pos.size and (pos.min() < 0 or pos.max() >= cos.shape[0]):
+        raise ValueError("rotary tables are shorter than an example")
+    shape = (pos.shape[0],) + (1,) * (x.ndim - 2) + (D // 2,)
+    c = cos[pos].reshape(shape)
+    s = sin[pos].reshape(shape)
+    if transpose:
+        s = -s
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    y = np.empty_like(x)
+    y[..., 0::2] = x0 * c - x1 * s
+    y[..., 1::2] = x0 * s + x1 * c
+    return y
+
+
+def rope_rotate(x, seq_offsets, cos, sin, transpose=False):
+    """Rotary embedding of every row of x [T, H, D] at its local position
+    (transpose=True: the transposed rotation, see _rotate_at)."""
+    return _rotate_at(x, positions(seq_offsets), cos, sin, transpose)
+
+
+def _as_operand(x, operand_dtype):
+    """Round the rotated operand to the dtype the products run in (None: keep fp64)."""
+    if operand_dtype is None:
+        return x
+    return torch.from_numpy(x).to(operand_dtype).to(torch.float64).numpy()
+
+
+def rope_fwd(seq_offsets, q, k, v, cos, sin, block, window, skip=None, operand_dtype=None, nthreads=None):
+    """Block attention of the rotated q and k. operand_dtype (e.g.
+    torch.bfloat16) rounds the rotated q and k to that dtype first, as a
+    library that feeds them to tensor-core products in the input dtype does."""
+    qr = _as_operand(rope_rotate(q, seq_offsets, cos, sin), operand_dtype)
+    kr = _as_operand(rope_rotate(k, seq_offsets, cos, sin), operand_dtype)
+    return fwd(seq_offsets, qr, kr, v, block, window, skip=skip, nthreads=nthreads)
+
+
+def rope_bwd(seq_offsets, q, k, v, dout, cos, sin, block, window, skip=None, operand_dtype=None,
+             nthreads=None):
+    """Gradients of rope_fwd: dv as for plain attention, dq and dk the
+    transposed rotations of the gradients with respect to the rotated q and
+    k (the rounding of operand_dtype counts as the identity)."""
+    qr = _as_operand(rope_rotate(q, seq_offsets, cos, sin), operand_dtype)
+    kr = _as_operand(rope_rotate(k, seq_offsets, cos, sin), operand_dtype)
+    dqr, dkr, dv = bwd(seq_offsets, qr, kr, v, dout, block, window, skip=skip, nthreads=nthreads)
+    return (rope_rotate(dqr, seq_offsets, cos, sin, transpose=True),
+            rope_rotate(dkr, seq_offsets, cos, sin, transpose=True), dv)
+
+
+def rope_rows(q_e, k_e, v_e, cos, sin, head, rows_idx, block, window, dout_e=None,
+              want=("out", "lse"), operand_dtype=None, nthreads=None):
+    """``rows`` for the rotated attention of one example (rows [L, H, D])."""
+    L = _f64(q_e).shape[0]
+    offs = np.array([0, L], dtype=np.int32)
+    qr = _as_operand(rope_rotate(q_e, offs, cos, sin), operand_dtype)
+    kr = _as_operand(rope_rotate(k_e, offs, cos, sin), operand_dtype)
+    res = rows(qr, kr, v_e, head, rows_idx, block, window, dout_e=dout_e, want=want, nthreads=nthreads)
+    pos = np.asarray(rows_idx, dtype=np.int64)
+    for name in ("dq", "dk"):
+        if name in res:
+            res[name] = _rotate_at(res[name], pos, cos, sin, transpose=True)
     return res

@@ -352,3 +352,144 @@ def test_sliding_window_gradients_match_masked_sdpa():
     o.backward(torch.tensor(do.transpose(1, 0, 2)))
     for name, got, ref in (("dq", dq, tq.grad), ("dk", dk, tk.grad), ("dv", dv, tv.grad)):
         np.testing.assert_allclose(got, ref.numpy().transpose(1, 0, 2), rtol=0, atol=1e-11, err_msg=name)
+
+
+# ------------------------------------------------- rotary embedding ---
+# Rotary position embedding on q and k ("GEM (Meta)", "Custom kernels": the
+# block-attention kernel fuses the backward pass of the rotary embedding).
+# RoFormer writes the rotation as a complex multiplication: the pair
+# (x[2k], x[2k+1]) read as x[2k] + i x[2k+1] is multiplied by exp(i p theta_k).
+# These pins check the oracle's real-arithmetic form against that, against
+# autograd through it, and against the relative-position property it exists
+# for.
+
+def _exact_tables(rows, D, base=10000.0):
+    ang = np.arange(rows, dtype=np.float64)[:, None] * base ** (-2.0 * np.arange(D // 2) / D)[None, :]
+    return np.cos(ang), np.sin(ang), ang
+
+
+def _complex_rotate(x, pos, ang):
+    z = x[..., 0::2] + 1j * x[..., 1::2]
+    z = z * np.exp(1j * ang[pos])[:, None, :]
+    y = np.empty_like(x)
+    y[..., 0::2] = z.real
+    y[..., 1::2] = z.imag
+    return y
+
+
+def test_rope_rotation_is_complex_multiplication():
+    rng = np.random.default_rng(500)
+    offs, q, _, _, _ = rand_case(rng, [17, 0, 40, 5], 3, 8)
+    cos, sin, ang = _exact_tables(64, 8)
+    pos = np.concatenate([np.arange(17), np.arange(40), np.arange(5)])
+    np.testing.assert_allclose(oracle.rope_rotate(q, offs, cos, sin), _complex_rotate(q, pos, ang),
+                               rtol=0, atol=1e-13)
+    # the transpose turns by the opposite angle: multiplication by the conjugate
+    np.testing.assert_allclose(oracle.rope_rotate(q, offs, cos, sin, transpose=True),
+                               _complex_rotate(q, pos, -ang), rtol=0, atol=1e-13)
+
+
+def test_rope_transpose_undoes_rotation_and_keeps_pair_norms():
+    rng = np.random.default_rng(501)
+    offs, q, _, _, _ = rand_case(rng, [33, 12], 2, 16)
+    cos, sin, _ = _exact_tables(40, 16)
+    y = oracle.rope_rotate(q, offs, cos, sin)
+    np.testing.assert_allclose(oracle.rope_rotate(y, offs, cos, sin, transpose=True), q, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(np.hypot(y[..., 0::2], y[..., 1::2]), np.hypot(q[..., 0::2], q[..., 1::2]),
+                               rtol=1e-13, atol=0)
+
+
+def test_rope_attention_depends_on_relative_position_only():
+    """RoFormer's property: rotating every position by a further constant
+    angle leaves q . k, hence out and lse, unchanged."""
+    rng = np.random.default_rng(502)
+    offs, q, k, v, _ = rand_case(rng, [45, 30], 2, 8, scale=2.0)
+    cos, sin, ang = _exact_tables(100, 8)
+    out0, lse0 = oracle.rope_fwd(offs, q, k, v, cos, sin, 8, 3)
+    out1, lse1 = oracle.rope_fwd(offs, q, k, v, np.cos(ang[37:]), np.sin(ang[37:]), 8, 3)
+    np.testing.assert_allclose(out1, out0, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse1, lse0, rtol=0, atol=1e-12)
+    # ... while a table that is not a rotation by p * theta does change them
+    out2, _ = oracle.rope_fwd(offs, q, k, v, cos[::-1].copy(), sin[::-1].copy(), 8, 3)
+    assert np.max(np.abs(out2 - out0)) > 1e-3
+
+
+def test_rope_gradients_match_autograd_of_complex_form():
+    """Backward against PyTorch autograd through the complex-number rotation
+    followed by masked attention (fp64), per example, jagged batch."""
+    rng = np.random.default_rng(503)
+    block, window, H, D = 4, 2, 2, 8
+    offs, q, k, v, do = rand_case(rng, [13, 0, 29], H, D, scale=1.5)
+    cos, sin, ang = _exact_tables(32, D)
+    dq, dk, dv = oracle.rope_bwd(offs, q, k, v, do, cos, sin, block, window)
+    out, _ = oracle.rope_fwd(offs, q, k, v, cos, sin, block, window)
+    for e in range(len(offs) - 1):
+        s0, s1 = int(offs[e]), int(offs[e + 1])
+        L = s1 - s0
+        if L == 0:
+            continue
+        i = torch.arange(L)[:, None]
+        j = torch.arange(L)[None, :]
+        mask = (j <= i) & (j // block >= i // block - (window - 1))
+        rot = torch.polar(torch.ones(L, D // 2, dtype=torch.float64),
+                          torch.tensor(ang[:L]))[None, :, :]                      # [1, L, D/2]
+        tq, tk, tv = (torch.tensor(x[s0:s1].transpose(1, 0, 2), dtype=torch.float64, requires_grad=True)
+                      for x in (q, k, v))
+        as_c = lambda t: torch.view_as_complex(t.reshape(H, L, D // 2, 2))
+        as_r = lambda z: torch.view_as_real(z).reshape(H, L, D)
+        o = torch.nn.functional.scaled_dot_product_attention(as_r(as_c(tq) * rot), as_r(as_c(tk) * rot), tv,
+                                                             attn_mask=mask)
+        o.backward(torch.tensor(do[s0:s1].transpose(1, 0, 2)))
+        t = lambda x: x.detach().numpy().transpose(1, 0, 2)
+        np.testing.assert_allclose(out[s0:s1], t(o), rtol=0, atol=1e-12)
+        for name, got, ref in (("dq", dq, tq.grad), ("dk", dk, tk.grad), ("dv", dv, tv.grad)):
+            np.testing.assert_allclose(got[s0:s1], t(ref), rtol=0, atol=1e-11, err_msg=f"{name} example {e}")
+
+
+def test_rope_identity_tables_give_plain_attention():
+    rng = np.random.default_rng(504)
+    offs, q, k, v, do = rand_case(rng, [20, 7], 2, 4)
+    one, zero = np.ones((20, 2)), np.zeros((20, 2))
+    for a, b in zip(oracle.rope_fwd(offs, q, k, v, one, zero, 4, 2), oracle.fwd(offs, q, k, v, 4, 2)):
+        np.testing.assert_array_equal(a, b)
+    for a, b in zip(oracle.rope_bwd(offs, q, k, v, do, one, zero, 4, 2), oracle.bwd(offs, q, k, v, do, 4, 2)):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_rope_positions_restart_in_every_example():
+    """A jagged batch equals each example run alone (positions are local);
+    dq and dk, unlike out, depend on the absolute position, so they would
+    differ if positions ran over the whole batch."""
+    rng = np.random.default_rng(505)
+    offs, q, k, v, do = rand_case(rng, [21, 34], 2, 8)
+    cos, sin, _ = _exact_tables(64, 8)
+    dq, dk, dv = oracle.rope_bwd(offs, q, k, v, do, cos, sin, 8, 2)
+    s = slice(21, 55)
+    one = np.array([0, 34], dtype=np.int32)
+    dq1, dk1, dv1 = oracle.rope_bwd(one, q[s], k[s], v[s], do[s], cos, sin, 8, 2)
+    np.testing.assert_allclose(dq[s], dq1, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dk[s], dk1, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dv[s], dv1, rtol=0, atol=1e-13)
+    glob = np.arange(55)[s]   # rows numbered over the batch instead
+    dq_glob = oracle._rotate_at(oracle.rope_rotate(dq1, one, cos, sin), glob, cos, sin, transpose=True)
+    assert np.max(np.abs(dq_glob - dq[s])) > 1e-3
+
+
+def test_rope_rows_match_full_computation():
+    rng = np.random.default_rng(506)
+    offs, q, k, v, do = rand_case(rng, [70], 2, 8)
+    cos, sin, _ = _exact_tables(80, 8)
+    out, lse = oracle.rope_fwd(offs, q, k, v, cos, sin, 16, 2)
+    dq, dk, dv = oracle.rope_bwd(offs, q, k, v, do, cos, sin, 16, 2)
+    idx = np.array([0, 5, 16, 31, 69])
+    r = oracle.rope_rows(q, k, v, cos, sin, 1, idx, 16, 2, dout_e=do, want=("out", "lse", "dq", "dk", "dv"))
+    for name, full in (("out", out), ("dq", dq), ("dk", dk), ("dv", dv)):
+        np.testing.assert_allclose(r[name], full[idx, 1], rtol=0, atol=1e-13, err_msg=name)
+    np.testing.assert_allclose(r["lse"], lse[1, idx], rtol=0, atol=1e-13)
+
+
+def test_rope_tables_shorter_than_an_example_are_rejected():
+    offs, q, k, v, _ = rand_case(np.random.default_rng(507), [10, 12], 1, 4)
+    cos, sin, _ = _exact_tables(11, 4)
+    with pytest.raises(ValueError):
+        oracle.rope_fwd(offs, q, k, v, cos, sin, 4, 1)
