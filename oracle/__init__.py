@@ -167,13 +167,15 @@ def positions(seq_offsets):
     return np.arange(int(offs[-1]), dtype=np.int64) - np.repeat(offs[:-1], lens)
 
 
-def _rotate_at(x, pos, cos, sin, transpose):
+def _rotate_at(x, pos, cos, sin, transpose, fp32=False):
     """Rotate the adjacent pairs of rows x[n, ..., D] sitting at positions pos[n]:
     y[2k] = x[2k] c - x[2k+1] s, y[2k+1] = x[2k] s + x[2k+1] c with c, s the
     tables' entries at [pos, k]. transpose=True applies the transposed 2 x 2
     map instead (c, s) -> (c, -s), which takes a gradient with respect to y
     to the gradient with respect to x; it is also the inverse when the
-    tables hold exact cosines and sines."""
+    tables hold exact cosines and sines. fp32=True evaluates the same
+    formula in float32, each product and the sum rounded once (used only to
+    decide the bf16 rounding of the rotated operands, see _rotated_operand)."""
     x = _f64(x)
     cos = np.asarray(cos, dtype=np.float64)
     sin = np.asarray(sin, dtype=np.float64)
@@ -189,31 +191,39 @@ def _rotate_at(x, pos, cos, sin, transpose):
     if transpose:
         s = -s
     x0, x1 = x[..., 0::2], x[..., 1::2]
-    y = np.empty_like(x)
+    if fp32:
+        x0, x1, c, s = (a.astype(np.float32) for a in (x0, x1, c, s))
+    y = np.empty(x.shape, dtype=x0.dtype)
     y[..., 0::2] = x0 * c - x1 * s
     y[..., 1::2] = x0 * s + x1 * c
-    return y
+    return y.astype(np.float64)
 
 
-def rope_rotate(x, seq_offsets, cos, sin, transpose=False):
+def rope_rotate(x, seq_offsets, cos, sin, transpose=False, fp32=False):
     """Rotary embedding of every row of x [T, H, D] at its local position
-    (transpose=True: the transposed rotation, see _rotate_at)."""
-    return _rotate_at(x, positions(seq_offsets), cos, sin, transpose)
+    (transpose=True: the transposed rotation; fp32: see _rotate_at)."""
+    return _rotate_at(x, positions(seq_offsets), cos, sin, transpose, fp32)
 
 
-def _as_operand(x, operand_dtype):
-    """Round the rotated operand to the dtype the products run in (None: keep fp64)."""
+def _rotated_operand(x, seq_offsets, cos, sin, operand_dtype):
+    """The rotated q or k as the attention's products take it. None: exact
+    (fp64). A dtype (torch.bfloat16): the rotation rounded to that dtype,
+    nearest even. Which way a value near a rounding tie goes is a
+    quantisation decision, so it is taken in the precision the library
+    takes it in: the float32 value of the formula, each product and the sum
+    rounded once."""
     if operand_dtype is None:
-        return x
-    return torch.from_numpy(x).to(operand_dtype).to(torch.float64).numpy()
+        return rope_rotate(x, seq_offsets, cos, sin)
+    y = rope_rotate(x, seq_offsets, cos, sin, fp32=True).astype(np.float32)
+    return torch.from_numpy(y).to(operand_dtype).to(torch.float64).numpy()
 
 
 def rope_fwd(seq_offsets, q, k, v, cos, sin, block, window, skip=None, operand_dtype=None, nthreads=None):
     """Block attention of the rotated q and k. operand_dtype (e.g.
     torch.bfloat16) rounds the rotated q and k to that dtype first, as a
     library that feeds them to tensor-core products in the input dtype does."""
-    qr = _as_operand(rope_rotate(q, seq_offsets, cos, sin), operand_dtype)
-    kr = _as_operand(rope_rotate(k, seq_offsets, cos, sin), operand_dtype)
+    qr = _rotated_operand(q, seq_offsets, cos, sin, operand_dtype)
+    kr = _rotated_operand(k, seq_offsets, cos, sin, operand_dtype)
     return fwd(seq_offsets, qr, kr, v, block, window, skip=skip, nthreads=nthreads)
 
 
@@ -222,8 +232,8 @@ def rope_bwd(seq_offsets, q, k, v, dout, cos, sin, block, window, skip=None, ope
     """Gradients of rope_fwd: dv as for plain attention, dq and dk the
     transposed rotations of the gradients with respect to the rotated q and
     k (the rounding of operand_dtype counts as the identity)."""
-    qr = _as_operand(rope_rotate(q, seq_offsets, cos, sin), operand_dtype)
-    kr = _as_operand(rope_rotate(k, seq_offsets, cos, sin), operand_dtype)
+    qr = _rotated_operand(q, seq_offsets, cos, sin, operand_dtype)
+    kr = _rotated_operand(k, seq_offsets, cos, sin, operand_dtype)
     dqr, dkr, dv = bwd(seq_offsets, qr, kr, v, dout, block, window, skip=skip, nthreads=nthreads)
     return (rope_rotate(dqr, seq_offsets, cos, sin, transpose=True),
             rope_rotate(dkr, seq_offsets, cos, sin, transpose=True), dv)
@@ -234,8 +244,8 @@ def rope_rows(q_e, k_e, v_e, cos, sin, head, rows_idx, block, window, dout_e=Non
     """``rows`` for the rotated attention of one example (rows [L, H, D])."""
     L = _f64(q_e).shape[0]
     offs = np.array([0, L], dtype=np.int32)
-    qr = _as_operand(rope_rotate(q_e, offs, cos, sin), operand_dtype)
-    kr = _as_operand(rope_rotate(k_e, offs, cos, sin), operand_dtype)
+    qr = _rotated_operand(q_e, offs, cos, sin, operand_dtype)
+    kr = _rotated_operand(k_e, offs, cos, sin, operand_dtype)
     res = rows(qr, kr, v_e, head, rows_idx, block, window, dout_e=dout_e, want=want, nthreads=nthreads)
     pos = np.asarray(rows_idx, dtype=np.int64)
     for name in ("dq", "dk"):

@@ -493,3 +493,29 @@ def test_rope_tables_shorter_than_an_example_are_rejected():
     cos, sin, _ = _exact_tables(11, 4)
     with pytest.raises(ValueError):
         oracle.rope_fwd(offs, q, k, v, cos, sin, 4, 1)
+
+
+def test_rope_float32_form_is_the_formula_rounded_per_operation():
+    """The float32 evaluation (used only to decide the bf16 rounding of the
+    rotated operands) is the same formula: within the error of three float32
+    roundings of the fp64 value, and the rounded operands it gives differ
+    from rounding the exact value by at most one bf16 step."""
+    rng = np.random.default_rng(508)
+    offs, q, _, _, _ = rand_case(rng, [50, 30], 2, 16, scale=3.0)
+    q = torch.from_numpy(q).to(torch.bfloat16).double().numpy()       # operands as the library sees them
+    cos, sin, _ = _exact_tables(64, 16)
+    cos, sin = cos.astype(np.float32).astype(np.float64), sin.astype(np.float32).astype(np.float64)
+    exact = oracle.rope_rotate(q, offs, cos, sin)
+    f32 = oracle.rope_rotate(q, offs, cos, sin, fp32=True)
+    pos = oracle.positions(offs)
+    c = cos[pos][:, None, :]
+    s = sin[pos][:, None, :]
+    mag = np.empty_like(q)
+    mag[..., 0::2] = np.abs(q[..., 0::2] * c) + np.abs(q[..., 1::2] * s)
+    mag[..., 1::2] = np.abs(q[..., 0::2] * s) + np.abs(q[..., 1::2] * c)
+    assert np.all(np.abs(f32 - exact) <= 3 * 2.0 ** -24 * mag * (1 + 1e-6))
+    a = oracle._rotated_operand(q, offs, cos, sin, torch.bfloat16)
+    b = torch.from_numpy(exact).to(torch.bfloat16).double().numpy()
+    step = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(b), 1e-30))) - 7)
+    assert np.all(np.abs(a - b) <= step * (1 + 1e-9))
+    assert np.mean(a == b) > 0.99
