@@ -4,7 +4,11 @@
 One step = ba_fwd + ba_bwd over a whole batch (every kernel of the path).
 Default workload: 256 user histories with lengths uniform in [64, 4096],
 8 heads, head_dim 128, block 256, window 2, bf16 (the jagged long-history
-case); --config picks another of the five workloads in workloads.py.
+case); --config picks another of the five workloads in workloads.py, --swa
+the sliding-window variant, --rope the rotary entry points (ba_rope_fwd +
+ba_rope_bwd: rotary embedding on q and k with tables covering the longest
+example, resident on the device like weights; the forward's rotated q and k
+are kept for the backward, as training keeps activations).
 
 Prints ONE JSON line (rank 0). ``value`` is useful TFLOP/s (14 * head_dim
 FLOPs per visible query/key pair and head, summed over all ranks) with the
@@ -34,7 +38,7 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from block_sparse_attention_kunlun_b200 import flops as F  # noqa: E402
-from block_sparse_attention_kunlun_b200.workloads import CONFIGS, make_inputs  # noqa: E402
+from block_sparse_attention_kunlun_b200.workloads import CONFIGS, make_inputs, rope_tables  # noqa: E402
 
 METRIC = "block-attention fwd+bwd useful TFLOP/s and tokens/s on 1 B200; % of bf16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -54,6 +58,8 @@ def parse():
     ap.add_argument("--swa", type=int, default=0, metavar="W",
                     help="time sliding-window attention (each query sees its last W tokens; block 1, "
                          "window W) on the config's shapes instead of block attention")
+    ap.add_argument("--rope", action="store_true",
+                    help="rotary embedding on q and k (ba_rope_fwd / ba_rope_bwd)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic-file", default=os.path.join(ROOT, "profiles", "traffic.json"),
@@ -72,16 +78,24 @@ def load_peaks():
 
 
 def config_workload(args):
-    """The config's workload, or its sliding-window variant under --swa."""
+    """The config's workload, or its sliding-window variant under --swa; --rope
+    adds the rotary embedding (the name says so)."""
     import re
     w = CONFIGS[args.config]
     if args.swa:
-        return w.replace(block=1, window=args.swa,
-                         name=re.sub(r"block \d+, window \d+", f"sliding window {args.swa} tokens", w.name))
-    if args.block or args.window:
+        w = w.replace(block=1, window=args.swa,
+                      name=re.sub(r"block \d+, window \d+", f"sliding window {args.swa} tokens", w.name))
+    elif args.block or args.window:
         b, win = args.block or w.block, args.window or w.window
         w = w.replace(block=b, window=win, name=re.sub(r"block \d+, window \d+", f"block {b}, window {win}", w.name))
+    if getattr(args, "rope", False):
+        w = w.replace(name=w.name + ", rotary q/k")
     return w
+
+
+def tables_for(lens, head_dim):
+    """Rotary tables covering the longest example (float32, CPU)."""
+    return rope_tables(max(1, int(max(lens, default=1))), head_dim)
 
 
 def workload(args, rank=0):
@@ -149,8 +163,9 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def cpu_baseline(w, inp, pairs_total, budget_frac=0.04):
-    """Times the CPU oracle (as it stands) on the first examples of the batch."""
+def cpu_baseline(w, inp, pairs_total, budget_frac=0.04, tables=None):
+    """Times the CPU oracle (as it stands) on the first examples of the batch
+    (its rotary form when tables are given)."""
     import oracle
     offs = inp["seq_offsets"].numpy()
     lens = np.diff(offs)
@@ -169,8 +184,13 @@ def cpu_baseline(w, inp, pairs_total, budget_frac=0.04):
     q, k, v, do = f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["dout"])
     threads = oracle.default_threads()
     t0 = time.perf_counter()
-    o, lse = oracle.fwd(sub_offs, q, k, v, w.block, w.window, skip=sub_skip, nthreads=threads)
-    oracle.bwd(sub_offs, q, k, v, do, w.block, w.window, skip=sub_skip, nthreads=threads)
+    if tables is None:
+        oracle.fwd(sub_offs, q, k, v, w.block, w.window, skip=sub_skip, nthreads=threads)
+        oracle.bwd(sub_offs, q, k, v, do, w.block, w.window, skip=sub_skip, nthreads=threads)
+    else:
+        c, s = (t.to(torch.float64).numpy() for t in tables)
+        oracle.rope_fwd(sub_offs, q, k, v, c, s, w.block, w.window, skip=sub_skip, nthreads=threads)
+        oracle.rope_bwd(sub_offs, q, k, v, do, c, s, w.block, w.window, skip=sub_skip, nthreads=threads)
     dt = time.perf_counter() - t0
     useful = F.step_flops(acc, w.heads, w.head_dim)["step"]
     return {"value": useful / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
@@ -201,7 +221,14 @@ def run_reference(args):
     pairs = F.visible_pairs([s1 - s0], w.block, w.window)
     useful = F.step_flops(pairs, w.heads, w.head_dim)["step"]
 
+    if args.rope:
+        c, s = (t.to(torch.float64).numpy() for t in tables_for(lens, w.head_dim))
+
     def step():
+        if args.rope:
+            oracle.rope_fwd(sub, q, k, v, c, s, w.block, w.window, nthreads=threads)
+            oracle.rope_bwd(sub, q, k, v, do, c, s, w.block, w.window, nthreads=threads)
+            return
         oracle.fwd(sub, q, k, v, w.block, w.window, nthreads=threads)
         oracle.bwd(sub, q, k, v, do, w.block, w.window, nthreads=threads)
 
@@ -269,16 +296,32 @@ def main():
     out, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
     lse = torch.empty((H, T), dtype=torch.float32, device=dev)
     prob = ba.make_problem(q, offs)
-    ws_f = ba.workspace_for(ba.ba_fwd_workspace_size(prob, w.block, w.window), dev)
-    ws_b = ba.workspace_for(ba.ba_bwd_workspace_size(prob, w.block, w.window), dev)
     stream = torch.cuda.current_stream(dev)
+    if args.rope:
+        tables = tables_for(lens, D)
+        cos_d, sin_d = (t.to(dev) for t in tables)
+        q_rot, k_rot = torch.empty_like(q), torch.empty_like(k)
+        rope = ba.make_rope(cos_d, sin_d, q_rot, k_rot)
+        ws_f = ba.workspace_for(ba.ba_fwd_workspace_size(prob, w.block, w.window), dev)
+        ws_b = ba.workspace_for(ba.ba_bwd_workspace_size(prob, w.block, w.window), dev)
+    else:
+        tables = None
+        ws_f = ba.workspace_for(ba.ba_fwd_workspace_size(prob, w.block, w.window), dev)
+        ws_b = ba.workspace_for(ba.ba_bwd_workspace_size(prob, w.block, w.window), dev)
 
     def step():
-        st = ba.ba_fwd(prob, q, k, v, offs, w.block, w.window, skip, out, lse, ws_f, stream=stream)
+        if args.rope:
+            st = ba.ba_rope_fwd(prob, rope, q, k, v, offs, w.block, w.window, skip, out, lse, ws_f, stream=stream)
+        else:
+            st = ba.ba_fwd(prob, q, k, v, offs, w.block, w.window, skip, out, lse, ws_f, stream=stream)
         if st != ba.BA_OK:
             raise ba.BAError(st, "ba_fwd")
-        st = ba.ba_bwd(prob, q, k, v, out, lse, dout, offs, w.block, w.window, skip, dq, dk, dv, ws_b,
-                       stream=stream)
+        if args.rope:
+            st = ba.ba_rope_bwd(prob, rope, q, k, v, out, lse, dout, offs, w.block, w.window, skip, dq, dk, dv,
+                                ws_b, stream=stream)
+        else:
+            st = ba.ba_bwd(prob, q, k, v, out, lse, dout, offs, w.block, w.window, skip, dq, dk, dv, ws_b,
+                           stream=stream)
         if st != ba.BA_OK:
             raise ba.BAError(st, "ba_bwd")
 
@@ -287,8 +330,12 @@ def main():
         if dist is not None:
             dist.barrier()
 
-    # ba_fwd: work list, (skip), attention; ba_bwd: work list, (skip), dQ, dK/dV
+    # ba_fwd: work list, (skip), attention; ba_bwd: work list, (skip), dQ, dK/dV;
+    # the rotary forward adds one rotation pass (the backward reads the kept rotated copies;
+    # fp32 adds a transposed pass after its backward kernels)
     launches_per_step = (2 + (skip is not None)) + (3 + (skip is not None))
+    if args.rope:
+        launches_per_step += 1 + (w.dtype == torch.float32)
 
     for _ in range(args.warmup):
         step()
@@ -391,6 +438,7 @@ def main():
             tr = json.load(f)
         key = f"{names[dom]}:config{args.config}" + (f":block{w.block}:window{w.window}"
                                                        if (args.swa or args.block or args.window) else "")
+        key += ":rope" if args.rope else ""
         if key in tr and tr[key].get("kernel_sha") == kernel_sha(dom):
             traffic = tr[key]["bytes_per_launch"]
     except (OSError, ValueError):
@@ -408,6 +456,7 @@ def main():
         "data": "synthetic",
         "config": {"workload": w.name, "batch": int(len(lens)), "total_tokens": int(T), "heads": H,
                    "head_dim": D, "block": w.block, "window": w.window, "seed": w.seed,
+                   "rotary": bool(args.rope),
                    "visible_pairs_per_head": pairs, "useful_flops_per_step": fl["step"],
                    "l2": f"inputs larger than L2 ({by['fwd'] + by['bwd']:.3g} B touched per step), no flush",
                    "parallelism": f"dp{world} (independent batches, no collective in the step)"},
@@ -421,7 +470,7 @@ def main():
         "clocks": clk,
     }
     if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(w, inp, pairs)
+        line["cpu_baseline"] = cpu_baseline(w, inp, pairs, tables=tables)
     print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

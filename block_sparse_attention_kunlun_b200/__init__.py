@@ -22,8 +22,10 @@ import torch
 __all__ = [
     "BAError", "ba_fwd", "ba_fwd_noalloc", "ba_bwd", "ba_fwd_workspace_size", "ba_bwd_workspace_size",
     "ba_swa_fwd", "ba_swa_bwd", "ba_swa_fwd_workspace_size", "ba_swa_bwd_workspace_size",
+    "ba_rope_fwd", "ba_rope_bwd", "ba_rope_fwd_workspace_size", "ba_rope_bwd_workspace_size",
     "ba_device_status", "ba_selftest_wait_timeout", "ba_set_profile_events", "ba_status_string", "ba_version",
     "block_attention_fwd", "block_attention_bwd", "sliding_window_attention_fwd", "sliding_window_attention_bwd",
+    "rope_block_attention_fwd", "rope_block_attention_bwd",
     "library_path",
 ]
 
@@ -38,6 +40,11 @@ _DTYPES = {torch.float32: BA_F32, torch.bfloat16: BA_BF16}
 class BAProblem(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("total_tokens", ctypes.c_int32),
                 ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("dtype", ctypes.c_int)]
+
+
+class BARope(ctypes.Structure):
+    _fields_ = [("cos", ctypes.c_void_p), ("sin", ctypes.c_void_p), ("rows", ctypes.c_int32),
+                ("q_rot", ctypes.c_void_p), ("k_rot", ctypes.c_void_p)]
 
 
 class BAError(RuntimeError):
@@ -91,6 +98,15 @@ def _load():
     lib.ba_swa_fwd.restype = ctypes.c_int
     lib.ba_swa_bwd.argtypes = [prob, P, P, P, P, P, P, P, i32, P, P, P, P, P, ctypes.c_size_t, P]
     lib.ba_swa_bwd.restype = ctypes.c_int
+    rope = ctypes.POINTER(BARope)
+    lib.ba_rope_fwd_workspace_size.argtypes = [prob, i32, i32]
+    lib.ba_rope_fwd_workspace_size.restype = ctypes.c_size_t
+    lib.ba_rope_bwd_workspace_size.argtypes = [prob, i32, i32]
+    lib.ba_rope_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.ba_rope_fwd.argtypes = [prob, rope, P, P, P, P, i32, i32, P, P, P, P, ctypes.c_size_t, P]
+    lib.ba_rope_fwd.restype = ctypes.c_int
+    lib.ba_rope_bwd.argtypes = [prob, rope, P, P, P, P, P, P, P, i32, i32, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.ba_rope_bwd.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -191,6 +207,46 @@ def ba_swa_bwd(problem, q, k, v, out, lse, dout, seq_offsets, window_tokens, ski
                                   _ptr(dout), _ptr(seq_offsets), int(window_tokens), _ptr(skip),
                                   _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), int(workspace_bytes),
                                   _stream(stream)))
+
+
+def make_rope(cos, sin, q_rot=None, k_rot=None) -> BARope:
+    """Rotary tables (float32 CUDA tensors [rows, head_dim / 2]) as the C
+    struct, with optional caller buffers for the rotated q and k."""
+    for name, t in (("cos", cos), ("sin", sin)):
+        if not isinstance(t, int) and (t.dtype != torch.float32 or t.dim() != 2 or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous float32 [rows, head_dim / 2] tensor")
+    rows = cos.shape[0] if not isinstance(cos, int) else 0
+    return BARope(_ptr(cos), _ptr(sin), int(rows), _ptr(q_rot), _ptr(k_rot))
+
+
+def ba_rope_fwd_workspace_size(problem: BAProblem, block: int, window: int) -> int:
+    return int(_load().ba_rope_fwd_workspace_size(ctypes.byref(problem), int(block), int(window)))
+
+
+def ba_rope_bwd_workspace_size(problem: BAProblem, block: int, window: int) -> int:
+    return int(_load().ba_rope_bwd_workspace_size(ctypes.byref(problem), int(block), int(window)))
+
+
+def ba_rope_fwd(problem, rope, q, k, v, seq_offsets, block, window, skip, out, lse, workspace,
+                workspace_bytes=None, stream=None) -> int:
+    """Direct call of the rotary forward (rope: BARope or None); returns its status code."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(_load().ba_rope_fwd(ctypes.byref(problem), ctypes.byref(rope) if rope is not None else None,
+                                   _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), int(block), int(window),
+                                   _ptr(skip), _ptr(out), _ptr(lse), _ptr(workspace), int(workspace_bytes),
+                                   _stream(stream)))
+
+
+def ba_rope_bwd(problem, rope, q, k, v, out, lse, dout, seq_offsets, block, window, skip, dq, dk, dv,
+                workspace, workspace_bytes=None, stream=None) -> int:
+    """Direct call of the rotary backward; returns its status code."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(_load().ba_rope_bwd(ctypes.byref(problem), ctypes.byref(rope) if rope is not None else None,
+                                   _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout),
+                                   _ptr(seq_offsets), int(block), int(window), _ptr(skip), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), _ptr(workspace), int(workspace_bytes), _stream(stream)))
 
 
 def ba_set_profile_events(which: int, start=None, stop=None) -> int:
@@ -299,4 +355,66 @@ def sliding_window_attention_bwd(q, k, v, out, lse, dout, seq_offsets, window_to
                     workspace, stream=stream)
     if st != BA_OK:
         raise BAError(st, "ba_swa_bwd")
+    return dq, dk, dv
+
+
+def _check_tables(cos, sin, q):
+    for name, t in (("cos", cos), ("sin", sin)):
+        if not t.is_cuda or t.dtype != torch.float32 or t.dim() != 2 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor [rows, head_dim / 2]")
+        if t.shape[1] != q.shape[2] // 2 or t.shape != cos.shape:
+            raise ValueError("cos and sin must both be [rows, head_dim / 2]")
+
+
+def _check_rotated(q_rot, k_rot, q):
+    if (q_rot is None) != (k_rot is None):
+        raise ValueError("pass both q_rot and k_rot, or neither")
+    for name, t in (("q_rot", q_rot), ("k_rot", k_rot)):
+        if t is not None and (not t.is_cuda or not t.is_contiguous() or t.shape != q.shape or t.dtype != q.dtype):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor like q")
+
+
+def rope_block_attention_fwd(q, k, v, seq_offsets, block, window, cos, sin, skip=None, out=None, lse=None,
+                             workspace=None, q_rot=None, k_rot=None, stream=None):
+    """Rotary embedding on q and k (tables cos, sin [rows, head_dim / 2];
+    rows must cover the longest example), then block attention: ba_rope_fwd.
+    Allocates out/lse (and a workspace) with torch. q_rot / k_rot: buffers
+    like q that receive the rotated q and k, to hand to the backward."""
+    _check_inputs(q, k, v, seq_offsets)
+    _check_tables(cos, sin, q)
+    _check_rotated(q_rot, k_rot, q)
+    prob = make_problem(q, seq_offsets)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        need = (ba_fwd_workspace_size if q_rot is not None else ba_rope_fwd_workspace_size)(prob, block, window)
+        workspace = workspace_for(need, q.device)
+    st = ba_rope_fwd(prob, make_rope(cos, sin, q_rot, k_rot), q, k, v, seq_offsets, block, window, skip, out,
+                     lse, workspace, stream=stream)
+    if st != BA_OK:
+        raise BAError(st, "ba_rope_fwd")
+    return out, lse
+
+
+def rope_block_attention_bwd(q, k, v, out, lse, dout, seq_offsets, block, window, cos, sin, skip=None,
+                             dq=None, dk=None, dv=None, workspace=None, q_rot=None, k_rot=None, stream=None):
+    """Gradients of rope_block_attention_fwd with respect to the unrotated q,
+    k and v: ba_rope_bwd. Allocates dq/dk/dv (and a workspace) with torch.
+    q_rot / k_rot: the forward's rotated copies (then no rotation pass runs)."""
+    _check_inputs(q, k, v, seq_offsets)
+    _check_tables(cos, sin, q)
+    _check_rotated(q_rot, k_rot, q)
+    prob = make_problem(q, seq_offsets)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if workspace is None:
+        need = (ba_bwd_workspace_size if q_rot is not None else ba_rope_bwd_workspace_size)(prob, block, window)
+        workspace = workspace_for(need, q.device)
+    st = ba_rope_bwd(prob, make_rope(cos, sin, q_rot, k_rot), q, k, v, out, lse, dout, seq_offsets, block,
+                     window, skip, dq, dk, dv, workspace, stream=stream)
+    if st != BA_OK:
+        raise BAError(st, "ba_rope_bwd")
     return dq, dk, dv

@@ -6,6 +6,10 @@
 //   ba_bwd: worklist -> skip passthrough -> bf16: dQ kernel (also writes
 //           Delta) -> dK/dV kernel; fp32: Delta pre-pass -> dQ and dK/dV
 //           SIMT kernels
+//   ba_rope_fwd / ba_rope_bwd: the same, with a rotary pass writing rotated
+//           copies of q and k into the workspace before the attention
+//           kernels read them; the bf16 backward turns dq and dk back inside
+//           the dQ and dK/dV epilogues, the fp32 one in a pass after them
 // Nothing here allocates, synchronises or falls back to another device.
 #include "ba.h"
 #include "ba_common.cuh"
@@ -121,6 +125,39 @@ Problem make_problem(const ba_problem &pp, const int32_t *offs, const uint8_t *s
     return p;
 }
 
+// Rotated q and k (the rotary entry points) follow the attention workspace.
+struct RopeLayout {
+    size_t qr, kr, total;
+};
+
+RopeLayout rope_layout(const ba_problem &P, size_t base_total)
+{
+    const size_t esz = P.dtype == BA_BF16 ? 2 : 4;
+    const size_t bytes = align256(size_t(P.total_tokens) * size_t(P.heads) * size_t(P.head_dim) * esz);
+    return RopeLayout{base_total, base_total + bytes, base_total + 2 * bytes};
+}
+
+ba_status check_rope(const ba_rope *r, const ba_problem &P)
+{
+    if (!r) return BA_ERR_INVALID_ARG;
+    if (P.total_tokens == 0) return BA_OK;
+    if (!r->cos || !r->sin || !aligned(r->cos, 16) || !aligned(r->sin, 16) || r->rows < 1 || P.head_dim % 2)
+        return BA_ERR_INVALID_ARG;
+    if (!r->q_rot != !r->k_rot) return BA_ERR_INVALID_ARG;
+    if (r->q_rot && (!aligned(r->q_rot, 16) || !aligned(r->k_rot, 16))) return BA_ERR_INVALID_ARG;
+    return BA_OK;
+}
+
+// Rotated copies in the caller's buffers (both set) or in the workspace.
+bool caller_rotated(const ba_rope *r) { return r && r->q_rot && r->k_rot; }
+
+void set_rope(Problem &p, const ba_rope *r)
+{
+    p.rope_cos = r->cos;
+    p.rope_sin = r->sin;
+    p.rope_rows = r->rows;
+}
+
 thread_local cudaEvent_t t_prof[3][2] = {{nullptr, nullptr}, {nullptr, nullptr}, {nullptr, nullptr}};
 
 cudaError_t prof_mark(int which, int edge, cudaStream_t stream)
@@ -134,25 +171,10 @@ cudaError_t prof_mark(int which, int edge, cudaStream_t stream)
         if ((expr) != cudaSuccess) return BA_ERR_CUDA;                                                    \
     } while (0)
 
-} // namespace
-
-extern "C" {
-
-size_t ba_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
-{
-    if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
-    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, false).total;
-}
-
-size_t ba_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
-{
-    if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
-    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, true).total;
-}
-
-ba_status ba_fwd(const ba_problem *pp, const void *q, const void *k, const void *v, const int32_t *seq_offsets,
-                 int32_t block, int32_t window, const uint8_t *skip, void *out, float *lse, void *workspace,
-                 size_t workspace_bytes, ba_stream_t stream_)
+// ba_fwd (rope == nullptr) and ba_rope_fwd.
+ba_status fwd_impl(const ba_problem *pp, const ba_rope *rope, const void *q, const void *k, const void *v,
+                   const int32_t *seq_offsets, int32_t block, int32_t window, const uint8_t *skip, void *out,
+                   float *lse, void *workspace, size_t workspace_bytes, ba_stream_t stream_, bool with_rope)
 {
     ba_status st = check_problem(pp, block, window);
     if (st != BA_OK) return st;
@@ -161,18 +183,31 @@ ba_status ba_fwd(const ba_problem *pp, const void *q, const void *k, const void 
     if (!seq_offsets || !aligned(seq_offsets, 4) || !tensor_ok(q, T) || !tensor_ok(k, T) || !tensor_ok(v, T) ||
         !tensor_ok(out, T) || (T > 0 && (!lse || !aligned(lse, 4))))
         return BA_ERR_INVALID_ARG;
+    if (with_rope && (st = check_rope(rope, P)) != BA_OK) return st;
     const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, false);
-    if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total) return BA_ERR_INVALID_ARG;
+    const RopeLayout rl = rope_layout(P, lay.total);
+    const size_t need = with_rope && !caller_rotated(rope) ? rl.total : lay.total;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return BA_ERR_INVALID_ARG;
     int num_sms = 0, cc = 0;
     if (!device_info(num_sms, cc)) return BA_ERR_CUDA;
     if (P.dtype == BA_BF16 && cc != 10) return BA_ERR_UNSUPPORTED;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
 
-    const Problem p = make_problem(P, seq_offsets, skip, block, window, workspace, lay);
+    Problem p = make_problem(P, seq_offsets, skip, block, window, workspace, lay);
     BA_TRY(launch_worklist(p, stream));
     if (T == 0) return BA_OK;
     const size_t esz = P.dtype == BA_BF16 ? 2 : 4;
     BA_TRY(launch_skip_fwd(p, esz, v, out, lse, stream));
+    if (with_rope) {
+        // the attention kernels read rotated copies of q and k
+        uint8_t *ws = static_cast<uint8_t *>(workspace);
+        void *qr = caller_rotated(rope) ? rope->q_rot : ws + rl.qr;
+        void *kr = caller_rotated(rope) ? rope->k_rot : ws + rl.kr;
+        set_rope(p, rope);
+        BA_TRY(launch_rope_rows(p, esz, false, q, k, qr, kr, num_sms, stream));
+        q = qr;
+        k = kr;
+    }
     if (P.dtype == BA_F32) {
         BA_TRY(prof_mark(0, 0, stream));
         BA_TRY(launch_fwd_f32(p, static_cast<const float *>(q), static_cast<const float *>(k),
@@ -191,10 +226,11 @@ ba_status ba_fwd(const ba_problem *pp, const void *q, const void *k, const void 
     return BA_OK;
 }
 
-ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void *v, const void *out,
-                 const float *lse, const void *dout, const int32_t *seq_offsets, int32_t block, int32_t window,
-                 const uint8_t *skip, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
-                 ba_stream_t stream_)
+// ba_bwd (rope == nullptr) and ba_rope_bwd.
+ba_status bwd_impl(const ba_problem *pp, const ba_rope *rope, const void *q, const void *k, const void *v,
+                   const void *out, const float *lse, const void *dout, const int32_t *seq_offsets, int32_t block,
+                   int32_t window, const uint8_t *skip, void *dq, void *dk, void *dv, void *workspace,
+                   size_t workspace_bytes, ba_stream_t stream_, bool with_rope)
 {
     ba_status st = check_problem(pp, block, window);
     if (st != BA_OK) return st;
@@ -204,15 +240,18 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
         !tensor_ok(out, T) || !tensor_ok(dout, T) || !tensor_ok(dq, T) || !tensor_ok(dk, T) || !tensor_ok(dv, T) ||
         (T > 0 && (!lse || !aligned(lse, 4))))
         return BA_ERR_INVALID_ARG;
+    if (with_rope && (st = check_rope(rope, P)) != BA_OK) return st;
     const bool bf16 = P.dtype == BA_BF16;
     const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, true);
-    if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total) return BA_ERR_INVALID_ARG;
+    const RopeLayout rl = rope_layout(P, lay.total);
+    const size_t need = with_rope && !caller_rotated(rope) ? rl.total : lay.total;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return BA_ERR_INVALID_ARG;
     int num_sms = 0, cc = 0;
     if (!device_info(num_sms, cc)) return BA_ERR_CUDA;
     if (bf16 && cc != 10) return BA_ERR_UNSUPPORTED;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
 
-    const Problem p = make_problem(P, seq_offsets, skip, block, window, workspace, lay);
+    Problem p = make_problem(P, seq_offsets, skip, block, window, workspace, lay);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     float *delta = reinterpret_cast<float *>(ws + lay.delta);
     float *nlse2 = reinterpret_cast<float *>(ws + lay.nlse2);
@@ -220,6 +259,20 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
     if (T == 0) return BA_OK;
     const size_t esz = bf16 ? 2 : 4;
     BA_TRY(launch_skip_bwd(p, esz, dout, dq, dk, dv, stream));
+    if (with_rope) {
+        // the rotated q and k the forward used: the caller's saved copies, or
+        // recomputed here; p.rope_* also tells the bf16 dQ and dK/dV epilogues to
+        // turn dq and dk back
+        set_rope(p, rope);
+        if (caller_rotated(rope)) {
+            q = rope->q_rot;
+            k = rope->k_rot;
+        } else {
+            BA_TRY(launch_rope_rows(p, esz, false, q, k, ws + rl.qr, ws + rl.kr, num_sms, stream));
+            q = ws + rl.qr;
+            k = ws + rl.kr;
+        }
+    }
     if (!bf16) {
         BA_TRY(launch_bwd_pre<float>(p, out, dout, delta, num_sms, stream));
         BA_TRY(prof_mark(1, 0, stream));
@@ -228,6 +281,7 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
                               static_cast<float *>(dq), static_cast<float *>(dk), static_cast<float *>(dv), num_sms,
                               stream));
         BA_TRY(prof_mark(2, 1, stream));
+        if (with_rope) BA_TRY(launch_rope_rows(p, esz, true, dq, dk, dq, dk, num_sms, stream));
         return BA_OK;
     }
     CUtensorMap tq, tk, tv, tdo, to, tdk, tdv;
@@ -249,6 +303,69 @@ ba_status ba_bwd(const ba_problem *pp, const void *q, const void *k, const void 
         BA_TRY(launch_bwd_dkdv_sm100<128>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, delta, dk, dv, num_sms, stream));
     BA_TRY(prof_mark(2, 1, stream));
     return BA_OK;
+}
+
+} // namespace
+
+extern "C" {
+
+size_t ba_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
+{
+    if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
+    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, false).total;
+}
+
+size_t ba_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
+{
+    if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
+    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, true).total;
+}
+
+ba_status ba_fwd(const ba_problem *p, const void *q, const void *k, const void *v, const int32_t *seq_offsets,
+                 int32_t block, int32_t window, const uint8_t *skip, void *out, float *lse, void *workspace,
+                 size_t workspace_bytes, ba_stream_t stream)
+{
+    return fwd_impl(p, nullptr, q, k, v, seq_offsets, block, window, skip, out, lse, workspace, workspace_bytes,
+                    stream, false);
+}
+
+ba_status ba_bwd(const ba_problem *p, const void *q, const void *k, const void *v, const void *out,
+                 const float *lse, const void *dout, const int32_t *seq_offsets, int32_t block, int32_t window,
+                 const uint8_t *skip, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                 ba_stream_t stream)
+{
+    return bwd_impl(p, nullptr, q, k, v, out, lse, dout, seq_offsets, block, window, skip, dq, dk, dv, workspace,
+                    workspace_bytes, stream, false);
+}
+
+// Rotary position embedding on q and k, then block attention.
+size_t ba_rope_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
+{
+    const size_t base = ba_fwd_workspace_size(p, block, window);
+    return base ? rope_layout(*p, base).total : 0;
+}
+
+size_t ba_rope_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
+{
+    const size_t base = ba_bwd_workspace_size(p, block, window);
+    return base ? rope_layout(*p, base).total : 0;
+}
+
+ba_status ba_rope_fwd(const ba_problem *p, const ba_rope *rope, const void *q, const void *k, const void *v,
+                      const int32_t *seq_offsets, int32_t block, int32_t window, const uint8_t *skip, void *out,
+                      float *lse, void *workspace, size_t workspace_bytes, ba_stream_t stream)
+{
+    return fwd_impl(p, rope, q, k, v, seq_offsets, block, window, skip, out, lse, workspace, workspace_bytes,
+                    stream, true);
+}
+
+ba_status ba_rope_bwd(const ba_problem *p, const ba_rope *rope, const void *q, const void *k, const void *v,
+                      const void *out, const float *lse, const void *dout, const int32_t *seq_offsets,
+                      int32_t block, int32_t window, const uint8_t *skip, void *dq, void *dk, void *dv,
+                      void *workspace, size_t workspace_bytes, ba_stream_t stream)
+{
+    return bwd_impl(p, rope, q, k, v, out, lse, dout, seq_offsets, block, window, skip, dq, dk, dv, workspace,
+                    workspace_bytes, stream, true);
 }
 
 // Sliding-window attention: the block rule with block = 1 (one token per block),
@@ -287,7 +404,8 @@ ba_status ba_device_status(const void *workspace, ba_stream_t stream_)
     if (cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
         cudaStreamSynchronize(stream) != cudaSuccess)
         return BA_ERR_CUDA;
-    return (word & kStatusTimeout) ? BA_ERR_TIMEOUT : BA_OK;
+    if (word & kStatusTimeout) return BA_ERR_TIMEOUT;
+    return (word & kStatusRopeRange) ? BA_ERR_INVALID_ARG : BA_OK;
 }
 
 ba_status ba_selftest_wait_timeout(void *workspace, size_t workspace_bytes, int32_t limit_us, ba_stream_t stream_)

@@ -93,7 +93,7 @@ __device__ __forceinline__ void query_tile_range(const TileRef &r, int64_t B, in
 
 } // namespace
 
-template <int D>
+template <int D, bool kRope>
 __global__ void __launch_bounds__(448, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -465,22 +465,44 @@ __global__ void __launch_bounds__(448, 1)
                 const bool is_k = part >= Lay::kChunks;
                 const int c = is_k ? part - Lay::kChunks : part;
                 const float sc = is_k ? p.scale : 1.f;
-                uint32_t rr[2][32];
-                tmem_ld32(tmem + lane_base + (is_k ? Lay::kColDK : Lay::kColDV) + 64 * c, rr[0]);
-                tmem_ld32(tmem + lane_base + (is_k ? Lay::kColDK : Lay::kColDV) + 64 * c + 32, rr[1]);
-                tmem_wait_ld();
-                reg_fence(rr[0]);
-                reg_fence(rr[1]);
-                if (c == Lay::kChunks - 1) { // all of dV (or dK) read: the next item may accumulate into it
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(is_k ? &sb.dk_free : &sb.dv_free);
-                }
+                auto release = [&] {
+                    if (c == Lay::kChunks - 1) { // all of dV (or dK) read: the next item may accumulate into it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(is_k ? &sb.dk_free : &sb.dv_free);
+                    }
+                };
                 uint32_t pk[32];
+                if (kRope && is_k) {
+                    // rotary embedding: dK is the gradient of the rotated k; turn its pairs back
+                    // (transposed rotation at this key row's position). One 32-column half at a
+                    // time, read, turned and packed before the next, to stay within registers.
 #pragma unroll
-                for (int x = 0; x < 32; ++x)
-                    pk[x] = pack_bf16x2(__uint_as_float(rr[x / 16][2 * (x % 16)]) * sc,
-                                        __uint_as_float(rr[x / 16][2 * (x % 16) + 1]) * sc);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t rh[32];
+                        tmem_ld32(tmem + lane_base + Lay::kColDK + 64 * c + 32 * hh, rh);
+                        tmem_wait_ld();
+                        reg_fence(rh);
+                        if (valid_k) rope_transpose_bits<4>(p, k, 32 * c + 16 * hh, rh);
+#pragma unroll
+                        for (int x = 0; x < 16; ++x)
+                            pk[16 * hh + x] =
+                                pack_bf16x2(__uint_as_float(rh[2 * x]) * sc, __uint_as_float(rh[2 * x + 1]) * sc);
+                    }
+                    release();
+                } else {
+                    uint32_t rr[2][32];
+                    tmem_ld32(tmem + lane_base + (is_k ? Lay::kColDK : Lay::kColDV) + 64 * c, rr[0]);
+                    tmem_ld32(tmem + lane_base + (is_k ? Lay::kColDK : Lay::kColDV) + 64 * c + 32, rr[1]);
+                    tmem_wait_ld();
+                    reg_fence(rr[0]);
+                    reg_fence(rr[1]);
+                    release();
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                        pk[x] = pack_bf16x2(__uint_as_float(rr[x / 16][2 * (x % 16)]) * sc,
+                                            __uint_as_float(rr[x / 16][2 * (x % 16) + 1]) * sc);
+                }
                 if (full_tile) {
                     if (leader) bulk_wait_group_read<0>(); // the previous store has left the buffer
                     if (!group_sync(&sb.epi_sync, sync_phase, abort)) { ok = false; break; }
@@ -519,7 +541,7 @@ cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
                                   int num_sms, cudaStream_t stream)
 {
     using Lay = DkvLayout<D>;
-    auto kern = bwd_dkdv_sm100_kernel<D>;
+    auto kern = p.rope_cos ? bwd_dkdv_sm100_kernel<D, true> : bwd_dkdv_sm100_kernel<D, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
     kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, neg_delta,

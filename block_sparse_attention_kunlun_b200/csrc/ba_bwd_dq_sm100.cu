@@ -75,7 +75,7 @@ __device__ __forceinline__ int first_key_tile(const TileRef &r, int64_t B, int64
 
 } // namespace
 
-template <int D>
+template <int D, bool kRope>
 __global__ void __launch_bounds__(384, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -446,6 +446,9 @@ __global__ void __launch_bounds__(384, 1)
                     tmem_wait_ld();
                     reg_fence(a);
                     if (valid) {
+                        // rotary embedding: the accumulator is the gradient of the rotated q; turn
+                        // its 16 pairs back (transposed rotation at this row's position)
+                        if constexpr (kRope) rope_transpose_bits<4>(p, i, (D / 4) * g + 16 * c, a);
                         uint4 *dst = reinterpret_cast<uint4 *>(qrow + 32 * c);
 #pragma unroll
                         for (int x = 0; x < 4; ++x)
@@ -481,7 +484,7 @@ cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, co
                                 float *neg_delta, float *nlse2, void *dq, int num_sms, cudaStream_t stream)
 {
     using Lay = DqLayout<D>;
-    auto kern = bwd_dq_sm100_kernel<D>;
+    auto kern = p.rope_cos ? bwd_dq_sm100_kernel<D, true> : bwd_dq_sm100_kernel<D, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
     // the register split only works if the CTA is launched with at least the budgets' sum

@@ -19,6 +19,7 @@ constexpr int kWorklistThreads = 1024;
 
 // Status bits the kernels OR into the workspace status word.
 constexpr int kStatusTimeout = 1;
+constexpr int kStatusRopeRange = 2; // a row's position was past the rotary tables
 
 // First key visible to query i: the start of block blk(i) - (window - 1),
 // clamped at 0. Indices are local to an example and fit in 32 bits; the
@@ -105,7 +106,61 @@ struct Problem {
     int *status;                // workspace status word
     int32_t batch, total_tokens, heads, head_dim, block, window;
     float scale;                // 1 / sqrt(head_dim)
+    // rotary tables [rope_rows, head_dim / 2] (cos, sin of position x
+    // frequency); rope_cos == nullptr: no rotation
+    const float *rope_cos = nullptr;
+    const float *rope_sin = nullptr;
+    int32_t rope_rows = 0;
 };
+
+// Rotary position embedding (RoFormer's rotation, adjacent pairs; "GEM
+// (Meta)", section "Custom kernels": the block-attention kernel fuses the
+// rotary embedding's backward pass). A row at local position pos turns its
+// pair (x0, x1) = (x[2k], x[2k+1]) by the angle whose cosine c and sine s
+// the tables hold at [pos, k]:
+//   forward:    (x0 c - x1 s,  x0 s + x1 c)
+//   transposed: (g0 c + g1 s, -g0 s + g1 c)   (gradient of the unrotated row)
+// The forward result is rounded to the input dtype for the tensor cores; it
+// is formed with each product and the sum rounded once (no fused
+// multiply-add), so which way a value near a rounding tie goes follows from
+// the formula evaluated in float32 alone.
+__device__ __forceinline__ float2 rope_pair(float x0, float x1, float c, float s)
+{
+    return make_float2(__fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, s)), __fadd_rn(__fmul_rn(x0, s), __fmul_rn(x1, c)));
+}
+
+__device__ __forceinline__ float2 rope_pair_t(float g0, float g1, float c, float s)
+{
+    return make_float2(fmaf(g0, c, g1 * s), fmaf(g1, c, -g0 * s));
+}
+
+// Transposed rotation, in place, of 4 * NQ adjacent pairs held as float bit
+// patterns v[2m], v[2m+1] (m < 4 * NQ), pair indices k0 .. k0 + 4 NQ - 1 of
+// the row at local position pos (k0 a multiple of 4). A position past the
+// tables sets kStatusRopeRange and leaves the values as they are.
+template <int NQ>
+__device__ __forceinline__ void rope_transpose_bits(const Problem &p, int64_t pos, int k0, uint32_t *v)
+{
+    if (pos >= p.rope_rows) {
+        atomicOr(p.status, kStatusRopeRange);
+        return;
+    }
+    const int64_t base = pos * (p.head_dim / 2) + k0;
+    const float4 *cs = reinterpret_cast<const float4 *>(p.rope_cos + base);
+    const float4 *sn = reinterpret_cast<const float4 *>(p.rope_sin + base);
+#pragma unroll
+    for (int u = 0; u < NQ; ++u) {
+        const float4 c = __ldg(cs + u), s = __ldg(sn + u);
+        const float cc[4] = {c.x, c.y, c.z, c.w}, ss[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int m = 4 * u + e;
+            const float2 r = rope_pair_t(__uint_as_float(v[2 * m]), __uint_as_float(v[2 * m + 1]), cc[e], ss[e]);
+            v[2 * m] = __float_as_uint(r.x);
+            v[2 * m + 1] = __float_as_uint(r.y);
+        }
+    }
+}
 
 // One 128-row tile of one (example, head).
 struct TileRef {

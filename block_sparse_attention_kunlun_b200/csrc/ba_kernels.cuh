@@ -21,6 +21,11 @@ cudaError_t launch_skip_fwd(const Problem &p, size_t elem_bytes, const void *v, 
 cudaError_t launch_skip_bwd(const Problem &p, size_t elem_bytes, const void *dout, void *dq, void *dk, void *dv,
                             cudaStream_t stream);
 
+// Rotary embedding over every row of the batch: (a_out, b_out) = R(pos) (a_in, b_in),
+// or with transpose = true R(pos)^T (in place when a_out == a_in, b_out == b_in).
+cudaError_t launch_rope_rows(const Problem &p, size_t elem_bytes, bool transpose, const void *a_in, const void *b_in,
+                             void *a_out, void *b_out, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_fwd_f32(const Problem &p, const float *q, const float *k, const float *v, float *out, float *lse,
                            int num_sms, cudaStream_t stream);
 cudaError_t launch_bwd_f32(const Problem &p, const float *q, const float *k, const float *v, const float *dout,

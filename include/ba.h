@@ -144,6 +144,71 @@ ba_status ba_swa_bwd(const ba_problem *p, const void *q, const void *k, const vo
                      ba_stream_t stream);
 
 /*
+ * Rotary position embedding fused with block attention ("GEM (Meta)",
+ * section "Custom kernels": the production block-attention kernel carries a
+ * fused rotary position embedding backward pass; the pages say nothing more
+ * about it). The reading this library implements is RoFormer's rotation
+ * applied to q and k (not v) before the scores. The adjacent pair
+ * (x[2m], x[2m+1]) of a row at position pos, its 0-based index within its
+ * own example (the origin the blocks use), becomes
+ *     (x[2m] c - x[2m+1] s,  x[2m] s + x[2m+1] c),
+ *     c = cos[pos * head_dim/2 + m],  s = sin[pos * head_dim/2 + m].
+ * The caller owns the tables and so picks the frequencies (RoFormer's are
+ * angle = pos * 10000^(-2m / head_dim)).
+ *
+ *  - ba_rope_fwd: block attention of the rotated q and k. A rotation pass
+ *    writes rotated copies of q and k, in the problem's dtype, into the
+ *    workspace; the attention kernels read those. q and k are not modified.
+ *    Every row is rotated, skipped examples' too.
+ *  - ba_rope_bwd: the gradients with respect to the UNROTATED q and k, which
+ *    are the transposed rotations of the gradients of the rotated ones
+ *    (g0 c + g1 s, -g0 s + g1 c). dv is as for ba_bwd. It recomputes the
+ *    rotated copies, then runs the bf16 dQ and dK/dV kernels, which turn dq
+ *    and dk back in their epilogues before the single store. The fp32 path
+ *    does that in a pass after its kernels. out and lse are ba_rope_fwd's.
+ *  - Rotated copies: by default ba_rope_fwd writes them into its workspace,
+ *    and ba_rope_bwd recomputes them. A caller that keeps activations from
+ *    the forward for the backward (as training does) can set q_rot and k_rot
+ *    in the struct. ba_rope_fwd then writes R q and R k there, and
+ *    ba_rope_bwd given the same buffers (holding those values, for the same
+ *    q, k and tables) reads them and runs no rotation pass. Either both are
+ *    NULL or both are set: DEVICE [total_tokens, heads, head_dim] tensors of
+ *    the problem's dtype, 16-byte aligned, not aliasing any other argument.
+ *  - Workspace: without q_rot / k_rot, the *_workspace_size of the plain
+ *    entry point plus two 256-byte-aligned copies of a [total_tokens, heads,
+ *    head_dim] tensor (ba_rope_*_workspace_size); with them, the plain entry
+ *    point's size suffices.
+ *  - Errors: as for ba_fwd / ba_bwd. In addition, BA_ERR_INVALID_ARG when
+ *    rope is NULL, or, with total_tokens > 0, when cos or sin is NULL or not
+ *    16-byte aligned, when rows < 1, or when exactly one of q_rot, k_rot is
+ *    set or either is not 16-byte aligned. Nothing is launched in those
+ *    cases.
+ *    An example longer than the tables cannot be seen on the host. Its rows
+ *    at positions >= rows are left unrotated (their results are wrong, but
+ *    no memory outside the tables is read), and the workspace status word
+ *    records it: ba_device_status then returns BA_ERR_INVALID_ARG.
+ */
+typedef struct {
+    const float *cos; /* DEVICE, float32 [rows, head_dim / 2], row-major, 16-byte aligned */
+    const float *sin; /* DEVICE, same layout */
+    int32_t rows;     /* table rows; must cover the longest example, skipped ones included */
+    void *q_rot;      /* optional DEVICE [total_tokens, heads, head_dim]: R q (see above) */
+    void *k_rot;      /* optional, likewise R k; both NULL or both set */
+} ba_rope;
+
+size_t ba_rope_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window);
+size_t ba_rope_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window);
+ba_status ba_rope_fwd(const ba_problem *p, const ba_rope *rope, const void *q, const void *k,
+                      const void *v, const int32_t *seq_offsets, int32_t block, int32_t window,
+                      const uint8_t *skip, void *out, float *lse, void *workspace,
+                      size_t workspace_bytes, ba_stream_t stream);
+ba_status ba_rope_bwd(const ba_problem *p, const ba_rope *rope, const void *q, const void *k,
+                      const void *v, const void *out, const float *lse, const void *dout,
+                      const int32_t *seq_offsets, int32_t block, int32_t window,
+                      const uint8_t *skip, void *dq, void *dk, void *dv, void *workspace,
+                      size_t workspace_bytes, ba_stream_t stream);
+
+/*
  * Forward pass that allocates nothing and takes no workspace (the pages have
  * no counterpart; this is a convenience of this library). For callers that
  * cannot allocate device memory: a serving loop that records its forward into
@@ -166,9 +231,14 @@ ba_status ba_fwd_noalloc(const ba_problem *p, const void *q, const void *k, cons
                          const uint8_t *skip, void *out, float *lse, ba_stream_t stream);
 
 /*
- * Waits for `stream`, then reads the status word a previous ba_fwd/ba_bwd
- * left in `workspace`: BA_OK, or BA_ERR_TIMEOUT if a kernel gave up waiting
- * (its outputs are then undefined). BA_ERR_CUDA if the read itself failed.
+ * Waits for `stream`, then reads the status word that previous calls (ba_fwd,
+ * ba_bwd and the other entry points) left in `workspace`. Returns:
+ *  - BA_OK;
+ *  - BA_ERR_TIMEOUT if a kernel gave up waiting (its outputs are then
+ *    undefined);
+ *  - BA_ERR_INVALID_ARG if a rotary call met an example longer than its
+ *    tables;
+ *  - BA_ERR_CUDA if the read itself failed.
  */
 ba_status ba_device_status(const void *workspace, ba_stream_t stream);
 

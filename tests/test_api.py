@@ -104,3 +104,54 @@ def test_bwd_rejects_small_workspace():
     p = prob(batch=2, T=300, H=4, D=64)
     need = ba.ba_bwd_workspace_size(p, 128, 2)
     assert call_bwd(p, ws_bytes=need - 1) == ba.BA_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------- rotary ---
+
+def test_rope_workspace_sizes():
+    p = prob(batch=3, T=1000, H=2, D=128)
+    for plain, rope, esz in ((ba.ba_fwd_workspace_size, ba.ba_rope_fwd_workspace_size, 2),
+                             (ba.ba_bwd_workspace_size, ba.ba_rope_bwd_workspace_size, 2)):
+        extra = 2 * ((1000 * 2 * 128 * esz + 255) // 256 * 256)   # rotated copies of q and k
+        assert rope(p, 128, 2) == plain(p, 128, 2) + extra
+    p32 = prob(batch=1, T=77, H=3, D=32, dt=ba.BA_F32)
+    assert ba.ba_rope_fwd_workspace_size(p32, 64, 1) == \
+        ba.ba_fwd_workspace_size(p32, 64, 1) + 2 * ((77 * 3 * 32 * 4 + 255) // 256 * 256)
+    assert ba.ba_rope_fwd_workspace_size(prob(batch=-1), 128, 2) == 0
+    assert ba.ba_rope_bwd_workspace_size(p, 128, 0) == 0
+
+
+def test_rope_rejects_bad_arguments_before_launching():
+    p = prob(batch=2, T=300, H=4, D=64)
+    need_f = ba.ba_rope_fwd_workspace_size(p, 128, 2)
+    need_b = ba.ba_rope_bwd_workspace_size(p, 128, 2)
+    good = ba.BARope(FAKE, FAKE, 300)
+
+    def fwd(rope, ws_bytes=need_f):
+        return ba.ba_rope_fwd(p, rope, FAKE, FAKE, FAKE, FAKE, 128, 2, None, FAKE, FAKE, FAKE,
+                              workspace_bytes=ws_bytes, stream=0)
+
+    def bwd(rope, ws_bytes=need_b):
+        return ba.ba_rope_bwd(p, rope, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 2, None, FAKE, FAKE, FAKE,
+                              FAKE, workspace_bytes=ws_bytes, stream=0)
+
+    for call in (fwd, bwd):
+        assert call(None) == ba.BA_ERR_INVALID_ARG                                   # no tables
+        assert call(ba.BARope(None, FAKE, 300)) == ba.BA_ERR_INVALID_ARG             # null cos
+        assert call(ba.BARope(FAKE, None, 300)) == ba.BA_ERR_INVALID_ARG             # null sin
+        assert call(ba.BARope(FAKE + 8, FAKE, 300)) == ba.BA_ERR_INVALID_ARG         # misaligned
+        assert call(ba.BARope(FAKE, FAKE, 0)) == ba.BA_ERR_INVALID_ARG               # no rows
+    # the plain entry points' workspace is too small: the rotated copies need room
+    assert fwd(good, ba.ba_fwd_workspace_size(p, 128, 2)) == ba.BA_ERR_INVALID_ARG
+    assert bwd(good, need_b - 1) == ba.BA_ERR_INVALID_ARG
+
+
+def test_rope_saved_copies_must_come_in_pairs():
+    p = prob(batch=2, T=300, H=4, D=64)
+    need_b = ba.ba_rope_bwd_workspace_size(p, 128, 2)
+    for rope in (ba.BARope(FAKE, FAKE, 300, FAKE, None), ba.BARope(FAKE, FAKE, 300, None, FAKE),
+                 ba.BARope(FAKE, FAKE, 300, FAKE + 4, FAKE), ba.BARope(FAKE, FAKE, 300, FAKE, FAKE + 2)):
+        assert ba.ba_rope_fwd(p, rope, FAKE, FAKE, FAKE, FAKE, 128, 2, None, FAKE, FAKE, FAKE,
+                              workspace_bytes=need_b, stream=0) == ba.BA_ERR_INVALID_ARG
+        assert ba.ba_rope_bwd(p, rope, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 2, None, FAKE, FAKE, FAKE,
+                              FAKE, workspace_bytes=need_b, stream=0) == ba.BA_ERR_INVALID_ARG

@@ -1,5 +1,6 @@
-"""bench.py's workload selection: --swa W runs the sliding window (block 1, window W) and
---block/--window override the block rule, on the config's own shapes and seeds."""
+"""bench.py's workload selection: --swa W runs the sliding window (block 1, window W),
+--block/--window override the block rule and --rope adds the rotary embedding, all on the
+config's own shapes and seeds."""
 import importlib.util
 import os
 
@@ -45,3 +46,16 @@ def test_block_window_overrides():
 def test_job_totals_single_rank_is_identity():
     b = _bench()
     assert b.job_totals(5.0, 7.0, 3.0) == (5.0, 7.0, 3.0)
+
+
+def test_rope_option_keeps_the_workload_and_covers_the_longest_example():
+    b = _bench()
+    a = Args()
+    a.rope = True
+    w = b.config_workload(a)
+    base = b.config_workload(Args())
+    assert w.name == base.name + ", rotary q/k"
+    assert (w.block, w.window, w.batch, w.heads, w.head_dim, w.seed) == \
+        (base.block, base.window, base.batch, base.heads, base.head_dim, base.seed)
+    cos, sin = b.tables_for([64, 4096, 17], 128)
+    assert cos.shape == sin.shape == (4096, 64)
