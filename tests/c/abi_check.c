@@ -1,0 +1,91 @@
+/*
+ * Plain-C client of the block-attention library: compiled with a C compiler
+ * against include/ba.h and linked against libba.so. It checks that the
+ * header is valid C99 and exercises only calls that never reach the device:
+ * status strings, the version, workspace-size arithmetic and argument
+ * errors that are returned before anything is launched.
+ * Exit status 0 = every check passed; otherwise the number of failures.
+ */
+#include "ba.h"
+
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+static int failures = 0;
+
+#define CHECK(cond)                                                                 \
+    do {                                                                            \
+        if (!(cond)) {                                                              \
+            fprintf(stderr, "%s:%d: check failed: %s\n", __FILE__, __LINE__, #cond); \
+            ++failures;                                                             \
+        }                                                                           \
+    } while (0)
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int main(void)
+{
+    /* a never-dereferenced, 256-byte-aligned address: every call below fails its checks first */
+    void *fake = (void *)(uintptr_t)(1u << 20);
+    ba_problem p;
+    ba_rope rope;
+    size_t f, b, rf, rb;
+
+    CHECK(strcmp(ba_status_string(BA_OK), "ok") == 0);
+    CHECK(strcmp(ba_status_string(BA_ERR_TIMEOUT), "device wait timed out") == 0);
+    CHECK(ba_version() >= 100);
+
+    p.batch = 3;
+    p.total_tokens = 1000;
+    p.heads = 2;
+    p.head_dim = 128;
+    p.dtype = BA_BF16;
+    f = ba_fwd_workspace_size(&p, 128, 2);
+    b = ba_bwd_workspace_size(&p, 128, 2);
+    CHECK(f > 0 && f % 256 == 0 && b > f);
+    /* the backward adds two float per-row buffers [heads, total_tokens] */
+    CHECK(b == f + 2 * align256(4u * 2 * 1000));
+    /* the rotary forms add two rotated copies of a [T, H, D] bf16 tensor */
+    rf = ba_rope_fwd_workspace_size(&p, 128, 2);
+    rb = ba_rope_bwd_workspace_size(&p, 128, 2);
+    CHECK(rf == f + 2 * align256((size_t)1000 * 2 * 128 * 2));
+    CHECK(rb == b + 2 * align256((size_t)1000 * 2 * 128 * 2));
+    /* sliding window = block 1 */
+    CHECK(ba_swa_fwd_workspace_size(&p, 64) == ba_fwd_workspace_size(&p, 1, 64));
+    /* invalid problems size to 0 */
+    CHECK(ba_fwd_workspace_size(&p, 0, 2) == 0);
+    CHECK(ba_fwd_workspace_size(NULL, 128, 2) == 0);
+
+    /* argument errors come back before any launch */
+    CHECK(ba_fwd(NULL, fake, fake, fake, fake, 128, 2, NULL, fake, fake, fake, f, NULL) == BA_ERR_INVALID_ARG);
+    CHECK(ba_fwd(&p, fake, fake, fake, fake, 0, 2, NULL, fake, fake, fake, f, NULL) == BA_ERR_INVALID_ARG);
+    CHECK(ba_fwd(&p, fake, fake, fake, fake, 128, 2, NULL, fake, fake, fake, f - 1, NULL) == BA_ERR_INVALID_ARG);
+    CHECK(ba_bwd(&p, fake, fake, fake, fake, fake, fake, fake, 128, 2, NULL, fake, fake, NULL, fake, b, NULL) ==
+          BA_ERR_INVALID_ARG);
+    p.head_dim = 96;
+    CHECK(ba_fwd(&p, fake, fake, fake, fake, 128, 2, NULL, fake, fake, fake, 1u << 30, NULL) == BA_ERR_UNSUPPORTED);
+    p.head_dim = 128;
+
+    memset(&rope, 0, sizeof(rope));
+    CHECK(ba_rope_fwd(&p, NULL, fake, fake, fake, fake, 128, 2, NULL, fake, fake, fake, rf, NULL) ==
+          BA_ERR_INVALID_ARG);
+    CHECK(ba_rope_fwd(&p, &rope, fake, fake, fake, fake, 128, 2, NULL, fake, fake, fake, rf, NULL) ==
+          BA_ERR_INVALID_ARG); /* no tables */
+    rope.cos = (const float *)fake;
+    rope.sin = (const float *)fake;
+    rope.rows = 1000;
+    rope.q_rot = fake; /* k_rot missing */
+    CHECK(ba_rope_bwd(&p, &rope, fake, fake, fake, fake, fake, fake, fake, 128, 2, NULL, fake, fake, fake, fake, rb,
+                      NULL) == BA_ERR_INVALID_ARG);
+    rope.q_rot = NULL;
+    CHECK(ba_rope_fwd(&p, &rope, fake, fake, fake, fake, 128, 2, NULL, fake, fake, fake, f, NULL) ==
+          BA_ERR_INVALID_ARG); /* the plain workspace has no room for the rotated copies */
+
+    CHECK(ba_selftest_wait_timeout(NULL, 256, 1000, NULL) == BA_ERR_INVALID_ARG);
+    CHECK(ba_set_profile_events(3, NULL, NULL) == BA_ERR_INVALID_ARG);
+    CHECK(ba_device_status(NULL, NULL) == BA_ERR_INVALID_ARG);
+
+    if (failures == 0) printf("abi_check: all checks passed\n");
+    return failures;
+}

@@ -155,3 +155,23 @@ def test_rope_saved_copies_must_come_in_pairs():
                               workspace_bytes=need_b, stream=0) == ba.BA_ERR_INVALID_ARG
         assert ba.ba_rope_bwd(p, rope, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 2, None, FAKE, FAKE, FAKE,
                               FAKE, workspace_bytes=need_b, stream=0) == ba.BA_ERR_INVALID_ARG
+
+
+def test_header_is_c99_and_a_c_client_links(tmp_path):
+    """tests/c/abi_check.c: a plain-C client compiled with -std=c99 -pedantic
+    against include/ba.h and linked against libba.so; it runs only calls that
+    never reach the device (sizes, status strings, argument errors)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    lib_dir = os.path.dirname(ba.library_path())
+    exe = str(tmp_path / "abi_check")
+    subprocess.run([cc, "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                    "-I", os.path.join(root, "include"), os.path.join(root, "tests", "c", "abi_check.c"),
+                    "-o", exe, "-L", lib_dir, "-l:libba.so", f"-Wl,-rpath,{lib_dir}"], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert "all checks passed" in r.stdout
