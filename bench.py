@@ -50,7 +50,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--config", type=int, default=3, choices=sorted(CONFIGS))
+    # config 1 is the fp32 forward parity configuration; the benchmark times the bf16 path
+    ap.add_argument("--config", type=int, default=3, choices=[c for c in sorted(CONFIGS) if c != 1])
     ap.add_argument("--examples", type=int, default=0,
                     help="keep only the first N examples (small cases for profiling)")
     ap.add_argument("--block", type=int, default=0, help="override the config's block size")

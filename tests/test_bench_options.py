@@ -59,3 +59,25 @@ def test_rope_option_keeps_the_workload_and_covers_the_longest_example():
         (base.block, base.window, base.batch, base.heads, base.head_dim, base.seed)
     cos, sin = b.tables_for([64, 4096, 17], 128)
     assert cos.shape == sin.shape == (4096, 64)
+
+
+def test_reference_arm_prints_one_contract_line():
+    """bench.py --impl reference (the oracle on the host cores) prints one JSON
+    line with the contract's keys; config 2 (one 1024-token example per step)
+    keeps it to seconds."""
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "2",
+                        "--steps", "2", "--warmup", "1"], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 2
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert "workload" in d["config"]
