@@ -167,15 +167,13 @@ def positions(seq_offsets):
     return np.arange(int(offs[-1]), dtype=np.int64) - np.repeat(offs[:-1], lens)
 
 
-def _rotate_at(x, pos, cos, sin, transpose, fp32=False):
+def _rotate_at(x, pos, cos, sin, transpose):
     """Rotate the adjacent pairs of rows x[n, ..., D] sitting at positions pos[n]:
     y[2k] = x[2k] c - x[2k+1] s, y[2k+1] = x[2k] s + x[2k+1] c with c, s the
-    tables' entries at [pos, k]. transpose=True applies the transposed 2 x 2
-    map instead (c, s) -> (c, -s), which takes a gradient with respect to y
-    to the gradient with respect to x; it is also the inverse when the
-    tables hold exact cosines and sines. fp32=True evaluates the same
-    formula in float32, each product and the sum rounded once (used only to
-    decide the bf16 rounding of the rotated operands, see _rotated_operand)."""
+    tables' entries at [pos, k], in fp64. transpose=True applies the
+    transposed 2 x 2 map instead (c, s) -> (c, -s), which takes a gradient
+    with respect to y to the gradient with respect to x; it is also the
+    inverse when the tables hold exact cosines and sines."""
     x = _f64(x)
     cos = np.asarray(cos, dtype=np.float64)
     sin = np.asarray(sin, dtype=np.float64)
@@ -191,37 +189,47 @@ def _rotate_at(x, pos, cos, sin, transpose, fp32=False):
     if transpose:
         s = -s
     x0, x1 = x[..., 0::2], x[..., 1::2]
-    if fp32:
-        x0, x1, c, s = (a.astype(np.float32) for a in (x0, x1, c, s))
-    y = np.empty(x.shape, dtype=x0.dtype)
+    y = np.empty_like(x)
     y[..., 0::2] = x0 * c - x1 * s
     y[..., 1::2] = x0 * s + x1 * c
-    return y.astype(np.float64)
+    return y
 
 
-def rope_rotate(x, seq_offsets, cos, sin, transpose=False, fp32=False):
-    """Rotary embedding of every row of x [T, H, D] at its local position
-    (transpose=True: the transposed rotation; fp32: see _rotate_at)."""
-    return _rotate_at(x, positions(seq_offsets), cos, sin, transpose, fp32)
+def rope_rotate(x, seq_offsets, cos, sin, transpose=False):
+    """Rotary embedding of every row of x [T, H, D] at its local position, in
+    fp64 (transpose=True: the transposed rotation)."""
+    return _rotate_at(x, positions(seq_offsets), cos, sin, transpose)
+
+
+def round_bf16(x):
+    """Round fp64 values to the nearest bfloat16 value, ties to the even
+    significand, straight from the definition: bfloat16 keeps 8 significant
+    bits and float32's exponent range, so with x = m 2^e (0.5 <= |m| < 1) the
+    result is rint(m 2^8) 2^(e - 8); numpy's rint rounds half to even and
+    m 2^8 is exact in fp64. Only finite values inside bfloat16's normal range
+    are used here (|x| in [2^-126, 2^128) or 0)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
 
 
 def _rotated_operand(x, seq_offsets, cos, sin, operand_dtype):
-    """The rotated q or k as the attention's products take it. None: exact
-    (fp64). A dtype (torch.bfloat16): the rotation rounded to that dtype,
-    nearest even. Which way a value near a rounding tie goes is a
-    quantisation decision, so it is taken in the precision the library
-    takes it in: the float32 value of the formula, each product and the sum
-    rounded once."""
+    """The rotated q or k as the attention's products take it. None: the
+    exact fp64 rotation. torch.bfloat16: that exact rotation rounded to the
+    nearest bfloat16 value (ties to even), the operand type of a library
+    whose tensor-core products take the input dtype."""
+    y = rope_rotate(x, seq_offsets, cos, sin)
     if operand_dtype is None:
-        return rope_rotate(x, seq_offsets, cos, sin)
-    y = rope_rotate(x, seq_offsets, cos, sin, fp32=True).astype(np.float32)
-    return torch.from_numpy(y).to(operand_dtype).to(torch.float64).numpy()
+        return y
+    if operand_dtype != torch.bfloat16:
+        raise ValueError("operand_dtype must be None or torch.bfloat16")
+    return round_bf16(y)
 
 
 def rope_fwd(seq_offsets, q, k, v, cos, sin, block, window, skip=None, operand_dtype=None, nthreads=None):
-    """Block attention of the rotated q and k. operand_dtype (e.g.
-    torch.bfloat16) rounds the rotated q and k to that dtype first, as a
-    library that feeds them to tensor-core products in the input dtype does."""
+    """Block attention of the rotated q and k. operand_dtype=torch.bfloat16
+    rounds the exact rotated q and k to bfloat16 first, as a library that
+    feeds them to tensor-core products in the input dtype holds them."""
     qr = _rotated_operand(q, seq_offsets, cos, sin, operand_dtype)
     kr = _rotated_operand(k, seq_offsets, cos, sin, operand_dtype)
     return fwd(seq_offsets, qr, kr, v, block, window, skip=skip, nthreads=nthreads)

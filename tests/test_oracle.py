@@ -495,27 +495,59 @@ def test_rope_tables_shorter_than_an_example_are_rejected():
         oracle.rope_fwd(offs, q, k, v, cos, sin, 4, 1)
 
 
-def test_rope_float32_form_is_the_formula_rounded_per_operation():
-    """The float32 evaluation (used only to decide the bf16 rounding of the
-    rotated operands) is the same formula: within the error of three float32
-    roundings of the fp64 value, and the rounded operands it gives differ
-    from rounding the exact value by at most one bf16 step."""
+def _bf16_neighbours(x):
+    """The two bfloat16 values around each fp64 x (x > 0), found by walking
+    float32 bit patterns whose low 16 bits are zero."""
+    f = np.float32(x)
+    bits = np.array([f]).view(np.uint32)[0] & np.uint32(0xFFFF0000)
+    lo = np.array([bits], dtype=np.uint32).view(np.float32)[0].astype(np.float64)
+    if lo > x:
+        bits -= np.uint32(0x10000)
+        lo = np.array([bits], dtype=np.uint32).view(np.float32)[0].astype(np.float64)
+    hi_bits = bits + np.uint32(0x10000)
+    hi = np.array([hi_bits], dtype=np.uint32).view(np.float32)[0].astype(np.float64)
+    return lo, hi, int(bits >> 16) & 1
+
+
+def test_round_bf16_is_nearest_with_ties_to_even():
+    """round_bf16 (the rounding of the rotated operands) against a brute-force
+    search of the two neighbouring bfloat16 values, exact midpoints (which
+    go to the even significand), values a hair off a midpoint (where
+    rounding through float32 first would land on the midpoint and go the
+    wrong way), and torch's float32 -> bfloat16 cast on float32 inputs."""
+    rng = np.random.default_rng(497)
+    xs = np.concatenate([rng.standard_normal(2000) * 10.0 ** rng.integers(-6, 6, 2000),
+                         rng.uniform(0.5, 8.0, 200)])
+    got = oracle.round_bf16(xs)
+    for x, g in zip(xs, got):
+        a = abs(x)
+        lo, hi, lo_odd = _bf16_neighbours(a)
+        want = lo if (a - lo < hi - a or (a - lo == hi - a and not lo_odd)) else hi
+        assert g == np.copysign(want, x), (x, g, want)
+    for a in (1.0, 3.0, 0.0078125, 1000.0):
+        lo, hi, lo_odd = _bf16_neighbours(a * (1 + 2.0 ** -20))
+        mid = (lo + hi) / 2
+        assert oracle.round_bf16(mid) == (hi if lo_odd else lo)
+        assert oracle.round_bf16(-mid) == -(hi if lo_odd else lo)
+        # just above the midpoint rounds up, even where float32 would first round onto the midpoint
+        above = mid * (1 + 2.0 ** -40)
+        assert np.float32(above) == np.float32(mid)
+        assert oracle.round_bf16(above) == hi
+    f32 = rng.standard_normal(5000).astype(np.float32)
+    ref = torch.from_numpy(f32).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(oracle.round_bf16(f32.astype(np.float64)), ref)
+    assert oracle.round_bf16(np.array([0.0]))[0] == 0.0
+
+
+def test_rotated_bf16_operands_are_the_exact_rotation_rounded():
     rng = np.random.default_rng(508)
     offs, q, _, _, _ = rand_case(rng, [50, 30], 2, 16, scale=3.0)
-    q = torch.from_numpy(q).to(torch.bfloat16).double().numpy()       # operands as the library sees them
+    q = torch.from_numpy(q).to(torch.bfloat16).double().numpy()
     cos, sin, _ = _exact_tables(64, 16)
-    cos, sin = cos.astype(np.float32).astype(np.float64), sin.astype(np.float32).astype(np.float64)
     exact = oracle.rope_rotate(q, offs, cos, sin)
-    f32 = oracle.rope_rotate(q, offs, cos, sin, fp32=True)
-    pos = oracle.positions(offs)
-    c = cos[pos][:, None, :]
-    s = sin[pos][:, None, :]
-    mag = np.empty_like(q)
-    mag[..., 0::2] = np.abs(q[..., 0::2] * c) + np.abs(q[..., 1::2] * s)
-    mag[..., 1::2] = np.abs(q[..., 0::2] * s) + np.abs(q[..., 1::2] * c)
-    assert np.all(np.abs(f32 - exact) <= 3 * 2.0 ** -24 * mag * (1 + 1e-6))
     a = oracle._rotated_operand(q, offs, cos, sin, torch.bfloat16)
-    b = torch.from_numpy(exact).to(torch.bfloat16).double().numpy()
-    step = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(b), 1e-30))) - 7)
-    assert np.all(np.abs(a - b) <= step * (1 + 1e-9))
-    assert np.mean(a == b) > 0.99
+    assert np.array_equal(a, oracle.round_bf16(exact))
+    assert np.array_equal(oracle._rotated_operand(q, offs, cos, sin, None), exact)
+    # each rounded value is within half a bfloat16 step of the exact one
+    step = 2.0 ** (np.floor(np.log2(np.abs(exact))) - 7)
+    assert np.all(np.abs(a - exact) <= step / 2)
