@@ -77,6 +77,7 @@ struct DkvBarriers {
     uint64_t q_full[4], q_empty[4], o_full[4], o_empty[4];
     uint64_t s_full, dp_full, pa_done[2], pb_done[2];
     uint64_t epi_sync; // group barrier of the epilogue warps
+    uint64_t tail;     // the TMA warp's own barrier for a Q or dO tile whose last rows it clears
     uint32_t tmem_base;
     int abort;
     // per Q slot: -lse in log2 units and -Delta of the tile's 128 queries
@@ -127,6 +128,7 @@ __global__ void __launch_bounds__(448, 1)
         mbar_init(&sb.s_full, 1);
         mbar_init(&sb.dp_full, 1);
         mbar_init(&sb.epi_sync, 128);
+        mbar_init(&sb.tail, 1);
         for (int g = 0; g < 2; ++g) {
             mbar_init(&sb.pa_done[g], 4);
             mbar_init(&sb.pb_done[g], 4);
@@ -155,7 +157,7 @@ __global__ void __launch_bounds__(448, 1)
 
     if (warp == 12) {
         // ------------------------------------------------ TMA producer ---
-        uint32_t it = 0, item_cnt = 0;
+        uint32_t it = 0, item_cnt = 0, tail_phase = 0;
         TileRef r;
         bool ok = true;
         ItemWalker items(p.tile_info, ntiles, p.heads);
@@ -168,11 +170,14 @@ __global__ void __launch_bounds__(448, 1)
                     ok = false;
                     break;
                 }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&sb.q_full[qs], Lay::kTileBytes);
-                    for (int c = 0; c < Lay::kChunks; ++c)
-                        tma_load_2d(smem + Lay::kQ0 + qs * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_q,
-                                    &sb.q_full[qs], r.h * D + c * 64, r.s0 + i * kTile);
+                // the example's last query tile: its rows past the example are cleared (Q here,
+                // dO below), since dK += dS^T Q and dV += P^T dO multiply them by zeros
+                const int valid = r.L - i * kTile;
+                if (!load_tile_zero_tail<Lay::kChunks>(smem + Lay::kQ0 + qs * Lay::kTileBytes, &tm_q, &sb.q_full[qs],
+                                                       &sb.tail, tail_phase, r.h * D, r.s0 + i * kTile, valid,
+                                                       abort)) {
+                    ok = false;
+                    break;
                 }
                 // the tile's -lse (log2 units) and -Delta, four queries per lane, copied
                 // asynchronously; each lane's copies arrive on q_full when they land. Rows past
@@ -217,11 +222,13 @@ __global__ void __launch_bounds__(448, 1)
                     ok = false;
                     break;
                 }
+                if (!load_tile_zero_tail<Lay::kChunks>(smem + Lay::kO0 + os * Lay::kTileBytes, &tm_do, &sb.o_full[os],
+                                                       &sb.tail, tail_phase, r.h * D, r.s0 + i * kTile, valid,
+                                                       abort)) {
+                    ok = false;
+                    break;
+                }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&sb.o_full[os], Lay::kTileBytes);
-                    for (int c = 0; c < Lay::kChunks; ++c)
-                        tma_load_2d(smem + Lay::kO0 + os * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_do,
-                                    &sb.o_full[os], r.h * D + c * 64, r.s0 + i * kTile);
                     // warm L2 two query tiles ahead, and with the next item's K, V and first tiles
                     if (i + 2 <= ihi)
                         for (int c = 0; c < Lay::kChunks; ++c) {

@@ -63,6 +63,7 @@ struct DqBarriers {
     uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
     uint64_t st_full, st_empty, qt_ready;
     uint64_t s_full, s_free, dp_full, ds_full[2], dq_done, dq_free;
+    uint64_t tail; // the TMA warp's own barrier for a K or V tile whose last rows it clears
     uint32_t tmem_base;
     int abort;
 };
@@ -108,6 +109,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(&sb.ds_full[1], 4);
         mbar_init(&sb.dq_done, 1);
         mbar_init(&sb.dq_free, 8);
+        mbar_init(&sb.tail, 1);
         sb.abort = 0;
         fence_mbar_init();
     }
@@ -136,7 +138,7 @@ __global__ void __launch_bounds__(384, 1)
         warpgroup_regs_dec<Lay::kRegsOther>();
         if (warp == 8) {
             // ------------------------------------------------ TMA producer ---
-            uint32_t kv_cnt = 0, item_cnt = 0;
+            uint32_t kv_cnt = 0, item_cnt = 0, tail_phase = 0;
             TileRef r;
             bool ok = true;
             ItemWalker items(p.tile_info, ntiles, p.heads);
@@ -158,28 +160,21 @@ __global__ void __launch_bounds__(384, 1)
                     const int st = kv_cnt % S;
                     uint8_t *kdst = smem + Lay::kKV0 + 2 * st * Lay::kTileBytes;
                     // K is read until dQ, V only by dP: they are released and refilled separately
-                    if (!mbar_wait(&sb.k_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
+                    // the example's last K and V tiles: rows past the example are cleared, since
+                    // dQ += dS K and the masked dS = P (dP - Delta) multiply them by zeros
+                    const int valid = r.L - j * kTile;
+                    if (!mbar_wait(&sb.k_empty[st], ((kv_cnt / S) & 1) ^ 1, abort) ||
+                        !load_tile_zero_tail<Lay::kChunks>(kdst, &tm_k, &sb.k_full[st], &sb.tail, tail_phase,
+                                                           r.h * D, r.s0 + j * kTile, valid, abort)) {
                         ok = false;
                         break;
                     }
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(&sb.k_full[st], Lay::kTileBytes);
-                        for (int c = 0; c < Lay::kChunks; ++c)
-                            tma_load_2d(kdst + c * Lay::kChunkBytes, &tm_k, &sb.k_full[st], r.h * D + c * 64,
-                                        r.s0 + j * kTile);
-                    }
-                    __syncwarp();
-                    if (!mbar_wait(&sb.v_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
+                    if (!mbar_wait(&sb.v_empty[st], ((kv_cnt / S) & 1) ^ 1, abort) ||
+                        !load_tile_zero_tail<Lay::kChunks>(kdst + Lay::kTileBytes, &tm_v, &sb.v_full[st], &sb.tail,
+                                                           tail_phase, r.h * D, r.s0 + j * kTile, valid, abort)) {
                         ok = false;
                         break;
                     }
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(&sb.v_full[st], Lay::kTileBytes);
-                        for (int c = 0; c < Lay::kChunks; ++c)
-                            tma_load_2d(kdst + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_v, &sb.v_full[st],
-                                        r.h * D + c * 64, r.s0 + j * kTile);
-                    }
-                    __syncwarp();
                 }
             }
         } else if (warp == 9) {

@@ -65,6 +65,7 @@ struct FwdBarriers {
     uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
     uint64_t o_ready[2]; // group w's softmax is done with its item: inv_l[w] holds 1 / l
     uint64_t epi_sync;   // group barrier of the epilogue warpgroup
+    uint64_t tail;       // the TMA warp's own barrier for a V tile whose last rows it clears
     float inv_l[2][kTile];
     uint32_t tmem_base;
     int abort;
@@ -113,6 +114,7 @@ __global__ void __launch_bounds__(512, 1)
             mbar_init(&sb.v_empty[i], 1);
         }
         mbar_init(&sb.epi_sync, 128);
+        mbar_init(&sb.tail, 1);
         sb.abort = 0;
         fence_mbar_init();
     }
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(512, 1)
         warpgroup_regs_dec<Lay::kRegsOther>();
         if (warp == 8) {
             // ------------------------------------------------ TMA producer ---
-            uint32_t kv_cnt = 0, item_cnt = 0;
+            uint32_t kv_cnt = 0, item_cnt = 0, tail_phase = 0;
             uint32_t qcnt[2] = {0, 0}; // query tiles loaded per group
             TileRef r;
             bool second;
@@ -195,13 +197,15 @@ __global__ void __launch_bounds__(512, 1)
                         ok = false;
                         break;
                     }
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(&sb.v_full[st], Lay::kTileBytes);
-                        for (int c = 0; c < Lay::kChunks; ++c)
-                            tma_load_2d(kdst + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_v, &sb.v_full[st],
-                                        r.h * D + c * 64, r.s0 + j * kTile);
+                    // the example's last V tile: its rows past the example are cleared, since
+                    // P V multiplies them by zero probabilities (K needs nothing: masked scores
+                    // are replaced, not multiplied)
+                    if (!load_tile_zero_tail<Lay::kChunks>(kdst + Lay::kTileBytes, &tm_v, &sb.v_full[st], &sb.tail,
+                                                           tail_phase, r.h * D, r.s0 + j * kTile,
+                                                           r.L - j * kTile, abort)) {
+                        ok = false;
+                        break;
                     }
-                    __syncwarp();
                 }
             }
         } else if (warp == 9) {

@@ -182,6 +182,48 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Loads one 128-row tile of a [rows, columns] bf16 tensor map (CHUNKS boxes of
+// 128 rows x 64 columns, each a 16 KB 128B-swizzled chunk at dst + c * 16 KB)
+// and signals `full`. When only the first `valid` rows belong to the current
+// example (valid < 128), the rows after them hold the next example's data,
+// which a masked product would still multiply by a zero probability (and
+// 0 x inf is NaN). Such a tile completes on the warp's private barrier
+// `tail` instead; the warp waits for it, clears the rows [valid, 128) of every
+// chunk (the swizzle permutes 16-byte units only within a row's own 128
+// bytes, so a row is the same 128 bytes swizzled or not), makes the clears
+// visible to the tensor core's operand reads and then arrives on `full` (one
+// plain arrival in place of the expect_tx one). Called by all 32 lanes of
+// the producer warp; false after a timed-out wait.
+template <int CHUNKS>
+__device__ __forceinline__ bool load_tile_zero_tail(uint8_t *dst, const CUtensorMap *map, uint64_t *full,
+                                                    uint64_t *tail, uint32_t &tail_phase, int32_t x, int32_t y,
+                                                    int valid, volatile int *abort)
+{
+    constexpr uint32_t kChunkBytes = 128 * 128;
+    const int lane = threadIdx.x & 31;
+    const bool clear = valid < 128;
+    if (lane == 0) {
+        uint64_t *bar = clear ? tail : full;
+        mbar_arrive_expect_tx(bar, CHUNKS * kChunkBytes);
+        for (int c = 0; c < CHUNKS; ++c) tma_load_2d(dst + c * kChunkBytes, map, bar, x + 64 * c, y);
+    }
+    __syncwarp();
+    if (!clear) return true;
+    if (!mbar_wait(tail, tail_phase, abort)) return false;
+    tail_phase ^= 1;
+    const int v = valid < 0 ? 0 : valid;
+    const int units = (128 - v) * 8; // 16-byte units from row v to the end of a chunk
+    for (int c = 0; c < CHUNKS; ++c) {
+        uint4 *z = reinterpret_cast<uint4 *>(dst + c * kChunkBytes + v * 128);
+        for (int u = lane; u < units; u += 32) z[u] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(full);
+    __syncwarp();
+    return true;
+}
+
 // -------------------------------------------------------------- tcgen05 ---
 
 // Whole warp: allocate `ncols` TMEM columns; the base address lands in *slot.

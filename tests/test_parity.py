@@ -263,3 +263,58 @@ def test_sliding_window_full_size_sampled():
             for n in ("out", "dq", "dk", "dv"):
                 check_bf16(f"swa e{e} h{h} {n}", f64(got[n][sl][rows, h]), ref[n])
             check_abs(f"swa e{e} h{h} lse", f64(got["lse"][h, s0:s0 + L][rows]), ref["lse"], 2e-3)
+
+
+# ------------------------------------------------ isolation of examples ---
+# The oracle's examples are independent (tests/test_oracle.py: a jagged batch
+# equals separate runs). On the GPU a 128-row tile at an example's end also
+# loads the next example's rows; these cases put Inf and NaN there (and in a
+# skipped example) and require every other example's results to be bit-equal
+# to a clean run and within tolerance of the oracle.
+
+ISOLATION = [
+    # (dtype, head_dim, block, window)
+    (torch.bfloat16, 128, 256, 2),
+    (torch.bfloat16, 64, 64, 1),
+    (torch.bfloat16, 128, 100, 3),
+    (torch.float32, 32, 48, 2),
+]
+
+
+def _poison(t, s0, n):
+    pattern = torch.tensor([float("inf"), float("nan"), float("-inf")], dtype=t.dtype)
+    rows = t[s0:s0 + n]
+    rows.copy_(pattern.repeat(rows.numel() // 3 + 1)[: rows.numel()].view_as(rows))
+
+
+@pytest.mark.parametrize("dtype,head_dim,block,window", ISOLATION)
+def test_examples_are_isolated_from_non_finite_neighbours(dtype, head_dim, block, window):
+    lengths = [300, 200, 1000, 129, 777, 90, 128, 5]
+    skip = torch.tensor([0, 0, 0, 1, 0, 0, 0, 0], dtype=torch.uint8)
+    base = CONFIGS[1] if dtype == torch.float32 else CONFIGS[3]
+    w = base.replace(head_dim=head_dim, block=block, window=window, heads=2, batch=len(lengths),
+                     fwd_only=False)
+    inp = make_inputs(w, lengths=lengths, seed=4242 + head_dim)
+    inp["skip"] = skip
+    offs = inp["seq_offsets"].numpy()
+    poisoned = {1: 40, 3: lengths[3], 5: lengths[5], 7: lengths[7]}  # example -> rows poisoned from its start
+    dirty = dict(inp)
+    for n in ("q", "k", "v", "dout"):
+        dirty[n] = inp[n].clone()
+        for e, rows in poisoned.items():
+            _poison(dirty[n], int(offs[e]), rows)
+    clean_got = run_gpu(inp, block, window)
+    dirty_got = run_gpu(dirty, block, window)
+    ref = run_oracle(inp, block, window)
+    for e in range(len(lengths)):
+        if e in poisoned or lengths[e] == 0:
+            continue
+        sl = slice(int(offs[e]), int(offs[e + 1]))
+        for n in ("out", "dq", "dk", "dv"):
+            assert torch.equal(dirty_got[n][sl], clean_got[n][sl]), f"example {e} {n} changed by a neighbour"
+            if dtype == torch.float32:
+                check_abs(f"e{e} {n}", dirty_got[n][sl], ref[n][sl], 1e-5)
+            else:
+                check_bf16(f"e{e} {n}", dirty_got[n][sl], ref[n][sl])
+        assert torch.equal(dirty_got["lse"][:, sl], clean_got["lse"][:, sl]), f"example {e} lse changed"
+        check_abs(f"e{e} lse", dirty_got["lse"][:, sl], ref["lse"][:, sl], 1e-5 if dtype == torch.float32 else 2e-3)
