@@ -1,18 +1,19 @@
 // ba_fwd_noalloc: the forward pass for callers that cannot allocate device
 // memory, with its scratch in a fixed array compiled into the library.
 //
-// Who needs it: a serving loop that records its forward pass into a CUDA
-// graph (device allocation is not allowed while a stream is being captured),
-// or a host framework that owns every byte of device memory through its own
-// pool and gives kernels only their inputs and outputs. Such a caller cannot
-// obtain the workspace ba_fwd asks for, so this entry point brings its own.
+// Who needs it: a host framework that owns every byte of device memory
+// through its own pool and gives kernels only their inputs and outputs, or a
+// plugin running inside such a framework without access to its allocator.
+// Such a caller cannot obtain the workspace ba_fwd asks for, so this entry
+// point brings its own.
 //
 // The scratch is one file-scope __device__ array of kScratchBytes; every GPU
 // that loads the library holds it until the process exits. Its device address
 // is looked up once per device, on the first call made with that device
-// current, and cached; that first call must therefore not be made while a
-// stream is being captured. All calls share the array: two calls whose work
-// may overlap on the GPU (different streams, or different host threads
+// current, and cached for the life of the process (a context destroyed and
+// created again may place the array elsewhere, so the entry point is not for
+// use across a device reset). All calls share the array: two calls whose
+// work may overlap on the GPU (different streams, or different host threads
 // without ordering) race on it. Every byte the forward reads from the scratch
 // is written earlier in the same call (the work-list kernel rewrites the
 // status word, the tile prefix and the tile table), so nothing left behind by

@@ -211,20 +211,27 @@ ba_status ba_rope_bwd(const ba_problem *p, const ba_rope *rope, const void *q, c
 /*
  * Forward pass that allocates nothing and takes no workspace (the pages have
  * no counterpart; this is a convenience of this library). For callers that
- * cannot allocate device memory: a serving loop that records its forward into
- * a CUDA graph (allocation is not allowed during stream capture), or a host
- * framework that owns all device memory and hands kernels only their inputs
- * and outputs. Same arguments and results as ba_fwd minus the workspace.
+ * cannot call cudaMalloc: a host framework that owns every byte of device
+ * memory through its own pool and hands kernels only their inputs and
+ * outputs, or a plugin running inside such a framework with no handle on its
+ * allocator. Same arguments and results as ba_fwd minus the workspace.
  *  - Scratch: a fixed 1 MiB array inside the library, held by every GPU that
- *    loads it until the process exits. Problems whose ba_fwd_workspace_size
- *    exceeds 1 MiB are rejected with BA_ERR_INVALID_ARG before anything runs
- *    (roughly: ceil(total_tokens / 128) + batch must stay below ~65,000).
- *  - The first call on each device looks up the array's device address;
- *    make that first call before any stream capture.
+ *    loads it until the process exits. A problem whose ba_fwd_workspace_size
+ *    exceeds 1 MiB is rejected with BA_ERR_INVALID_ARG before anything runs.
+ *    The size is about 16 bytes per 128-row tile plus 16 per pair of tiles
+ *    plus 8 per example (and 1 KiB of fixed overhead), so one example of up
+ *    to about 5.5 million tokens fits; compare ba_fwd_workspace_size with
+ *    1 MiB to know for sure.
+ *  - The first call on each device, with that device current, looks up the
+ *    array's device address and caches it for the process. A context that is
+ *    destroyed and created again (cudaDeviceReset) may load the library's
+ *    device code elsewhere; do not use this entry point across such a reset.
  *  - All calls share the array: calls that may overlap on the GPU race and
  *    must be ordered by the caller (one stream, or events). Nothing a call
  *    reads from the array is left over from an earlier call.
- *  - ba_device_status cannot be used with this entry point (no workspace).
+ *  - ba_device_status cannot be used with this entry point (no workspace), so
+ *    a kernel wait that timed out here is not reported; use ba_fwd where that
+ *    matters.
  */
 ba_status ba_fwd_noalloc(const ba_problem *p, const void *q, const void *k, const void *v,
                          const int32_t *seq_offsets, int32_t block, int32_t window,
@@ -256,6 +263,20 @@ ba_status ba_device_status(const void *workspace, ba_stream_t stream);
  */
 ba_status ba_selftest_wait_timeout(void *workspace, size_t workspace_bytes, int32_t limit_us,
                                    ba_stream_t stream);
+
+/*
+ * Self-test of the attention kernels' FMA-pipe 2^x (the pages have no
+ * counterpart). To take load off the special-function unit, the softmax in
+ * the bf16 kernels evaluates some of its exponentials on the fused
+ * multiply-add pipe: x is split into the nearest integer n and f = x - n in
+ * [-1/2, 1/2], 2^f comes from a cubic fitted to it (relative error below
+ * 1e-4), and n is added to the exponent field; x below -125 is first raised
+ * to -125 (such values are far below anything a bf16 probability can hold
+ * next to the row maximum). This writes y[i] = that 2^x(i) for the n DEVICE
+ * floats x (y: DEVICE, n floats, not aliasing x), asynchronously on stream.
+ * Returns BA_ERR_INVALID_ARG for n < 0 or null/misaligned pointers.
+ */
+ba_status ba_selftest_exp2(const float *x, float *y, int64_t n, ba_stream_t stream);
 
 /*
  * Profiling hook. Until changed, calls made from THIS host thread record
