@@ -23,9 +23,10 @@ __all__ = [
     "BAError", "ba_fwd", "ba_fwd_noalloc", "ba_bwd", "ba_fwd_workspace_size", "ba_bwd_workspace_size",
     "ba_swa_fwd", "ba_swa_bwd", "ba_swa_fwd_workspace_size", "ba_swa_bwd_workspace_size",
     "ba_rope_fwd", "ba_rope_bwd", "ba_rope_fwd_workspace_size", "ba_rope_bwd_workspace_size",
-    "ba_device_status", "ba_selftest_wait_timeout", "ba_set_profile_events", "ba_status_string", "ba_version",
+    "ba_device_status", "ba_selftest_wait_timeout", "ba_selftest_exp2", "ba_set_profile_events", "ba_status_string", "ba_version",
     "block_attention_fwd", "block_attention_bwd", "sliding_window_attention_fwd", "sliding_window_attention_bwd",
     "rope_block_attention_fwd", "rope_block_attention_bwd",
+    "ba_gdpa_workspace_size", "ba_gdpa_fwd", "ba_gdpa_bwd", "gdpa_fwd", "gdpa_bwd",
     "library_path",
 ]
 
@@ -34,6 +35,8 @@ _LIB_PATH = os.path.join(_HERE, "libba.so")
 
 BA_OK, BA_ERR_INVALID_ARG, BA_ERR_UNSUPPORTED, BA_ERR_CUDA, BA_ERR_TIMEOUT = range(5)
 BA_F32, BA_BF16 = 0, 1
+BA_ACT_GELU, BA_ACT_SILU = 1, 2
+_ACTS = {"gelu": BA_ACT_GELU, "silu": BA_ACT_SILU}
 _DTYPES = {torch.float32: BA_F32, torch.bfloat16: BA_BF16}
 
 
@@ -90,6 +93,8 @@ def _load():
     lib.ba_version.restype = ctypes.c_int32
     lib.ba_selftest_wait_timeout.argtypes = [P, ctypes.c_size_t, i32, P]
     lib.ba_selftest_wait_timeout.restype = ctypes.c_int
+    lib.ba_selftest_exp2.argtypes = [P, P, ctypes.c_int64, P]
+    lib.ba_selftest_exp2.restype = ctypes.c_int
     lib.ba_swa_fwd_workspace_size.argtypes = [prob, i32]
     lib.ba_swa_fwd_workspace_size.restype = ctypes.c_size_t
     lib.ba_swa_bwd_workspace_size.argtypes = [prob, i32]
@@ -98,6 +103,12 @@ def _load():
     lib.ba_swa_fwd.restype = ctypes.c_int
     lib.ba_swa_bwd.argtypes = [prob, P, P, P, P, P, P, P, i32, P, P, P, P, P, ctypes.c_size_t, P]
     lib.ba_swa_bwd.restype = ctypes.c_int
+    lib.ba_gdpa_workspace_size.argtypes = [prob, i32, i32]
+    lib.ba_gdpa_workspace_size.restype = ctypes.c_size_t
+    lib.ba_gdpa_fwd.argtypes = [prob, ctypes.c_int, P, P, P, P, i32, i32, P, P, ctypes.c_size_t, P]
+    lib.ba_gdpa_fwd.restype = ctypes.c_int
+    lib.ba_gdpa_bwd.argtypes = [prob, ctypes.c_int, P, P, P, P, P, i32, i32, P, P, P, P, ctypes.c_size_t, P]
+    lib.ba_gdpa_bwd.restype = ctypes.c_int
     rope = ctypes.POINTER(BARope)
     lib.ba_rope_fwd_workspace_size.argtypes = [prob, i32, i32]
     lib.ba_rope_fwd_workspace_size.restype = ctypes.c_size_t
@@ -209,6 +220,71 @@ def ba_swa_bwd(problem, q, k, v, out, lse, dout, seq_offsets, window_tokens, ski
                                   _stream(stream)))
 
 
+def _act(activation) -> int:
+    if isinstance(activation, str):
+        if activation not in _ACTS:
+            raise ValueError(f"activation must be one of {sorted(_ACTS)}")
+        return _ACTS[activation]
+    return int(activation)
+
+
+def ba_gdpa_workspace_size(problem: BAProblem, block: int, window: int) -> int:
+    return int(_load().ba_gdpa_workspace_size(ctypes.byref(problem), int(block), int(window)))
+
+
+def ba_gdpa_fwd(problem, activation, q, k, v, seq_offsets, block, window, out, workspace,
+                workspace_bytes=None, stream=None) -> int:
+    """Direct call of the generalized-attention forward; returns its status code."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(_load().ba_gdpa_fwd(ctypes.byref(problem), _act(activation), _ptr(q), _ptr(k), _ptr(v),
+                                   _ptr(seq_offsets), int(block), int(window), _ptr(out), _ptr(workspace),
+                                   int(workspace_bytes), _stream(stream)))
+
+
+def ba_gdpa_bwd(problem, activation, q, k, v, dout, seq_offsets, block, window, dq, dk, dv, workspace,
+                workspace_bytes=None, stream=None) -> int:
+    """Direct call of the generalized-attention backward; returns its status code."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(_load().ba_gdpa_bwd(ctypes.byref(problem), _act(activation), _ptr(q), _ptr(k), _ptr(v),
+                                   _ptr(dout), _ptr(seq_offsets), int(block), int(window), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def gdpa_fwd(q, k, v, seq_offsets, block, window, activation="gelu", out=None, workspace=None, stream=None):
+    """Generalized dot-product attention (activation in place of the softmax,
+    block rule, no normalisation): allocates out (and a workspace) with torch
+    and runs ba_gdpa_fwd."""
+    _check_inputs(q, k, v, seq_offsets)
+    prob = make_problem(q, seq_offsets)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = workspace_for(ba_gdpa_workspace_size(prob, block, window), q.device)
+    st = ba_gdpa_fwd(prob, activation, q, k, v, seq_offsets, block, window, out, workspace, stream=stream)
+    if st != BA_OK:
+        raise BAError(st, "ba_gdpa_fwd")
+    return out
+
+
+def gdpa_bwd(q, k, v, dout, seq_offsets, block, window, activation="gelu", dq=None, dk=None, dv=None,
+             workspace=None, stream=None):
+    """Gradients of gdpa_fwd: allocates dq/dk/dv (and a workspace) with torch and runs ba_gdpa_bwd."""
+    _check_inputs(q, k, v, seq_offsets)
+    prob = make_problem(q, seq_offsets)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if workspace is None:
+        workspace = workspace_for(ba_gdpa_workspace_size(prob, block, window), q.device)
+    st = ba_gdpa_bwd(prob, activation, q, k, v, dout, seq_offsets, block, window, dq, dk, dv, workspace,
+                     stream=stream)
+    if st != BA_OK:
+        raise BAError(st, "ba_gdpa_bwd")
+    return dq, dk, dv
+
+
 def make_rope(cos, sin, q_rot=None, k_rot=None) -> BARope:
     """Rotary tables (float32 CUDA tensors [rows, head_dim / 2]) as the C
     struct, with optional caller buffers for the rotated q and k."""
@@ -268,6 +344,13 @@ def ba_selftest_wait_timeout(workspace, limit_us: int, workspace_bytes=None, str
         workspace_bytes = workspace.numel() * workspace.element_size()
     return int(_load().ba_selftest_wait_timeout(_ptr(workspace), int(workspace_bytes), int(limit_us),
                                                 _stream(stream)))
+
+
+def ba_selftest_exp2(x, y, stream=None) -> int:
+    """y = the kernels' FMA-pipe 2^x for float32 CUDA tensors x, y of equal size."""
+    if x.dtype != torch.float32 or y.dtype != torch.float32 or x.numel() != y.numel():
+        raise ValueError("x and y must be float32 tensors of equal size")
+    return int(_load().ba_selftest_exp2(_ptr(x), _ptr(y), int(x.numel()), _stream(stream)))
 
 
 def ba_device_status(workspace, stream=None) -> int:

@@ -6,6 +6,8 @@
 //   ba_bwd: worklist -> skip passthrough -> bf16: dQ kernel (also writes
 //           Delta) -> dK/dV kernel; fp32: Delta pre-pass -> dQ and dK/dV
 //           SIMT kernels
+//   ba_gdpa_fwd / ba_gdpa_bwd: worklist -> the same tensor-core kernels
+//           instantiated with an activation in place of the softmax
 //   ba_rope_fwd / ba_rope_bwd: the same, with a rotary pass writing rotated
 //           copies of q and k into the workspace before the attention
 //           kernels read them; the bf16 backward turns dq and dk back inside
@@ -166,9 +168,9 @@ cudaError_t prof_mark(int which, int edge, cudaStream_t stream)
     return e ? cudaEventRecord(e, stream) : cudaSuccess;
 }
 
-#define BA_TRY(expr)                                                                                      \
+#define BA_TRY(...)                                                                                       \
     do {                                                                                                  \
-        if ((expr) != cudaSuccess) return BA_ERR_CUDA;                                                    \
+        if ((__VA_ARGS__) != cudaSuccess) return BA_ERR_CUDA;                                             \
     } while (0)
 
 // ba_fwd (rope == nullptr) and ba_rope_fwd.
@@ -220,8 +222,8 @@ ba_status fwd_impl(const ba_problem *pp, const ba_rope *rope, const void *q, con
         !encode_bf16_rows(&tv, v, T, P.heads, P.head_dim) || !encode_bf16_rows(&to, out, T, P.heads, P.head_dim))
         return BA_ERR_CUDA;
     BA_TRY(prof_mark(0, 0, stream));
-    if (P.head_dim == 64) BA_TRY(launch_fwd_bf16_sm100<64>(tq, tk, tv, to, p, out, lse, num_sms, stream));
-    else BA_TRY(launch_fwd_bf16_sm100<128>(tq, tk, tv, to, p, out, lse, num_sms, stream));
+    if (P.head_dim == 64) BA_TRY(launch_fwd_bf16_sm100<64, kSoftmax>(tq, tk, tv, to, p, out, lse, num_sms, stream));
+    else BA_TRY(launch_fwd_bf16_sm100<128, kSoftmax>(tq, tk, tv, to, p, out, lse, num_sms, stream));
     BA_TRY(prof_mark(0, 1, stream));
     return BA_OK;
 }
@@ -292,17 +294,87 @@ ba_status bwd_impl(const ba_problem *pp, const ba_rope *rope, const void *q, con
         return BA_ERR_CUDA;
     BA_TRY(prof_mark(1, 0, stream));
     if (P.head_dim == 64)
-        BA_TRY(launch_bwd_dq_sm100<64>(tq, tk, tv, tdo, to, p, lse, delta, nlse2, dq, num_sms, stream));
+        BA_TRY(launch_bwd_dq_sm100<64, kSoftmax>(tq, tk, tv, tdo, to, p, lse, delta, nlse2, dq, num_sms, stream));
     else
-        BA_TRY(launch_bwd_dq_sm100<128>(tq, tk, tv, tdo, to, p, lse, delta, nlse2, dq, num_sms, stream));
+        BA_TRY(launch_bwd_dq_sm100<128, kSoftmax>(tq, tk, tv, tdo, to, p, lse, delta, nlse2, dq, num_sms, stream));
     BA_TRY(prof_mark(1, 1, stream));
     BA_TRY(prof_mark(2, 0, stream));
     if (P.head_dim == 64)
-        BA_TRY(launch_bwd_dkdv_sm100<64>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, delta, dk, dv, num_sms, stream));
+        BA_TRY(launch_bwd_dkdv_sm100<64, kSoftmax>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, delta, dk, dv, num_sms, stream));
     else
-        BA_TRY(launch_bwd_dkdv_sm100<128>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, delta, dk, dv, num_sms, stream));
+        BA_TRY(launch_bwd_dkdv_sm100<128, kSoftmax>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, delta, dk, dv, num_sms, stream));
     BA_TRY(prof_mark(2, 1, stream));
     return BA_OK;
+}
+
+// ba_gdpa_fwd / ba_gdpa_bwd: the block-attention kernels with the softmax
+// replaced by the activation (no lse, no Delta).
+template <int A>
+cudaError_t gdpa_launch(bool bwd, int D, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                        const CUtensorMap &tdo, const CUtensorMap &to, const CUtensorMap &tdk, const CUtensorMap &tdv,
+                        const Problem &p, void *out, void *dq, void *dk, void *dv, int num_sms, cudaStream_t stream)
+{
+    cudaError_t e;
+    if (!bwd) {
+        if ((e = prof_mark(0, 0, stream)) != cudaSuccess) return e;
+        e = D == 64 ? launch_fwd_bf16_sm100<64, A>(tq, tk, tv, to, p, out, nullptr, num_sms, stream)
+                    : launch_fwd_bf16_sm100<128, A>(tq, tk, tv, to, p, out, nullptr, num_sms, stream);
+        if (e != cudaSuccess) return e;
+        return prof_mark(0, 1, stream);
+    }
+    if ((e = prof_mark(1, 0, stream)) != cudaSuccess) return e;
+    e = D == 64 ? launch_bwd_dq_sm100<64, A>(tq, tk, tv, tdo, to, p, nullptr, nullptr, nullptr, dq, num_sms, stream)
+                : launch_bwd_dq_sm100<128, A>(tq, tk, tv, tdo, to, p, nullptr, nullptr, nullptr, dq, num_sms, stream);
+    if (e != cudaSuccess) return e;
+    if ((e = prof_mark(1, 1, stream)) != cudaSuccess || (e = prof_mark(2, 0, stream)) != cudaSuccess) return e;
+    e = D == 64 ? launch_bwd_dkdv_sm100<64, A>(tq, tk, tv, tdo, tdk, tdv, p, nullptr, nullptr, dk, dv, num_sms, stream)
+                : launch_bwd_dkdv_sm100<128, A>(tq, tk, tv, tdo, tdk, tdv, p, nullptr, nullptr, dk, dv, num_sms,
+                                                stream);
+    if (e != cudaSuccess) return e;
+    return prof_mark(2, 1, stream);
+}
+
+ba_status gdpa_impl(bool bwd, const ba_problem *pp, ba_activation act, const void *q, const void *k, const void *v,
+                    const void *dout, const int32_t *seq_offsets, int32_t block, int32_t window, void *out, void *dq,
+                    void *dk, void *dv, void *workspace, size_t workspace_bytes, ba_stream_t stream_)
+{
+    ba_status st = check_problem(pp, block, window);
+    if (st != BA_OK) return st;
+    if (act != BA_ACT_GELU && act != BA_ACT_SILU) return BA_ERR_INVALID_ARG;
+    const ba_problem &P = *pp;
+    const int64_t T = P.total_tokens;
+    if (!seq_offsets || !aligned(seq_offsets, 4) || !tensor_ok(q, T) || !tensor_ok(k, T) || !tensor_ok(v, T))
+        return BA_ERR_INVALID_ARG;
+    if (!bwd && !tensor_ok(out, T)) return BA_ERR_INVALID_ARG;
+    if (bwd && (!tensor_ok(dout, T) || !tensor_ok(dq, T) || !tensor_ok(dk, T) || !tensor_ok(dv, T)))
+        return BA_ERR_INVALID_ARG;
+    if (P.dtype != BA_BF16) return BA_ERR_UNSUPPORTED;
+    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, false);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total) return BA_ERR_INVALID_ARG;
+    int num_sms = 0, cc = 0;
+    if (!device_info(num_sms, cc)) return BA_ERR_CUDA;
+    if (cc != 10) return BA_ERR_UNSUPPORTED;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    Problem p = make_problem(P, seq_offsets, nullptr, block, window, workspace, lay);
+    BA_TRY(launch_worklist(p, stream));
+    if (T == 0) return BA_OK;
+    CUtensorMap tq, tk, tv, tdo, to, tdk, tdv;
+    if (!encode_bf16_rows(&tq, q, T, P.heads, P.head_dim) || !encode_bf16_rows(&tk, k, T, P.heads, P.head_dim) ||
+        !encode_bf16_rows(&tv, v, T, P.heads, P.head_dim))
+        return BA_ERR_CUDA;
+    if (!bwd && !encode_bf16_rows(&to, out, T, P.heads, P.head_dim)) return BA_ERR_CUDA;
+    if (bwd && (!encode_bf16_rows(&tdo, dout, T, P.heads, P.head_dim) ||
+                !encode_bf16_rows(&tdk, dk, T, P.heads, P.head_dim) ||
+                !encode_bf16_rows(&tdv, dv, T, P.heads, P.head_dim)))
+        return BA_ERR_CUDA;
+    if (bwd) to = tdo; // the dQ pass reads no `out` here; any valid map fills the slot
+    else tdo = tdk = tdv = to;
+    const cudaError_t e = act == BA_ACT_GELU
+                              ? gdpa_launch<kGelu>(bwd, P.head_dim, tq, tk, tv, tdo, to, tdk, tdv, p, out, dq, dk, dv,
+                                                   num_sms, stream)
+                              : gdpa_launch<kSilu>(bwd, P.head_dim, tq, tk, tv, tdo, to, tdk, tdv, p, out, dq, dk, dv,
+                                                   num_sms, stream);
+    return e == cudaSuccess ? BA_OK : BA_ERR_CUDA;
 }
 
 } // namespace
@@ -396,6 +468,27 @@ ba_status ba_swa_bwd(const ba_problem *p, const void *q, const void *k, const vo
                   workspace_bytes, stream);
 }
 
+size_t ba_gdpa_workspace_size(const ba_problem *p, int32_t block, int32_t window)
+{
+    return ba_fwd_workspace_size(p, block, window);
+}
+
+ba_status ba_gdpa_fwd(const ba_problem *p, ba_activation act, const void *q, const void *k, const void *v,
+                      const int32_t *seq_offsets, int32_t block, int32_t window, void *out, void *workspace,
+                      size_t workspace_bytes, ba_stream_t stream)
+{
+    return gdpa_impl(false, p, act, q, k, v, nullptr, seq_offsets, block, window, out, nullptr, nullptr, nullptr,
+                     workspace, workspace_bytes, stream);
+}
+
+ba_status ba_gdpa_bwd(const ba_problem *p, ba_activation act, const void *q, const void *k, const void *v,
+                      const void *dout, const int32_t *seq_offsets, int32_t block, int32_t window, void *dq, void *dk,
+                      void *dv, void *workspace, size_t workspace_bytes, ba_stream_t stream)
+{
+    return gdpa_impl(true, p, act, q, k, v, dout, seq_offsets, block, window, nullptr, dq, dk, dv, workspace,
+                     workspace_bytes, stream);
+}
+
 ba_status ba_device_status(const void *workspace, ba_stream_t stream_)
 {
     if (!workspace) return BA_ERR_INVALID_ARG;
@@ -416,6 +509,13 @@ ba_status ba_selftest_wait_timeout(void *workspace, size_t workspace_bytes, int3
     int *status = static_cast<int *>(workspace);
     if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return BA_ERR_CUDA;
     BA_TRY(launch_wait_selftest(status, uint64_t(limit_us) * 1000, stream));
+    return BA_OK;
+}
+
+ba_status ba_selftest_exp2(const float *x, float *y, int64_t n, ba_stream_t stream_)
+{
+    if (n < 0 || (n > 0 && (!x || !y || !aligned(x, 4) || !aligned(y, 4)))) return BA_ERR_INVALID_ARG;
+    BA_TRY(launch_exp2_selftest(x, y, n, reinterpret_cast<cudaStream_t>(stream_)));
     return BA_OK;
 }
 

@@ -1,12 +1,14 @@
 // Small memory-bound kernels around the attention kernels:
-//   worklist_kernel   per-example count of live 128-row tiles -> exclusive
-//                     prefix sum (the persistent kernels' work list); resets
+//   worklist_kernel   the persistent kernels' work list: every live 128-row
+//                     tile (and pair of tiles), examples longest first; resets
 //                     the status word
 //   bwd_pre_kernel    Delta = rowsum(dout * out) in fp32 (the fp32 path; the
 //                     bf16 dQ pass computes Delta itself)
 //   wait_selftest_kernel  one warp waits on a barrier nothing completes, with a
 //                     short limit, through the same bounded wait the attention
 //                     kernels use, and reports the timeout in the status word
+//   exp2_selftest_kernel  the attention kernels' FMA-pipe 2^x on a caller's array
+//                     (its accuracy is tested against 2^x computed on the host)
 //   skip_*_kernel     component skip: flagged examples pass v through
 //                     ("Meta Scales GEM Ads Model Across Platforms and
 //                     Thousands of GPUs", section "Kunlun changes how GEM
@@ -61,6 +63,17 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t local, int32_t *
     return incl - local + (wid > 0 ? warp_tot[wid - 1] : 0);
 }
 
+// The persistent kernels deal their work items out round-robin (item n to CTA
+// n mod grid) in table order. The table lists examples longest first, each
+// example's tiles together and in order: the long examples' items, which see
+// the most key tiles, go out first and the short examples' cheap ones fill in
+// at the end, so the CTAs finish close together (longest-processing-time-first
+// dealing), while the tiles of one example, which share K/V tiles, still run
+// at about the same time. Examples are bucketed by their live tile count
+// (counts of kSortBuckets - 1 and more share the first bucket); the order
+// inside a bucket is whatever order the examples claim their slots in.
+constexpr int kSortBuckets = kWorklistThreads;
+
 // Per live example: its 128-row tiles, and pairs of consecutive tiles (the
 // forward processes two query tiles of one example together).
 __global__ void __launch_bounds__(kWorklistThreads)
@@ -69,28 +82,37 @@ __global__ void __launch_bounds__(kWorklistThreads)
                     int32_t *__restrict__ pair_prefix, int4 *__restrict__ pair_info, int *__restrict__ status)
 {
     __shared__ int32_t warp_tot[kWorklistThreads / 32];
+    __shared__ int32_t bucket_tiles[kSortBuckets], bucket_pairs[kSortBuckets];
     const int tid = threadIdx.x;
-    const int per = (batch + kWorklistThreads - 1) / kWorklistThreads;
-    const int b0 = tid * per;
-    const int b1 = min(batch, b0 + per);
-    int32_t ltiles = 0, lpairs = 0;
-    for (int b = b0; b < b1; ++b) {
+    auto bucket = [](int32_t nt) { return kSortBuckets - 1 - (nt < kSortBuckets - 1 ? nt : kSortBuckets - 1); };
+    bucket_tiles[tid] = 0;
+    bucket_pairs[tid] = 0;
+    __syncthreads();
+    for (int b = tid; b < batch; b += kWorklistThreads) {
         const int32_t nt = live_tiles(offs, skip, b);
-        ltiles += nt;
-        lpairs += (nt + 1) / 2;
+        if (nt == 0) continue;
+        atomicAdd(&bucket_tiles[bucket(nt)], nt);
+        atomicAdd(&bucket_pairs[bucket(nt)], (nt + 1) / 2);
     }
+    __syncthreads();
     int32_t ttot, ptot;
-    int32_t trun = block_exclusive_scan(ltiles, warp_tot, ttot);
-    int32_t prun = block_exclusive_scan(lpairs, warp_tot, ptot);
-    for (int b = b0; b < b1; ++b) {
-        tile_prefix[b] = trun;
-        pair_prefix[b] = prun;
+    const int32_t tstart = block_exclusive_scan(bucket_tiles[tid], warp_tot, ttot);
+    const int32_t pstart = block_exclusive_scan(bucket_pairs[tid], warp_tot, ptot);
+    bucket_tiles[tid] = tstart; // every thread read its bucket before the scans' barriers
+    bucket_pairs[tid] = pstart;
+    __syncthreads();
+    for (int b = tid; b < batch; b += kWorklistThreads) {
         const int32_t nt = live_tiles(offs, skip, b);
         const int32_t s0 = offs[b], L = offs[b + 1] - s0;
-        for (int32_t t = 0; t < nt; ++t) tile_info[trun + t] = make_int4(s0, L, t, b);
-        for (int32_t t = 0; t < nt; t += 2) pair_info[prun + t / 2] = make_int4(s0, L, t, b);
-        trun += nt;
-        prun += (nt + 1) / 2;
+        int32_t t0 = ttot, p0 = ptot; // an example without live tiles owns no slots
+        if (nt > 0) {
+            t0 = atomicAdd(&bucket_tiles[bucket(nt)], nt);
+            p0 = atomicAdd(&bucket_pairs[bucket(nt)], (nt + 1) / 2);
+        }
+        tile_prefix[b] = t0;
+        pair_prefix[b] = p0;
+        for (int32_t t = 0; t < nt; ++t) tile_info[t0 + t] = make_int4(s0, L, t, b);
+        for (int32_t t = 0; t < nt; t += 2) pair_info[p0 + t / 2] = make_int4(s0, L, t, b);
     }
     if (tid == kWorklistThreads - 1) {
         tile_prefix[batch] = ttot;
@@ -244,6 +266,20 @@ __global__ void __launch_bounds__(32) wait_selftest_kernel(int *status, uint64_t
 cudaError_t launch_wait_selftest(int *status, uint64_t limit_ns, cudaStream_t stream)
 {
     wait_selftest_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+    return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(256) exp2_selftest_kernel(const float *__restrict__ x, float *__restrict__ y, int64_t n)
+{
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
+        y[i] = exp2_fma(x[i]);
+}
+
+cudaError_t launch_exp2_selftest(const float *x, float *y, int64_t n, cudaStream_t stream)
+{
+    if (n == 0) return cudaSuccess;
+    const int64_t g = (n + 255) / 256;
+    exp2_selftest_kernel<<<int(g < 4096 ? g : 4096), 256, 0, stream>>>(x, y, n);
     return cudaGetLastError();
 }
 

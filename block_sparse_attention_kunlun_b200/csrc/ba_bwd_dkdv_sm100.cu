@@ -94,7 +94,7 @@ __device__ __forceinline__ void query_tile_range(const TileRef &r, int64_t B, in
 
 } // namespace
 
-template <int D, bool kRope>
+template <int D, bool kRope, int A>
 __global__ void __launch_bounds__(448, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -182,15 +182,19 @@ __global__ void __launch_bounds__(448, 1)
                 // the tile's -lse (log2 units) and -Delta, four queries per lane, copied
                 // asynchronously; each lane's copies arrive on q_full when they land. Rows past
                 // the example's end copy its last row (those queries are masked out).
+                if constexpr (A == kSoftmax) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int qr = 4 * lane + e;
-                    const int64_t q = int64_t(i) * kTile + qr;
-                    const int64_t gi = int64_t(r.h) * T + r.s0 + (q < r.L ? q : r.L - 1);
-                    cp_async_4(&sb.stat[qs][0][qr], nlse2 + gi);
-                    cp_async_4(&sb.stat[qs][1][qr], neg_delta + gi);
+                    for (int e = 0; e < 4; ++e) {
+                        const int qr = 4 * lane + e;
+                        const int64_t q = int64_t(i) * kTile + qr;
+                        const int64_t gi = int64_t(r.h) * T + r.s0 + (q < r.L ? q : r.L - 1);
+                        cp_async_4(&sb.stat[qs][0][qr], nlse2 + gi);
+                        cp_async_4(&sb.stat[qs][1][qr], neg_delta + gi);
+                    }
+                    cp_async_arrive_noinc(&sb.q_full[qs]);
+                } else {
+                    mbar_arrive(&sb.q_full[qs]); // generalized attention has no per-query statistics
                 }
-                cp_async_arrive_noinc(&sb.q_full[qs]);
                 __syncwarp();
                 if (i == ilo) {
                     // the item's K and V, once the previous item's last S^T (K) and dP^T (V)
@@ -392,26 +396,45 @@ __global__ void __launch_bounds__(448, 1)
                     uint32_t(&cur)[16] = sr[q4 & 1];
                     reg_fence(cur);
                     if (q4 < 3) tmem_ld16(tmem + lane_base + Lay::kColS + 64 * g + 16 * (q4 + 1), sr[(q4 + 1) & 1]);
+                    if constexpr (A == kSoftmax) {
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const float4 l4 = l2v[4 * q4 + c4]; // -lse of 4 queries
-                        const float2 x01 = ffma2(make_float2(__uint_as_float(cur[4 * c4]), __uint_as_float(cur[4 * c4 + 1])),
-                                                 sc2, make_float2(l4.x, l4.y));
-                        const float2 x23 = ffma2(make_float2(__uint_as_float(cur[4 * c4 + 2]), __uint_as_float(cur[4 * c4 + 3])),
-                                                 sc2, make_float2(l4.z, l4.w));
-                        // one value in four goes through the FMA pipe to offload the MUFU unit
-                        float ev[4] = {ex2_approx(x01.x), ex2_approx(x01.y), ex2_approx(x23.x), exp2_fma(x23.y)};
-                        if (!full) {
+                        for (int c4 = 0; c4 < 4; ++c4) {
+                            const float4 l4 = l2v[4 * q4 + c4]; // -lse of 4 queries
+                            const float2 x01 = ffma2(make_float2(__uint_as_float(cur[4 * c4]), __uint_as_float(cur[4 * c4 + 1])),
+                                                     sc2, make_float2(l4.x, l4.y));
+                            const float2 x23 = ffma2(make_float2(__uint_as_float(cur[4 * c4 + 2]), __uint_as_float(cur[4 * c4 + 3])),
+                                                     sc2, make_float2(l4.z, l4.w));
+                            // one value in four goes through the FMA pipe to offload the MUFU unit
+                            float ev[4] = {ex2_approx(x01.x), ex2_approx(x01.y), ex2_approx(x23.x), exp2_fma(x23.y)};
+                            if (!full) {
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int cc = 16 * q4 + 4 * c4 + e;
-                                ev[e] = (cc >= lo_c && cc <= hi_c) ? ev[e] : 0.f;
+                                for (int e = 0; e < 4; ++e) {
+                                    const int cc = 16 * q4 + 4 * c4 + e;
+                                    ev[e] = (cc >= lo_c && cc <= hi_c) ? ev[e] : 0.f;
+                                }
                             }
+                            pp[q4][2 * c4] = pack_bf16x2(ev[0], ev[1]);
+                            pp[q4][2 * c4 + 1] = pack_bf16x2(ev[2], ev[3]);
                         }
-                        pp[q4][2 * c4] = pack_bf16x2(ev[0], ev[1]);
-                        pp[q4][2 * c4 + 1] = pack_bf16x2(ev[2], ev[3]);
+                        tmem_st8(tmem + lane_base + Lay::kColS + 64 * g + 8 * q4, pp[q4]);
+                    } else {
+                        // generalized attention: act(S^T / sqrt(D)) goes to TMEM for dV; act' stays
+                        // in registers for dS^T = act' dP^T (Delta is 0)
+                        uint32_t pa[8];
+#pragma unroll
+                        for (int c2 = 0; c2 < 8; ++c2) {
+                            float2 v0 = act_value_grad<A>(__uint_as_float(cur[2 * c2]) * p.scale);
+                            float2 v1 = act_value_grad<A>(__uint_as_float(cur[2 * c2 + 1]) * p.scale);
+                            if (!full) {
+                                const int cc = 16 * q4 + 2 * c2;
+                                if (!(cc >= lo_c && cc <= hi_c)) v0 = make_float2(0.f, 0.f);
+                                if (!(cc + 1 >= lo_c && cc + 1 <= hi_c)) v1 = make_float2(0.f, 0.f);
+                            }
+                            pa[c2] = pack_bf16x2(v0.x, v1.x);
+                            pp[q4][c2] = pack_bf16x2(v0.y, v1.y);
+                        }
+                        tmem_st8(tmem + lane_base + Lay::kColS + 64 * g + 8 * q4, pa);
                     }
-                    tmem_st8(tmem + lane_base + Lay::kColS + 64 * g + 8 * q4, pp[q4]);
                     if (q4 < 3) tmem_wait_ld();
                 }
                 tmem_wait_st();
@@ -431,7 +454,7 @@ __global__ void __launch_bounds__(448, 1)
                     uint32_t dk16[16];
 #pragma unroll
                     for (int c2 = 0; c2 < 16; ++c2) {
-                        const float2 d2 = dlv2[16 * h2 + c2]; // -Delta of 2 queries
+                        const float2 d2 = A == kSoftmax ? dlv2[16 * h2 + c2] : make_float2(0.f, 0.f); // -Delta
                         const uint32_t pw = pp[2 * h2 + c2 / 8][c2 % 8];
                         const float2 p2 = make_float2(__uint_as_float(pw << 16), __uint_as_float(pw & 0xffff0000u));
                         const float2 ds = fmul2(p2, fadd2(make_float2(__uint_as_float(dr[2 * c2]),
@@ -541,14 +564,16 @@ __global__ void __launch_bounds__(448, 1)
     if (threadIdx.x == 0 && sb.abort) atomicOr(p.status, kStatusTimeout);
 }
 
-template <int D>
+template <int D, int A>
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
                                   const Problem &p, const float *nlse2, const float *neg_delta, void *dk, void *dv,
                                   int num_sms, cudaStream_t stream)
 {
     using Lay = DkvLayout<D>;
-    auto kern = p.rope_cos ? bwd_dkdv_sm100_kernel<D, true> : bwd_dkdv_sm100_kernel<D, false>;
+    // the rotary epilogue exists for block attention only
+    auto kern = (A == kSoftmax && p.rope_cos) ? bwd_dkdv_sm100_kernel<D, A == kSoftmax, A>
+                                              : bwd_dkdv_sm100_kernel<D, false, A>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
     kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, neg_delta,
@@ -557,13 +582,16 @@ cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
     return cudaGetLastError();
 }
 
-template cudaError_t launch_bwd_dkdv_sm100<64>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                                               const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                                               const Problem &, const float *, const float *, void *, void *, int,
-                                               cudaStream_t);
-template cudaError_t launch_bwd_dkdv_sm100<128>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                                                const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                                                const Problem &, const float *, const float *, void *, void *, int,
-                                                cudaStream_t);
+#define BA_DKDV_INST(D, A)                                                                                   \
+    template cudaError_t launch_bwd_dkdv_sm100<D, A>(const CUtensorMap &, const CUtensorMap &,                \
+                                                     const CUtensorMap &, const CUtensorMap &, const CUtensorMap &, \
+                                                     const CUtensorMap &, const Problem &, const float *,       \
+                                                     const float *, void *, void *, int, cudaStream_t);
+BA_DKDV_INST(64, kSoftmax)
+BA_DKDV_INST(128, kSoftmax)
+BA_DKDV_INST(64, kGelu)
+BA_DKDV_INST(128, kGelu)
+BA_DKDV_INST(64, kSilu)
+BA_DKDV_INST(128, kSilu)
 
 } // namespace ba

@@ -76,7 +76,7 @@ __device__ __forceinline__ int first_key_tile(const TileRef &r, int64_t B, int64
 
 } // namespace
 
-template <int D, bool kRope>
+template <int D, bool kRope, int A>
 __global__ void __launch_bounds__(384, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -146,13 +146,15 @@ __global__ void __launch_bounds__(384, 1)
                 const int jlo = first_key_tile(r, B, W);
                 if (!mbar_wait(&sb.st_empty, (item_cnt & 1) ^ 1, abort)) break;
                 if (lane == 0) {
+                    // Q, dO and (for Delta; the softmax only) out
                     uint8_t *st = smem + Lay::kStaging;
-                    mbar_arrive_expect_tx(&sb.st_full, 3 * Lay::kTileBytes);
+                    mbar_arrive_expect_tx(&sb.st_full, (A == kSoftmax ? 3 : 2) * Lay::kTileBytes);
                     for (int c = 0; c < Lay::kChunks; ++c) {
                         const int x = r.h * D + c * 64, y = r.s0 + r.t * kTile;
                         tma_load_2d(st + c * Lay::kChunkBytes, &tm_q, &sb.st_full, x, y);
                         tma_load_2d(st + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_do, &sb.st_full, x, y);
-                        tma_load_2d(st + 2 * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_o, &sb.st_full, x, y);
+                        if (A == kSoftmax)
+                            tma_load_2d(st + 2 * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_o, &sb.st_full, x, y);
                     }
                 }
                 __syncwarp();
@@ -295,13 +297,17 @@ __global__ void __launch_bounds__(384, 1)
                         const int u = 4 * hh + u4;
                         const int off = c * Lay::kChunkBytes + row * 128 + ((u ^ (row & 7)) * 16);
                         const uint4 d4 = *reinterpret_cast<const uint4 *>(dsrc + off);
-                        const uint4 o4 = *reinterpret_cast<const uint4 *>(osrc + off);
-                        const uint32_t dw[4] = {d4.x, d4.y, d4.z, d4.w}, ow[4] = {o4.x, o4.y, o4.z, o4.w};
+                        if constexpr (A == kSoftmax) {
+                            const uint4 o4 = *reinterpret_cast<const uint4 *>(osrc + off);
+                            const uint32_t dw[4] = {d4.x, d4.y, d4.z, d4.w}, ow[4] = {o4.x, o4.y, o4.z, o4.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 df = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&dw[e]));
-                            const float2 of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ow[e]));
-                            dl = fmaf(df.x, of.x, fmaf(df.y, of.y, dl));
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 df =
+                                    __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&dw[e]));
+                                const float2 of =
+                                    __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ow[e]));
+                                dl = fmaf(df.x, of.x, fmaf(df.y, of.y, dl));
+                            }
                         }
                         const uint4 a = g == 0 ? *reinterpret_cast<const uint4 *>(qsrc + off) : d4;
                         w[4 * u4] = a.x;
@@ -323,7 +329,7 @@ __global__ void __launch_bounds__(384, 1)
             delta_row = dl;
             const int64_t i = int64_t(rr.t) * kTile + row;
             // for the dK/dV pass: -Delta (group 0) and -lse in log2 units (group 1)
-            if (i < rr.L) {
+            if (A == kSoftmax && i < rr.L) {
                 if (g == 0) neg_delta[int64_t(rr.h) * T + rr.s0 + i] = -dl;
                 else nlse2[int64_t(rr.h) * T + rr.s0 + i] = -lse_val * 1.4426950408889634f;
             }
@@ -337,6 +343,7 @@ __global__ void __launch_bounds__(384, 1)
         // lse of this thread's query row (log2 units), loaded an item ahead
         auto load_l2 = [&](const TileRef &rr) -> float {
             const int64_t q = int64_t(rr.t) * kTile + row;
+            if (A != kSoftmax) return 0.f;
             return q < rr.L ? lse[int64_t(rr.h) * T + rr.s0 + q] : INFINITY;
         };
         float lse_row = have ? load_l2(r) : 0.f;
@@ -382,8 +389,16 @@ __global__ void __launch_bounds__(384, 1)
                         for (int c2 = 0; c2 < 8; ++c2) {
                             const float2 x = ffma2(make_float2(__uint_as_float(cur[2 * c2]), __uint_as_float(cur[2 * c2 + 1])),
                                                    sc2, nl2);
-                            // one value in four goes through the FMA pipe to offload the MUFU unit
-                            float e0 = ex2_approx(x.x), e1 = (c2 & 1) ? exp2_fma(x.y) : ex2_approx(x.y);
+                            float e0, e1;
+                            if constexpr (A == kSoftmax) {
+                                // one value in four goes through the FMA pipe to offload the MUFU unit
+                                e0 = ex2_approx(x.x);
+                                e1 = (c2 & 1) ? exp2_fma(x.y) : ex2_approx(x.y);
+                            } else {
+                                // generalized attention: dS = act'(S / sqrt(D)) dP (Delta is 0)
+                                e0 = act_grad<A>(__uint_as_float(cur[2 * c2]) * p.scale);
+                                e1 = act_grad<A>(__uint_as_float(cur[2 * c2 + 1]) * p.scale);
+                            }
                             if (!full) {
                                 const int cc = 16 * q4 + 2 * c2;
                                 e0 = (cc >= lo_c && cc <= hi_c) ? e0 : 0.f;
@@ -473,13 +488,14 @@ __global__ void __launch_bounds__(384, 1)
     if (threadIdx.x == 0 && sb.abort) atomicOr(p.status, kStatusTimeout);
 }
 
-template <int D>
+template <int D, int A>
 cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const CUtensorMap &tdo, const CUtensorMap &to, const Problem &p, const float *lse,
                                 float *neg_delta, float *nlse2, void *dq, int num_sms, cudaStream_t stream)
 {
     using Lay = DqLayout<D>;
-    auto kern = p.rope_cos ? bwd_dq_sm100_kernel<D, true> : bwd_dq_sm100_kernel<D, false>;
+    // the rotary epilogue exists for block attention only
+    auto kern = (A == kSoftmax && p.rope_cos) ? bwd_dq_sm100_kernel<D, A == kSoftmax, A> : bwd_dq_sm100_kernel<D, false, A>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
     // the register split only works if the CTA is launched with at least the budgets' sum
@@ -493,11 +509,16 @@ cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, co
     return cudaGetLastError();
 }
 
-template cudaError_t launch_bwd_dq_sm100<64>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                                             const CUtensorMap &, const CUtensorMap &, const Problem &, const float *,
-                                             float *, float *, void *, int, cudaStream_t);
-template cudaError_t launch_bwd_dq_sm100<128>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                                              const CUtensorMap &, const CUtensorMap &, const Problem &, const float *,
-                                              float *, float *, void *, int, cudaStream_t);
+#define BA_DQ_INST(D, A)                                                                                   \
+    template cudaError_t launch_bwd_dq_sm100<D, A>(const CUtensorMap &, const CUtensorMap &,                \
+                                                   const CUtensorMap &, const CUtensorMap &, const CUtensorMap &, \
+                                                   const Problem &, const float *, float *, float *, void *, int, \
+                                                   cudaStream_t);
+BA_DQ_INST(64, kSoftmax)
+BA_DQ_INST(128, kSoftmax)
+BA_DQ_INST(64, kGelu)
+BA_DQ_INST(128, kGelu)
+BA_DQ_INST(64, kSilu)
+BA_DQ_INST(128, kSilu)
 
 } // namespace ba

@@ -46,11 +46,14 @@ __host__ __device__ __forceinline__ bool visible(int64_t i, int64_t j, int64_t b
 
 // Workspace layout (all offsets 256-byte aligned):
 //   [0, 256)            status word (int32)
-//   tile_prefix         int32[batch + 1]: live 128-row tiles before example b
+//   tile_prefix         int32[batch + 1]: slot of example b's first tile in
+//                       tile_info; [batch] = number of live tiles
 //   tile_info           int4[max_tiles]: per live tile {first row of its
 //                       example, example length, tile index in the example,
-//                       example index}, max_tiles = ceil(T / 128) + batch
-//   pair_prefix         int32[batch + 1]: live pairs of consecutive tiles
+//                       example index}, max_tiles = ceil(T / 128) + batch;
+//                       examples longest first, an example's tiles in order
+//   pair_prefix         int32[batch + 1]: likewise for pairs of consecutive
+//                       tiles; [batch] = number of live pairs
 //   pair_info           int4[max_pairs]: per pair {row0, length, first tile,
 //                       example}, max_pairs = ceil(T / 256) + batch
 //   delta   (bwd only)  float[heads * total_tokens]: Delta (fp32 path) or -Delta
@@ -159,6 +162,54 @@ __device__ __forceinline__ void rope_transpose_bits(const Problem &p, int64_t po
             v[2 * m] = __float_as_uint(r.x);
             v[2 * m + 1] = __float_as_uint(r.y);
         }
+    }
+}
+
+// What replaces exp(s - lse) in the attention. kSoftmax: block attention.
+// kGelu / kSilu: generalized dot-product attention ("GEM (Meta)", section
+// "Custom kernels": GEM's self-, cross- and pooled attention with the softmax
+// replaced by an activation such as GELU or SiLU), out_i = sum_j act(s_ij) v_j
+// over the visible keys with s_ij = q_i . k_j / sqrt(D), no normalisation,
+// so no running maximum and no lse.
+enum Act : int { kSoftmax = 0, kGelu = 1, kSilu = 2 };
+
+// GELU (exact form x Phi(x), Phi the standard normal distribution function)
+// and SiLU (x sigma(x)).
+template <int A>
+__device__ __forceinline__ float act_value(float x)
+{
+    static_assert(A == kGelu || A == kSilu, "an activation");
+    if constexpr (A == kGelu) return 0.5f * x * (1.f + erff(x * 0.70710678118654752f));
+    else return x / (1.f + __expf(-x));
+}
+
+// The activation and its derivative: GELU' = Phi(x) + x phi(x) with phi the
+// standard normal density; SiLU' = sigma(x) (1 + x (1 - sigma(x))).
+template <int A>
+__device__ __forceinline__ float2 act_value_grad(float x)
+{
+    static_assert(A == kGelu || A == kSilu, "an activation");
+    if constexpr (A == kGelu) {
+        const float cdf = 0.5f * (1.f + erff(x * 0.70710678118654752f));
+        const float pdf = 0.39894228040143268f * __expf(-0.5f * x * x);
+        return make_float2(x * cdf, fmaf(x, pdf, cdf));
+    } else {
+        const float sg = 1.f / (1.f + __expf(-x));
+        return make_float2(x * sg, sg * fmaf(x, 1.f - sg, 1.f));
+    }
+}
+
+// The activation's derivative alone.
+template <int A>
+__device__ __forceinline__ float act_grad(float x)
+{
+    static_assert(A == kGelu || A == kSilu, "an activation");
+    if constexpr (A == kGelu) {
+        const float cdf = 0.5f * (1.f + erff(x * 0.70710678118654752f));
+        return fmaf(x, 0.39894228040143268f * __expf(-0.5f * x * x), cdf);
+    } else {
+        const float sg = 1.f / (1.f + __expf(-x));
+        return sg * fmaf(x, 1.f - sg, 1.f);
     }
 }
 

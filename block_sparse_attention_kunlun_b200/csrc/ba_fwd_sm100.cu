@@ -79,7 +79,7 @@ __device__ __forceinline__ int first_key_tile(int t, int64_t B, int64_t W)
 
 } // namespace
 
-template <int D>
+template <int D, int A>
 __global__ void __launch_bounds__(512, 1)
     fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -395,12 +395,38 @@ __global__ void __launch_bounds__(512, 1)
                     const float2 a = fadd2(a01, a23);
                     rs = a.x + a.y;
                 };
-                if (full) softmax_tile(std::true_type{});
+                // generalized attention: P = act(S / sqrt(D)) on the visible keys, nothing to normalise
+                auto activation_tile = [&](auto full_t) {
+                    constexpr bool FULL = decltype(full_t)::value;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const int c0 = 64 * hh + 2 * c;
+                            float p0 = 0.f, p1 = 0.f;
+                            if constexpr (A != kSoftmax) {
+                                p0 = act_value<A>(__uint_as_float(sr[c0 / 32][c0 % 32]) * p.scale);
+                                p1 = act_value<A>(__uint_as_float(sr[c0 / 32][c0 % 32 + 1]) * p.scale);
+                            }
+                            if (!FULL) {
+                                p0 = (c0 >= lo_c && c0 <= hi_c) ? p0 : 0.f;
+                                p1 = (c0 + 1 >= lo_c && c0 + 1 <= hi_c) ? p1 : 0.f;
+                            }
+                            pk[c] = pack_bf16x2(p0, p1);
+                        }
+                        tmem_st32(s_addr + 32 * hh, pk);
+                    }
+                };
+                if constexpr (A != kSoftmax) {
+                    if (full) activation_tile(std::true_type{});
+                    else activation_tile(std::false_type{});
+                } else if (full) softmax_tile(std::true_type{});
                 else softmax_tile(std::false_type{});
                 l = l * alpha + rs;
                 tmem_wait_st();
                 // O holds the earlier tiles' P V (complete: this S was issued after it).
-                if (j > jlo && __any_sync(0xffffffffu, grow)) {
+                if (A == kSoftmax && j > jlo && __any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t orr[32];
@@ -419,9 +445,13 @@ __global__ void __launch_bounds__(512, 1)
             }
             if (!ok) break;
             // hand 1 / l to the epilogue warps, write lse, and go on with the next item
-            sb.inv_l[w][row] = valid ? 1.f / l : 0.f;
-            if (valid)
-                lse[int64_t(r.h) * p.total_tokens + r.s0 + i] = (m_ref + log2f(l)) * 0.6931471805599453f;
+            if constexpr (A == kSoftmax) {
+                sb.inv_l[w][row] = valid ? 1.f / l : 0.f;
+                if (valid)
+                    lse[int64_t(r.h) * p.total_tokens + r.s0 + i] = (m_ref + log2f(l)) * 0.6931471805599453f;
+            } else {
+                sb.inv_l[w][row] = valid ? 1.f : 0.f;
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sb.o_ready[w]);
         }
@@ -516,13 +546,13 @@ __global__ void __launch_bounds__(512, 1)
     if (threadIdx.x == 0 && sb.abort) atomicOr(p.status, kStatusTimeout);
 }
 
-template <int D>
+template <int D, int A>
 cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &to, const Problem &p, void *out, float *lse, int num_sms,
                                   cudaStream_t stream)
 {
     using Lay = FwdLayout<D>;
-    auto kern = fwd_bf16_sm100_kernel<D>;
+    auto kern = fwd_bf16_sm100_kernel<D, A>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
     // the register split only works if the CTA is launched with at least the budgets' sum
@@ -536,11 +566,15 @@ cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
     return cudaGetLastError();
 }
 
-template cudaError_t launch_fwd_bf16_sm100<64>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                                               const CUtensorMap &, const Problem &, void *, float *, int,
-                                               cudaStream_t);
-template cudaError_t launch_fwd_bf16_sm100<128>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                                                const CUtensorMap &, const Problem &, void *, float *, int,
-                                                cudaStream_t);
+#define BA_FWD_INST(D, A)                                                                                  \
+    template cudaError_t launch_fwd_bf16_sm100<D, A>(const CUtensorMap &, const CUtensorMap &,              \
+                                                     const CUtensorMap &, const CUtensorMap &, const Problem &, \
+                                                     void *, float *, int, cudaStream_t);
+BA_FWD_INST(64, kSoftmax)
+BA_FWD_INST(128, kSoftmax)
+BA_FWD_INST(64, kGelu)
+BA_FWD_INST(128, kGelu)
+BA_FWD_INST(64, kSilu)
+BA_FWD_INST(128, kSilu)
 
 } // namespace ba

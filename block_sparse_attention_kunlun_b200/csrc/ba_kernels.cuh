@@ -11,6 +11,7 @@ namespace ba {
 
 cudaError_t launch_worklist(const Problem &p, cudaStream_t stream);
 cudaError_t launch_wait_selftest(int *status, uint64_t limit_ns, cudaStream_t stream);
+cudaError_t launch_exp2_selftest(const float *x, float *y, int64_t n, cudaStream_t stream);
 
 template <typename T>
 cudaError_t launch_bwd_pre(const Problem &p, const void *out, const void *dout, float *delta, int num_sms,
@@ -32,16 +33,16 @@ cudaError_t launch_bwd_f32(const Problem &p, const float *q, const float *k, con
                            const float *lse, const float *delta, float *dq, float *dk, float *dv, int num_sms,
                            cudaStream_t stream);
 
-template <int D>
+template <int D, int A>
 cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &to, const Problem &p, void *out, float *lse, int num_sms,
                                   cudaStream_t stream);
 
-template <int D>
+template <int D, int A>
 cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const CUtensorMap &tdo, const CUtensorMap &to, const Problem &p, const float *lse,
                                 float *neg_delta, float *nlse2, void *dq, int num_sms, cudaStream_t stream);
-template <int D>
+template <int D, int A>
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
                                   const Problem &p, const float *nlse2, const float *neg_delta, void *dk, void *dv,

@@ -121,6 +121,33 @@ ba_status ba_bwd(const ba_problem *p, const void *q, const void *k, const void *
                  void *workspace, size_t workspace_bytes, ba_stream_t stream);
 
 /*
+ * Generalized dot-product attention (GDPA): "GEM (Meta)", section "Custom
+ * kernels", describes GEM's self-, cross- and pooled attention with the
+ * softmax replaced by an activation such as GELU or SiLU; "Scaling Meta's
+ * Generative Ads Model (GEM) for Ads Recommendations", section "Kunlun
+ * Architecture Details", adds that per-example feed-forward networks were
+ * recast as it. The pages give no formula; the reading implemented here is
+ * that the activation takes the softmax's place and nothing else changes:
+ *     out_i = sum over visible j of act(q_i . k_j / sqrt(head_dim)) v_j
+ * with the block rule above for visibility, no normalisation (hence no lse),
+ * act = GELU (x Phi(x), exact erf form) or SiLU (x sigma(x)). The backward
+ * writes the exact gradients dq, dk, dv of sum(out * dout).
+ *  - BF16 only (BA_ERR_UNSUPPORTED for BA_F32); head_dim 64 or 128; no skip
+ *    flags. Same tensor layouts, ownership and errors as ba_fwd / ba_bwd.
+ *  - Workspace: ba_gdpa_workspace_size bytes, for either direction.
+ *  - act outside the enumeration: BA_ERR_INVALID_ARG.
+ */
+typedef enum { BA_ACT_GELU = 1, BA_ACT_SILU = 2 } ba_activation;
+
+size_t ba_gdpa_workspace_size(const ba_problem *p, int32_t block, int32_t window);
+ba_status ba_gdpa_fwd(const ba_problem *p, ba_activation act, const void *q, const void *k, const void *v,
+                      const int32_t *seq_offsets, int32_t block, int32_t window, void *out, void *workspace,
+                      size_t workspace_bytes, ba_stream_t stream);
+ba_status ba_gdpa_bwd(const ba_problem *p, ba_activation act, const void *q, const void *k, const void *v,
+                      const void *dout, const int32_t *seq_offsets, int32_t block, int32_t window, void *dq,
+                      void *dk, void *dv, void *workspace, size_t workspace_bytes, ba_stream_t stream);
+
+/*
  * Token-granular sliding-window attention, the predecessor that block
  * attention replaced ("GEM (Meta)", section "Custom kernels": long
  * user-history self-attention first moved to a sliding window, then to
@@ -282,8 +309,8 @@ ba_status ba_selftest_exp2(const float *x, float *y, int64_t n, ba_stream_t stre
  * Profiling hook. Until changed, calls made from THIS host thread record
  * `start` on their stream right before one kernel and `stop` right after it,
  * so that cudaEventElapsedTime(start, stop) is that kernel's own duration:
- * which = 0 the forward attention kernel of ba_fwd, 1 the dQ kernel of
- * ba_bwd, 2 its dK/dV kernel. The events are cudaEvent_t handles owned by
+ * which = 0 the forward attention kernel of ba_fwd (or ba_gdpa_fwd), 1 the
+ * dQ kernel of ba_bwd (ba_gdpa_bwd), 2 its dK/dV kernel. The events are cudaEvent_t handles owned by
  * the caller; pass NULL, NULL to stop recording. Returns BA_ERR_INVALID_ARG
  * for another `which`. Only the hook pointers are stored (thread-local);
  * nothing is synchronised.

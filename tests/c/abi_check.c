@@ -83,6 +83,16 @@ int main(void)
           BA_ERR_INVALID_ARG); /* the plain workspace has no room for the rotated copies */
 
     CHECK(ba_selftest_wait_timeout(NULL, 256, 1000, NULL) == BA_ERR_INVALID_ARG);
+    CHECK(ba_gdpa_workspace_size(&p, 128, 2) == f);
+    CHECK(ba_gdpa_fwd(&p, (ba_activation)7, fake, fake, fake, fake, 128, 2, fake, fake, f, NULL) ==
+          BA_ERR_INVALID_ARG); /* not an activation */
+    CHECK(ba_gdpa_fwd(&p, BA_ACT_GELU, fake, fake, fake, fake, 128, 2, fake, fake, 16, NULL) ==
+          BA_ERR_INVALID_ARG); /* workspace too small */
+    CHECK(ba_gdpa_bwd(&p, BA_ACT_SILU, fake, fake, fake, NULL, fake, 128, 2, fake, fake, fake, fake, f, NULL) ==
+          BA_ERR_INVALID_ARG); /* no dout */
+    CHECK(ba_selftest_exp2(NULL, NULL, 5, NULL) == BA_ERR_INVALID_ARG);
+    CHECK(ba_selftest_exp2((const float *)fake, (float *)fake, -1, NULL) == BA_ERR_INVALID_ARG);
+    CHECK(ba_selftest_exp2(NULL, NULL, 0, NULL) == BA_OK); /* nothing to do, nothing launched */
     CHECK(ba_set_profile_events(3, NULL, NULL) == BA_ERR_INVALID_ARG);
     CHECK(ba_device_status(NULL, NULL) == BA_ERR_INVALID_ARG);
 

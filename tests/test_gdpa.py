@@ -1,0 +1,94 @@
+"""GPU parity of generalized dot-product attention (ba_gdpa_fwd / ba_gdpa_bwd,
+called through the C ABI) against the fp64 oracle in oracle/gdpa.py.
+
+GDPA replaces the softmax with an activation such as GELU or SiLU ("GEM
+(Meta)", section "Custom kernels"); the reading implemented on both sides:
+out_i = sum over visible j of act(q_i . k_j / sqrt(D)) v_j under the block
+rule, no normalisation. The activation values fed to the P V product and
+their derivatives fed to dS are rounded to bf16, like the softmax path's
+probabilities, so the tolerances are the project's bf16 ones (parity_util):
+max-abs 2e-2 and relative L2 1e-2 on out, dq, dk, dv, the max-abs bound
+taken relative to max(1, max|ref|) on peaked inputs whose outputs run to
+tens or hundreds (no normalisation keeps them small).
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_kunlun_b200 as ba
+from block_sparse_attention_kunlun_b200.workloads import CONFIGS, make_inputs
+from oracle import gdpa as G
+from parity_util import check_bf16, f64
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # (head_dim, block, window, lengths)
+    (128, 256, 2, [64, 4096, 1000, 257, 129]),      # the jagged long-history shapes, reduced batch
+    (64, 128, 2, [1024, 1024, 0, 300]),
+    (128, 64, 1, [0, 1, 127, 128, 129, 383]),       # independent 64-token blocks
+    (64, 100, 3, [1, 99, 250, 640]),
+]
+
+
+def run_gpu(inp, block, window, act):
+    q, k, v, dout = (inp[n].cuda() for n in ("q", "k", "v", "dout"))
+    offs = inp["seq_offsets"].cuda()
+    out = ba.gdpa_fwd(q, k, v, offs, block, window, act)
+    dq, dk, dv = ba.gdpa_bwd(q, k, v, dout, offs, block, window, act)
+    torch.cuda.synchronize()
+    return {n: t.cpu() for n, t in dict(out=out, dq=dq, dk=dk, dv=dv).items()}
+
+
+def run_oracle(inp, block, window, act):
+    args = (inp["seq_offsets"].numpy(), f64(inp["q"]), f64(inp["k"]), f64(inp["v"]))
+    out = G.fwd(*args, block, window, act)
+    dq, dk, dv = G.bwd(*args, f64(inp["dout"]), block, window, act)
+    return dict(out=out, dq=dq, dk=dk, dv=dv)
+
+
+@pytest.mark.parametrize("act", ["gelu", "silu"])
+@pytest.mark.parametrize("head_dim,block,window,lengths", CASES)
+@pytest.mark.parametrize("peaked", [False, True], ids=["config", "peaked"])
+def test_gdpa_matches_oracle(act, head_dim, block, window, lengths, peaked):
+    w = CONFIGS[3].replace(head_dim=head_dim, block=block, window=window, heads=2, batch=len(lengths))
+    q_gain = 1.0
+    if peaked:
+        w = w.replace(qkv_scale=1.0)
+        q_gain = 3.0
+    inp = make_inputs(w, q_gain=q_gain, lengths=lengths, seed=300 + head_dim + block)
+    got = run_gpu(inp, block, window, act)
+    ref = run_oracle(inp, block, window, act)
+    for n in ("out", "dq", "dk", "dv"):
+        check_bf16(f"{act} {n}", got[n], ref[n], peaked=peaked)
+
+
+def test_gdpa_examples_are_isolated_and_deterministic():
+    """Examples do not see each other (a jagged batch equals its examples run
+    one by one, bit for bit), and a second call gives the same bits."""
+    w = CONFIGS[3].replace(heads=2, batch=3)
+    lengths = [300, 129, 700]
+    inp = make_inputs(w, lengths=lengths, seed=11)
+    got = run_gpu(inp, w.block, w.window, "gelu")
+    again = run_gpu(inp, w.block, w.window, "gelu")
+    offs = inp["seq_offsets"].numpy()
+    for n in got:
+        assert torch.equal(got[n], again[n]), n
+    for e in range(3):
+        sl = slice(int(offs[e]), int(offs[e + 1]))
+        one = {n: inp[n][sl].clone() for n in ("q", "k", "v", "dout")}
+        one["seq_offsets"] = torch.tensor([0, lengths[e]], dtype=torch.int32)
+        alone = run_gpu(one, w.block, w.window, "gelu")
+        for n in got:
+            assert torch.equal(got[n][sl], alone[n]), (e, n)
+
+
+def test_gdpa_rejects_fp32_and_unknown_activations():
+    q = torch.zeros((128, 2, 64), device="cuda")
+    offs = torch.tensor([0, 128], dtype=torch.int32, device="cuda")
+    prob = ba.make_problem(q, offs)
+    ws = ba.workspace_for(ba.ba_gdpa_workspace_size(prob, 64, 1), q.device)
+    assert ba.ba_gdpa_fwd(prob, "gelu", q, q, q, offs, 64, 1, q.clone(), ws) == ba.BA_ERR_UNSUPPORTED
+    qb = q.to(torch.bfloat16)
+    prob = ba.make_problem(qb, offs)
+    assert ba.ba_gdpa_fwd(prob, 7, qb, qb, qb, offs, 64, 1, qb.clone(), ws) == ba.BA_ERR_INVALID_ARG
