@@ -15,8 +15,14 @@ FLOPs per visible query/key pair and head, summed over all ranks) with the
 inputs resident in HBM; ``e2e`` is the same metric with pinned-host inputs
 copied in and the results copied out inside the timed region.
 
-Multi-GPU (torchrun): every rank runs its own batch (seeded per rank) with
-no collective on the data path; the step time is the max over ranks.
+The same line carries ``other_configs``: the long-context workload (8 x 32768,
+block 512, window 4) and the jagged workload with component skip, each timed
+the same way (N = 1 only).
+
+Multi-GPU: every rank runs its own batch (seeded per rank) with no
+collective on the data path; the step time is the max over ranks. Launched
+as ``bench.py --gpus N`` without torchrun, the script starts N ranks itself
+(torch.distributed.run, one process per GPU); under torchrun it is one rank.
 ``--impl reference`` times the CPU oracle on bounded samples instead.
 """
 from __future__ import annotations
@@ -44,7 +50,7 @@ METRIC = "block-attention fwd+bwd useful TFLOP/s and tokens/s on 1 B200; % of bf
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
@@ -61,11 +67,14 @@ def parse():
                          "window W) on the config's shapes instead of block attention")
     ap.add_argument("--rope", action="store_true",
                     help="rotary embedding on q and k (ba_rope_fwd / ba_rope_bwd)")
+    ap.add_argument("--gdpa", choices=["gelu", "silu"], default=None,
+                    help="generalized dot-product attention (ba_gdpa_fwd / ba_gdpa_bwd): the activation "
+                         "in place of the softmax, same block rule and shapes")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic-file", default=os.path.join(ROOT, "profiles", "traffic.json"),
                     help="per-launch DRAM bytes of the dominant kernel from an ncu capture")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def load_peaks():
@@ -76,6 +85,36 @@ def load_peaks():
         return d, "measured"
     except (OSError, ValueError):
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def spawn_ranks(n: int, argv, script: str = None, **run_kw) -> subprocess.CompletedProcess:
+    """Runs `script argv` as n ranks on this node (one process per GPU) through
+    torch.distributed.run on 127.0.0.1 and waits for them. Each rank finds
+    RANK / LOCAL_RANK / WORLD_SIZE / MASTER_* in its environment; rank 0 alone
+    prints the JSON line. run_kw goes to subprocess.run (e.g. capture_output)."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()),
+           script or os.path.abspath(__file__), *argv]
+    return subprocess.run(cmd, **run_kw)
 
 
 def config_workload(args):
@@ -91,6 +130,10 @@ def config_workload(args):
         w = w.replace(block=b, window=win, name=re.sub(r"block \d+, window \d+", f"block {b}, window {win}", w.name))
     if getattr(args, "rope", False):
         w = w.replace(name=w.name + ", rotary q/k")
+    if getattr(args, "gdpa", None):
+        if w.skip_p > 0:
+            raise SystemExit("--gdpa takes no skip flags: pick a workload without component skip")
+        w = w.replace(name=w.name + f", GDPA {args.gdpa}")
     return w
 
 
@@ -194,7 +237,7 @@ def cpu_baseline(w, inp, pairs_total, budget_frac=0.04, tables=None):
         oracle.rope_bwd(sub_offs, q, k, v, do, c, s, w.block, w.window, skip=sub_skip, nthreads=threads)
     dt = time.perf_counter() - t0
     useful = F.step_flops(acc, w.heads, w.head_dim)["step"]
-    return {"value": useful / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+    return {"value": useful / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "cpu": cpu_model(), "kind": "oracle",
             "sample": f"fwd+bwd of the first {n} of {len(lens)} examples ({s1} tokens, all heads, "
                       f"{acc / max(pairs_total, 1):.1%} of the batch's visible pairs), {dt:.1f} s"}
 
@@ -226,6 +269,11 @@ def run_reference(args):
         c, s = (t.to(torch.float64).numpy() for t in tables_for(lens, w.head_dim))
 
     def step():
+        if args.gdpa:
+            from oracle import gdpa
+            gdpa.fwd(sub, q, k, v, w.block, w.window, args.gdpa)
+            gdpa.bwd(sub, q, k, v, do, w.block, w.window, args.gdpa)
+            return
         if args.rope:
             oracle.rope_fwd(sub, q, k, v, c, s, w.block, w.window, nthreads=threads)
             oracle.rope_bwd(sub, q, k, v, do, c, s, w.block, w.window, nthreads=threads)
@@ -245,8 +293,8 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": w.name, "sample": sample},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "cpu": cpu_model(),
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -264,128 +312,201 @@ def job_totals(flops, tokens, ms, dist=None, device="cpu"):
     return tuple(float(x) for x in totals.tolist())
 
 
-def main():
-    args = parse()
+KERNEL_NAMES = {"fwd": "fwd_bf16_sm100_kernel", "bwd_dq": "bwd_dq_sm100_kernel",
+                "bwd_dkdv": "bwd_dkdv_sm100_kernel"}
+
+
+class Runner:
+    """Device buffers and one training step (ba_fwd + ba_bwd, or the rotary
+    entry points) of one workload through the library's public API."""
+
+    def __init__(self, ba, w, inp, dev, rope=False, gdpa=None):
+        self.ba, self.w, self.inp, self.dev, self.rope, self.gdpa = ba, w, inp, dev, rope, gdpa
+        self.lens = inp["lengths"].numpy()
+        self.skip_np = inp["skip"].numpy() if inp["skip"] is not None else None
+        T, H, D = inp["q"].shape
+        self.T, self.H, self.D = T, H, D
+        self.pairs = F.visible_pairs(self.lens, w.block, w.window, self.skip_np)
+        self.flops = F.step_flops(self.pairs, H, D)
+        self.bytes = F.step_bytes(T, H, D)
+        self.q, self.k, self.v, self.dout = (inp[n].to(dev) for n in ("q", "k", "v", "dout"))
+        self.offs = inp["seq_offsets"].to(dev)
+        self.skip = inp["skip"].to(dev) if inp["skip"] is not None else None
+        self.out, self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(4))
+        self.lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+        self.prob = ba.make_problem(self.q, self.offs)
+        self.stream = torch.cuda.current_stream(dev)
+        self.tables = None
+        if rope:
+            self.tables = tables_for(self.lens, D)
+            self.cos_d, self.sin_d = (t.to(dev) for t in self.tables)
+            self.q_rot, self.k_rot = torch.empty_like(self.q), torch.empty_like(self.k)
+            self.rope_arg = ba.make_rope(self.cos_d, self.sin_d, self.q_rot, self.k_rot)
+        self.ws_f = ba.workspace_for(ba.ba_fwd_workspace_size(self.prob, w.block, w.window), dev)
+        self.ws_b = ba.workspace_for(ba.ba_bwd_workspace_size(self.prob, w.block, w.window), dev)
+        # ba_fwd: work list, (skip), attention; ba_bwd: work list, (skip), dQ, dK/dV; the rotary
+        # forward adds one rotation pass (the backward reads the kept rotated copies)
+        self.launches_per_step = (2 + (self.skip is not None)) + (3 + (self.skip is not None)) + (1 if rope else 0)
+        if gdpa:
+            self.launches_per_step = 5  # work list + forward; work list + dQ + dK/dV
+
+    def step(self):
+        ba, w, s = self.ba, self.w, self
+        if s.gdpa:
+            st = ba.ba_gdpa_fwd(s.prob, s.gdpa, s.q, s.k, s.v, s.offs, w.block, w.window, s.out, s.ws_f,
+                                stream=s.stream)
+            if st != ba.BA_OK:
+                raise ba.BAError(st, "ba_gdpa_fwd")
+            st = ba.ba_gdpa_bwd(s.prob, s.gdpa, s.q, s.k, s.v, s.dout, s.offs, w.block, w.window, s.dq, s.dk,
+                                s.dv, s.ws_f, stream=s.stream)
+            if st != ba.BA_OK:
+                raise ba.BAError(st, "ba_gdpa_bwd")
+            return
+        if s.rope:
+            st = ba.ba_rope_fwd(s.prob, s.rope_arg, s.q, s.k, s.v, s.offs, w.block, w.window, s.skip, s.out,
+                                s.lse, s.ws_f, stream=s.stream)
+        else:
+            st = ba.ba_fwd(s.prob, s.q, s.k, s.v, s.offs, w.block, w.window, s.skip, s.out, s.lse, s.ws_f,
+                           stream=s.stream)
+        if st != ba.BA_OK:
+            raise ba.BAError(st, "ba_fwd")
+        if s.rope:
+            st = ba.ba_rope_bwd(s.prob, s.rope_arg, s.q, s.k, s.v, s.out, s.lse, s.dout, s.offs, w.block,
+                                w.window, s.skip, s.dq, s.dk, s.dv, s.ws_b, stream=s.stream)
+        else:
+            st = ba.ba_bwd(s.prob, s.q, s.k, s.v, s.out, s.lse, s.dout, s.offs, w.block, w.window, s.skip,
+                           s.dq, s.dk, s.dv, s.ws_b, stream=s.stream)
+        if st != ba.BA_OK:
+            raise ba.BAError(st, "ba_bwd")
+
+    def check_status(self, when):
+        if self.ba.ba_device_status(self.ws_f) != self.ba.BA_OK or \
+                (not self.gdpa and self.ba.ba_device_status(self.ws_b) != self.ba.BA_OK):
+            raise RuntimeError(f"a kernel timed out {when}")
+
+    def timed(self, K, warmup, barrier, clocks=None):
+        """W warm-up steps, then K steps between two events on the launching
+        stream; per-kernel events through ba_set_profile_events. Returns the
+        total ms and the mean ms of each attention kernel."""
+        ba = self.ba
+        for _ in range(warmup):
+            self.step()
+        barrier()
+        self.check_status("during warm-up")
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        per = {n: [(ev(), ev()) for _ in range(K)] for n in KERNEL_NAMES}
+        for pairs in per.values():  # torch creates the CUDA event on its first record
+            for a, b in pairs:
+                a.record(self.stream)
+                b.record(self.stream)
+        t_start, t_stop = ev(), ev()
+        if clocks is not None:
+            time.sleep(0.3)
+        barrier()
+        if clocks is not None:
+            clocks.mark("t0")
+        t_start.record(self.stream)
+        for i in range(K):
+            for which, n in enumerate(KERNEL_NAMES):
+                ba.ba_set_profile_events(which, *per[n][i])
+            self.step()
+        t_stop.record(self.stream)
+        for which in range(3):
+            ba.ba_set_profile_events(which)
+        barrier()
+        if clocks is not None:
+            clocks.mark("t1")
+        self.check_status("during the timed steps")
+        ms_k = {n: statistics.mean(a.elapsed_time(b) for a, b in per[n]) for n in KERNEL_NAMES}
+        return t_start.elapsed_time(t_stop), ms_k
+
+    def kernel_stats(self, ms_k):
+        # Per kernel, the FLOPs its own tensor-core work does on visible pairs: forward 4 D (S, PV),
+        # dQ pass 6 D (S, dP, dQ), dK/dV pass 8 D (S, dP, dV, dK); per visible pair and head.
+        unit = self.pairs * self.H * self.D
+        fl = {"fwd": 4 * unit, "bwd_dq": 6 * unit, "bwd_dkdv": 8 * unit}
+        return {n: {"ms": ms_k[n], "tflops": fl[n] / (ms_k[n] / 1e3) / 1e12, "flops_per_launch": fl[n]}
+                for n in KERNEL_NAMES}
+
+
+def other_config_line(ba, cfg, dev, K, warmup, local):
+    """One more workload timed like the main one (its own process memory is
+    released afterwards)."""
+    w = CONFIGS[cfg]
+    inp = make_inputs(w)
+    run = Runner(ba, w, inp, dev)
+    clocks = ClockSampler(local)
+    ms_total, ms_k = run.timed(K, warmup, lambda: torch.cuda.synchronize(dev), clocks)
+    clk = clocks.stop()
+    ms = ms_total / K
+    d = {"workload": w.name, "ms_per_step": ms, "useful_tflops": run.flops["step"] / (ms / 1e3) / 1e12,
+         "tokens_per_s": run.T / (ms / 1e3), "total_tokens": int(run.T),
+         "visible_pairs_per_head": run.pairs, "useful_flops_per_step": run.flops["step"],
+         "steps": K, "warmup": warmup, "kernels": run.kernel_stats(ms_k), "clocks": clk}
+    if run.skip_np is not None:
+        d["live_tokens"] = F.live_tokens(run.lens, run.skip_np)
+        d["skipped_examples"] = int(run.skip_np.sum())
+    del run, inp
+    torch.cuda.empty_cache()
+    return d
+
+
+def main(argv=None, runner_cls=None):
+    """The benchmark. runner_cls replaces Runner (the GPU step) with a stand-in
+    of the same interface; it then runs on the CPU with gloo ranks, which is
+    how the multi-rank launch and report are tested without a GPU."""
+    args = parse(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU, launched here; each rank re-enters main() below
+        sys.exit(spawn_ranks(args.gpus, sys.argv[1:] if argv is None else argv).returncode)
 
     import block_sparse_attention_kunlun_b200 as ba
 
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
+    on_gpu = runner_cls is None
+    if on_gpu:
+        torch.cuda.set_device(local)
+        dev = torch.device("cuda", local)
+    else:
+        dev = torch.device("cpu")
     dist = None
     if world > 1:
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+        if on_gpu:
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=300))
 
     w, inp = workload(args, rank)
-    offs_h = inp["seq_offsets"]
-    lens = inp["lengths"].numpy()
-    skip_np = inp["skip"].numpy() if inp["skip"] is not None else None
-    T, H, D = inp["q"].shape
-    pairs = F.visible_pairs(lens, w.block, w.window, skip_np)
-    fl = F.step_flops(pairs, H, D)
-    by = F.step_bytes(T, H, D)
-
-    # device buffers
-    q, k, v, dout = (inp[n].to(dev) for n in ("q", "k", "v", "dout"))
-    offs = offs_h.to(dev)
-    skip = inp["skip"].to(dev) if inp["skip"] is not None else None
-    out, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
-    lse = torch.empty((H, T), dtype=torch.float32, device=dev)
-    prob = ba.make_problem(q, offs)
-    stream = torch.cuda.current_stream(dev)
-    if args.rope:
-        tables = tables_for(lens, D)
-        cos_d, sin_d = (t.to(dev) for t in tables)
-        q_rot, k_rot = torch.empty_like(q), torch.empty_like(k)
-        rope = ba.make_rope(cos_d, sin_d, q_rot, k_rot)
-        ws_f = ba.workspace_for(ba.ba_fwd_workspace_size(prob, w.block, w.window), dev)
-        ws_b = ba.workspace_for(ba.ba_bwd_workspace_size(prob, w.block, w.window), dev)
-    else:
-        tables = None
-        ws_f = ba.workspace_for(ba.ba_fwd_workspace_size(prob, w.block, w.window), dev)
-        ws_b = ba.workspace_for(ba.ba_bwd_workspace_size(prob, w.block, w.window), dev)
-
-    def step():
-        if args.rope:
-            st = ba.ba_rope_fwd(prob, rope, q, k, v, offs, w.block, w.window, skip, out, lse, ws_f, stream=stream)
-        else:
-            st = ba.ba_fwd(prob, q, k, v, offs, w.block, w.window, skip, out, lse, ws_f, stream=stream)
-        if st != ba.BA_OK:
-            raise ba.BAError(st, "ba_fwd")
-        if args.rope:
-            st = ba.ba_rope_bwd(prob, rope, q, k, v, out, lse, dout, offs, w.block, w.window, skip, dq, dk, dv,
-                                ws_b, stream=stream)
-        else:
-            st = ba.ba_bwd(prob, q, k, v, out, lse, dout, offs, w.block, w.window, skip, dq, dk, dv, ws_b,
-                           stream=stream)
-        if st != ba.BA_OK:
-            raise ba.BAError(st, "ba_bwd")
+    run = (runner_cls or Runner)(ba, w, inp, dev, rope=args.rope, gdpa=args.gdpa)
+    T, H, D = run.T, run.H, run.D
+    fl, by = run.flops, run.bytes
 
     def barrier():
-        torch.cuda.synchronize(dev)
+        if on_gpu:
+            torch.cuda.synchronize(dev)
         if dist is not None:
             dist.barrier()
 
-    # ba_fwd: work list, (skip), attention; ba_bwd: work list, (skip), dQ, dK/dV;
-    # the rotary forward adds one rotation pass (the backward reads the kept rotated copies;
-    # fp32 adds a transposed pass after its backward kernels)
-    launches_per_step = (2 + (skip is not None)) + (3 + (skip is not None))
-    if args.rope:
-        launches_per_step += 1 + (w.dtype == torch.float32)
-
-    for _ in range(args.warmup):
-        step()
-    barrier()
-    if ba.ba_device_status(ws_f) != ba.BA_OK or ba.ba_device_status(ws_b) != ba.BA_OK:
-        raise RuntimeError("a kernel timed out during warm-up")
-
     K = args.steps
-    ev = lambda: torch.cuda.Event(enable_timing=True)
-    kf = [(ev(), ev()) for _ in range(K)]
-    kq = [(ev(), ev()) for _ in range(K)]
-    kb = [(ev(), ev()) for _ in range(K)]
-    for pair in kf + kq + kb:  # torch creates the CUDA event on its first record
-        for e in pair:
-            e.record(stream)
-    t_start, t_stop = ev(), ev()
-    clocks = ClockSampler(local)
-    time.sleep(0.3)
-    barrier()
-    clocks.mark("t0")
-    t_start.record(stream)
-    for i in range(K):
-        ba.ba_set_profile_events(0, *kf[i])
-        ba.ba_set_profile_events(1, *kq[i])
-        ba.ba_set_profile_events(2, *kb[i])
-        step()
-    t_stop.record(stream)
-    for which in range(3):
-        ba.ba_set_profile_events(which)
-    barrier()
-    clocks.mark("t1")
-    clk = clocks.stop()
-    ms_total = t_start.elapsed_time(t_stop)
-    ms_fwd_k = statistics.mean(a.elapsed_time(b) for a, b in kf)
-    ms_dq_k = statistics.mean(a.elapsed_time(b) for a, b in kq)
-    ms_dkv_k = statistics.mean(a.elapsed_time(b) for a, b in kb)
-    if ba.ba_device_status(ws_f) != ba.BA_OK or ba.ba_device_status(ws_b) != ba.BA_OK:
-        raise RuntimeError("a kernel timed out during the timed steps")
+    clocks = ClockSampler(local) if on_gpu else None
+    ms_total, ms_k = run.timed(K, args.warmup, barrier, clocks)
+    clk = clocks.stop() if clocks is not None else None
 
     job_flops, job_tokens, ms_max = job_totals(fl["step"] * K, T * K, ms_total, dist, dev)
     value = job_flops / (ms_max / 1e3) / 1e12
 
     # end to end through the same API: pinned host in, results out
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and on_gpu:
         host_in = [inp[n].pin_memory() for n in ("q", "k", "v", "dout")]
-        offs_pin = offs_h.pin_memory()
+        offs_pin = inp["seq_offsets"].pin_memory()
         skip_pin = inp["skip"].pin_memory() if inp["skip"] is not None else None
-        host_out = [torch.empty_like(out, device="cpu").pin_memory() for _ in range(4)]
+        host_out = [torch.empty_like(run.out, device="cpu").pin_memory() for _ in range(4)]
         lse_out = torch.empty((H, T), dtype=torch.float32).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in host_in) + offs_pin.numel() * 4 + (
             skip_pin.numel() if skip_pin is not None else 0)
@@ -393,23 +514,24 @@ def main():
         Ke = max(3, min(K, 10))
 
         def e2e_step():
-            for dst, src in zip((q, k, v, dout), host_in):
+            for dst, src in zip((run.q, run.k, run.v, run.dout), host_in):
                 dst.copy_(src, non_blocking=True)
-            offs.copy_(offs_pin, non_blocking=True)
+            run.offs.copy_(offs_pin, non_blocking=True)
             if skip_pin is not None:
-                skip.copy_(skip_pin, non_blocking=True)
-            step()
-            for dst, src in zip(host_out, (out, dq, dk, dv)):
+                run.skip.copy_(skip_pin, non_blocking=True)
+            run.step()
+            for dst, src in zip(host_out, (run.out, run.dq, run.dk, run.dv)):
                 dst.copy_(src, non_blocking=True)
-            lse_out.copy_(lse, non_blocking=True)
+            lse_out.copy_(run.lse, non_blocking=True)
 
         e2e_step()
         barrier()
+        ev = lambda: torch.cuda.Event(enable_timing=True)
         a, b = ev(), ev()
-        a.record(stream)
+        a.record(run.stream)
         for _ in range(Ke):
             e2e_step()
-        b.record(stream)
+        b.record(run.stream)
         barrier()
         ms_e2e = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
         if dist is not None:
@@ -424,54 +546,70 @@ def main():
         return
 
     peaks, peaks_src = load_peaks()
-    tensor_peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    burst_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    # Per kernel, the FLOPs its own tensor-core work does on visible pairs: forward 4 D (S, PV),
-    # dQ pass 6 D (S, dP, dQ), dK/dV pass 8 D (S, dP, dV, dK); per visible pair and head.
-    unit = pairs * H * D
-    kern = {"fwd": (4 * unit, ms_fwd_k), "bwd_dq": (6 * unit, ms_dq_k), "bwd_dkdv": (8 * unit, ms_dkv_k)}
-    kstats = {n: {"ms": ms, "tflops": f / (ms / 1e3) / 1e12, "flops_per_launch": f} for n, (f, ms) in kern.items()}
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    timed_s = ms_total / 1e3
+    # the burst figure for a region shorter than the seconds the sustained figure takes to settle
+    long_region = timed_s >= 5.0
+    tensor_peak = sustained if long_region else burst
+    kstats = run.kernel_stats(ms_k)
     dom = max(kstats, key=lambda n: kstats[n]["ms"])
-    names = {"fwd": "fwd_bf16_sm100_kernel", "bwd_dq": "bwd_dq_sm100_kernel", "bwd_dkdv": "bwd_dkdv_sm100_kernel"}
     traffic = None
     try:
         with open(args.traffic_file) as f:
             tr = json.load(f)
-        key = f"{names[dom]}:config{args.config}" + (f":block{w.block}:window{w.window}"
-                                                       if (args.swa or args.block or args.window) else "")
+        key = f"{KERNEL_NAMES[dom]}:config{args.config}" + (f":block{w.block}:window{w.window}"
+                                                            if (args.swa or args.block or args.window) else "")
         key += ":rope" if args.rope else ""
+        key += f":gdpa-{args.gdpa}" if args.gdpa else ""
         if key in tr and tr[key].get("kernel_sha") == kernel_sha(dom):
             traffic = tr[key]["bytes_per_launch"]
     except (OSError, ValueError):
         pass
     achieved = kstats[dom]["tflops"]
-    roofline = {"kernel": names[dom], "bound": "tensor", "achieved": achieved, "peak": tensor_peak,
+    flops_launch = kstats[dom]["flops_per_launch"]
+    roofline = {"kernel": KERNEL_NAMES[dom], "bound": "tensor", "achieved": achieved, "peak": tensor_peak,
                 "unit": "TFLOP/s", "frac": achieved / tensor_peak, "traffic": traffic,
-                "peak_source": f"{peaks_src} bf16_tflops_sustained",
-                "algorithmic_flops_per_launch": kstats[dom]["flops_per_launch"],
+                "peak_source": f"{peaks_src} {'bf16_tflops_sustained' if long_region else 'bf16_tflops (burst)'};"
+                               f" timed region {timed_s:.2f} s",
+                "algorithmic_flops_per_launch": flops_launch,
                 "ms_per_launch": kstats[dom]["ms"], "share_of_step": kstats[dom]["ms"] * K / ms_total}
+    if traffic:
+        # the roof this kernel can reach at its measured arithmetic intensity
+        intensity = flops_launch / traffic
+        attainable = min(tensor_peak, intensity * hbm / 1e3)
+        roofline.update({"intensity_flop_per_byte": intensity, "hbm_peak_gbs": hbm,
+                         "attainable": attainable, "frac_of_attainable": achieved / attainable})
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
         "data": "synthetic",
-        "config": {"workload": w.name, "batch": int(len(lens)), "total_tokens": int(T), "heads": H,
+        "config": {"workload": w.name, "batch": int(len(run.lens)), "total_tokens": int(T), "heads": H,
                    "head_dim": D, "block": w.block, "window": w.window, "seed": w.seed,
-                   "rotary": bool(args.rope),
-                   "visible_pairs_per_head": pairs, "useful_flops_per_step": fl["step"],
+                   "rotary": bool(args.rope), "attention": f"gdpa-{args.gdpa}" if args.gdpa else "softmax",
+                   "visible_pairs_per_head": run.pairs, "useful_flops_per_step": fl["step"],
                    "l2": f"inputs larger than L2 ({by['fwd'] + by['bwd']:.3g} B touched per step), no flush",
                    "parallelism": f"dp{world} (independent batches, no collective in the step)"},
         "tokens_per_s": job_tokens / (ms_max / 1e3),
-        "pct_of_bf16_peak": {"sustained": value / tensor_peak, "burst": value / burst_peak,
-                             "source": peaks_src},
+        "pct_of_bf16_peak": {"burst": value / burst, "sustained": value / sustained, "source": peaks_src},
         "kernels": kstats,
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": launches_per_step * K,
+        "gpu_launches": run.launches_per_step * K,
         "clocks": clk,
     }
-    if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(w, inp, pairs, tables=tables)
+    pairs, lens = run.pairs, run.lens
+    if world == 1 and on_gpu and not args.examples and not (args.swa or args.block or args.window or args.rope
+                                                            or args.gdpa):
+        del run
+        torch.cuda.empty_cache()
+        Ko = max(5, min(K, 20))
+        line["other_configs"] = {f"config{c}": other_config_line(ba, c, dev, Ko, max(3, args.warmup), local)
+                                 for c in (4, 5) if c != args.config}
+    if not args.no_cpu_baseline and world == 1 and on_gpu and not args.gdpa:
+        line["cpu_baseline"] = cpu_baseline(w, inp, pairs, tables=tables_for(lens, D) if args.rope else None)
     print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

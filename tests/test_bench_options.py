@@ -81,3 +81,15 @@ def test_reference_arm_prints_one_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert "workload" in d["config"]
+
+
+def test_gdpa_option_names_the_activation_and_refuses_skip_flags():
+    import pytest
+    b = _bench()
+    a = Args()
+    a.gdpa = "silu"
+    w = b.config_workload(a)
+    assert w.name.endswith(", GDPA silu") and (w.block, w.window) == (256, 2)
+    a.config = 5
+    with pytest.raises(SystemExit):
+        b.config_workload(a)
