@@ -27,6 +27,8 @@ __all__ = [
     "block_attention_fwd", "block_attention_bwd", "sliding_window_attention_fwd", "sliding_window_attention_bwd",
     "rope_block_attention_fwd", "rope_block_attention_bwd",
     "ba_gdpa_workspace_size", "ba_gdpa_fwd", "ba_gdpa_bwd", "gdpa_fwd", "gdpa_bwd",
+    "ba_gdpa_cross_workspace_size", "ba_gdpa_cross_fwd", "ba_gdpa_cross_bwd", "gdpa_cross_fwd", "gdpa_cross_bwd",
+    "ba_mx_quantize", "ba_mx_fwd_workspace_size", "ba_mx_fwd", "mx_quantize", "mx_block_attention_fwd",
     "library_path",
 ]
 
@@ -109,6 +111,18 @@ def _load():
     lib.ba_gdpa_fwd.restype = ctypes.c_int
     lib.ba_gdpa_bwd.argtypes = [prob, ctypes.c_int, P, P, P, P, P, i32, i32, P, P, P, P, ctypes.c_size_t, P]
     lib.ba_gdpa_bwd.restype = ctypes.c_int
+    lib.ba_gdpa_cross_workspace_size.argtypes = [prob, i32]
+    lib.ba_gdpa_cross_workspace_size.restype = ctypes.c_size_t
+    lib.ba_gdpa_cross_fwd.argtypes = [prob, i32, ctypes.c_int, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.ba_gdpa_cross_fwd.restype = ctypes.c_int
+    lib.ba_gdpa_cross_bwd.argtypes = [prob, i32, ctypes.c_int, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.ba_gdpa_cross_bwd.restype = ctypes.c_int
+    lib.ba_mx_quantize.argtypes = [P, ctypes.c_int64, i32, i32, P, P, P]
+    lib.ba_mx_quantize.restype = ctypes.c_int
+    lib.ba_mx_fwd_workspace_size.argtypes = [prob, i32, i32]
+    lib.ba_mx_fwd_workspace_size.restype = ctypes.c_size_t
+    lib.ba_mx_fwd.argtypes = [prob, P, P, P, P, i32, i32, P, P, P, P, ctypes.c_size_t, P]
+    lib.ba_mx_fwd.restype = ctypes.c_int
     rope = ctypes.POINTER(BARope)
     lib.ba_rope_fwd_workspace_size.argtypes = [prob, i32, i32]
     lib.ba_rope_fwd_workspace_size.restype = ctypes.c_size_t
@@ -283,6 +297,130 @@ def gdpa_bwd(q, k, v, dout, seq_offsets, block, window, activation="gelu", dq=No
     if st != BA_OK:
         raise BAError(st, "ba_gdpa_bwd")
     return dq, dk, dv
+
+
+def ba_gdpa_cross_workspace_size(problem: BAProblem, kv_total_tokens: int) -> int:
+    return int(_load().ba_gdpa_cross_workspace_size(ctypes.byref(problem), int(kv_total_tokens)))
+
+
+def ba_gdpa_cross_fwd(problem, kv_total_tokens, activation, q, k, v, q_offsets, kv_offsets, out, workspace,
+                      workspace_bytes=None, stream=None) -> int:
+    """Direct call of the cross-attention GDPA forward; returns its status code."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(_load().ba_gdpa_cross_fwd(ctypes.byref(problem), int(kv_total_tokens), _act(activation), _ptr(q),
+                                         _ptr(k), _ptr(v), _ptr(q_offsets), _ptr(kv_offsets), _ptr(out),
+                                         _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def ba_gdpa_cross_bwd(problem, kv_total_tokens, activation, q, k, v, dout, q_offsets, kv_offsets, dq, dk, dv,
+                      workspace, workspace_bytes=None, stream=None) -> int:
+    """Direct call of the cross-attention GDPA backward; returns its status code."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(_load().ba_gdpa_cross_bwd(ctypes.byref(problem), int(kv_total_tokens), _act(activation), _ptr(q),
+                                         _ptr(k), _ptr(v), _ptr(dout), _ptr(q_offsets), _ptr(kv_offsets),
+                                         _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), int(workspace_bytes),
+                                         _stream(stream)))
+
+
+def _check_cross(q, k, v, q_offsets, kv_offsets):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != q.dtype or t.dim() != 3:
+            raise ValueError(f"{name} must be a contiguous CUDA tensor like q")
+    if k.shape != v.shape or k.shape[1:] != q.shape[1:]:
+        raise ValueError("k and v must be [kv_total_tokens, heads, head_dim] like q's heads and head_dim")
+    for name, t in (("q_offsets", q_offsets), ("kv_offsets", kv_offsets)):
+        if t.dtype != torch.int32 or not t.is_cuda:
+            raise ValueError(f"{name} must be an int32 CUDA tensor")
+    if q_offsets.numel() != kv_offsets.numel():
+        raise ValueError("q_offsets and kv_offsets must describe the same examples")
+
+
+def gdpa_cross_fwd(q, k, v, q_offsets, kv_offsets, activation="gelu", out=None, workspace=None, stream=None):
+    """Cross-attention GDPA: example b's queries see every key of its own
+    key/value set (no mask). Allocates out (and a workspace) with torch and
+    runs ba_gdpa_cross_fwd."""
+    _check_cross(q, k, v, q_offsets, kv_offsets)
+    prob = make_problem(q, q_offsets)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = workspace_for(ba_gdpa_cross_workspace_size(prob, k.shape[0]), q.device)
+    st = ba_gdpa_cross_fwd(prob, k.shape[0], activation, q, k, v, q_offsets, kv_offsets, out, workspace,
+                           stream=stream)
+    if st != BA_OK:
+        raise BAError(st, "ba_gdpa_cross_fwd")
+    return out
+
+
+def gdpa_cross_bwd(q, k, v, dout, q_offsets, kv_offsets, activation="gelu", dq=None, dk=None, dv=None,
+                   workspace=None, stream=None):
+    """Gradients of gdpa_cross_fwd (ba_gdpa_cross_bwd)."""
+    _check_cross(q, k, v, q_offsets, kv_offsets)
+    prob = make_problem(q, q_offsets)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = workspace_for(ba_gdpa_cross_workspace_size(prob, k.shape[0]), q.device)
+    st = ba_gdpa_cross_bwd(prob, k.shape[0], activation, q, k, v, dout, q_offsets, kv_offsets, dq, dk, dv,
+                           workspace, stream=stream)
+    if st != BA_OK:
+        raise BAError(st, "ba_gdpa_cross_bwd")
+    return dq, dk, dv
+
+
+def ba_mx_quantize(x, elements, scales, stream=None) -> int:
+    """Direct call of the MX (E4M3 / E8M0) quantisation of x [rows, heads, head_dim] bf16."""
+    rows, heads, head_dim = x.shape
+    return int(_load().ba_mx_quantize(_ptr(x), int(rows), int(heads), int(head_dim), _ptr(elements),
+                                      _ptr(scales), _stream(stream)))
+
+
+def mx_quantize(x, stream=None):
+    """MX quantisation of a bf16 CUDA tensor [rows, heads, head_dim]: returns
+    (elements uint8 [rows, heads, head_dim] holding E4M3 codes, scales uint8
+    [rows, heads rounded up to 4, head_dim / 32] holding E8M0 codes)."""
+    rows, heads, head_dim = x.shape
+    elements = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scales = torch.zeros((rows, (heads + 3) // 4 * 4, head_dim // 32), dtype=torch.uint8, device=x.device)
+    st = ba_mx_quantize(x, elements, scales, stream)
+    if st != BA_OK:
+        raise BAError(st, "ba_mx_quantize")
+    return elements, scales
+
+
+def ba_mx_fwd_workspace_size(problem: BAProblem, block: int, window: int) -> int:
+    return int(_load().ba_mx_fwd_workspace_size(ctypes.byref(problem), int(block), int(window)))
+
+
+def ba_mx_fwd(problem, q, k, v, seq_offsets, block, window, skip, out, lse, workspace, workspace_bytes=None,
+              stream=None) -> int:
+    """Direct call of the MXFP8-operand forward; returns its status code."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(_load().ba_mx_fwd(ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), int(block),
+                                 int(window), _ptr(skip), _ptr(out), _ptr(lse), _ptr(workspace),
+                                 int(workspace_bytes), _stream(stream)))
+
+
+def mx_block_attention_fwd(q, k, v, seq_offsets, block, window, skip=None, out=None, lse=None, workspace=None,
+                           stream=None):
+    """Block attention with MXFP8 Q and K in the score product (ba_mx_fwd);
+    allocates out/lse (and a workspace) with torch."""
+    _check_inputs(q, k, v, seq_offsets)
+    prob = make_problem(q, seq_offsets)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = workspace_for(ba_mx_fwd_workspace_size(prob, block, window), q.device)
+    st = ba_mx_fwd(prob, q, k, v, seq_offsets, block, window, skip, out, lse, workspace, stream=stream)
+    if st != BA_OK:
+        raise BAError(st, "ba_mx_fwd")
+    return out, lse
 
 
 def make_rope(cos, sin, q_rot=None, k_rot=None) -> BARope:

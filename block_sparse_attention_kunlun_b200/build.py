@@ -19,7 +19,7 @@ LIB = os.path.join(HERE, "libba.so")
 OBJDIR = os.path.join(HERE, "_build")
 
 SOURCES = ["ba_api.cu", "ba_aux.cu", "ba_simt.cu", "ba_fwd_sm100.cu", "ba_bwd_dq_sm100.cu",
-           "ba_bwd_dkdv_sm100.cu", "ba_noalloc.cu", "ba_rope.cu"]
+           "ba_bwd_dkdv_sm100.cu", "ba_noalloc.cu", "ba_rope.cu", "ba_mx.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -23,6 +23,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <type_traits>
 
 namespace {
 
@@ -78,6 +79,22 @@ bool encode_bf16_rows(CUtensorMap *map, const void *base, int64_t T, int64_t H, 
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D byte views for the MXFP8 forward: E4M3 rows [T, H * D] in 128 x 128-byte
+// boxes (one 128-byte swizzled row per head at head_dim 128), and scale words
+// [T, heads_pad * 4] in 128-row x 16-byte boxes (four heads' words).
+bool encode_u8_rows(CUtensorMap *map, const void *base, int64_t T, int64_t row_bytes, uint32_t box_x, bool swizzle)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cuuint64_t(row_bytes), cuuint64_t(T)};
+    cuuint64_t strides[1] = {cuuint64_t(row_bytes)};
+    cuuint32_t box[2] = {box_x, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -377,6 +394,151 @@ ba_status gdpa_impl(bool bwd, const ba_problem *pp, ba_activation act, const voi
     return e == cudaSuccess ? BA_OK : BA_ERR_CUDA;
 }
 
+// Cross-attention GDPA: query tiles against their example's key/value set
+// (forward, dQ pass), key tiles against their example's query set (dK/dV
+// pass); rows whose other side is empty get zeros.
+ba_status gdpa_cross_impl(bool bwd, const ba_problem *pp, int32_t kv_total, ba_activation act, const void *q,
+                          const void *k, const void *v, const void *dout, const int32_t *q_offsets,
+                          const int32_t *kv_offsets, void *out, void *dq, void *dk, void *dv, void *workspace,
+                          size_t workspace_bytes, ba_stream_t stream_)
+{
+    ba_status st = check_problem(pp, 1, 1);
+    if (st != BA_OK) return st;
+    if (act != BA_ACT_GELU && act != BA_ACT_SILU) return BA_ERR_INVALID_ARG;
+    const ba_problem &P = *pp;
+    const int64_t Tq = P.total_tokens, Tk = kv_total;
+    if (kv_total < 0 || (P.batch == 0 && kv_total != 0)) return BA_ERR_INVALID_ARG;
+    if (max_tiles(P.batch, Tk) * P.heads > INT32_MAX) return BA_ERR_UNSUPPORTED;
+    if (!q_offsets || !aligned(q_offsets, 4) || !kv_offsets || !aligned(kv_offsets, 4) || !tensor_ok(q, Tq) ||
+        !tensor_ok(k, Tk) || !tensor_ok(v, Tk))
+        return BA_ERR_INVALID_ARG;
+    if (!bwd && !tensor_ok(out, Tq)) return BA_ERR_INVALID_ARG;
+    if (bwd && (!tensor_ok(dout, Tq) || !tensor_ok(dq, Tq) || !tensor_ok(dk, Tk) || !tensor_ok(dv, Tk)))
+        return BA_ERR_INVALID_ARG;
+    if (P.dtype != BA_BF16) return BA_ERR_UNSUPPORTED;
+    const WorkspaceLayout lay = workspace_layout(P.batch, Tq > Tk ? Tq : Tk, P.heads, P.head_dim, false);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total) return BA_ERR_INVALID_ARG;
+    int num_sms = 0, cc = 0;
+    if (!device_info(num_sms, cc)) return BA_ERR_CUDA;
+    if (cc != 10) return BA_ERR_UNSUPPORTED;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    const size_t row_bytes = size_t(P.heads) * P.head_dim * 2;
+    // the query-tile side: tables over the query sets, each paired with its key/value set
+    Problem pq = make_problem(P, q_offsets, nullptr, 1, 1, workspace, lay);
+    pq.other_offsets = kv_offsets;
+    BA_TRY(launch_worklist(pq, stream));
+    if (Tq > 0) BA_TRY(launch_zero_unpaired_rows(q_offsets, kv_offsets, P.batch, row_bytes, bwd ? dq : out, nullptr,
+                                                 stream));
+    if (Tq == 0 || Tk == 0) {
+        if (bwd && Tk > 0)
+            BA_TRY(launch_zero_unpaired_rows(kv_offsets, q_offsets, P.batch, row_bytes, dk, dv, stream));
+        return BA_OK;
+    }
+    CUtensorMap tq, tk, tv, tdo, to, tdk, tdv;
+    if (!encode_bf16_rows(&tq, q, Tq, P.heads, P.head_dim) || !encode_bf16_rows(&tk, k, Tk, P.heads, P.head_dim) ||
+        !encode_bf16_rows(&tv, v, Tk, P.heads, P.head_dim))
+        return BA_ERR_CUDA;
+    const auto run = [&](auto act_c, bool dkdv_pass, const Problem &p) -> cudaError_t {
+        constexpr int A = decltype(act_c)::value;
+        const int D = P.head_dim;
+        if (!bwd) {
+            cudaError_t e = prof_mark(0, 0, stream);
+            if (e == cudaSuccess)
+                e = D == 64 ? launch_fwd_bf16_sm100<64, A>(tq, tk, tv, to, p, out, nullptr, num_sms, stream)
+                            : launch_fwd_bf16_sm100<128, A>(tq, tk, tv, to, p, out, nullptr, num_sms, stream);
+            return e == cudaSuccess ? prof_mark(0, 1, stream) : e;
+        }
+        const int w = dkdv_pass ? 2 : 1;
+        cudaError_t e = prof_mark(w, 0, stream);
+        if (e != cudaSuccess) return e;
+        if (!dkdv_pass)
+            e = D == 64 ? launch_bwd_dq_sm100<64, A>(tq, tk, tv, tdo, tdo, p, nullptr, nullptr, nullptr, dq, num_sms,
+                                                     stream)
+                        : launch_bwd_dq_sm100<128, A>(tq, tk, tv, tdo, tdo, p, nullptr, nullptr, nullptr, dq, num_sms,
+                                                      stream);
+        else
+            e = D == 64 ? launch_bwd_dkdv_sm100<64, A>(tq, tk, tv, tdo, tdk, tdv, p, nullptr, nullptr, dk, dv,
+                                                       num_sms, stream)
+                        : launch_bwd_dkdv_sm100<128, A>(tq, tk, tv, tdo, tdk, tdv, p, nullptr, nullptr, dk, dv,
+                                                        num_sms, stream);
+        return e == cudaSuccess ? prof_mark(w, 1, stream) : e;
+    };
+    const auto run_act = [&](bool dkdv_pass, const Problem &p) -> cudaError_t {
+        return act == BA_ACT_GELU ? run(std::integral_constant<int, kGelu>{}, dkdv_pass, p)
+                                  : run(std::integral_constant<int, kSilu>{}, dkdv_pass, p);
+    };
+    if (!bwd) {
+        if (!encode_bf16_rows(&to, out, Tq, P.heads, P.head_dim)) return BA_ERR_CUDA;
+        BA_TRY(run_act(false, pq));
+        return BA_OK;
+    }
+    if (!encode_bf16_rows(&tdo, dout, Tq, P.heads, P.head_dim) || !encode_bf16_rows(&tdk, dk, Tk, P.heads, P.head_dim) ||
+        !encode_bf16_rows(&tdv, dv, Tk, P.heads, P.head_dim))
+        return BA_ERR_CUDA;
+    BA_TRY(run_act(false, pq));
+    // the key-tile side: tables over the key/value sets, each paired with its query set (the
+    // dQ pass's status word is kept)
+    ba_problem Pk = P;
+    Pk.total_tokens = int32_t(Tk);
+    Problem pk = make_problem(Pk, kv_offsets, nullptr, 1, 1, workspace, lay);
+    pk.other_offsets = q_offsets;
+    BA_TRY(launch_worklist(pk, stream, false));
+    BA_TRY(launch_zero_unpaired_rows(kv_offsets, q_offsets, P.batch, row_bytes, dk, dv, stream));
+    BA_TRY(run_act(true, pk));
+    return BA_OK;
+}
+
+// MXFP8 operands in the workspace after the forward's own regions: E4M3 q and
+// k [T, H, D], then their scale bytes [T, heads_pad, D / 32].
+struct MxLayout {
+    size_t q8, k8, qs, ks, total;
+};
+
+MxLayout mx_layout(const ba_problem &P, size_t base_total)
+{
+    const size_t e = align256(size_t(P.total_tokens) * size_t(P.heads) * size_t(P.head_dim));
+    const size_t sc = align256(size_t(P.total_tokens) * size_t((P.heads + 3) / 4 * 4) * size_t(P.head_dim / 32));
+    return MxLayout{base_total, base_total + e, base_total + 2 * e, base_total + 2 * e + sc, base_total + 2 * e + 2 * sc};
+}
+
+ba_status mx_fwd_impl(const ba_problem *pp, const void *q, const void *k, const void *v, const int32_t *seq_offsets,
+                      int32_t block, int32_t window, const uint8_t *skip, void *out, float *lse, void *workspace,
+                      size_t workspace_bytes, ba_stream_t stream_)
+{
+    ba_status st = check_problem(pp, block, window);
+    if (st != BA_OK) return st;
+    const ba_problem &P = *pp;
+    const int64_t T = P.total_tokens;
+    if (!seq_offsets || !aligned(seq_offsets, 4) || !tensor_ok(q, T) || !tensor_ok(k, T) || !tensor_ok(v, T) ||
+        !tensor_ok(out, T) || (T > 0 && (!lse || !aligned(lse, 4))))
+        return BA_ERR_INVALID_ARG;
+    if (P.dtype != BA_BF16 || P.head_dim != 128) return BA_ERR_UNSUPPORTED;
+    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, false);
+    const MxLayout ml = mx_layout(P, lay.total);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < ml.total) return BA_ERR_INVALID_ARG;
+    int num_sms = 0, cc = 0;
+    if (!device_info(num_sms, cc)) return BA_ERR_CUDA;
+    if (cc != 10) return BA_ERR_UNSUPPORTED;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    Problem p = make_problem(P, seq_offsets, skip, block, window, workspace, lay);
+    BA_TRY(launch_worklist(p, stream));
+    if (T == 0) return BA_OK;
+    BA_TRY(launch_skip_fwd(p, 2, v, out, lse, stream));
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    BA_TRY(launch_mx_quantize(q, T, P.heads, P.head_dim, ws + ml.q8, ws + ml.qs, num_sms, stream));
+    BA_TRY(launch_mx_quantize(k, T, P.heads, P.head_dim, ws + ml.k8, ws + ml.ks, num_sms, stream));
+    const int64_t row8 = int64_t(P.heads) * P.head_dim, rows = int64_t((P.heads + 3) / 4 * 4) * 4;
+    CUtensorMap tq, tk, tv, to, tqs, tks;
+    if (!encode_u8_rows(&tq, ws + ml.q8, T, row8, 128, true) || !encode_u8_rows(&tk, ws + ml.k8, T, row8, 128, true) ||
+        !encode_u8_rows(&tqs, ws + ml.qs, T, rows, 16, false) || !encode_u8_rows(&tks, ws + ml.ks, T, rows, 16, false) ||
+        !encode_bf16_rows(&tv, v, T, P.heads, P.head_dim) || !encode_bf16_rows(&to, out, T, P.heads, P.head_dim))
+        return BA_ERR_CUDA;
+    BA_TRY(prof_mark(0, 0, stream));
+    BA_TRY(launch_fwd_bf16_sm100<128, kSoftmax>(tq, tk, tv, to, p, out, lse, num_sms, stream, &tqs, &tks));
+    BA_TRY(prof_mark(0, 1, stream));
+    return BA_OK;
+}
+
 } // namespace
 
 extern "C" {
@@ -487,6 +649,56 @@ ba_status ba_gdpa_bwd(const ba_problem *p, ba_activation act, const void *q, con
 {
     return gdpa_impl(true, p, act, q, k, v, dout, seq_offsets, block, window, nullptr, dq, dk, dv, workspace,
                      workspace_bytes, stream);
+}
+
+size_t ba_gdpa_cross_workspace_size(const ba_problem *p, int32_t kv_total_tokens)
+{
+    if (check_problem(p, 1, 1) == BA_ERR_INVALID_ARG || kv_total_tokens < 0) return 0;
+    const int64_t t = p->total_tokens > kv_total_tokens ? p->total_tokens : kv_total_tokens;
+    return workspace_layout(p->batch, t, p->heads, p->head_dim, false).total;
+}
+
+ba_status ba_gdpa_cross_fwd(const ba_problem *p, int32_t kv_total_tokens, ba_activation act, const void *q,
+                            const void *k, const void *v, const int32_t *q_offsets, const int32_t *kv_offsets,
+                            void *out, void *workspace, size_t workspace_bytes, ba_stream_t stream)
+{
+    return gdpa_cross_impl(false, p, kv_total_tokens, act, q, k, v, nullptr, q_offsets, kv_offsets, out, nullptr,
+                           nullptr, nullptr, workspace, workspace_bytes, stream);
+}
+
+ba_status ba_gdpa_cross_bwd(const ba_problem *p, int32_t kv_total_tokens, ba_activation act, const void *q,
+                            const void *k, const void *v, const void *dout, const int32_t *q_offsets,
+                            const int32_t *kv_offsets, void *dq, void *dk, void *dv, void *workspace,
+                            size_t workspace_bytes, ba_stream_t stream)
+{
+    return gdpa_cross_impl(true, p, kv_total_tokens, act, q, k, v, dout, q_offsets, kv_offsets, nullptr, dq, dk, dv,
+                           workspace, workspace_bytes, stream);
+}
+
+ba_status ba_mx_quantize(const void *x, int64_t rows, int32_t heads, int32_t head_dim, void *elements,
+                         void *scales, ba_stream_t stream)
+{
+    if (rows < 0 || heads < 1 || head_dim < 32 || head_dim % 32 || rows > (int64_t(1) << 40)) return BA_ERR_INVALID_ARG;
+    if (rows > 0 && (!x || !elements || !scales || !aligned(x, 16) || !aligned(elements, 16)))
+        return BA_ERR_INVALID_ARG;
+    int num_sms = 0, cc = 0;
+    if (rows > 0 && !device_info(num_sms, cc)) return BA_ERR_CUDA;
+    BA_TRY(launch_mx_quantize(x, rows, heads, head_dim, elements, scales, num_sms,
+                              reinterpret_cast<cudaStream_t>(stream)));
+    return BA_OK;
+}
+
+size_t ba_mx_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
+{
+    const size_t base = ba_fwd_workspace_size(p, block, window);
+    return base ? mx_layout(*p, base).total : 0;
+}
+
+ba_status ba_mx_fwd(const ba_problem *p, const void *q, const void *k, const void *v, const int32_t *seq_offsets,
+                    int32_t block, int32_t window, const uint8_t *skip, void *out, float *lse, void *workspace,
+                    size_t workspace_bytes, ba_stream_t stream)
+{
+    return mx_fwd_impl(p, q, k, v, seq_offsets, block, window, skip, out, lse, workspace, workspace_bytes, stream);
 }
 
 ba_status ba_device_status(const void *workspace, ba_stream_t stream_)

@@ -16,6 +16,7 @@
 #include "ba_common.cuh"
 #include "ba_kernels.cuh"
 #include "ba_ptx.cuh"
+#include "ba_sched.cuh"
 
 #include <cuda_bf16.h>
 
@@ -23,9 +24,13 @@ namespace ba {
 
 namespace {
 
-__device__ __forceinline__ int32_t live_tiles(const int32_t *offs, const uint8_t *skip, int32_t b)
+// Live 128-row tiles of example b: none if it is skipped, or (cross-attention)
+// if its other side is empty.
+__device__ __forceinline__ int32_t live_tiles(const int32_t *offs, const uint8_t *skip, const int32_t *other,
+                                              int32_t b)
 {
     if (skip && skip[b]) return 0;
+    if (other && other[b + 1] == other[b]) return 0;
     const int32_t L = offs[b + 1] - offs[b];
     return L > 0 ? (L + kTile - 1) / kTile : 0;
 }
@@ -77,9 +82,10 @@ constexpr int kSortBuckets = kWorklistThreads;
 // Per live example: its 128-row tiles, and pairs of consecutive tiles (the
 // forward processes two query tiles of one example together).
 __global__ void __launch_bounds__(kWorklistThreads)
-    worklist_kernel(const int32_t *__restrict__ offs, const uint8_t *__restrict__ skip, int32_t batch,
-                    int32_t *__restrict__ tile_prefix, int4 *__restrict__ tile_info,
-                    int32_t *__restrict__ pair_prefix, int4 *__restrict__ pair_info, int *__restrict__ status)
+    worklist_kernel(const int32_t *__restrict__ offs, const uint8_t *__restrict__ skip,
+                    const int32_t *__restrict__ other, int32_t batch, int32_t *__restrict__ tile_prefix,
+                    int4 *__restrict__ tile_info, int32_t *__restrict__ pair_prefix, int4 *__restrict__ pair_info,
+                    int *__restrict__ status, int reset_status)
 {
     __shared__ int32_t warp_tot[kWorklistThreads / 32];
     __shared__ int32_t bucket_tiles[kSortBuckets], bucket_pairs[kSortBuckets];
@@ -89,7 +95,7 @@ __global__ void __launch_bounds__(kWorklistThreads)
     bucket_pairs[tid] = 0;
     __syncthreads();
     for (int b = tid; b < batch; b += kWorklistThreads) {
-        const int32_t nt = live_tiles(offs, skip, b);
+        const int32_t nt = live_tiles(offs, skip, other, b);
         if (nt == 0) continue;
         atomicAdd(&bucket_tiles[bucket(nt)], nt);
         atomicAdd(&bucket_pairs[bucket(nt)], (nt + 1) / 2);
@@ -102,7 +108,7 @@ __global__ void __launch_bounds__(kWorklistThreads)
     bucket_pairs[tid] = pstart;
     __syncthreads();
     for (int b = tid; b < batch; b += kWorklistThreads) {
-        const int32_t nt = live_tiles(offs, skip, b);
+        const int32_t nt = live_tiles(offs, skip, other, b);
         const int32_t s0 = offs[b], L = offs[b + 1] - s0;
         int32_t t0 = ttot, p0 = ptot; // an example without live tiles owns no slots
         if (nt > 0) {
@@ -117,7 +123,9 @@ __global__ void __launch_bounds__(kWorklistThreads)
     if (tid == kWorklistThreads - 1) {
         tile_prefix[batch] = ttot;
         pair_prefix[batch] = ptot;
-        *status = 0;
+        if (reset_status) *status = 0;
+        // the attention kernels' item counters (one per kernel of a call)
+        for (int c = kCounterFwd; c <= kCounterDkdv; ++c) status[c] = 0;
     }
 }
 
@@ -192,11 +200,40 @@ __global__ void __launch_bounds__(256)
 
 // ---------------------------------------------------------------- launchers
 
-cudaError_t launch_worklist(const Problem &p, cudaStream_t stream)
+cudaError_t launch_worklist(const Problem &p, cudaStream_t stream, bool reset_status)
 {
     worklist_kernel<<<1, kWorklistThreads, 0, stream>>>(
-        p.seq_offsets, p.skip, p.batch, const_cast<int32_t *>(p.tile_prefix), const_cast<int4 *>(p.tile_info),
-        const_cast<int32_t *>(p.pair_prefix), const_cast<int4 *>(p.pair_info), p.status);
+        p.seq_offsets, p.skip, p.other_offsets, p.batch, const_cast<int32_t *>(p.tile_prefix),
+        const_cast<int4 *>(p.tile_info), const_cast<int32_t *>(p.pair_prefix), const_cast<int4 *>(p.pair_info),
+        p.status, reset_status ? 1 : 0);
+    return cudaGetLastError();
+}
+
+// Cross-attention: rows of examples whose other side is empty get zeros (an
+// empty sum) in a and, when given, b. grid.x = example.
+__global__ void __launch_bounds__(256)
+    zero_unpaired_rows_kernel(const int32_t *__restrict__ offs, const int32_t *__restrict__ other, int64_t row_bytes,
+                              uint8_t *__restrict__ a, uint8_t *__restrict__ b)
+{
+    const int e = blockIdx.x;
+    if (other[e + 1] != other[e]) return;
+    const int64_t s0 = offs[e], L = offs[e + 1] - s0;
+    const int64_t nvec = L * row_bytes / 16;
+    uint4 *av = reinterpret_cast<uint4 *>(a + s0 * row_bytes);
+    uint4 *bv = b ? reinterpret_cast<uint4 *>(b + s0 * row_bytes) : nullptr;
+    const int64_t stride = int64_t(gridDim.y) * blockDim.x;
+    for (int64_t x = int64_t(blockIdx.y) * blockDim.x + threadIdx.x; x < nvec; x += stride) {
+        av[x] = make_uint4(0, 0, 0, 0);
+        if (bv) bv[x] = make_uint4(0, 0, 0, 0);
+    }
+}
+
+cudaError_t launch_zero_unpaired_rows(const int32_t *offs, const int32_t *other, int32_t batch, size_t row_bytes,
+                                      void *a, void *b, cudaStream_t stream)
+{
+    if (batch == 0) return cudaSuccess;
+    zero_unpaired_rows_kernel<<<dim3(batch, 8), 256, 0, stream>>>(offs, other, int64_t(row_bytes),
+                                                                 static_cast<uint8_t *>(a), static_cast<uint8_t *>(b));
     return cudaGetLastError();
 }
 

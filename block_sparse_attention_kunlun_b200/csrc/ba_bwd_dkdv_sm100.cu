@@ -42,6 +42,7 @@
 #include "ba_common.cuh"
 #include "ba_kernels.cuh"
 #include "ba_ptx.cuh"
+#include "ba_sched.cuh"
 
 #include <cuda_bf16.h>
 
@@ -78,6 +79,7 @@ struct DkvBarriers {
     uint64_t s_full, dp_full, pa_done[2], pb_done[2];
     uint64_t epi_sync; // group barrier of the epilogue warps
     uint64_t tail;     // the TMA warp's own barrier for a Q or dO tile whose last rows it clears
+    ItemRing ring;     // items claimed by the TMA warp, read by the MMA, compute and epilogue warps
     uint32_t tmem_base;
     int abort;
     // per Q slot: -lse in log2 units and -Delta of the tile's 128 queries
@@ -85,8 +87,14 @@ struct DkvBarriers {
     __align__(16) float stat[4][2][kTile];
 };
 
+template <bool kCross>
 __device__ __forceinline__ void query_tile_range(const TileRef &r, int64_t B, int64_t W, int &ilo, int &ihi)
 {
+    if (kCross) { // cross-attention: every query tile of the example's own query set
+        ilo = 0;
+        ihi = (r.oL + kTile - 1) / kTile - 1;
+        return;
+    }
     const int64_t kmax = (int64_t(r.t) * kTile + kTile < r.L ? int64_t(r.t) * kTile + kTile : r.L) - 1;
     ilo = r.t;
     ihi = int(last_query_seeing(kmax, r.L, B, W) / kTile);
@@ -94,7 +102,7 @@ __device__ __forceinline__ void query_tile_range(const TileRef &r, int64_t B, in
 
 } // namespace
 
-template <int D, bool kRope, int A>
+template <int D, bool kRope, int A, bool kCross>
 __global__ void __launch_bounds__(448, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -129,6 +137,7 @@ __global__ void __launch_bounds__(448, 1)
         mbar_init(&sb.dp_full, 1);
         mbar_init(&sb.epi_sync, 128);
         mbar_init(&sb.tail, 1);
+        item_ring_init(sb.ring, 1 + 8 + 4); // MMA warp, compute warps, epilogue warps
         for (int g = 0; g < 2; ++g) {
             mbar_init(&sb.pa_done[g], 4);
             mbar_init(&sb.pb_done[g], 4);
@@ -160,10 +169,10 @@ __global__ void __launch_bounds__(448, 1)
         uint32_t it = 0, item_cnt = 0, tail_phase = 0;
         TileRef r;
         bool ok = true;
-        ItemWalker items(p.tile_info, ntiles, p.heads);
-        for (; ok && items.advance(r); ++item_cnt) {
+        ItemSource items(p.tile_info, ntiles, p.heads, p.status + kCounterDkdv, p.other_offsets);
+        for (; ok && items.advance(r, sb.ring, abort, ok); ++item_cnt) {
             int ilo, ihi;
-            query_tile_range(r, B, W, ilo, ihi);
+            query_tile_range<kCross>(r, B, W, ilo, ihi);
             for (int i = ilo; i <= ihi; ++i, ++it) {
                 const int qs = it % QS, os = it % OS;
                 if (!mbar_wait(&sb.q_empty[qs], ((it / QS) & 1) ^ 1, abort)) {
@@ -172,9 +181,9 @@ __global__ void __launch_bounds__(448, 1)
                 }
                 // the example's last query tile: its rows past the example are cleared (Q here,
                 // dO below), since dK += dS^T Q and dV += P^T dO multiply them by zeros
-                const int valid = r.L - i * kTile;
+                const int valid = r.oL - i * kTile; // query rows: the example's own, or its query set
                 if (!load_tile_zero_tail<Lay::kChunks>(smem + Lay::kQ0 + qs * Lay::kTileBytes, &tm_q, &sb.q_full[qs],
-                                                       &sb.tail, tail_phase, r.h * D, r.s0 + i * kTile, valid,
+                                                       &sb.tail, tail_phase, r.h * D, r.os0 + i * kTile, valid,
                                                        abort)) {
                     ok = false;
                     break;
@@ -227,7 +236,7 @@ __global__ void __launch_bounds__(448, 1)
                     break;
                 }
                 if (!load_tile_zero_tail<Lay::kChunks>(smem + Lay::kO0 + os * Lay::kTileBytes, &tm_do, &sb.o_full[os],
-                                                       &sb.tail, tail_phase, r.h * D, r.s0 + i * kTile, valid,
+                                                       &sb.tail, tail_phase, r.h * D, r.os0 + i * kTile, valid,
                                                        abort)) {
                     ok = false;
                     break;
@@ -236,19 +245,19 @@ __global__ void __launch_bounds__(448, 1)
                     // warm L2 two query tiles ahead, and with the next item's K, V and first tiles
                     if (i + 2 <= ihi)
                         for (int c = 0; c < Lay::kChunks; ++c) {
-                            tma_prefetch_l2_2d(&tm_q, r.h * D + c * 64, r.s0 + (i + 2) * kTile);
-                            tma_prefetch_l2_2d(&tm_do, r.h * D + c * 64, r.s0 + (i + 2) * kTile);
+                            tma_prefetch_l2_2d(&tm_q, r.h * D + c * 64, r.os0 + (i + 2) * kTile);
+                            tma_prefetch_l2_2d(&tm_do, r.h * D + c * 64, r.os0 + (i + 2) * kTile);
                         }
                     TileRef rn;
                     if (i == ilo && items.peek(rn)) {
                         int nlo, nhi;
-                        query_tile_range(rn, B, W, nlo, nhi);
+                        query_tile_range<kCross>(rn, B, W, nlo, nhi);
                         for (int c = 0; c < Lay::kChunks; ++c) {
                             tma_prefetch_l2_2d(&tm_k, rn.h * D + c * 64, rn.s0 + rn.t * kTile);
                             tma_prefetch_l2_2d(&tm_v, rn.h * D + c * 64, rn.s0 + rn.t * kTile);
                             for (int i2 = nlo; i2 <= nhi && i2 < nlo + 2; ++i2) {
-                                tma_prefetch_l2_2d(&tm_q, rn.h * D + c * 64, rn.s0 + i2 * kTile);
-                                tma_prefetch_l2_2d(&tm_do, rn.h * D + c * 64, rn.s0 + i2 * kTile);
+                                tma_prefetch_l2_2d(&tm_q, rn.h * D + c * 64, rn.os0 + i2 * kTile);
+                                tma_prefetch_l2_2d(&tm_do, rn.h * D + c * 64, rn.os0 + i2 * kTile);
                             }
                         }
                     }
@@ -264,10 +273,10 @@ __global__ void __launch_bounds__(448, 1)
         TileRef r;
         bool ok = true;
         const uint32_t k_addr = smem_base + Lay::kK, v_addr = smem_base + Lay::kV;
-        ItemWalker items(p.tile_info, ntiles, p.heads);
-        for (; ok && items.advance(r); ++item_cnt) {
+        ItemSink items;
+        for (; ok && items.advance(r, sb.ring, abort, ok); ++item_cnt) {
             int ilo, ihi;
-            query_tile_range(r, B, W, ilo, ihi);
+            query_tile_range<kCross>(r, B, W, ilo, ihi);
             const int nq = ihi - ilo + 1;
             // S^T = K Q^T of query tile m of this item; after the item's last one K is not read again
             auto issue_s = [&](int m) -> bool {
@@ -359,17 +368,19 @@ __global__ void __launch_bounds__(448, 1)
         uint32_t it = 0;
         TileRef r;
         bool ok = true;
-        ItemWalker items(p.tile_info, ntiles, p.heads);
-        while (ok && items.advance(r)) {
+        ItemSink items;
+        while (ok && items.advance(r, sb.ring, abort, ok)) {
             int ilo, ihi;
-            query_tile_range(r, B, W, ilo, ihi);
+            query_tile_range<kCross>(r, B, W, ilo, ihi);
             const int64_t k = int64_t(r.t) * kTile + row; // local key index
             const bool valid_k = k < r.L;
-            const int64_t qmax = valid_k ? last_query_seeing(k, r.L, B, W) : -1;
+            // visible queries [qmin, qmax]: the block rule, or (cross-attention) the whole query set
+            const int64_t qmax = valid_k ? (kCross ? int64_t(r.oL) - 1 : last_query_seeing(k, r.L, B, W)) : -1;
+            const int64_t qmin = kCross ? 0 : k;
             for (int i = ilo; i <= ihi && ok; ++i, ++it) {
                 const int qs = it % QS;
                 const int64_t q0 = int64_t(i) * kTile + 64 * g;
-                int64_t lo64 = k - q0, hi64 = qmax - q0;
+                int64_t lo64 = qmin - q0, hi64 = qmax - q0;
                 if (!valid_k) { lo64 = 1; hi64 = 0; }
                 const int lo_c = int(lo64 < -1 ? -1 : (lo64 > 64 ? 64 : lo64));
                 const int hi_c = int(hi64 < -1 ? -1 : (hi64 > 64 ? 64 : hi64));
@@ -481,8 +492,8 @@ __global__ void __launch_bounds__(448, 1)
         uint32_t item_cnt = 0, sync_phase = 0;
         bool ok = true;
         TileRef r;
-        ItemWalker items(p.tile_info, ntiles, p.heads);
-        for (; ok && items.advance(r); ++item_cnt) {
+        ItemSink items;
+        for (; ok && items.advance(r, sb.ring, abort, ok); ++item_cnt) {
             const int64_t k = int64_t(r.t) * kTile + row;
             const bool valid_k = k < r.L;
             const bool full_tile = int64_t(r.t) * kTile + kTile <= r.L;
@@ -571,9 +582,10 @@ cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
                                   int num_sms, cudaStream_t stream)
 {
     using Lay = DkvLayout<D>;
-    // the rotary epilogue exists for block attention only
-    auto kern = (A == kSoftmax && p.rope_cos) ? bwd_dkdv_sm100_kernel<D, A == kSoftmax, A>
-                                              : bwd_dkdv_sm100_kernel<D, false, A>;
+    // the rotary epilogue exists for block attention only, cross-attention for the generalized one
+    auto kern = (A == kSoftmax && p.rope_cos)        ? bwd_dkdv_sm100_kernel<D, A == kSoftmax, A, false>
+                : (A != kSoftmax && p.other_offsets) ? bwd_dkdv_sm100_kernel<D, false, A, A != kSoftmax>
+                                                     : bwd_dkdv_sm100_kernel<D, false, A, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
     kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, neg_delta,

@@ -34,6 +34,7 @@
 #include "ba_common.cuh"
 #include "ba_kernels.cuh"
 #include "ba_ptx.cuh"
+#include "ba_sched.cuh"
 
 #include <cuda_bf16.h>
 
@@ -64,6 +65,7 @@ struct DqBarriers {
     uint64_t st_full, st_empty, qt_ready;
     uint64_t s_full, s_free, dp_full, ds_full[2], dq_done, dq_free;
     uint64_t tail; // the TMA warp's own barrier for a K or V tile whose last rows it clears
+    ItemRing ring; // items claimed by the TMA warp, read by the MMA and compute warps
     uint32_t tmem_base;
     int abort;
 };
@@ -76,7 +78,7 @@ __device__ __forceinline__ int first_key_tile(const TileRef &r, int64_t B, int64
 
 } // namespace
 
-template <int D, bool kRope, int A>
+template <int D, bool kRope, int A, bool kCross>
 __global__ void __launch_bounds__(384, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -110,6 +112,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(&sb.dq_done, 1);
         mbar_init(&sb.dq_free, 8);
         mbar_init(&sb.tail, 1);
+        item_ring_init(sb.ring, 1 + 8); // MMA warp, compute warps
         sb.abort = 0;
         fence_mbar_init();
     }
@@ -141,9 +144,11 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t kv_cnt = 0, item_cnt = 0, tail_phase = 0;
             TileRef r;
             bool ok = true;
-            ItemWalker items(p.tile_info, ntiles, p.heads);
-            for (; ok && items.advance(r); ++item_cnt) {
-                const int jlo = first_key_tile(r, B, W);
+            ItemSource items(p.tile_info, ntiles, p.heads, p.status + kCounterDq, p.other_offsets);
+            for (; ok && items.advance(r, sb.ring, abort, ok); ++item_cnt) {
+                // key tiles [jlo, jend]: the block rule, or (cross-attention) the example's whole key/value set
+                const int jlo = kCross ? 0 : first_key_tile(r, B, W);
+                const int jend = kCross ? (r.oL + kTile - 1) / kTile - 1 : r.t;
                 if (!mbar_wait(&sb.st_empty, (item_cnt & 1) ^ 1, abort)) break;
                 if (lane == 0) {
                     // Q, dO and (for Delta; the softmax only) out
@@ -158,22 +163,22 @@ __global__ void __launch_bounds__(384, 1)
                     }
                 }
                 __syncwarp();
-                for (int j = jlo; j <= r.t; ++j, ++kv_cnt) {
+                for (int j = jlo; j <= jend; ++j, ++kv_cnt) {
                     const int st = kv_cnt % S;
                     uint8_t *kdst = smem + Lay::kKV0 + 2 * st * Lay::kTileBytes;
                     // K is read until dQ, V only by dP: they are released and refilled separately
                     // the example's last K and V tiles: rows past the example are cleared, since
                     // dQ += dS K and the masked dS = P (dP - Delta) multiply them by zeros
-                    const int valid = r.L - j * kTile;
+                    const int valid = r.oL - j * kTile;
                     if (!mbar_wait(&sb.k_empty[st], ((kv_cnt / S) & 1) ^ 1, abort) ||
                         !load_tile_zero_tail<Lay::kChunks>(kdst, &tm_k, &sb.k_full[st], &sb.tail, tail_phase,
-                                                           r.h * D, r.s0 + j * kTile, valid, abort)) {
+                                                           r.h * D, r.os0 + j * kTile, valid, abort)) {
                         ok = false;
                         break;
                     }
                     if (!mbar_wait(&sb.v_empty[st], ((kv_cnt / S) & 1) ^ 1, abort) ||
                         !load_tile_zero_tail<Lay::kChunks>(kdst + Lay::kTileBytes, &tm_v, &sb.v_full[st], &sb.tail,
-                                                           tail_phase, r.h * D, r.s0 + j * kTile, valid, abort)) {
+                                                           tail_phase, r.h * D, r.os0 + j * kTile, valid, abort)) {
                         ok = false;
                         break;
                     }
@@ -213,10 +218,10 @@ __global__ void __launch_bounds__(384, 1)
                 ++d_cnt;
                 return true;
             };
-            ItemWalker items(p.tile_info, ntiles, p.heads);
-            for (; ok && items.advance(r); ++item_cnt) {
-                const int jlo = first_key_tile(r, B, W);
-                const int nkv = r.t - jlo + 1;
+            ItemSink items;
+            for (; ok && items.advance(r, sb.ring, abort, ok); ++item_cnt) {
+                const int jlo = kCross ? 0 : first_key_tile(r, B, W);
+                const int nkv = kCross ? (r.oL + kTile - 1) / kTile : r.t - jlo + 1;
                 if (!mbar_wait(&sb.qt_ready, item_cnt & 1, abort)) break;
                 tc_fence_after();
                 for (int m = 0; m < nkv; ++m, ++kv_cnt, ++s_cnt) {
@@ -337,8 +342,8 @@ __global__ void __launch_bounds__(384, 1)
         };
 
         TileRef r;
-        ItemWalker items(p.tile_info, ntiles, p.heads);
-        bool have = items.advance(r);
+        ItemSink items;
+        bool have = items.advance(r, sb.ring, abort, ok);
         float delta_row = 0.f;
         // lse of this thread's query row (log2 units), loaded an item ahead
         auto load_l2 = [&](const TileRef &rr) -> float {
@@ -349,16 +354,18 @@ __global__ void __launch_bounds__(384, 1)
         float lse_row = have ? load_l2(r) : 0.f;
         if (have) ok = fill(r, 0, delta_row, lse_row);
         while (have && ok) {
-            const int jlo = first_key_tile(r, B, W);
-            const int nkv = r.t - jlo + 1;
+            const int jlo = kCross ? 0 : first_key_tile(r, B, W);
+            const int nkv = kCross ? (r.oL + kTile - 1) / kTile : r.t - jlo + 1;
             const int64_t i = int64_t(r.t) * kTile + row;
             const bool valid = i < r.L;
-            const int64_t ws = window_start(i, B, W);
+            // visible keys [ws, last]: the block rule, or (cross-attention) the whole key/value set
+            const int64_t ws = kCross ? 0 : window_start(i, B, W);
+            const int64_t last = kCross ? int64_t(r.oL) - 1 : i;
             const float l2 = lse_row * 1.4426950408889634f;
             const float dl = delta_row;
             for (int m = 0; m < nkv; ++m, ++s_cnt) {
                 const int64_t key0 = int64_t(jlo + m) * kTile + 64 * g;
-                int64_t lo64 = ws - key0, hi64 = i - key0;
+                int64_t lo64 = ws - key0, hi64 = last - key0;
                 if (!valid) { lo64 = 1; hi64 = 0; }
                 const int lo_c = int(lo64 < -1 ? -1 : (lo64 > 64 ? 64 : lo64));
                 const int hi_c = int(hi64 < -1 ? -1 : (hi64 > 64 ? 64 : hi64));
@@ -440,7 +447,8 @@ __global__ void __launch_bounds__(384, 1)
             if (!ok) break;
             // the next item's Q / dO go into TMEM now: this item's last S and dP have completed
             TileRef rn;
-            const bool have_next = items.advance(rn);
+            const bool have_next = items.advance(rn, sb.ring, abort, ok);
+            if (!ok) break;
             float delta_next = 0.f;
             const float lse_next = have_next ? load_l2(rn) : 0.f;
             if (have_next && !fill(rn, item_cnt + 1, delta_next, lse_next)) break;
@@ -494,8 +502,10 @@ cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, co
                                 float *neg_delta, float *nlse2, void *dq, int num_sms, cudaStream_t stream)
 {
     using Lay = DqLayout<D>;
-    // the rotary epilogue exists for block attention only
-    auto kern = (A == kSoftmax && p.rope_cos) ? bwd_dq_sm100_kernel<D, A == kSoftmax, A> : bwd_dq_sm100_kernel<D, false, A>;
+    // the rotary epilogue exists for block attention only, cross-attention for the generalized one
+    auto kern = (A == kSoftmax && p.rope_cos)        ? bwd_dq_sm100_kernel<D, A == kSoftmax, A, false>
+                : (A != kSoftmax && p.other_offsets) ? bwd_dq_sm100_kernel<D, false, A, A != kSoftmax>
+                                                     : bwd_dq_sm100_kernel<D, false, A, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
     // the register split only works if the CTA is launched with at least the budgets' sum

@@ -114,6 +114,10 @@ struct Problem {
     const float *rope_cos = nullptr;
     const float *rope_sin = nullptr;
     int32_t rope_rows = 0;
+    // cross-attention (generalized attention only): the other side's offsets
+    // [batch + 1] (key/value rows for the query-tile kernels, query rows for
+    // the key-tile kernel); nullptr for self-attention
+    const int32_t *other_offsets = nullptr;
 };
 
 // Rotary position embedding (RoFormer's rotation, adjacent pairs; "GEM
@@ -217,6 +221,8 @@ __device__ __forceinline__ float act_grad(float x)
 struct TileRef {
     int32_t h, t;      // head, tile index within the example
     int32_t s0, L;     // first global row of the example, its length
+    int32_t os0, oL;   // the other side's rows (cross-attention: the example's key/value set
+                       // for a query tile, its queries for a key tile); self-attention: s0, L
 };
 
 // Number of live tiles (read once per kernel role).
@@ -253,40 +259,6 @@ __device__ __forceinline__ bool decode_pair(const Problem &p, int32_t npairs, in
     second = int64_t(r.t + 1) * kTile < r.L;
     return true;
 }
-
-// Walks one CTA's work items n = blockIdx.x, blockIdx.x + gridDim.x, ...
-// (item n is entry n / heads of a tile or pair table, head n % heads; the
-// host checks that entries * heads fits in 31 bits). Each item's table entry
-// is loaded one item ahead, so its global-memory latency overlaps the
-// previous item's work, and the index arithmetic is 32-bit.
-struct ItemWalker {
-    const int4 *table;
-    uint32_t total, heads, n;
-    int4 next;
-    __device__ __forceinline__ ItemWalker(const int4 *t, int32_t entries, int32_t h)
-        : table(t), total(uint32_t(entries) * uint32_t(h)), heads(uint32_t(h)), n(blockIdx.x), next()
-    {
-        if (n < total) next = table[n / heads];
-    }
-    // The next item into r; false once the CTA's items are done.
-    __device__ __forceinline__ bool advance(TileRef &r)
-    {
-        if (!peek(r)) return false;
-        n += gridDim.x;
-        if (n < total) next = table[n / heads];
-        return true;
-    }
-    // The item advance() would return next, without moving on.
-    __device__ __forceinline__ bool peek(TileRef &r) const
-    {
-        if (n >= total) return false;
-        r.h = int32_t(n % heads);
-        r.s0 = next.x;
-        r.L = next.y;
-        r.t = next.z;
-        return true;
-    }
-};
 
 // Whether a pair item (first tile r.t) has its second tile.
 __device__ __forceinline__ bool pair_has_second(const TileRef &r) { return int64_t(r.t + 1) * kTile < r.L; }

@@ -30,6 +30,7 @@
 #include "ba_common.cuh"
 #include "ba_kernels.cuh"
 #include "ba_ptx.cuh"
+#include "ba_sched.cuh"
 
 #include <cuda_bf16.h>
 #include <type_traits>
@@ -57,6 +58,15 @@ struct FwdLayout {
     static constexpr uint32_t kRegsCompute = D == 64 ? 168 : 184, kRegsEpi = 64, kRegsOther = D == 64 ? 112 : 80;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColO = 256;
+    // MXFP8 mode (one softmax group, single query tiles): Q and K are E4M3 (one
+    // 16 KB chunk per 128 x 128 tile, in the bf16 slots); the Q tile's scale words
+    // (a 128-row x 16-byte box: four heads' words per row) sit in group 1's Q slot,
+    // the K stages' boxes after it; the scale factors go to TMEM columns that
+    // group 1's S would use: A (the Q tile's) at 128..131, B (the K tile's) at 132..135.
+    static constexpr int kQScale = kQ + kTileBytes;
+    static constexpr int kScaleBox = kTile * 16;
+    static constexpr int kFp8TileBytes = kTile * 128;
+    static constexpr uint32_t kColSFA = 128, kColSFB = 132;
 };
 
 struct FwdBarriers {
@@ -66,6 +76,8 @@ struct FwdBarriers {
     uint64_t o_ready[2]; // group w's softmax is done with its item: inv_l[w] holds 1 / l
     uint64_t epi_sync;   // group barrier of the epilogue warpgroup
     uint64_t tail;       // the TMA warp's own barrier for a V tile whose last rows it clears
+    uint64_t sf_ready;   // MXFP8: the item's scale factors (Q tile and first K tile) are in TMEM
+    ItemRing ring;       // items claimed by the TMA warp, read by the MMA, softmax and epilogue warps
     float inv_l[2][kTile];
     uint32_t tmem_base;
     int abort;
@@ -79,10 +91,11 @@ __device__ __forceinline__ int first_key_tile(int t, int64_t B, int64_t W)
 
 } // namespace
 
-template <int D, int A>
+template <int D, int A, bool kCross, bool kMx>
 __global__ void __launch_bounds__(512, 1)
     fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                          const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_ks,
                           const Problem p,
                           __nv_bfloat16 *__restrict__ out, float *__restrict__ lse)
 {
@@ -115,6 +128,8 @@ __global__ void __launch_bounds__(512, 1)
         }
         mbar_init(&sb.epi_sync, 128);
         mbar_init(&sb.tail, 1);
+        item_ring_init(sb.ring, 1 + 8 + 4); // MMA warp, softmax warps, epilogue warps
+        mbar_init(&sb.sf_ready, 4);
         sb.abort = 0;
         fence_mbar_init();
     }
@@ -133,7 +148,10 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t tmem = sb.tmem_base;
     volatile int *abort = &sb.abort;
     const int64_t B = p.block, W = p.window;
-    const int32_t npairs = live_pair_count(p);
+    // MXFP8 mode walks single query tiles (one softmax group), the others pairs of them
+    const int32_t nitems = kMx ? live_tile_count(p) : live_pair_count(p);
+    const int4 *item_table = kMx ? p.tile_info : p.pair_info;
+    static_assert(!kMx || (D == 128 && A == kSoftmax && !kCross), "MXFP8 mode: head_dim 128, softmax, self-attention");
 
     if (warp >= 8 && warp < 12) {
         // warps 8-11 (one warpgroup: TMA, MMA, two idle) hand registers to the softmax warpgroups
@@ -145,11 +163,12 @@ __global__ void __launch_bounds__(512, 1)
             TileRef r;
             bool second;
             bool ok = true;
-            ItemWalker items(p.pair_info, npairs, p.heads);
-            for (; ok && items.advance(r); ++item_cnt) {
-                second = pair_has_second(r);
-                const int jlo = first_key_tile(r.t, B, W);
-                const int jhi = r.t + (second ? 1 : 0);
+            ItemSource items(item_table, nitems, p.heads, p.status + kCounterFwd, p.other_offsets);
+            for (; ok && items.advance(r, sb.ring, abort, ok); ++item_cnt) {
+                second = !kMx && pair_has_second(r);
+                // cross-attention: every key tile of the example's own key/value set
+                const int jlo = kCross ? 0 : first_key_tile(r.t, B, W);
+                const int jhi = kCross ? (r.oL + kTile - 1) / kTile - 1 : r.t + (second ? 1 : 0);
                 // each group's query tile as soon as that group's previous one is done with
                 for (int w = 0; w < (second ? 2 : 1) && ok; ++w) {
                     if (!mbar_wait(&sb.q_empty[w], (qcnt[w] & 1) ^ 1, abort)) {
@@ -157,10 +176,16 @@ __global__ void __launch_bounds__(512, 1)
                         break;
                     }
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(&sb.q_full[w], Lay::kTileBytes);
-                        for (int c = 0; c < Lay::kChunks; ++c)
-                            tma_load_2d(smem + Lay::kQ + w * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_q,
-                                        &sb.q_full[w], r.h * D + c * 64, r.s0 + (r.t + w) * kTile);
+                        if constexpr (kMx) { // E4M3 tile (128 bytes a row) and its rows' scale words
+                            mbar_arrive_expect_tx(&sb.q_full[w], Lay::kFp8TileBytes + Lay::kScaleBox);
+                            tma_load_2d(smem + Lay::kQ, &tm_q, &sb.q_full[w], r.h * D, r.s0 + r.t * kTile);
+                            tma_load_2d(smem + Lay::kQScale, &tm_qs, &sb.q_full[w], (r.h / 4) * 16, r.s0 + r.t * kTile);
+                        } else {
+                            mbar_arrive_expect_tx(&sb.q_full[w], Lay::kTileBytes);
+                            for (int c = 0; c < Lay::kChunks; ++c)
+                                tma_load_2d(smem + Lay::kQ + w * Lay::kTileBytes + c * Lay::kChunkBytes, &tm_q,
+                                            &sb.q_full[w], r.h * D + c * 64, r.s0 + (r.t + w) * kTile);
+                        }
                     }
                     __syncwarp();
                     ++qcnt[w];
@@ -170,7 +195,7 @@ __global__ void __launch_bounds__(512, 1)
                     // warm L2 with the next item's query tiles
                     TileRef rn;
                     if (items.peek(rn)) {
-                        const bool sn = pair_has_second(rn);
+                        const bool sn = !kMx && pair_has_second(rn);
                         for (int w = 0; w < (sn ? 2 : 1); ++w)
                             for (int c = 0; c < Lay::kChunks; ++c)
                                 tma_prefetch_l2_2d(&tm_q, rn.h * D + c * 64, rn.s0 + (rn.t + w) * kTile);
@@ -187,10 +212,17 @@ __global__ void __launch_bounds__(512, 1)
                         break;
                     }
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(&sb.k_full[st], Lay::kTileBytes);
-                        for (int c = 0; c < Lay::kChunks; ++c)
-                            tma_load_2d(kdst + c * Lay::kChunkBytes, &tm_k, &sb.k_full[st], r.h * D + c * 64,
-                                        r.s0 + j * kTile);
+                        if constexpr (kMx) {
+                            mbar_arrive_expect_tx(&sb.k_full[st], Lay::kFp8TileBytes + Lay::kScaleBox);
+                            tma_load_2d(kdst, &tm_k, &sb.k_full[st], r.h * D, r.os0 + j * kTile);
+                            tma_load_2d(smem + Lay::kQScale + (1 + st) * Lay::kScaleBox, &tm_ks, &sb.k_full[st],
+                                        (r.h / 4) * 16, r.os0 + j * kTile);
+                        } else {
+                            mbar_arrive_expect_tx(&sb.k_full[st], Lay::kTileBytes);
+                            for (int c = 0; c < Lay::kChunks; ++c)
+                                tma_load_2d(kdst + c * Lay::kChunkBytes, &tm_k, &sb.k_full[st], r.h * D + c * 64,
+                                            r.os0 + j * kTile);
+                        }
                     }
                     __syncwarp();
                     if (!mbar_wait(&sb.v_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
@@ -201,8 +233,8 @@ __global__ void __launch_bounds__(512, 1)
                     // P V multiplies them by zero probabilities (K needs nothing: masked scores
                     // are replaced, not multiplied)
                     if (!load_tile_zero_tail<Lay::kChunks>(kdst + Lay::kTileBytes, &tm_v, &sb.v_full[st], &sb.tail,
-                                                           tail_phase, r.h * D, r.s0 + j * kTile,
-                                                           r.L - j * kTile, abort)) {
+                                                           tail_phase, r.h * D, r.os0 + j * kTile,
+                                                           r.oL - j * kTile, abort)) {
                         ok = false;
                         break;
                     }
@@ -219,11 +251,13 @@ __global__ void __launch_bounds__(512, 1)
             TileRef r;
             bool second;
             bool ok = true;
-            ItemWalker items(p.pair_info, npairs, p.heads);
-            for (; ok && items.advance(r); ++item_cnt) {
-                second = pair_has_second(r);
-                const int lo[2] = {first_key_tile(r.t, B, W), second ? first_key_tile(r.t + 1, B, W) : 1};
-                const int hi[2] = {r.t, second ? r.t + 1 : 0};
+            ItemSink items;
+            for (; ok && items.advance(r, sb.ring, abort, ok); ++item_cnt) {
+                second = !kMx && pair_has_second(r);
+                const int nkt = (r.oL + kTile - 1) / kTile; // cross-attention: key tiles of the example
+                const int lo[2] = {kCross ? 0 : first_key_tile(r.t, B, W),
+                                   second ? (kCross ? 0 : first_key_tile(r.t + 1, B, W)) : 1};
+                const int hi[2] = {kCross ? nkt - 1 : r.t, second ? (kCross ? nkt - 1 : r.t + 1) : 0};
                 const int jlo = lo[0], jhi = second ? hi[1] : hi[0];
                 // O_w += P_w V for key tile j of group w (V from ring stage st)
                 auto issue_pv = [&](int w, int j, int st) -> bool {
@@ -247,16 +281,29 @@ __global__ void __launch_bounds__(512, 1)
                 auto issue_s = [&](int w, int j, int st) -> bool {
                     if (j == lo[w]) { // this group's query tile of the item
                         if (!mbar_wait(&sb.q_full[w], qf[w] & 1, abort)) return false;
+                        // MXFP8: the softmax warps have put the item's scale factors in TMEM
+                        if (kMx && !mbar_wait(&sb.sf_ready, qf[w] & 1, abort)) return false;
                         tc_fence_after();
                     }
                     {
                         const uint32_t q_addr = smem_base + Lay::kQ + w * Lay::kTileBytes;
                         const uint32_t k_addr = smem_base + Lay::kK0 + 2 * st * Lay::kTileBytes;
+                        if constexpr (kMx) {
+                            // four K = 32 products along head_dim, k-block kk scaled by byte kk of
+                            // each row's scale word
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t off = (kk / 4) * Lay::kChunkBytes + (kk % 4) * 32;
-                            mma_ss(tmem + 128 * w, sdesc_sw128(q_addr + off, 16, 1024),
-                                   sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                            for (uint32_t kk = 0; kk < 4; ++kk)
+                                mma_mx_ss(tmem, sdesc_sw128(q_addr + kk * 32, 16, 1024),
+                                          sdesc_sw128(k_addr + kk * 32, 16, 1024), idesc_mx_e4m3(128, 128, kk, kk),
+                                          (tmem + Lay::kColSFA) | (kk << 30), (tmem + Lay::kColSFB) | (kk << 30),
+                                          kk > 0 ? 1u : 0u);
+                        } else {
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint32_t off = (kk / 4) * Lay::kChunkBytes + (kk % 4) * 32;
+                                mma_ss(tmem + 128 * w, sdesc_sw128(q_addr + off, 16, 1024),
+                                       sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                            }
                         }
                         tc_commit(&sb.s_full[w]);
                         if (j == hi[w]) tc_commit(&sb.q_empty[w]); // its last S: the tile may be replaced
@@ -312,22 +359,52 @@ __global__ void __launch_bounds__(512, 1)
         const uint32_t o_addr = tmem + lane_base + Lay::kColO + D * w;
         const float scale_log2 = p.scale * 1.4426950408889634f;
         uint32_t cnt = 0; // tiles this group has processed
+        uint32_t mx_items = 0;
         TileRef r;
         bool second;
         bool ok = true;
-        ItemWalker items(p.pair_info, npairs, p.heads);
-        while (ok && items.advance(r)) {
-            second = pair_has_second(r);
+        // MXFP8: move the scale words of 128 rows (a TMA box of 16 bytes a row, this head's word
+        // at 4 (h % 4)) into TMEM columns col .. col + 3 in the block-scaled MMA's layout: lane
+        // l of every lane quarter holds, in column m, the word of row l + 32 m (byte k: k-block k)
+        auto put_scales = [&](const uint8_t *box, uint32_t col, int head) {
+            uint32_t wd[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                wd[m] = *reinterpret_cast<const uint32_t *>(box + (lane + 32 * m) * 16 + (head % 4) * 4);
+            tmem_st4(tmem + lane_base + col, wd);
+        };
+        ItemSink items;
+        while (ok && items.advance(r, sb.ring, abort, ok)) {
+            second = !kMx && pair_has_second(r);
             if (w == 1 && !second) continue;
+            if constexpr (kMx) {
+                // the Q tile's and the first K tile's scale factors, before the item's first S
+                const uint32_t st0 = cnt % S;
+                if (!mbar_wait(&sb.q_full[0], mx_items & 1, abort) ||
+                    !mbar_wait(&sb.k_full[st0], (cnt / S) & 1, abort)) {
+                    ok = false;
+                    break;
+                }
+                put_scales(smem + Lay::kQScale, Lay::kColSFA, r.h);
+                put_scales(smem + Lay::kQScale + (1 + st0) * Lay::kScaleBox, Lay::kColSFB, r.h);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sb.sf_ready);
+                ++mx_items;
+            }
             const int t = r.t + w;
-            const int jlo = first_key_tile(t, B, W);
+            const int jlo = kCross ? 0 : first_key_tile(t, B, W);
+            const int jend = kCross ? (r.oL + kTile - 1) / kTile - 1 : t;
             const int64_t i = int64_t(t) * kTile + row;
             const bool valid = i < r.L;
-            const int64_t ws = window_start(i, B, W);
+            // visible keys [ws, last]: the block rule, or (cross-attention) the whole key/value set
+            const int64_t ws = kCross ? 0 : window_start(i, B, W);
+            const int64_t last = kCross ? int64_t(r.oL) - 1 : i;
             float m_ref = -INFINITY, l = 0.f;
-            for (int j = jlo; j <= t; ++j, ++cnt) {
+            for (int j = jlo; j <= jend; ++j, ++cnt) {
                 const int64_t key0 = int64_t(j) * kTile;
-                int64_t lo64 = ws - key0, hi64 = i - key0;
+                int64_t lo64 = ws - key0, hi64 = last - key0;
                 if (!valid) { lo64 = 1; hi64 = 0; }
                 const int lo_c = int(lo64 < -1 ? -1 : (lo64 > 128 ? 128 : lo64));
                 const int hi_c = int(hi64 < -1 ? -1 : (hi64 > 128 ? 128 : hi64));
@@ -439,6 +516,16 @@ __global__ void __launch_bounds__(512, 1)
                     }
                     tmem_wait_st();
                 }
+                if constexpr (kMx) {
+                    // the next K tile's scale factors go to TMEM before P is released: the MMA warp
+                    // issues that tile's S right after this tile's P V
+                    if (j < jend) {
+                        const uint32_t st1 = (cnt + 1) % S;
+                        if (!mbar_wait(&sb.k_full[st1], ((cnt + 1) / S) & 1, abort)) { ok = false; break; }
+                        put_scales(smem + Lay::kQScale + (1 + st1) * Lay::kScaleBox, Lay::kColSFB, r.h);
+                        tmem_wait_st();
+                    }
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sb.p_full[w]);
@@ -468,9 +555,9 @@ __global__ void __launch_bounds__(512, 1)
         uint32_t done[2] = {0, 0}, sync_phase = 0, nstored = 0;
         TileRef r;
         bool ok = true;
-        ItemWalker items(p.pair_info, npairs, p.heads);
-        while (ok && items.advance(r)) {
-            const bool second = pair_has_second(r);
+        ItemSink items;
+        while (ok && items.advance(r, sb.ring, abort, ok)) {
+            const bool second = !kMx && pair_has_second(r);
             for (int w = 0; w < (second ? 2 : 1) && ok; ++w) {
                 if (!mbar_wait(&sb.o_ready[w], done[w] & 1, abort) ||
                     !mbar_wait(&sb.o_final[w], done[w] & 1, abort)) {
@@ -549,10 +636,17 @@ __global__ void __launch_bounds__(512, 1)
 template <int D, int A>
 cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &to, const Problem &p, void *out, float *lse, int num_sms,
-                                  cudaStream_t stream)
+                                  cudaStream_t stream, const CUtensorMap *tqs, const CUtensorMap *tks)
 {
     using Lay = FwdLayout<D>;
-    auto kern = fwd_bf16_sm100_kernel<D, A>;
+    // cross-attention exists for the generalized attention only, the MXFP8 mode (scale maps
+    // given) for block attention at head_dim 128
+    constexpr bool kCanMx = D == 128 && A == kSoftmax;
+    const bool mx = kCanMx && tqs && tks;
+    if (!kCanMx && (tqs || tks)) return cudaErrorInvalidValue;
+    auto kern = mx ? fwd_bf16_sm100_kernel<D, A, false, kCanMx>
+                   : (A != kSoftmax && p.other_offsets) ? fwd_bf16_sm100_kernel<D, A, A != kSoftmax, false>
+                                                        : fwd_bf16_sm100_kernel<D, A, false, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
     // the register split only works if the CTA is launched with at least the budgets' sum
@@ -561,15 +655,16 @@ cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
     if (e != cudaSuccess) return e;
     if (fa.numRegs * Lay::kThreads < int(256 * Lay::kRegsCompute + 128 * Lay::kRegsEpi + 128 * Lay::kRegsOther))
         return cudaErrorInvalidConfiguration;
-    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, to, p, static_cast<__nv_bfloat16 *>(out),
-                                                          lse);
+    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, to, mx ? *tqs : tq, mx ? *tks : tk, p,
+                                                          static_cast<__nv_bfloat16 *>(out), lse);
     return cudaGetLastError();
 }
 
 #define BA_FWD_INST(D, A)                                                                                  \
     template cudaError_t launch_fwd_bf16_sm100<D, A>(const CUtensorMap &, const CUtensorMap &,              \
                                                      const CUtensorMap &, const CUtensorMap &, const Problem &, \
-                                                     void *, float *, int, cudaStream_t);
+                                                     void *, float *, int, cudaStream_t, const CUtensorMap *,   \
+                                                     const CUtensorMap *);
 BA_FWD_INST(64, kSoftmax)
 BA_FWD_INST(128, kSoftmax)
 BA_FWD_INST(64, kGelu)

@@ -9,7 +9,12 @@
 
 namespace ba {
 
-cudaError_t launch_worklist(const Problem &p, cudaStream_t stream);
+// Builds the work tables; reset_status = false keeps the status word (a second
+// table for the same call).
+cudaError_t launch_worklist(const Problem &p, cudaStream_t stream, bool reset_status = true);
+// Cross-attention: zero the rows (of a, and of b unless nullptr) of examples whose other side is empty.
+cudaError_t launch_zero_unpaired_rows(const int32_t *offs, const int32_t *other, int32_t batch, size_t row_bytes,
+                                      void *a, void *b, cudaStream_t stream);
 cudaError_t launch_wait_selftest(int *status, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_exp2_selftest(const float *x, float *y, int64_t n, cudaStream_t stream);
 
@@ -27,16 +32,24 @@ cudaError_t launch_skip_bwd(const Problem &p, size_t elem_bytes, const void *dou
 cudaError_t launch_rope_rows(const Problem &p, size_t elem_bytes, bool transpose, const void *a_in, const void *b_in,
                              void *a_out, void *b_out, int num_sms, cudaStream_t stream);
 
+// MX quantisation (E4M3 elements, E8M0 scales per 32 along head_dim) of a
+// [rows, heads, head_dim] bf16 tensor; scales [rows, heads rounded up to 4, head_dim / 32].
+cudaError_t launch_mx_quantize(const void *x, int64_t rows, int32_t heads, int32_t head_dim, void *elems,
+                               void *scales, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_fwd_f32(const Problem &p, const float *q, const float *k, const float *v, float *out, float *lse,
                            int num_sms, cudaStream_t stream);
 cudaError_t launch_bwd_f32(const Problem &p, const float *q, const float *k, const float *v, const float *dout,
                            const float *lse, const float *delta, float *dq, float *dk, float *dv, int num_sms,
                            cudaStream_t stream);
 
+// tqs / tks: the MXFP8 mode's maps of the Q and K scale words (q, k then E4M3);
+// nullptr for the bf16 operands.
 template <int D, int A>
 cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &to, const Problem &p, void *out, float *lse, int num_sms,
-                                  cudaStream_t stream);
+                                  cudaStream_t stream, const CUtensorMap *tqs = nullptr,
+                                  const CUtensorMap *tks = nullptr);
 
 template <int D, int A>
 cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,

@@ -182,6 +182,27 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// The rare half of load_tile_zero_tail, kept out of line so that the hot
+// loops around its call sites stay small in the instruction cache.
+static __device__ __noinline__ bool finish_tail_tile(uint8_t *dst, int chunks, uint64_t *full, uint64_t *tail,
+                                              uint32_t tail_phase, int valid, volatile int *abort)
+{
+    constexpr uint32_t kChunkBytes = 128 * 128;
+    const int lane = threadIdx.x & 31;
+    if (!mbar_wait(tail, tail_phase, abort)) return false;
+    const int v = valid < 0 ? 0 : valid;
+    const int units = (128 - v) * 8; // 16-byte units from row v to the end of a chunk
+    for (int c = 0; c < chunks; ++c) {
+        uint4 *z = reinterpret_cast<uint4 *>(dst + c * kChunkBytes + v * 128);
+        for (int u = lane; u < units; u += 32) z[u] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(full);
+    __syncwarp();
+    return true;
+}
+
 // Loads one 128-row tile of a [rows, columns] bf16 tensor map (CHUNKS boxes of
 // 128 rows x 64 columns, each a 16 KB 128B-swizzled chunk at dst + c * 16 KB)
 // and signals `full`. When only the first `valid` rows belong to the current
@@ -200,28 +221,17 @@ __device__ __forceinline__ bool load_tile_zero_tail(uint8_t *dst, const CUtensor
                                                     int valid, volatile int *abort)
 {
     constexpr uint32_t kChunkBytes = 128 * 128;
-    const int lane = threadIdx.x & 31;
     const bool clear = valid < 128;
-    if (lane == 0) {
+    if ((threadIdx.x & 31) == 0) {
         uint64_t *bar = clear ? tail : full;
         mbar_arrive_expect_tx(bar, CHUNKS * kChunkBytes);
         for (int c = 0; c < CHUNKS; ++c) tma_load_2d(dst + c * kChunkBytes, map, bar, x + 64 * c, y);
     }
     __syncwarp();
     if (!clear) return true;
-    if (!mbar_wait(tail, tail_phase, abort)) return false;
+    const uint32_t ph = tail_phase;
     tail_phase ^= 1;
-    const int v = valid < 0 ? 0 : valid;
-    const int units = (128 - v) * 8; // 16-byte units from row v to the end of a chunk
-    for (int c = 0; c < CHUNKS; ++c) {
-        uint4 *z = reinterpret_cast<uint4 *>(dst + c * kChunkBytes + v * 128);
-        for (int u = lane; u < units; u += 32) z[u] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(full);
-    __syncwarp();
-    return true;
+    return finish_tail_tile(dst, CHUNKS, full, tail, ph, valid, abort);
 }
 
 // -------------------------------------------------------------- tcgen05 ---
@@ -297,6 +307,32 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
                  : "memory");
 }
 
+// D[tmem] (+)= (A[smem] * B[smem]^T) with MX block scaling: A, B E4M3 (K = 32
+// per instruction), each row of A and of B scaled by the E8M0 factor held in
+// TMEM at sfa / sfb (the byte given by the address's top two bits, which the
+// instruction descriptor repeats). Warp-collective like mma_ss.
+__device__ __forceinline__ void mma_mx_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p, e;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+                     d_tmem),
+                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+                 : "memory");
+}
+
+// Instruction descriptor of the block-scaled kind::mxf8f6f4 MMA with E4M3 A
+// and B (K-major) and E8M0 scale factors; fp32 accumulator. Bits: [4,6) B
+// scale-factor byte, [7,10) A format (0 = E4M3), [10,13) B format, [17,23)
+// N >> 3, 23 scale format (1 = E8M0), [24,29) M >> 4, [29,31) A scale-factor
+// byte; K = 32.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, uint32_t sfa_byte, uint32_t sfb_byte)
+{
+    return (sfb_byte << 4) | (uint32_t(N >> 3) << 17) | (1u << 23) | (uint32_t(M >> 4) << 24) | (sfa_byte << 29);
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulator.
 // Bits: [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B
 // format, 15 A major (1 = MN), 16 B major, [17,23) N >> 3, [24,29) M >> 4.
@@ -355,6 +391,13 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
                    "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
                    "=r"(r[14]), "=r"(r[15])
                  : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3])
+                 : "memory");
 }
 
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])

@@ -148,6 +148,65 @@ ba_status ba_gdpa_bwd(const ba_problem *p, ba_activation act, const void *q, con
                       void *dk, void *dv, void *workspace, size_t workspace_bytes, ba_stream_t stream);
 
 /*
+ * GDPA cross-attention, GEM's cross- and pooled attention ("GEM (Meta)",
+ * section "Custom kernels": the generalized attention serves them too and is
+ * fastest with short keys/values). Example b's queries, rows
+ * q_offsets[b] .. q_offsets[b+1]-1 of q (and of out, dout, dq), see every key
+ * of example b's own key/value set, rows kv_offsets[b] .. kv_offsets[b+1]-1
+ * of k and v (and of dk, dv); there is no mask:
+ *     out_i = sum over the example's keys j of act(q_i . k_j / sqrt(head_dim)) v_j.
+ * An example with no keys gets out = 0 (the empty sum) and dq = 0; one with no
+ * queries gets dk = dv = 0. Pooled attention is this with a set of seed
+ * queries repeated for every example (the caller sums the seeds' dq over
+ * examples).
+ *  - p describes the queries: batch, total_tokens = q_offsets[batch], heads,
+ *    head_dim, dtype (BF16 only); kv_total_tokens = kv_offsets[batch]. Both
+ *    offset arrays are DEVICE int32 [batch + 1], non-decreasing from 0.
+ *  - q, out, dout, dq: DEVICE [total_tokens, heads, head_dim]; k, v, dk, dv:
+ *    DEVICE [kv_total_tokens, heads, head_dim]; 16-byte aligned.
+ *  - Workspace: ba_gdpa_cross_workspace_size bytes, for either direction.
+ *  - Errors as for ba_gdpa_fwd / ba_gdpa_bwd.
+ */
+size_t ba_gdpa_cross_workspace_size(const ba_problem *p, int32_t kv_total_tokens);
+ba_status ba_gdpa_cross_fwd(const ba_problem *p, int32_t kv_total_tokens, ba_activation act, const void *q,
+                            const void *k, const void *v, const int32_t *q_offsets, const int32_t *kv_offsets,
+                            void *out, void *workspace, size_t workspace_bytes, ba_stream_t stream);
+ba_status ba_gdpa_cross_bwd(const ba_problem *p, int32_t kv_total_tokens, ba_activation act, const void *q,
+                            const void *k, const void *v, const void *dout, const int32_t *q_offsets,
+                            const int32_t *kv_offsets, void *dq, void *dk, void *dv, void *workspace,
+                            size_t workspace_bytes, ba_stream_t stream);
+
+/*
+ * MXFP8 operands for the score product ("Meta Scales GEM Ads Model Across
+ * Platforms and Thousands of GPUs", opening section: GEM trains attention in
+ * MXFP8; the pages define neither the format nor the operands). The format is
+ * the public OCP Microscaling one: 32 consecutive elements along head_dim
+ * share a power-of-two scale 2^e stored as an E8M0 byte (e + 127), with
+ * e = floor(log2 max|v|) - 8 clamped to [-127, 127] (e = -8 for an all-zero
+ * block); each element is v / 2^e rounded to the nearest E4M3 value, ties to
+ * even, magnitudes above 448 clamped to 448.
+ *
+ * ba_mx_quantize: x DEVICE bf16 [rows, heads, head_dim] (head_dim a multiple
+ * of 32) -> elements DEVICE E4M3 bytes [rows, heads, head_dim] and scales
+ * DEVICE E8M0 bytes [rows, heads_pad, head_dim / 32], heads_pad = heads
+ * rounded up to a multiple of 4 (padding entries are not written).
+ *
+ * ba_mx_fwd: block attention (same rule, arguments, outputs and errors as
+ * ba_fwd) whose score product Q K^T takes MXFP8 Q and K: it quantises q and k
+ * into its workspace and runs the block-scaled tensor-core product (E4M3
+ * operands, E8M0 scale factors); softmax and P V are unchanged (bf16 P and
+ * V). The result is block attention of the dequantised Q and K. BF16 with
+ * head_dim 128 only (BA_ERR_UNSUPPORTED otherwise). Workspace:
+ * ba_mx_fwd_workspace_size bytes.
+ */
+ba_status ba_mx_quantize(const void *x, int64_t rows, int32_t heads, int32_t head_dim, void *elements,
+                         void *scales, ba_stream_t stream);
+size_t ba_mx_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window);
+ba_status ba_mx_fwd(const ba_problem *p, const void *q, const void *k, const void *v, const int32_t *seq_offsets,
+                    int32_t block, int32_t window, const uint8_t *skip, void *out, float *lse, void *workspace,
+                    size_t workspace_bytes, ba_stream_t stream);
+
+/*
  * Token-granular sliding-window attention, the predecessor that block
  * attention replaced ("GEM (Meta)", section "Custom kernels": long
  * user-history self-attention first moved to a sliding window, then to

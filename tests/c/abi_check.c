@@ -90,6 +90,17 @@ int main(void)
           BA_ERR_INVALID_ARG); /* workspace too small */
     CHECK(ba_gdpa_bwd(&p, BA_ACT_SILU, fake, fake, fake, NULL, fake, 128, 2, fake, fake, fake, fake, f, NULL) ==
           BA_ERR_INVALID_ARG); /* no dout */
+    CHECK(ba_gdpa_cross_workspace_size(&p, 5000) >= ba_gdpa_cross_workspace_size(&p, 10));
+    CHECK(ba_gdpa_cross_workspace_size(&p, -1) == 0);
+    CHECK(ba_gdpa_cross_fwd(&p, 500, BA_ACT_GELU, fake, fake, fake, fake, NULL, fake, fake, f, NULL) ==
+          BA_ERR_INVALID_ARG); /* no key/value offsets */
+    CHECK(ba_gdpa_cross_bwd(&p, -3, BA_ACT_SILU, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, f,
+                            NULL) == BA_ERR_INVALID_ARG); /* negative key/value count */
+    CHECK(ba_mx_quantize(NULL, 10, 2, 128, NULL, NULL, NULL) == BA_ERR_INVALID_ARG);
+    CHECK(ba_mx_quantize(fake, 10, 2, 100, fake, fake, NULL) == BA_ERR_INVALID_ARG); /* head_dim not a multiple of 32 */
+    CHECK(ba_mx_fwd_workspace_size(&p, 128, 2) > f);
+    CHECK(ba_mx_fwd(&p, fake, fake, fake, fake, 128, 2, NULL, fake, fake, fake, f, NULL) ==
+          BA_ERR_INVALID_ARG); /* the plain workspace has no room for the MXFP8 operands */
     CHECK(ba_selftest_exp2(NULL, NULL, 5, NULL) == BA_ERR_INVALID_ARG);
     CHECK(ba_selftest_exp2((const float *)fake, (float *)fake, -1, NULL) == BA_ERR_INVALID_ARG);
     CHECK(ba_selftest_exp2(NULL, NULL, 0, NULL) == BA_OK); /* nothing to do, nothing launched */

@@ -92,3 +92,52 @@ def test_gdpa_rejects_fp32_and_unknown_activations():
     qb = q.to(torch.bfloat16)
     prob = ba.make_problem(qb, offs)
     assert ba.ba_gdpa_fwd(prob, 7, qb, qb, qb, offs, 64, 1, qb.clone(), ws) == ba.BA_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------- cross-attention ---
+# Example b's queries against every key of its own key/value set
+# (oracle/gdpa.py cross_fwd / cross_bwd): GEM's cross- and pooled attention,
+# the short-key/value case. Query and key/value sets are jagged separately,
+# with empty sets on either side.
+
+CROSS = [
+    # (head_dim, query lengths, key/value lengths)
+    (128, [300, 1, 1000, 0, 129], [64, 200, 17, 50, 0]),
+    (64, [256, 700, 33], [128, 1, 300]),
+    (128, [64, 64, 64, 64], [500, 128, 129, 1]),   # pooled shape: few seeds per example, longer sequences
+]
+
+
+def _cross_inputs(head_dim, lq, lk, seed, scale):
+    g = torch.Generator().manual_seed(seed)
+    H = 2
+    q = (torch.randn(sum(lq), H, head_dim, generator=g) * scale).to(torch.bfloat16)
+    k = (torch.randn(sum(lk), H, head_dim, generator=g) * scale).to(torch.bfloat16)
+    v = (torch.randn(sum(lk), H, head_dim, generator=g) * scale).to(torch.bfloat16)
+    dout = torch.randn(sum(lq), H, head_dim, generator=g).to(torch.bfloat16)
+    qo = torch.tensor([0, *np.cumsum(lq)], dtype=torch.int32)
+    ko = torch.tensor([0, *np.cumsum(lk)], dtype=torch.int32)
+    return q, k, v, dout, qo, ko
+
+
+@pytest.mark.parametrize("act", ["gelu", "silu"])
+@pytest.mark.parametrize("head_dim,lq,lk", CROSS)
+@pytest.mark.parametrize("peaked", [False, True], ids=["config", "peaked"])
+def test_gdpa_cross_matches_oracle(act, head_dim, lq, lk, peaked):
+    q, k, v, dout, qo, ko = _cross_inputs(head_dim, lq, lk, 77 + head_dim, 1.0 if peaked else head_dim ** -0.5)
+    dev = [t.cuda() for t in (q, k, v, dout, qo, ko)]
+    out = ba.gdpa_cross_fwd(*dev[:3], dev[4], dev[5], act)
+    dq, dk, dv = ba.gdpa_cross_bwd(*dev[:4], dev[4], dev[5], act)
+    torch.cuda.synchronize()
+    args = (qo.numpy(), ko.numpy(), f64(q), f64(k), f64(v))
+    ref_out = G.cross_fwd(*args, act)
+    ref_dq, ref_dk, ref_dv = G.cross_bwd(*args, f64(dout), act)
+    for name, got, ref in (("out", out, ref_out), ("dq", dq, ref_dq), ("dk", dk, ref_dk), ("dv", dv, ref_dv)):
+        check_bf16(f"cross {act} {name}", got.cpu(), ref, peaked=peaked)
+    # empty sets: no keys -> out = dq = 0; no queries -> dk = dv = 0
+    for e in range(len(lq)):
+        qs, ks = slice(int(qo[e]), int(qo[e + 1])), slice(int(ko[e]), int(ko[e + 1]))
+        if lk[e] == 0:
+            assert not out[qs].any() and not dq[qs].any()
+        if lq[e] == 0:
+            assert not dk[ks].any() and not dv[ks].any()
