@@ -99,6 +99,22 @@ bool encode_u8_rows(CUtensorMap *map, const void *base, int64_t T, int64_t row_b
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// The dK/dV pass's partial query tiles: each example's last query tile, when
+// it has fewer than 128 rows, copied from q and dout (query rows given by
+// offs) into the workspace with zeros past the example, and the tensor maps
+// the pass reads them through (rows 128 b .. 128 b + 127 for example b).
+bool stage_query_tails(const ba_problem &P, const int32_t *offs, const uint8_t *skip, const void *q,
+                       const void *dout, uint8_t *ws, const WorkspaceLayout &lay, CUtensorMap &tqt, CUtensorMap &tdot,
+                       cudaStream_t stream)
+{
+    const int64_t rows = int64_t(P.batch) * kTile;
+    if (!encode_bf16_rows(&tqt, ws + lay.tail_q, rows, P.heads, P.head_dim) ||
+        !encode_bf16_rows(&tdot, ws + lay.tail_do, rows, P.heads, P.head_dim))
+        return false;
+    return launch_stage_query_tails(offs, skip, P.batch, size_t(P.heads) * P.head_dim * 2, q, dout, ws + lay.tail_q,
+                                    ws + lay.tail_do, stream) == cudaSuccess;
+}
+
 bool head_dim_supported(const ba_problem &p)
 {
     if (p.dtype == BA_BF16) return p.head_dim == 64 || p.head_dim == 128;
@@ -115,8 +131,9 @@ ba_status check_problem(const ba_problem *p, int32_t block, int32_t window)
     if (p->batch == 0 && p->total_tokens != 0) return BA_ERR_INVALID_ARG;
     // element offsets of one tensor must stay below 2^62 and rows below 2^31
     if (int64_t(p->heads) * p->head_dim > (int64_t(1) << 24)) return BA_ERR_UNSUPPORTED;
-    // work items (128-row tiles x heads) are numbered in 31 bits
-    if (max_tiles(p->batch, p->total_tokens) * p->heads > INT32_MAX) return BA_ERR_UNSUPPORTED;
+    // work items (128-row tiles x heads) and the staged tail rows (128 per example) are numbered in 31 bits
+    if (max_tiles(p->batch, p->total_tokens) * p->heads > INT32_MAX || int64_t(p->batch) * kTile > INT32_MAX)
+        return BA_ERR_UNSUPPORTED;
     if (!head_dim_supported(*p)) return BA_ERR_UNSUPPORTED;
     return BA_OK;
 }
@@ -261,7 +278,7 @@ ba_status bwd_impl(const ba_problem *pp, const ba_rope *rope, const void *q, con
         return BA_ERR_INVALID_ARG;
     if (with_rope && (st = check_rope(rope, P)) != BA_OK) return st;
     const bool bf16 = P.dtype == BA_BF16;
-    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, true);
+    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, true, bf16);
     const RopeLayout rl = rope_layout(P, lay.total);
     const size_t need = with_rope && !caller_rotated(rope) ? rl.total : lay.total;
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return BA_ERR_INVALID_ARG;
@@ -303,11 +320,12 @@ ba_status bwd_impl(const ba_problem *pp, const ba_rope *rope, const void *q, con
         if (with_rope) BA_TRY(launch_rope_rows(p, esz, true, dq, dk, dq, dk, num_sms, stream));
         return BA_OK;
     }
-    CUtensorMap tq, tk, tv, tdo, to, tdk, tdv;
+    CUtensorMap tq, tk, tv, tdo, to, tdk, tdv, tqt, tdot;
     if (!encode_bf16_rows(&tq, q, T, P.heads, P.head_dim) || !encode_bf16_rows(&tk, k, T, P.heads, P.head_dim) ||
         !encode_bf16_rows(&tv, v, T, P.heads, P.head_dim) || !encode_bf16_rows(&tdo, dout, T, P.heads, P.head_dim) ||
         !encode_bf16_rows(&to, out, T, P.heads, P.head_dim) || !encode_bf16_rows(&tdk, dk, T, P.heads, P.head_dim) ||
-        !encode_bf16_rows(&tdv, dv, T, P.heads, P.head_dim))
+        !encode_bf16_rows(&tdv, dv, T, P.heads, P.head_dim) ||
+        !stage_query_tails(P, seq_offsets, skip, q, dout, ws, lay, tqt, tdot, stream))
         return BA_ERR_CUDA;
     BA_TRY(prof_mark(1, 0, stream));
     if (P.head_dim == 64)
@@ -317,9 +335,11 @@ ba_status bwd_impl(const ba_problem *pp, const ba_rope *rope, const void *q, con
     BA_TRY(prof_mark(1, 1, stream));
     BA_TRY(prof_mark(2, 0, stream));
     if (P.head_dim == 64)
-        BA_TRY(launch_bwd_dkdv_sm100<64, kSoftmax>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, delta, dk, dv, num_sms, stream));
+        BA_TRY(launch_bwd_dkdv_sm100<64, kSoftmax>(tq, tk, tv, tdo, tdk, tdv, tqt, tdot, p, nlse2, delta, dk, dv,
+                                                   num_sms, stream));
     else
-        BA_TRY(launch_bwd_dkdv_sm100<128, kSoftmax>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, delta, dk, dv, num_sms, stream));
+        BA_TRY(launch_bwd_dkdv_sm100<128, kSoftmax>(tq, tk, tv, tdo, tdk, tdv, tqt, tdot, p, nlse2, delta, dk, dv,
+                                                    num_sms, stream));
     BA_TRY(prof_mark(2, 1, stream));
     return BA_OK;
 }
@@ -329,7 +349,7 @@ ba_status bwd_impl(const ba_problem *pp, const ba_rope *rope, const void *q, con
 template <int A>
 cudaError_t gdpa_launch(bool bwd, int D, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                         const CUtensorMap &tdo, const CUtensorMap &to, const CUtensorMap &tdk, const CUtensorMap &tdv,
-                        const Problem &p, void *out, void *dq, void *dk, void *dv, int num_sms, cudaStream_t stream)
+                        const CUtensorMap &tqt, const CUtensorMap &tdot, const Problem &p, void *out, void *dq, void *dk, void *dv, int num_sms, cudaStream_t stream)
 {
     cudaError_t e;
     if (!bwd) {
@@ -344,9 +364,10 @@ cudaError_t gdpa_launch(bool bwd, int D, const CUtensorMap &tq, const CUtensorMa
                 : launch_bwd_dq_sm100<128, A>(tq, tk, tv, tdo, to, p, nullptr, nullptr, nullptr, dq, num_sms, stream);
     if (e != cudaSuccess) return e;
     if ((e = prof_mark(1, 1, stream)) != cudaSuccess || (e = prof_mark(2, 0, stream)) != cudaSuccess) return e;
-    e = D == 64 ? launch_bwd_dkdv_sm100<64, A>(tq, tk, tv, tdo, tdk, tdv, p, nullptr, nullptr, dk, dv, num_sms, stream)
-                : launch_bwd_dkdv_sm100<128, A>(tq, tk, tv, tdo, tdk, tdv, p, nullptr, nullptr, dk, dv, num_sms,
-                                                stream);
+    e = D == 64 ? launch_bwd_dkdv_sm100<64, A>(tq, tk, tv, tdo, tdk, tdv, tqt, tdot, p, nullptr, nullptr, dk, dv,
+                                               num_sms, stream)
+                : launch_bwd_dkdv_sm100<128, A>(tq, tk, tv, tdo, tdk, tdv, tqt, tdot, p, nullptr, nullptr, dk, dv,
+                                                num_sms, stream);
     if (e != cudaSuccess) return e;
     return prof_mark(2, 1, stream);
 }
@@ -366,7 +387,7 @@ ba_status gdpa_impl(bool bwd, const ba_problem *pp, ba_activation act, const voi
     if (bwd && (!tensor_ok(dout, T) || !tensor_ok(dq, T) || !tensor_ok(dk, T) || !tensor_ok(dv, T)))
         return BA_ERR_INVALID_ARG;
     if (P.dtype != BA_BF16) return BA_ERR_UNSUPPORTED;
-    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, false);
+    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, false, true);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total) return BA_ERR_INVALID_ARG;
     int num_sms = 0, cc = 0;
     if (!device_info(num_sms, cc)) return BA_ERR_CUDA;
@@ -375,22 +396,24 @@ ba_status gdpa_impl(bool bwd, const ba_problem *pp, ba_activation act, const voi
     Problem p = make_problem(P, seq_offsets, nullptr, block, window, workspace, lay);
     BA_TRY(launch_worklist(p, stream));
     if (T == 0) return BA_OK;
-    CUtensorMap tq, tk, tv, tdo, to, tdk, tdv;
+    CUtensorMap tq, tk, tv, tdo, to, tdk, tdv, tqt, tdot;
     if (!encode_bf16_rows(&tq, q, T, P.heads, P.head_dim) || !encode_bf16_rows(&tk, k, T, P.heads, P.head_dim) ||
         !encode_bf16_rows(&tv, v, T, P.heads, P.head_dim))
         return BA_ERR_CUDA;
     if (!bwd && !encode_bf16_rows(&to, out, T, P.heads, P.head_dim)) return BA_ERR_CUDA;
     if (bwd && (!encode_bf16_rows(&tdo, dout, T, P.heads, P.head_dim) ||
                 !encode_bf16_rows(&tdk, dk, T, P.heads, P.head_dim) ||
-                !encode_bf16_rows(&tdv, dv, T, P.heads, P.head_dim)))
+                !encode_bf16_rows(&tdv, dv, T, P.heads, P.head_dim) ||
+                !stage_query_tails(P, seq_offsets, nullptr, q, dout, static_cast<uint8_t *>(workspace), lay, tqt,
+                                   tdot, stream)))
         return BA_ERR_CUDA;
     if (bwd) to = tdo; // the dQ pass reads no `out` here; any valid map fills the slot
-    else tdo = tdk = tdv = to;
+    else tdo = tdk = tdv = tqt = tdot = to;
     const cudaError_t e = act == BA_ACT_GELU
-                              ? gdpa_launch<kGelu>(bwd, P.head_dim, tq, tk, tv, tdo, to, tdk, tdv, p, out, dq, dk, dv,
-                                                   num_sms, stream)
-                              : gdpa_launch<kSilu>(bwd, P.head_dim, tq, tk, tv, tdo, to, tdk, tdv, p, out, dq, dk, dv,
-                                                   num_sms, stream);
+                              ? gdpa_launch<kGelu>(bwd, P.head_dim, tq, tk, tv, tdo, to, tdk, tdv, tqt, tdot, p, out,
+                                                   dq, dk, dv, num_sms, stream)
+                              : gdpa_launch<kSilu>(bwd, P.head_dim, tq, tk, tv, tdo, to, tdk, tdv, tqt, tdot, p, out,
+                                                   dq, dk, dv, num_sms, stream);
     return e == cudaSuccess ? BA_OK : BA_ERR_CUDA;
 }
 
@@ -416,7 +439,7 @@ ba_status gdpa_cross_impl(bool bwd, const ba_problem *pp, int32_t kv_total, ba_a
     if (bwd && (!tensor_ok(dout, Tq) || !tensor_ok(dq, Tq) || !tensor_ok(dk, Tk) || !tensor_ok(dv, Tk)))
         return BA_ERR_INVALID_ARG;
     if (P.dtype != BA_BF16) return BA_ERR_UNSUPPORTED;
-    const WorkspaceLayout lay = workspace_layout(P.batch, Tq > Tk ? Tq : Tk, P.heads, P.head_dim, false);
+    const WorkspaceLayout lay = workspace_layout(P.batch, Tq > Tk ? Tq : Tk, P.heads, P.head_dim, false, true);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total) return BA_ERR_INVALID_ARG;
     int num_sms = 0, cc = 0;
     if (!device_info(num_sms, cc)) return BA_ERR_CUDA;
@@ -434,7 +457,7 @@ ba_status gdpa_cross_impl(bool bwd, const ba_problem *pp, int32_t kv_total, ba_a
             BA_TRY(launch_zero_unpaired_rows(kv_offsets, q_offsets, P.batch, row_bytes, dk, dv, stream));
         return BA_OK;
     }
-    CUtensorMap tq, tk, tv, tdo, to, tdk, tdv;
+    CUtensorMap tq, tk, tv, tdo, to, tdk, tdv, tqt, tdot;
     if (!encode_bf16_rows(&tq, q, Tq, P.heads, P.head_dim) || !encode_bf16_rows(&tk, k, Tk, P.heads, P.head_dim) ||
         !encode_bf16_rows(&tv, v, Tk, P.heads, P.head_dim))
         return BA_ERR_CUDA;
@@ -457,10 +480,10 @@ ba_status gdpa_cross_impl(bool bwd, const ba_problem *pp, int32_t kv_total, ba_a
                         : launch_bwd_dq_sm100<128, A>(tq, tk, tv, tdo, tdo, p, nullptr, nullptr, nullptr, dq, num_sms,
                                                       stream);
         else
-            e = D == 64 ? launch_bwd_dkdv_sm100<64, A>(tq, tk, tv, tdo, tdk, tdv, p, nullptr, nullptr, dk, dv,
-                                                       num_sms, stream)
-                        : launch_bwd_dkdv_sm100<128, A>(tq, tk, tv, tdo, tdk, tdv, p, nullptr, nullptr, dk, dv,
-                                                        num_sms, stream);
+            e = D == 64 ? launch_bwd_dkdv_sm100<64, A>(tq, tk, tv, tdo, tdk, tdv, tqt, tdot, p, nullptr, nullptr, dk,
+                                                       dv, num_sms, stream)
+                        : launch_bwd_dkdv_sm100<128, A>(tq, tk, tv, tdo, tdk, tdv, tqt, tdot, p, nullptr, nullptr, dk,
+                                                        dv, num_sms, stream);
         return e == cudaSuccess ? prof_mark(w, 1, stream) : e;
     };
     const auto run_act = [&](bool dkdv_pass, const Problem &p) -> cudaError_t {
@@ -473,7 +496,8 @@ ba_status gdpa_cross_impl(bool bwd, const ba_problem *pp, int32_t kv_total, ba_a
         return BA_OK;
     }
     if (!encode_bf16_rows(&tdo, dout, Tq, P.heads, P.head_dim) || !encode_bf16_rows(&tdk, dk, Tk, P.heads, P.head_dim) ||
-        !encode_bf16_rows(&tdv, dv, Tk, P.heads, P.head_dim))
+        !encode_bf16_rows(&tdv, dv, Tk, P.heads, P.head_dim) ||
+        !stage_query_tails(P, q_offsets, nullptr, q, dout, static_cast<uint8_t *>(workspace), lay, tqt, tdot, stream))
         return BA_ERR_CUDA;
     BA_TRY(run_act(false, pq));
     // the key-tile side: tables over the key/value sets, each paired with its query set (the
@@ -552,7 +576,7 @@ size_t ba_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
 size_t ba_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
 {
     if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
-    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, true).total;
+    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, true, p->dtype == BA_BF16).total;
 }
 
 ba_status ba_fwd(const ba_problem *p, const void *q, const void *k, const void *v, const int32_t *seq_offsets,
@@ -632,7 +656,8 @@ ba_status ba_swa_bwd(const ba_problem *p, const void *q, const void *k, const vo
 
 size_t ba_gdpa_workspace_size(const ba_problem *p, int32_t block, int32_t window)
 {
-    return ba_fwd_workspace_size(p, block, window);
+    if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
+    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, false, true).total;
 }
 
 ba_status ba_gdpa_fwd(const ba_problem *p, ba_activation act, const void *q, const void *k, const void *v,
@@ -655,7 +680,7 @@ size_t ba_gdpa_cross_workspace_size(const ba_problem *p, int32_t kv_total_tokens
 {
     if (check_problem(p, 1, 1) == BA_ERR_INVALID_ARG || kv_total_tokens < 0) return 0;
     const int64_t t = p->total_tokens > kv_total_tokens ? p->total_tokens : kv_total_tokens;
-    return workspace_layout(p->batch, t, p->heads, p->head_dim, false).total;
+    return workspace_layout(p->batch, t, p->heads, p->head_dim, false, true).total;
 }
 
 ba_status ba_gdpa_cross_fwd(const ba_problem *p, int32_t kv_total_tokens, ba_activation act, const void *q,

@@ -2,6 +2,8 @@
 //   worklist_kernel   the persistent kernels' work list: every live 128-row
 //                     tile (and pair of tiles), examples longest first; resets
 //                     the status word
+//   stage_query_tails_kernel  the last, partial query tile of each example
+//                     (q and dout), zero-padded, for the dK/dV pass
 //   bwd_pre_kernel    Delta = rowsum(dout * out) in fp32 (the fp32 path; the
 //                     bf16 dQ pass computes Delta itself)
 //   wait_selftest_kernel  one warp waits on a barrier nothing completes, with a
@@ -234,6 +236,48 @@ cudaError_t launch_zero_unpaired_rows(const int32_t *offs, const int32_t *other,
     if (batch == 0) return cudaSuccess;
     zero_unpaired_rows_kernel<<<dim3(batch, 8), 256, 0, stream>>>(offs, other, int64_t(row_bytes),
                                                                  static_cast<uint8_t *>(a), static_cast<uint8_t *>(b));
+    return cudaGetLastError();
+}
+
+// The dK/dV pass's partial query tiles: example b's last query tile, when it
+// has fewer than 128 rows, is copied from a (q) and b (dout) to rows
+// [128 b, 128 b + 128) of ta and tb with zeros in the rows past the example,
+// so that the pass never multiplies a neighbour's rows, finite or not, by its
+// zero probabilities. Examples whose length is a multiple of 128 (or zero) or
+// that are skipped are left alone. grid = (example, 8 slices of 16 rows).
+__global__ void __launch_bounds__(256)
+    stage_query_tails_kernel(const int32_t *__restrict__ offs, const uint8_t *__restrict__ skip, int64_t row_bytes,
+                             const uint8_t *__restrict__ a, const uint8_t *__restrict__ b, uint8_t *__restrict__ ta,
+                             uint8_t *__restrict__ tb)
+{
+    const int e = blockIdx.x;
+    if (skip && skip[e]) return;
+    const int64_t L = offs[e + 1] - offs[e];
+    const int64_t valid = L % kTile;
+    if (valid == 0) return;
+    const int64_t first = offs[e] + (L - valid); // first row of the partial tile
+    const int64_t units = row_bytes / 16;        // 16-byte units per row
+    const int64_t r0 = int64_t(blockIdx.y) * (kTile / 8);
+    for (int64_t x = threadIdx.x; x < (kTile / 8) * units; x += blockDim.x) {
+        const int64_t r = r0 + x / units, u = x % units;
+        const int64_t dst = (int64_t(e) * kTile + r) * units + u;
+        uint4 va = make_uint4(0, 0, 0, 0), vb = va;
+        if (r < valid) {
+            va = reinterpret_cast<const uint4 *>(a)[(first + r) * units + u];
+            vb = reinterpret_cast<const uint4 *>(b)[(first + r) * units + u];
+        }
+        reinterpret_cast<uint4 *>(ta)[dst] = va;
+        reinterpret_cast<uint4 *>(tb)[dst] = vb;
+    }
+}
+
+cudaError_t launch_stage_query_tails(const int32_t *offs, const uint8_t *skip, int32_t batch, size_t row_bytes,
+                                     const void *a, const void *b, void *ta, void *tb, cudaStream_t stream)
+{
+    if (batch == 0) return cudaSuccess;
+    stage_query_tails_kernel<<<dim3(batch, 8), 256, 0, stream>>>(
+        offs, skip, int64_t(row_bytes), static_cast<const uint8_t *>(a), static_cast<const uint8_t *>(b),
+        static_cast<uint8_t *>(ta), static_cast<uint8_t *>(tb));
     return cudaGetLastError();
 }
 

@@ -78,8 +78,7 @@ struct DkvBarriers {
     uint64_t q_full[4], q_empty[4], o_full[4], o_empty[4];
     uint64_t s_full, dp_full, pa_done[2], pb_done[2];
     uint64_t epi_sync; // group barrier of the epilogue warps
-    uint64_t tail;     // the TMA warp's own barrier for a Q or dO tile whose last rows it clears
-    ItemRing ring;     // items claimed by the TMA warp, read by the MMA, compute and epilogue warps
+    ItemRing ring;     // unused: this pass deals its items statically (StaticItems)
     uint32_t tmem_base;
     int abort;
     // per Q slot: -lse in log2 units and -Delta of the tile's 128 queries
@@ -107,6 +106,7 @@ __global__ void __launch_bounds__(448, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                           const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
+                          const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_dot,
                           const Problem p, const float *__restrict__ nlse2, const float *__restrict__ neg_delta,
                           __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv)
 {
@@ -136,8 +136,6 @@ __global__ void __launch_bounds__(448, 1)
         mbar_init(&sb.s_full, 1);
         mbar_init(&sb.dp_full, 1);
         mbar_init(&sb.epi_sync, 128);
-        mbar_init(&sb.tail, 1);
-        item_ring_init(sb.ring, 1 + 8 + 4); // MMA warp, compute warps, epilogue warps
         for (int g = 0; g < 2; ++g) {
             mbar_init(&sb.pa_done[g], 4);
             mbar_init(&sb.pb_done[g], 4);
@@ -150,6 +148,8 @@ __global__ void __launch_bounds__(448, 1)
         tma_prefetch_map(&tm_k);
         tma_prefetch_map(&tm_v);
         tma_prefetch_map(&tm_do);
+        tma_prefetch_map(&tm_qt);
+        tma_prefetch_map(&tm_dot);
     }
     if (warp == 13) {
         tmem_alloc(&sb.tmem_base, Lay::kTmemCols);
@@ -166,10 +166,10 @@ __global__ void __launch_bounds__(448, 1)
 
     if (warp == 12) {
         // ------------------------------------------------ TMA producer ---
-        uint32_t it = 0, item_cnt = 0, tail_phase = 0;
+        uint32_t it = 0, item_cnt = 0;
         TileRef r;
         bool ok = true;
-        ItemSource items(p.tile_info, ntiles, p.heads, p.status + kCounterDkdv, p.other_offsets);
+        StaticItems items(p.tile_info, ntiles, p.heads, p.other_offsets);
         for (; ok && items.advance(r, sb.ring, abort, ok); ++item_cnt) {
             int ilo, ihi;
             query_tile_range<kCross>(r, B, W, ilo, ihi);
@@ -179,14 +179,18 @@ __global__ void __launch_bounds__(448, 1)
                     ok = false;
                     break;
                 }
-                // the example's last query tile: its rows past the example are cleared (Q here,
-                // dO below), since dK += dS^T Q and dV += P^T dO multiply them by zeros
-                const int valid = r.oL - i * kTile; // query rows: the example's own, or its query set
-                if (!load_tile_zero_tail<Lay::kChunks>(smem + Lay::kQ0 + qs * Lay::kTileBytes, &tm_q, &sb.q_full[qs],
-                                                       &sb.tail, tail_phase, r.h * D, r.os0 + i * kTile, valid,
-                                                       abort)) {
-                    ok = false;
-                    break;
+                // the example's last query tile, when partial, comes from the staged copy whose
+                // rows past the example are zeros (Q here, dO below): dK += dS^T Q and
+                // dV += P^T dO multiply those rows by zeros, which must not meet a neighbour's
+                // Inf or NaN
+                const bool part = r.oL - i * kTile < kTile; // query rows: the example's own, or its query set
+                const CUtensorMap *mq = part ? &tm_qt : &tm_q, *mo = part ? &tm_dot : &tm_do;
+                const int32_t qy = part ? r.b * kTile : r.os0 + i * kTile;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sb.q_full[qs], Lay::kTileBytes);
+                    for (int c = 0; c < Lay::kChunks; ++c)
+                        tma_load_2d(smem + Lay::kQ0 + qs * Lay::kTileBytes + c * Lay::kChunkBytes, mq,
+                                    &sb.q_full[qs], r.h * D + c * 64, qy);
                 }
                 // the tile's -lse (log2 units) and -Delta, four queries per lane, copied
                 // asynchronously; each lane's copies arrive on q_full when they land. Rows past
@@ -235,13 +239,11 @@ __global__ void __launch_bounds__(448, 1)
                     ok = false;
                     break;
                 }
-                if (!load_tile_zero_tail<Lay::kChunks>(smem + Lay::kO0 + os * Lay::kTileBytes, &tm_do, &sb.o_full[os],
-                                                       &sb.tail, tail_phase, r.h * D, r.os0 + i * kTile, valid,
-                                                       abort)) {
-                    ok = false;
-                    break;
-                }
                 if (lane == 0) {
+                    mbar_arrive_expect_tx(&sb.o_full[os], Lay::kTileBytes);
+                    for (int c = 0; c < Lay::kChunks; ++c)
+                        tma_load_2d(smem + Lay::kO0 + os * Lay::kTileBytes + c * Lay::kChunkBytes, mo,
+                                    &sb.o_full[os], r.h * D + c * 64, qy);
                     // warm L2 two query tiles ahead, and with the next item's K, V and first tiles
                     if (i + 2 <= ihi)
                         for (int c = 0; c < Lay::kChunks; ++c) {
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(448, 1)
         TileRef r;
         bool ok = true;
         const uint32_t k_addr = smem_base + Lay::kK, v_addr = smem_base + Lay::kV;
-        ItemSink items;
+        StaticItems items(p.tile_info, ntiles, p.heads, p.other_offsets);
         for (; ok && items.advance(r, sb.ring, abort, ok); ++item_cnt) {
             int ilo, ihi;
             query_tile_range<kCross>(r, B, W, ilo, ihi);
@@ -368,7 +370,7 @@ __global__ void __launch_bounds__(448, 1)
         uint32_t it = 0;
         TileRef r;
         bool ok = true;
-        ItemSink items;
+        StaticItems items(p.tile_info, ntiles, p.heads, p.other_offsets);
         while (ok && items.advance(r, sb.ring, abort, ok)) {
             int ilo, ihi;
             query_tile_range<kCross>(r, B, W, ilo, ihi);
@@ -492,7 +494,7 @@ __global__ void __launch_bounds__(448, 1)
         uint32_t item_cnt = 0, sync_phase = 0;
         bool ok = true;
         TileRef r;
-        ItemSink items;
+        StaticItems items(p.tile_info, ntiles, p.heads, p.other_offsets);
         for (; ok && items.advance(r, sb.ring, abort, ok); ++item_cnt) {
             const int64_t k = int64_t(r.t) * kTile + row;
             const bool valid_k = k < r.L;
@@ -578,8 +580,9 @@ __global__ void __launch_bounds__(448, 1)
 template <int D, int A>
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
-                                  const Problem &p, const float *nlse2, const float *neg_delta, void *dk, void *dv,
-                                  int num_sms, cudaStream_t stream)
+                                  const CUtensorMap &tqt, const CUtensorMap &tdot, const Problem &p,
+                                  const float *nlse2, const float *neg_delta, void *dk, void *dv, int num_sms,
+                                  cudaStream_t stream)
 {
     using Lay = DkvLayout<D>;
     // the rotary epilogue exists for block attention only, cross-attention for the generalized one
@@ -588,7 +591,7 @@ cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
                                                      : bwd_dkdv_sm100_kernel<D, false, A, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, tdk, tdv, p, nlse2, neg_delta,
+    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, tdk, tdv, tqt, tdot, p, nlse2, neg_delta,
                                                           static_cast<__nv_bfloat16 *>(dk),
                                                           static_cast<__nv_bfloat16 *>(dv));
     return cudaGetLastError();
@@ -597,7 +600,8 @@ cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
 #define BA_DKDV_INST(D, A)                                                                                   \
     template cudaError_t launch_bwd_dkdv_sm100<D, A>(const CUtensorMap &, const CUtensorMap &,                \
                                                      const CUtensorMap &, const CUtensorMap &, const CUtensorMap &, \
-                                                     const CUtensorMap &, const Problem &, const float *,       \
+                                                     const CUtensorMap &, const CUtensorMap &, const CUtensorMap &, \
+                                                     const Problem &, const float *,                            \
                                                      const float *, void *, void *, int, cudaStream_t);
 BA_DKDV_INST(64, kSoftmax)
 BA_DKDV_INST(128, kSoftmax)

@@ -170,17 +170,45 @@ __global__ void __launch_bounds__(384, 1)
                     // the example's last K and V tiles: rows past the example are cleared, since
                     // dQ += dS K and the masked dS = P (dP - Delta) multiply them by zeros
                     const int valid = r.oL - j * kTile;
-                    if (!mbar_wait(&sb.k_empty[st], ((kv_cnt / S) & 1) ^ 1, abort) ||
-                        !load_tile_zero_tail<Lay::kChunks>(kdst, &tm_k, &sb.k_full[st], &sb.tail, tail_phase,
-                                                           r.h * D, r.os0 + j * kTile, valid, abort)) {
+                    if (!mbar_wait(&sb.k_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
                         ok = false;
                         break;
                     }
-                    if (!mbar_wait(&sb.v_empty[st], ((kv_cnt / S) & 1) ^ 1, abort) ||
-                        !load_tile_zero_tail<Lay::kChunks>(kdst + Lay::kTileBytes, &tm_v, &sb.v_full[st], &sb.tail,
-                                                           tail_phase, r.h * D, r.os0 + j * kTile, valid, abort)) {
+                    if (valid >= kTile) {
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(&sb.k_full[st], Lay::kTileBytes);
+                            for (int c = 0; c < Lay::kChunks; ++c)
+                                tma_load_2d(kdst + c * Lay::kChunkBytes, &tm_k, &sb.k_full[st], r.h * D + c * 64,
+                                            r.os0 + j * kTile);
+                        }
+                        __syncwarp();
+                    } else {
+                        if (!load_tail_tile(kdst, Lay::kChunks, &tm_k, &sb.k_full[st], &sb.tail, tail_phase, r.h * D,
+                                            r.os0 + j * kTile, valid, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tail_phase ^= 1;
+                    }
+                    if (!mbar_wait(&sb.v_empty[st], ((kv_cnt / S) & 1) ^ 1, abort)) {
                         ok = false;
                         break;
+                    }
+                    if (valid >= kTile) {
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(&sb.v_full[st], Lay::kTileBytes);
+                            for (int c = 0; c < Lay::kChunks; ++c)
+                                tma_load_2d(kdst + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_v, &sb.v_full[st],
+                                            r.h * D + c * 64, r.os0 + j * kTile);
+                        }
+                        __syncwarp();
+                    } else {
+                        if (!load_tail_tile(kdst + Lay::kTileBytes, Lay::kChunks, &tm_v, &sb.v_full[st], &sb.tail,
+                                            tail_phase, r.h * D, r.os0 + j * kTile, valid, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tail_phase ^= 1;
                     }
                 }
             }

@@ -59,8 +59,12 @@ __host__ __device__ __forceinline__ bool visible(int64_t i, int64_t j, int64_t b
 //   delta   (bwd only)  float[heads * total_tokens]: Delta (fp32 path) or -Delta
 //                       (bf16 path, written by the dQ pass for the dK/dV pass)
 //   nlse2   (bwd only)  float[heads * total_tokens]: -lse in log2 units (bf16 path)
+//   tail_q, tail_do     (bf16 backward only) bf16[batch * 128, heads * head_dim]
+//                       each: rows 128b .. 128b + 127 hold example b's last,
+//                       partial query tile of q (dout), zeros past the example
+//                       (the dK/dV pass reads that tile from here)
 struct WorkspaceLayout {
-    size_t status, tile_prefix, tile_info, pair_prefix, pair_info, delta, nlse2, total;
+    size_t status, tile_prefix, tile_info, pair_prefix, pair_info, delta, nlse2, tail_q, tail_do, total;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -77,7 +81,7 @@ __host__ __device__ inline int64_t max_pairs(int64_t batch, int64_t total_tokens
 
 __host__ __device__ inline WorkspaceLayout workspace_layout(int64_t batch, int64_t total_tokens,
                                                             int64_t heads, int64_t head_dim,
-                                                            bool with_delta)
+                                                            bool with_delta, bool tail_rows = false)
 {
     WorkspaceLayout w;
     w.status = 0;
@@ -94,7 +98,10 @@ __host__ __device__ inline WorkspaceLayout workspace_layout(int64_t batch, int64
     if (with_delta) off = align256(off + sizeof(float) * size_t(heads * total_tokens));
     w.nlse2 = off;
     if (with_delta) off = align256(off + sizeof(float) * size_t(heads * total_tokens));
-    w.total = off;
+    const size_t tail_bytes = tail_rows ? align256(size_t(batch) * kTile * size_t(heads * head_dim) * 2) : 0;
+    w.tail_q = off;
+    w.tail_do = off + tail_bytes;
+    w.total = off + 2 * tail_bytes;
     return w;
 }
 
@@ -219,6 +226,7 @@ __device__ __forceinline__ float act_grad(float x)
 
 // One 128-row tile of one (example, head).
 struct TileRef {
+    int32_t b;         // example index
     int32_t h, t;      // head, tile index within the example
     int32_t s0, L;     // first global row of the example, its length
     int32_t os0, oL;   // the other side's rows (cross-attention: the example's key/value set
@@ -236,6 +244,7 @@ __device__ __forceinline__ bool decode_item(const Problem &p, int32_t ntiles, in
     const int32_t tile = int32_t(n / p.heads);
     r.h = int32_t(n % p.heads);
     const int4 info = p.tile_info[tile];
+    r.b = info.w;
     r.s0 = info.x;
     r.L = info.y;
     r.t = info.z;
@@ -253,6 +262,7 @@ __device__ __forceinline__ bool decode_pair(const Problem &p, int32_t npairs, in
     const int32_t pair = int32_t(n / p.heads);
     r.h = int32_t(n % p.heads);
     const int4 info = p.pair_info[pair];
+    r.b = info.w;
     r.s0 = info.x;
     r.L = info.y;
     r.t = info.z;

@@ -58,12 +58,16 @@ struct FwdLayout {
     static constexpr uint32_t kRegsCompute = D == 64 ? 168 : 184, kRegsEpi = 64, kRegsOther = D == 64 ? 112 : 80;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColO = 256;
-    // MXFP8 mode (one softmax group, single query tiles): Q and K are E4M3 (one
-    // 16 KB chunk per 128 x 128 tile, in the bf16 slots); the Q tile's scale words
-    // (a 128-row x 16-byte box: four heads' words per row) sit in group 1's Q slot,
-    // the K stages' boxes after it; the scale factors go to TMEM columns that
-    // group 1's S would use: A (the Q tile's) at 128..131, B (the K tile's) at 132..135.
-    static constexpr int kQScale = kQ + kTileBytes;
+};
+
+// MXFP8 mode of the head_dim-128 layout (one softmax group, single query
+// tiles): Q and K are E4M3 (one 16 KB chunk per 128 x 128 tile, in the bf16
+// slots); the Q tile's scale words (a 128-row x 16-byte box: four heads' words
+// per row) sit in group 1's Q slot, the K stages' boxes after it; the scale
+// factors go to TMEM columns that group 1's S would use: A (the Q tile's) at
+// 128..131, B (the K tile's) at 132..135.
+struct FwdMx {
+    static constexpr int kQScale = FwdLayout<128>::kQ + FwdLayout<128>::kTileBytes;
     static constexpr int kScaleBox = kTile * 16;
     static constexpr int kFp8TileBytes = kTile * 128;
     static constexpr uint32_t kColSFA = 128, kColSFB = 132;
@@ -77,7 +81,7 @@ struct FwdBarriers {
     uint64_t epi_sync;   // group barrier of the epilogue warpgroup
     uint64_t tail;       // the TMA warp's own barrier for a V tile whose last rows it clears
     uint64_t sf_ready;   // MXFP8: the item's scale factors (Q tile and first K tile) are in TMEM
-    ItemRing ring;       // items claimed by the TMA warp, read by the MMA, softmax and epilogue warps
+    ItemRing ring;       // unused: this kernel deals its items statically (StaticItems)
     float inv_l[2][kTile];
     uint32_t tmem_base;
     int abort;
@@ -128,7 +132,6 @@ __global__ void __launch_bounds__(512, 1)
         }
         mbar_init(&sb.epi_sync, 128);
         mbar_init(&sb.tail, 1);
-        item_ring_init(sb.ring, 1 + 8 + 4); // MMA warp, softmax warps, epilogue warps
         mbar_init(&sb.sf_ready, 4);
         sb.abort = 0;
         fence_mbar_init();
@@ -163,7 +166,7 @@ __global__ void __launch_bounds__(512, 1)
             TileRef r;
             bool second;
             bool ok = true;
-            ItemSource items(item_table, nitems, p.heads, p.status + kCounterFwd, p.other_offsets);
+            StaticItems items(item_table, nitems, p.heads, p.other_offsets);
             for (; ok && items.advance(r, sb.ring, abort, ok); ++item_cnt) {
                 second = !kMx && pair_has_second(r);
                 // cross-attention: every key tile of the example's own key/value set
@@ -177,9 +180,9 @@ __global__ void __launch_bounds__(512, 1)
                     }
                     if (lane == 0) {
                         if constexpr (kMx) { // E4M3 tile (128 bytes a row) and its rows' scale words
-                            mbar_arrive_expect_tx(&sb.q_full[w], Lay::kFp8TileBytes + Lay::kScaleBox);
+                            mbar_arrive_expect_tx(&sb.q_full[w], FwdMx::kFp8TileBytes + FwdMx::kScaleBox);
                             tma_load_2d(smem + Lay::kQ, &tm_q, &sb.q_full[w], r.h * D, r.s0 + r.t * kTile);
-                            tma_load_2d(smem + Lay::kQScale, &tm_qs, &sb.q_full[w], (r.h / 4) * 16, r.s0 + r.t * kTile);
+                            tma_load_2d(smem + FwdMx::kQScale, &tm_qs, &sb.q_full[w], (r.h / 4) * 16, r.s0 + r.t * kTile);
                         } else {
                             mbar_arrive_expect_tx(&sb.q_full[w], Lay::kTileBytes);
                             for (int c = 0; c < Lay::kChunks; ++c)
@@ -213,9 +216,9 @@ __global__ void __launch_bounds__(512, 1)
                     }
                     if (lane == 0) {
                         if constexpr (kMx) {
-                            mbar_arrive_expect_tx(&sb.k_full[st], Lay::kFp8TileBytes + Lay::kScaleBox);
+                            mbar_arrive_expect_tx(&sb.k_full[st], FwdMx::kFp8TileBytes + FwdMx::kScaleBox);
                             tma_load_2d(kdst, &tm_k, &sb.k_full[st], r.h * D, r.os0 + j * kTile);
-                            tma_load_2d(smem + Lay::kQScale + (1 + st) * Lay::kScaleBox, &tm_ks, &sb.k_full[st],
+                            tma_load_2d(smem + FwdMx::kQScale + (1 + st) * FwdMx::kScaleBox, &tm_ks, &sb.k_full[st],
                                         (r.h / 4) * 16, r.os0 + j * kTile);
                         } else {
                             mbar_arrive_expect_tx(&sb.k_full[st], Lay::kTileBytes);
@@ -232,11 +235,22 @@ __global__ void __launch_bounds__(512, 1)
                     // the example's last V tile: its rows past the example are cleared, since
                     // P V multiplies them by zero probabilities (K needs nothing: masked scores
                     // are replaced, not multiplied)
-                    if (!load_tile_zero_tail<Lay::kChunks>(kdst + Lay::kTileBytes, &tm_v, &sb.v_full[st], &sb.tail,
-                                                           tail_phase, r.h * D, r.os0 + j * kTile,
-                                                           r.oL - j * kTile, abort)) {
-                        ok = false;
-                        break;
+                    const int valid = r.oL - j * kTile;
+                    if (valid >= kTile) {
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(&sb.v_full[st], Lay::kTileBytes);
+                            for (int c = 0; c < Lay::kChunks; ++c)
+                                tma_load_2d(kdst + Lay::kTileBytes + c * Lay::kChunkBytes, &tm_v, &sb.v_full[st],
+                                            r.h * D + c * 64, r.os0 + j * kTile);
+                        }
+                        __syncwarp();
+                    } else {
+                        if (!load_tail_tile(kdst + Lay::kTileBytes, Lay::kChunks, &tm_v, &sb.v_full[st], &sb.tail,
+                                            tail_phase, r.h * D, r.os0 + j * kTile, valid, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tail_phase ^= 1;
                     }
                 }
             }
@@ -251,7 +265,7 @@ __global__ void __launch_bounds__(512, 1)
             TileRef r;
             bool second;
             bool ok = true;
-            ItemSink items;
+            StaticItems items(item_table, nitems, p.heads, p.other_offsets);
             for (; ok && items.advance(r, sb.ring, abort, ok); ++item_cnt) {
                 second = !kMx && pair_has_second(r);
                 const int nkt = (r.oL + kTile - 1) / kTile; // cross-attention: key tiles of the example
@@ -295,7 +309,7 @@ __global__ void __launch_bounds__(512, 1)
                             for (uint32_t kk = 0; kk < 4; ++kk)
                                 mma_mx_ss(tmem, sdesc_sw128(q_addr + kk * 32, 16, 1024),
                                           sdesc_sw128(k_addr + kk * 32, 16, 1024), idesc_mx_e4m3(128, 128, kk, kk),
-                                          (tmem + Lay::kColSFA) | (kk << 30), (tmem + Lay::kColSFB) | (kk << 30),
+                                          (tmem + FwdMx::kColSFA) | (kk << 30), (tmem + FwdMx::kColSFB) | (kk << 30),
                                           kk > 0 ? 1u : 0u);
                         } else {
 #pragma unroll
@@ -373,7 +387,7 @@ __global__ void __launch_bounds__(512, 1)
                 wd[m] = *reinterpret_cast<const uint32_t *>(box + (lane + 32 * m) * 16 + (head % 4) * 4);
             tmem_st4(tmem + lane_base + col, wd);
         };
-        ItemSink items;
+        StaticItems items(item_table, nitems, p.heads, p.other_offsets);
         while (ok && items.advance(r, sb.ring, abort, ok)) {
             second = !kMx && pair_has_second(r);
             if (w == 1 && !second) continue;
@@ -385,8 +399,8 @@ __global__ void __launch_bounds__(512, 1)
                     ok = false;
                     break;
                 }
-                put_scales(smem + Lay::kQScale, Lay::kColSFA, r.h);
-                put_scales(smem + Lay::kQScale + (1 + st0) * Lay::kScaleBox, Lay::kColSFB, r.h);
+                put_scales(smem + FwdMx::kQScale, FwdMx::kColSFA, r.h);
+                put_scales(smem + FwdMx::kQScale + (1 + st0) * FwdMx::kScaleBox, FwdMx::kColSFB, r.h);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -522,7 +536,7 @@ __global__ void __launch_bounds__(512, 1)
                     if (j < jend) {
                         const uint32_t st1 = (cnt + 1) % S;
                         if (!mbar_wait(&sb.k_full[st1], ((cnt + 1) / S) & 1, abort)) { ok = false; break; }
-                        put_scales(smem + Lay::kQScale + (1 + st1) * Lay::kScaleBox, Lay::kColSFB, r.h);
+                        put_scales(smem + FwdMx::kQScale + (1 + st1) * FwdMx::kScaleBox, FwdMx::kColSFB, r.h);
                         tmem_wait_st();
                     }
                 }
@@ -555,7 +569,7 @@ __global__ void __launch_bounds__(512, 1)
         uint32_t done[2] = {0, 0}, sync_phase = 0, nstored = 0;
         TileRef r;
         bool ok = true;
-        ItemSink items;
+        StaticItems items(item_table, nitems, p.heads, p.other_offsets);
         while (ok && items.advance(r, sb.ring, abort, ok)) {
             const bool second = !kMx && pair_has_second(r);
             for (int w = 0; w < (second ? 2 : 1) && ok; ++w) {

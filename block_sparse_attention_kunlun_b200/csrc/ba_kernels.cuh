@@ -15,6 +15,9 @@ cudaError_t launch_worklist(const Problem &p, cudaStream_t stream, bool reset_st
 // Cross-attention: zero the rows (of a, and of b unless nullptr) of examples whose other side is empty.
 cudaError_t launch_zero_unpaired_rows(const int32_t *offs, const int32_t *other, int32_t batch, size_t row_bytes,
                                       void *a, void *b, cudaStream_t stream);
+// The dK/dV pass's partial query tiles of a (q) and b (dout), zero-padded to 128 rows, into ta and tb.
+cudaError_t launch_stage_query_tails(const int32_t *offs, const uint8_t *skip, int32_t batch, size_t row_bytes,
+                                     const void *a, const void *b, void *ta, void *tb, cudaStream_t stream);
 cudaError_t launch_wait_selftest(int *status, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_exp2_selftest(const float *x, float *y, int64_t n, cudaStream_t stream);
 
@@ -58,7 +61,8 @@ cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, co
 template <int D, int A>
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
-                                  const Problem &p, const float *nlse2, const float *neg_delta, void *dk, void *dv,
-                                  int num_sms, cudaStream_t stream);
+                                  const CUtensorMap &tqt, const CUtensorMap &tdot, const Problem &p,
+                                  const float *nlse2, const float *neg_delta, void *dk, void *dv, int num_sms,
+                                  cudaStream_t stream);
 
 } // namespace ba

@@ -182,10 +182,21 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// The rare half of load_tile_zero_tail, kept out of line so that the hot
-// loops around its call sites stay small in the instruction cache.
+// A 128-row tile whose first `valid` rows (valid < 128) belong to the current
+// example holds the next example's rows after them, which a masked product
+// would still multiply by a zero probability (and 0 x inf is NaN). Such a
+// tile is loaded by load_tail_tile: the TMA (CHUNKS boxes of 128 rows x 64
+// columns, each a 16 KB 128B-swizzled chunk at dst + c * 16 KB) completes on
+// the producer warp's private barrier `tail`; the warp waits for it, clears
+// rows [valid, 128) of every chunk (the swizzle permutes 16-byte units only
+// within a row's own 128 bytes, so a row is the same 128 bytes swizzled or
+// not), makes the clears visible to the tensor core's operand reads and then
+// arrives on `full` (one plain arrival in place of the expect_tx one). Both
+// functions are out of line, so that the kernels' hot loops (whose code sits
+// at the edge of the instruction cache) carry only the common full-tile load.
+// Called by all 32 lanes of the producer warp; false after a timed-out wait.
 static __device__ __noinline__ bool finish_tail_tile(uint8_t *dst, int chunks, uint64_t *full, uint64_t *tail,
-                                              uint32_t tail_phase, int valid, volatile int *abort)
+                                                     uint32_t tail_phase, int valid, volatile int *abort)
 {
     constexpr uint32_t kChunkBytes = 128 * 128;
     const int lane = threadIdx.x & 31;
@@ -203,35 +214,17 @@ static __device__ __noinline__ bool finish_tail_tile(uint8_t *dst, int chunks, u
     return true;
 }
 
-// Loads one 128-row tile of a [rows, columns] bf16 tensor map (CHUNKS boxes of
-// 128 rows x 64 columns, each a 16 KB 128B-swizzled chunk at dst + c * 16 KB)
-// and signals `full`. When only the first `valid` rows belong to the current
-// example (valid < 128), the rows after them hold the next example's data,
-// which a masked product would still multiply by a zero probability (and
-// 0 x inf is NaN). Such a tile completes on the warp's private barrier
-// `tail` instead; the warp waits for it, clears the rows [valid, 128) of every
-// chunk (the swizzle permutes 16-byte units only within a row's own 128
-// bytes, so a row is the same 128 bytes swizzled or not), makes the clears
-// visible to the tensor core's operand reads and then arrives on `full` (one
-// plain arrival in place of the expect_tx one). Called by all 32 lanes of
-// the producer warp; false after a timed-out wait.
-template <int CHUNKS>
-__device__ __forceinline__ bool load_tile_zero_tail(uint8_t *dst, const CUtensorMap *map, uint64_t *full,
-                                                    uint64_t *tail, uint32_t &tail_phase, int32_t x, int32_t y,
-                                                    int valid, volatile int *abort)
+static __device__ __noinline__ bool load_tail_tile(uint8_t *dst, int chunks, const CUtensorMap *map, uint64_t *full,
+                                                   uint64_t *tail, uint32_t tail_phase, int32_t x, int32_t y,
+                                                   int valid, volatile int *abort)
 {
     constexpr uint32_t kChunkBytes = 128 * 128;
-    const bool clear = valid < 128;
     if ((threadIdx.x & 31) == 0) {
-        uint64_t *bar = clear ? tail : full;
-        mbar_arrive_expect_tx(bar, CHUNKS * kChunkBytes);
-        for (int c = 0; c < CHUNKS; ++c) tma_load_2d(dst + c * kChunkBytes, map, bar, x + 64 * c, y);
+        mbar_arrive_expect_tx(tail, chunks * kChunkBytes);
+        for (int c = 0; c < chunks; ++c) tma_load_2d(dst + c * kChunkBytes, map, tail, x + 64 * c, y);
     }
     __syncwarp();
-    if (!clear) return true;
-    const uint32_t ph = tail_phase;
-    tail_phase ^= 1;
-    return finish_tail_tile(dst, CHUNKS, full, tail, ph, valid, abort);
+    return finish_tail_tile(dst, chunks, full, tail, tail_phase, valid, abort);
 }
 
 // -------------------------------------------------------------- tcgen05 ---

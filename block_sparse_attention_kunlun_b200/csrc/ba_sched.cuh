@@ -81,6 +81,7 @@ struct ItemSource {
 
     __device__ __forceinline__ void decode(uint32_t n, const int4 &info, const int2 &oth, TileRef &r) const
     {
+        r.b = info.w;
         r.h = int32_t(n % heads);
         r.s0 = info.x;
         r.L = info.y;
@@ -143,12 +144,55 @@ struct ItemSink {
         if ((threadIdx.x & 31) == 0) mbar_arrive(&q.empty[slot]);
         ++taken;
         if (it.w < 0) return false;
+        r.b = -1; // not carried by the ring (no consumer of these kernels reads it)
         r.s0 = it.x;
         r.L = it.y;
         r.t = it.z;
         r.h = it.w;
         r.os0 = ot.x;
         r.oL = ot.y;
+        return true;
+    }
+};
+
+// Static dealing for kernels where the ring's extra code costs more than the
+// balance gains (measured: the dK/dV pass, whose instruction footprint is at
+// the edge of the instruction cache): CTA c takes items c, c + grid, ... in
+// table order; each role walks the same sequence itself (same interface as
+// ItemSink / ItemSource, ring unused).
+struct StaticItems {
+    const int4 *table;
+    const int32_t *other;
+    uint32_t total, heads, n;
+    int4 next;
+    __device__ __forceinline__ StaticItems(const int4 *t, int32_t entries, int32_t h, const int32_t *other_offsets)
+        : table(t), other(other_offsets), total(uint32_t(entries) * uint32_t(h)), heads(uint32_t(h)), n(blockIdx.x),
+          next()
+    {
+        if (n < total) next = table[n / heads];
+    }
+    __device__ __forceinline__ bool peek(TileRef &r) const
+    {
+        if (n >= total) return false;
+        r.b = next.w;
+        r.h = int32_t(n % heads);
+        r.s0 = next.x;
+        r.L = next.y;
+        r.t = next.z;
+        if (other) {
+            r.os0 = other[next.w];
+            r.oL = other[next.w + 1] - r.os0;
+        } else {
+            r.os0 = r.s0;
+            r.oL = r.L;
+        }
+        return true;
+    }
+    __device__ __forceinline__ bool advance(TileRef &r, ItemRing &, volatile int *, bool &)
+    {
+        if (!peek(r)) return false;
+        n += gridDim.x;
+        if (n < total) next = table[n / heads];
         return true;
     }
 };

@@ -93,7 +93,11 @@ typedef struct {
  * problem): a status word and a work table of about 16 bytes per 128-row
  * tile, plus, for the backward, two float32 per-row buffers [heads,
  * total_tokens]: the row dot product Delta = dO . out and (bf16) the
- * forward's lse in the form the dK/dV pass reads.
+ * forward's lse in the form the dK/dV pass reads, and (bf16) 128 rows of q
+ * and 128 of dout per example, 2 * batch * 128 * heads * head_dim bf16
+ * values in all: each example's last query tile, when partial, staged with
+ * zeros past the example's end for the key-side gradient pass. A batch of
+ * more than 2^31 / 128 examples is BA_ERR_UNSUPPORTED.
  */
 size_t ba_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window);
 size_t ba_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window);
@@ -134,7 +138,9 @@ ba_status ba_bwd(const ba_problem *p, const void *q, const void *k, const void *
  * writes the exact gradients dq, dk, dv of sum(out * dout).
  *  - BF16 only (BA_ERR_UNSUPPORTED for BA_F32); head_dim 64 or 128; no skip
  *    flags. Same tensor layouts, ownership and errors as ba_fwd / ba_bwd.
- *  - Workspace: ba_gdpa_workspace_size bytes, for either direction.
+ *  - Workspace: ba_gdpa_workspace_size bytes, for either direction (the
+ *    backward's size, which includes the staged query tiles described at
+ *    ba_bwd_workspace_size).
  *  - act outside the enumeration: BA_ERR_INVALID_ARG.
  */
 typedef enum { BA_ACT_GELU = 1, BA_ACT_SILU = 2 } ba_activation;
@@ -164,7 +170,8 @@ ba_status ba_gdpa_bwd(const ba_problem *p, ba_activation act, const void *q, con
  *    offset arrays are DEVICE int32 [batch + 1], non-decreasing from 0.
  *  - q, out, dout, dq: DEVICE [total_tokens, heads, head_dim]; k, v, dk, dv:
  *    DEVICE [kv_total_tokens, heads, head_dim]; 16-byte aligned.
- *  - Workspace: ba_gdpa_cross_workspace_size bytes, for either direction.
+ *  - Workspace: ba_gdpa_cross_workspace_size bytes, for either direction
+ *    (it includes 128 staged rows of q and of dout per example).
  *  - Errors as for ba_gdpa_fwd / ba_gdpa_bwd.
  */
 size_t ba_gdpa_cross_workspace_size(const ba_problem *p, int32_t kv_total_tokens);

@@ -30,7 +30,7 @@ int main(void)
     void *fake = (void *)(uintptr_t)(1u << 20);
     ba_problem p;
     ba_rope rope;
-    size_t f, b, rf, rb;
+    size_t f, b, rf, rb, staged;
 
     CHECK(strcmp(ba_status_string(BA_OK), "ok") == 0);
     CHECK(strcmp(ba_status_string(BA_ERR_TIMEOUT), "device wait timed out") == 0);
@@ -44,8 +44,10 @@ int main(void)
     f = ba_fwd_workspace_size(&p, 128, 2);
     b = ba_bwd_workspace_size(&p, 128, 2);
     CHECK(f > 0 && f % 256 == 0 && b > f);
-    /* the backward adds two float per-row buffers [heads, total_tokens] */
-    CHECK(b == f + 2 * align256(4u * 2 * 1000));
+    /* the backward adds two float per-row buffers [heads, total_tokens] and
+       (bf16) 128 staged rows of q and of dout per example */
+    staged = 2 * align256((size_t)3 * 128 * 2 * 128 * 2);
+    CHECK(b == f + 2 * align256(4u * 2 * 1000) + staged);
     /* the rotary forms add two rotated copies of a [T, H, D] bf16 tensor */
     rf = ba_rope_fwd_workspace_size(&p, 128, 2);
     rb = ba_rope_bwd_workspace_size(&p, 128, 2);
@@ -83,7 +85,7 @@ int main(void)
           BA_ERR_INVALID_ARG); /* the plain workspace has no room for the rotated copies */
 
     CHECK(ba_selftest_wait_timeout(NULL, 256, 1000, NULL) == BA_ERR_INVALID_ARG);
-    CHECK(ba_gdpa_workspace_size(&p, 128, 2) == f);
+    CHECK(ba_gdpa_workspace_size(&p, 128, 2) == f + staged);
     CHECK(ba_gdpa_fwd(&p, (ba_activation)7, fake, fake, fake, fake, 128, 2, fake, fake, f, NULL) ==
           BA_ERR_INVALID_ARG); /* not an activation */
     CHECK(ba_gdpa_fwd(&p, BA_ACT_GELU, fake, fake, fake, fake, 128, 2, fake, fake, 16, NULL) ==

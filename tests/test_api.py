@@ -43,8 +43,16 @@ def test_workspace_sizes():
     f = ba.ba_fwd_workspace_size(p, 128, 2)
     b = ba.ba_bwd_workspace_size(p, 128, 2)
     assert f >= 256 + 4 * 4 and f % 256 == 0
-    # backward adds two per-row float buffers (Delta and lse for the dK/dV pass), H*T floats each
-    assert f + 2 * 4 * 2 * 1000 <= b <= f + 2 * 4 * 2 * 1000 + 512
+    # backward adds two per-row float buffers (Delta and lse for the dK/dV pass), H*T floats each,
+    # and (bf16) 128 staged rows of q and of dout per example
+    staged = 2 * 3 * 128 * 2 * 128 * 2
+    assert f + 2 * 4 * 2 * 1000 + staged <= b <= f + 2 * 4 * 2 * 1000 + staged + 1024
+    # float32 has no staged rows
+    p32 = prob(batch=3, T=1000, H=2, D=64, dt=ba.BA_F32)
+    f32, b32 = ba.ba_fwd_workspace_size(p32, 128, 2), ba.ba_bwd_workspace_size(p32, 128, 2)
+    assert f32 + 2 * 4 * 2 * 1000 <= b32 <= f32 + 2 * 4 * 2 * 1000 + 512
+    # the generalized attention's workspace (either direction) is the backward's
+    assert ba.ba_gdpa_workspace_size(p, 128, 2) == f + staged
     # the work table grows with the number of 128-row tiles
     assert ba.ba_fwd_workspace_size(prob(batch=3, T=100000, H=2, D=128), 128, 2) >= 16 * (100000 // 128)
     assert ba.ba_fwd_workspace_size(prob(batch=-1), 128, 2) == 0
