@@ -70,6 +70,8 @@ def parse(argv=None):
     ap.add_argument("--gdpa", choices=["gelu", "silu"], default=None,
                     help="generalized dot-product attention (ba_gdpa_fwd / ba_gdpa_bwd): the activation "
                          "in place of the softmax, same block rule and shapes")
+    ap.add_argument("--mx", action="store_true",
+                    help="MXFP8 Q and K in the score product (ba_mx_fwd / ba_mx_bwd), head_dim 128")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-configs", action="store_true",
@@ -132,6 +134,10 @@ def config_workload(args):
         w = w.replace(block=b, window=win, name=re.sub(r"block \d+, window \d+", f"block {b}, window {win}", w.name))
     if getattr(args, "rope", False):
         w = w.replace(name=w.name + ", rotary q/k")
+    if getattr(args, "mx", False):
+        if getattr(args, "rope", False) or getattr(args, "gdpa", None):
+            raise SystemExit("--mx takes neither --rope nor --gdpa")
+        w = w.replace(name=w.name + ", MXFP8 Q/K")
     if getattr(args, "gdpa", None):
         if w.skip_p > 0:
             raise SystemExit("--gdpa takes no skip flags: pick a workload without component skip")
@@ -276,6 +282,11 @@ def run_reference(args):
             gdpa.fwd(sub, q, k, v, w.block, w.window, args.gdpa)
             gdpa.bwd(sub, q, k, v, do, w.block, w.window, args.gdpa)
             return
+        if args.mx:
+            from oracle import mx
+            mx.fwd(sub, q, k, v, w.block, w.window, nthreads=threads)
+            mx.bwd(sub, q, k, v, do, w.block, w.window, nthreads=threads)
+            return
         if args.rope:
             oracle.rope_fwd(sub, q, k, v, c, s, w.block, w.window, nthreads=threads)
             oracle.rope_bwd(sub, q, k, v, do, c, s, w.block, w.window, nthreads=threads)
@@ -322,8 +333,8 @@ class Runner:
     """Device buffers and one training step (ba_fwd + ba_bwd, or the rotary
     entry points) of one workload through the library's public API."""
 
-    def __init__(self, ba, w, inp, dev, rope=False, gdpa=None):
-        self.ba, self.w, self.inp, self.dev, self.rope, self.gdpa = ba, w, inp, dev, rope, gdpa
+    def __init__(self, ba, w, inp, dev, rope=False, gdpa=None, mx=False):
+        self.ba, self.w, self.inp, self.dev, self.rope, self.gdpa, self.mx = ba, w, inp, dev, rope, gdpa, mx
         self.lens = inp["lengths"].numpy()
         self.skip_np = inp["skip"].numpy() if inp["skip"] is not None else None
         T, H, D = inp["q"].shape
@@ -344,15 +355,19 @@ class Runner:
             self.cos_d, self.sin_d = (t.to(dev) for t in self.tables)
             self.q_rot, self.k_rot = torch.empty_like(self.q), torch.empty_like(self.k)
             self.rope_arg = ba.make_rope(self.cos_d, self.sin_d, self.q_rot, self.k_rot)
-        size_f = (ba.ba_gdpa_workspace_size if gdpa else ba.ba_fwd_workspace_size)(self.prob, w.block, w.window)
+        size_f = (ba.ba_gdpa_workspace_size if gdpa else ba.ba_mx_fwd_workspace_size if mx
+                  else ba.ba_fwd_workspace_size)(self.prob, w.block, w.window)
+        size_b = (ba.ba_mx_bwd_workspace_size if mx else ba.ba_bwd_workspace_size)(self.prob, w.block, w.window)
         self.ws_f = ba.workspace_for(size_f, dev)
-        self.ws_b = ba.workspace_for(ba.ba_bwd_workspace_size(self.prob, w.block, w.window), dev)
+        self.ws_b = ba.workspace_for(size_b, dev)
         # ba_fwd: work list, (skip), attention; ba_bwd: work list, (skip), staging of the partial query
         # tiles, dQ, dK/dV; the rotary forward adds one rotation pass (the backward reads the kept
         # rotated copies)
         self.launches_per_step = (2 + (self.skip is not None)) + (4 + (self.skip is not None)) + (1 if rope else 0)
         if gdpa:
             self.launches_per_step = 6  # work list + forward; work list + staging + dQ + dK/dV
+        if mx:  # two quantisation passes in the forward, two round trips in the backward
+            self.launches_per_step += 4
 
     def step(self):
         ba, w, s = self.ba, self.w, self
@@ -365,6 +380,16 @@ class Runner:
                                 s.dv, s.ws_f, stream=s.stream)
             if st != ba.BA_OK:
                 raise ba.BAError(st, "ba_gdpa_bwd")
+            return
+        if s.mx:
+            st = ba.ba_mx_fwd(s.prob, s.q, s.k, s.v, s.offs, w.block, w.window, s.skip, s.out, s.lse, s.ws_f,
+                              stream=s.stream)
+            if st != ba.BA_OK:
+                raise ba.BAError(st, "ba_mx_fwd")
+            st = ba.ba_mx_bwd(s.prob, s.q, s.k, s.v, s.out, s.lse, s.dout, s.offs, w.block, w.window, s.skip,
+                              s.dq, s.dk, s.dv, s.ws_b, stream=s.stream)
+            if st != ba.BA_OK:
+                raise ba.BAError(st, "ba_mx_bwd")
             return
         if s.rope:
             st = ba.ba_rope_fwd(s.prob, s.rope_arg, s.q, s.k, s.v, s.offs, w.block, w.window, s.skip, s.out,
@@ -486,7 +511,7 @@ def main(argv=None, runner_cls=None):
             dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=300))
 
     w, inp = workload(args, rank)
-    run = (runner_cls or Runner)(ba, w, inp, dev, rope=args.rope, gdpa=args.gdpa)
+    run = (runner_cls or Runner)(ba, w, inp, dev, rope=args.rope, gdpa=args.gdpa, mx=args.mx)
     T, H, D = run.T, run.H, run.D
     fl, by = run.flops, run.bytes
 
@@ -596,6 +621,7 @@ def main(argv=None, runner_cls=None):
                                                             if (args.swa or args.block or args.window) else "")
         key += ":rope" if args.rope else ""
         key += f":gdpa-{args.gdpa}" if args.gdpa else ""
+        key += ":mx" if args.mx else ""
         if key in tr and tr[key].get("kernel_sha") == kernel_sha(dom):
             traffic = tr[key]["bytes_per_launch"]
     except (OSError, ValueError):
@@ -622,6 +648,7 @@ def main(argv=None, runner_cls=None):
         "config": {"workload": w.name, "batch": int(len(run.lens)), "total_tokens": int(T), "heads": H,
                    "head_dim": D, "block": w.block, "window": w.window, "seed": w.seed,
                    "rotary": bool(args.rope), "attention": f"gdpa-{args.gdpa}" if args.gdpa else "softmax",
+                   "score_operands": "MXFP8 (E4M3, E8M0 per 32)" if args.mx else "bf16",
                    "visible_pairs_per_head": run.pairs, "useful_flops_per_step": fl["step"],
                    "l2": f"inputs larger than L2 ({by['fwd'] + by['bwd']:.3g} B touched per step), no flush",
                    "parallelism": f"dp{world} (independent batches, no collective in the step)"},
@@ -635,13 +662,13 @@ def main(argv=None, runner_cls=None):
     }
     pairs, lens = run.pairs, run.lens
     if world == 1 and on_gpu and not args.examples and not args.no_other_configs and \
-            not (args.swa or args.block or args.window or args.rope or args.gdpa):
+            not (args.swa or args.block or args.window or args.rope or args.gdpa or args.mx):
         del run
         torch.cuda.empty_cache()
         Ko = max(5, min(K, 20))
         line["other_configs"] = {f"config{c}": other_config_line(ba, c, dev, Ko, max(3, args.warmup), local)
                                  for c in (4, 5) if c != args.config}
-    if not args.no_cpu_baseline and world == 1 and on_gpu and not args.gdpa:
+    if not args.no_cpu_baseline and world == 1 and on_gpu and not args.gdpa and not args.mx:
         line["cpu_baseline"] = cpu_baseline(w, inp, pairs, tables=tables_for(lens, D) if args.rope else None)
     print(json.dumps(line), flush=True)
     if dist is not None:

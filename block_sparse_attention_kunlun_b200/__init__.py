@@ -29,6 +29,7 @@ __all__ = [
     "ba_gdpa_workspace_size", "ba_gdpa_fwd", "ba_gdpa_bwd", "gdpa_fwd", "gdpa_bwd",
     "ba_gdpa_cross_workspace_size", "ba_gdpa_cross_fwd", "ba_gdpa_cross_bwd", "gdpa_cross_fwd", "gdpa_cross_bwd",
     "ba_mx_quantize", "ba_mx_fwd_workspace_size", "ba_mx_fwd", "mx_quantize", "mx_block_attention_fwd",
+    "ba_mx_bwd_workspace_size", "ba_mx_bwd", "mx_block_attention_bwd",
     "library_path",
 ]
 
@@ -123,6 +124,10 @@ def _load():
     lib.ba_mx_fwd_workspace_size.restype = ctypes.c_size_t
     lib.ba_mx_fwd.argtypes = [prob, P, P, P, P, i32, i32, P, P, P, P, ctypes.c_size_t, P]
     lib.ba_mx_fwd.restype = ctypes.c_int
+    lib.ba_mx_bwd_workspace_size.argtypes = [prob, i32, i32]
+    lib.ba_mx_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.ba_mx_bwd.argtypes = [prob, P, P, P, P, P, P, P, i32, i32, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.ba_mx_bwd.restype = ctypes.c_int
     rope = ctypes.POINTER(BARope)
     lib.ba_rope_fwd_workspace_size.argtypes = [prob, i32, i32]
     lib.ba_rope_fwd_workspace_size.restype = ctypes.c_size_t
@@ -421,6 +426,39 @@ def mx_block_attention_fwd(q, k, v, seq_offsets, block, window, skip=None, out=N
     if st != BA_OK:
         raise BAError(st, "ba_mx_fwd")
     return out, lse
+
+
+def ba_mx_bwd_workspace_size(problem: BAProblem, block: int, window: int) -> int:
+    return int(_load().ba_mx_bwd_workspace_size(ctypes.byref(problem), int(block), int(window)))
+
+
+def ba_mx_bwd(problem, q, k, v, out, lse, dout, seq_offsets, block, window, skip, dq, dk, dv,
+              workspace, workspace_bytes=None, stream=None) -> int:
+    """Direct call of the MXFP8-operand backward; returns its status code."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(_load().ba_mx_bwd(ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                 _ptr(dout), _ptr(seq_offsets), int(block), int(window), _ptr(skip),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), int(workspace_bytes),
+                                 _stream(stream)))
+
+
+def mx_block_attention_bwd(q, k, v, out, lse, dout, seq_offsets, block, window, skip=None,
+                           dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """The backward of mx_block_attention_fwd (ba_mx_bwd); allocates dq/dk/dv
+    (and a workspace) with torch."""
+    _check_inputs(q, k, v, seq_offsets)
+    prob = make_problem(q, seq_offsets)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if workspace is None:
+        workspace = workspace_for(ba_mx_bwd_workspace_size(prob, block, window), q.device)
+    st = ba_mx_bwd(prob, q, k, v, out, lse, dout, seq_offsets, block, window, skip, dq, dk, dv, workspace,
+                   stream=stream)
+    if st != BA_OK:
+        raise BAError(st, "ba_mx_bwd")
+    return dq, dk, dv
 
 
 def make_rope(cos, sin, q_rot=None, k_rot=None) -> BARope:

@@ -563,6 +563,44 @@ ba_status mx_fwd_impl(const ba_problem *pp, const void *q, const void *k, const 
     return BA_OK;
 }
 
+// ba_mx_bwd: the bf16 backward on the MX round trips of q and k (the
+// operands the MXFP8 forward's score product used), kept in the workspace
+// after the backward's own regions (so that the status word stays first).
+size_t mx_bwd_operand_bytes(const ba_problem &P)
+{
+    return align256(size_t(P.total_tokens) * size_t(P.heads) * size_t(P.head_dim) * 2);
+}
+
+ba_status mx_bwd_impl(const ba_problem *pp, const void *q, const void *k, const void *v, const void *out,
+                      const float *lse, const void *dout, const int32_t *seq_offsets, int32_t block, int32_t window,
+                      const uint8_t *skip, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                      ba_stream_t stream_)
+{
+    ba_status st = check_problem(pp, block, window);
+    if (st != BA_OK) return st;
+    const ba_problem &P = *pp;
+    const int64_t T = P.total_tokens;
+    if (!seq_offsets || !aligned(seq_offsets, 4) || !tensor_ok(q, T) || !tensor_ok(k, T) || !tensor_ok(v, T) ||
+        !tensor_ok(out, T) || !tensor_ok(dout, T) || !tensor_ok(dq, T) || !tensor_ok(dk, T) || !tensor_ok(dv, T) ||
+        (T > 0 && (!lse || !aligned(lse, 4))))
+        return BA_ERR_INVALID_ARG;
+    if (P.dtype != BA_BF16 || P.head_dim != 128) return BA_ERR_UNSUPPORTED;
+    const size_t rt = mx_bwd_operand_bytes(P);
+    const size_t base = workspace_layout(P.batch, T, P.heads, P.head_dim, true, true).total;
+    const size_t need = base + 2 * rt;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return BA_ERR_INVALID_ARG;
+    int num_sms = 0, cc = 0;
+    if (!device_info(num_sms, cc)) return BA_ERR_CUDA;
+    if (cc != 10) return BA_ERR_UNSUPPORTED;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    uint8_t *qr = static_cast<uint8_t *>(workspace) + base, *kr = qr + rt;
+    const int64_t elems = T * P.heads * P.head_dim;
+    BA_TRY(launch_mx_round_trip(q, elems, qr, num_sms, stream));
+    BA_TRY(launch_mx_round_trip(k, elems, kr, num_sms, stream));
+    return bwd_impl(pp, nullptr, qr, kr, v, out, lse, dout, seq_offsets, block, window, skip, dq, dk, dv, workspace,
+                    workspace_bytes, stream_, false);
+}
+
 } // namespace
 
 extern "C" {
@@ -724,6 +762,22 @@ ba_status ba_mx_fwd(const ba_problem *p, const void *q, const void *k, const voi
                     size_t workspace_bytes, ba_stream_t stream)
 {
     return mx_fwd_impl(p, q, k, v, seq_offsets, block, window, skip, out, lse, workspace, workspace_bytes, stream);
+}
+
+size_t ba_mx_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
+{
+    if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
+    return 2 * mx_bwd_operand_bytes(*p) +
+           workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, true, p->dtype == BA_BF16).total;
+}
+
+ba_status ba_mx_bwd(const ba_problem *p, const void *q, const void *k, const void *v, const void *out,
+                    const float *lse, const void *dout, const int32_t *seq_offsets, int32_t block, int32_t window,
+                    const uint8_t *skip, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                    ba_stream_t stream)
+{
+    return mx_bwd_impl(p, q, k, v, out, lse, dout, seq_offsets, block, window, skip, dq, dk, dv, workspace,
+                       workspace_bytes, stream);
 }
 
 ba_status ba_device_status(const void *workspace, ba_stream_t stream_)

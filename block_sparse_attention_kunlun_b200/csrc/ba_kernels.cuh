@@ -39,6 +39,8 @@ cudaError_t launch_rope_rows(const Problem &p, size_t elem_bytes, bool transpose
 // [rows, heads, head_dim] bf16 tensor; scales [rows, heads rounded up to 4, head_dim / 32].
 cudaError_t launch_mx_quantize(const void *x, int64_t rows, int32_t heads, int32_t head_dim, void *elems,
                                void *scales, int num_sms, cudaStream_t stream);
+// The same quantisation followed by dequantisation, bf16 to bf16 (elems a multiple of 32).
+cudaError_t launch_mx_round_trip(const void *x, int64_t elems, void *y, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_fwd_f32(const Problem &p, const float *q, const float *k, const float *v, float *out, float *lse,
                            int num_sms, cudaStream_t stream);

@@ -214,6 +214,28 @@ ba_status ba_mx_fwd(const ba_problem *p, const void *q, const void *k, const voi
                     size_t workspace_bytes, ba_stream_t stream);
 
 /*
+ * ba_mx_bwd: the backward of ba_mx_fwd (the pages say GEM's training uses
+ * MXFP8 in forward and backward). Reading: the score product is recomputed
+ * from the same MXFP8 Q and K as the forward, and the gradient passes
+ * through the quantisation unchanged (its derivative taken as the identity),
+ * so dq and dk are the gradients with respect to the dequantised q and k and
+ * dv is the usual P^T dout. It writes the MX round trips of q and k (quantise,
+ * then dequantise; exact in bf16 unless a block's largest magnitude is below
+ * 2^-118) into its workspace and runs ba_bwd's kernels on them, so the
+ * backward's products are bf16 MMAs of the dequantised values: the same
+ * products, summed in another order, as the forward's block-scaled MMA.
+ * Arguments, layouts, outputs and errors as ba_bwd; out and lse come from
+ * ba_mx_fwd. BF16 with head_dim 128 only (BA_ERR_UNSUPPORTED otherwise).
+ * Workspace: ba_mx_bwd_workspace_size bytes (ba_bwd_workspace_size plus two
+ * bf16 [total_tokens, heads, head_dim] copies); ba_device_status reads it.
+ */
+size_t ba_mx_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window);
+ba_status ba_mx_bwd(const ba_problem *p, const void *q, const void *k, const void *v, const void *out,
+                    const float *lse, const void *dout, const int32_t *seq_offsets, int32_t block, int32_t window,
+                    const uint8_t *skip, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                    ba_stream_t stream);
+
+/*
  * Token-granular sliding-window attention, the predecessor that block
  * attention replaced ("GEM (Meta)", section "Custom kernels": long
  * user-history self-attention first moved to a sliding window, then to

@@ -20,8 +20,13 @@ here from its definition:
 Reading for attention (the plainest one the sentence supports): the
 operands of the score product Q K^T are MXFP8, blocked along head_dim, the
 contraction of that product. The softmax and P V are unchanged, so the
-result is block attention of the dequantised Q and K. Everything else is
-the fp64 oracle of oracle/oracle.c. Pins: tests/test_oracle_mx.py.
+result is block attention of the dequantised Q and K. The backward, which
+the same sentence puts in MXFP8 too, recomputes the scores from the same
+MXFP8 Q and K and passes the gradient through the quantisation unchanged
+(its derivative taken as the identity, the usual reading for training
+through a rounding step): dq and dk are the gradients with respect to the
+dequantised operands. Everything else is the fp64 oracle of
+oracle/oracle.c. Pins: tests/test_oracle_mx.py.
 """
 from __future__ import annotations
 
@@ -85,4 +90,12 @@ def fwd(seq_offsets, q, k, v, block, window, fmt="e4m3", skip=None, nthreads=Non
     """Block attention with Q and K as MXFP8 operands (blocks of 32 along
     head_dim). Returns (out, lse) like oracle.fwd."""
     return oracle.fwd(seq_offsets, mx_round(q, fmt), mx_round(k, fmt), v, block, window, skip=skip,
+                      nthreads=nthreads)
+
+
+def bwd(seq_offsets, q, k, v, dout, block, window, fmt="e4m3", skip=None, nthreads=None):
+    """Backward of fwd: the gradients of block attention of the dequantised
+    Q and K, taken with respect to those dequantised operands (the rounding
+    passed through unchanged). Returns (dq, dk, dv) like oracle.bwd."""
+    return oracle.bwd(seq_offsets, mx_round(q, fmt), mx_round(k, fmt), v, dout, block, window, skip=skip,
                       nthreads=nthreads)

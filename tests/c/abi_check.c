@@ -103,6 +103,12 @@ int main(void)
     CHECK(ba_mx_fwd_workspace_size(&p, 128, 2) > f);
     CHECK(ba_mx_fwd(&p, fake, fake, fake, fake, 128, 2, NULL, fake, fake, fake, f, NULL) ==
           BA_ERR_INVALID_ARG); /* the plain workspace has no room for the MXFP8 operands */
+    /* the MXFP8 backward: the backward's workspace plus two bf16 round-trip copies of q and k */
+    CHECK(ba_mx_bwd_workspace_size(&p, 128, 2) == b + 2 * align256((size_t)1000 * 2 * 128 * 2));
+    CHECK(ba_mx_bwd(&p, fake, fake, fake, fake, (const float *)fake, fake, fake, 128, 2, NULL, fake, fake, fake,
+                    fake, b, NULL) == BA_ERR_INVALID_ARG); /* the plain backward's workspace is too small */
+    CHECK(ba_mx_bwd(&p, fake, fake, fake, fake, NULL, fake, fake, 128, 2, NULL, fake, fake, fake, fake, 1u << 30,
+                    NULL) == BA_ERR_INVALID_ARG); /* no lse */
     CHECK(ba_selftest_exp2(NULL, NULL, 5, NULL) == BA_ERR_INVALID_ARG);
     CHECK(ba_selftest_exp2((const float *)fake, (float *)fake, -1, NULL) == BA_ERR_INVALID_ARG);
     CHECK(ba_selftest_exp2(NULL, NULL, 0, NULL) == BA_OK); /* nothing to do, nothing launched */

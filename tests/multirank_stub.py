@@ -16,7 +16,7 @@ from block_sparse_attention_kunlun_b200 import flops as F  # noqa: E402
 
 
 class StubRunner:
-    def __init__(self, ba, w, inp, dev, rope=False, gdpa=None):
+    def __init__(self, ba, w, inp, dev, rope=False, gdpa=None, mx=False):
         self.w, self.inp = w, inp
         self.lens = inp["lengths"].numpy()
         self.skip_np = inp["skip"].numpy() if inp["skip"] is not None else None

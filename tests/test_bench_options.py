@@ -93,3 +93,16 @@ def test_gdpa_option_names_the_activation_and_refuses_skip_flags():
     a.config = 5
     with pytest.raises(SystemExit):
         b.config_workload(a)
+
+
+def test_mx_option_names_the_operands_and_refuses_rope_and_gdpa():
+    import pytest
+    b = _bench()
+    a = Args()
+    a.mx = True
+    w = b.config_workload(a)
+    assert w.name.endswith(", MXFP8 Q/K") and w.head_dim == 128
+    a.rope = True
+    with pytest.raises(SystemExit):
+        b.config_workload(a)
+    assert b.parse(["--mx"]).mx and not b.parse([]).mx

@@ -155,3 +155,47 @@ def test_attention_on_mx_representable_operands_is_plain_attention():
     out_mx, _ = mx.fwd(offs, q2, k, v, 16, 2)
     out, _ = oracle.fwd(offs, q2, k, v, 16, 2)
     assert 0 < np.max(np.abs(out_mx - out)) < 0.1
+
+
+def test_mx_backward_on_mx_representable_operands_is_plain_backward():
+    rng = np.random.default_rng(806)
+    offs = np.array([0, 40, 40, 77], dtype=np.int32)
+    H, D = 2, 64
+    q = mx.mx_round(rng.standard_normal((77, H, D)) * 2.0)
+    k = mx.mx_round(rng.standard_normal((77, H, D)))
+    v, do = rng.standard_normal((77, H, D)), rng.standard_normal((77, H, D))
+    for x, y in zip(mx.bwd(offs, q, k, v, do, 16, 2), oracle.bwd(offs, q, k, v, do, 16, 2)):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_mx_backward_is_straight_through_autograd():
+    """The backward against PyTorch autograd of masked attention whose q and k
+    pass through the MX round trip in the forward and straight through it in
+    the backward (x + (round(x) - x).detach()), fp64, per example."""
+    rng = np.random.default_rng(807)
+    block, window, H, D = 8, 2, 2, 64
+    offs = np.array([0, 23, 23, 60], dtype=np.int32)
+    T = int(offs[-1])
+    q, k = rng.standard_normal((T, H, D)) * 1.5, rng.standard_normal((T, H, D))
+    v, do = rng.standard_normal((T, H, D)), rng.standard_normal((T, H, D))
+    dq, dk, dv = mx.bwd(offs, q, k, v, do, block, window)
+    plain = oracle.bwd(offs, q, k, v, do, block, window)
+    assert np.max(np.abs(dq - plain[0])) > 1e-6  # the rounding is not skipped
+    for e in range(len(offs) - 1):
+        s0, s1 = int(offs[e]), int(offs[e + 1])
+        L = s1 - s0
+        if L == 0:
+            continue
+        i = torch.arange(L)[:, None]
+        j = torch.arange(L)[None, :]
+        mask = (j <= i) & (j // block >= i // block - (window - 1))
+        tq, tk, tv = (torch.tensor(x[s0:s1].transpose(1, 0, 2), dtype=torch.float64, requires_grad=True)
+                      for x in (q, k, v))
+        rq = torch.tensor(mx.mx_round(q[s0:s1]).transpose(1, 0, 2))
+        rk = torch.tensor(mx.mx_round(k[s0:s1]).transpose(1, 0, 2))
+        o = torch.nn.functional.scaled_dot_product_attention(tq + (rq - tq).detach(), tk + (rk - tk).detach(), tv,
+                                                             attn_mask=mask)
+        o.backward(torch.tensor(do[s0:s1].transpose(1, 0, 2)))
+        t = lambda x: x.detach().numpy().transpose(1, 0, 2)
+        for name, got, ref in (("dq", dq, tq.grad), ("dk", dk, tk.grad), ("dv", dv, tv.grad)):
+            np.testing.assert_allclose(got[s0:s1], t(ref), rtol=0, atol=1e-11, err_msg=f"{name} example {e}")
