@@ -417,8 +417,8 @@ __global__ void __launch_bounds__(448, 1)
                                                      sc2, make_float2(l4.x, l4.y));
                             const float2 x23 = ffma2(make_float2(__uint_as_float(cur[4 * c4 + 2]), __uint_as_float(cur[4 * c4 + 3])),
                                                      sc2, make_float2(l4.z, l4.w));
-                            // one value in four goes through the FMA pipe to offload the MUFU unit
-                            float ev[4] = {ex2_approx(x01.x), ex2_approx(x01.y), ex2_approx(x23.x), exp2_fma(x23.y)};
+                            // all on MUFU: these warps are bound by instruction issue (measured)
+                            float ev[4] = {ex2_approx(x01.x), ex2_approx(x01.y), ex2_approx(x23.x), ex2_approx(x23.y)};
                             if (!full) {
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
