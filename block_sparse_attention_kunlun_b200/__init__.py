@@ -23,7 +23,7 @@ __all__ = [
     "BAError", "ba_fwd", "ba_fwd_noalloc", "ba_bwd", "ba_fwd_workspace_size", "ba_bwd_workspace_size",
     "ba_swa_fwd", "ba_swa_bwd", "ba_swa_fwd_workspace_size", "ba_swa_bwd_workspace_size",
     "ba_rope_fwd", "ba_rope_bwd", "ba_rope_fwd_workspace_size", "ba_rope_bwd_workspace_size",
-    "ba_device_status", "ba_selftest_wait_timeout", "ba_selftest_exp2", "ba_set_profile_events", "ba_status_string", "ba_version",
+    "ba_device_status", "ba_selftest_wait_timeout", "ba_selftest_exp2", "ba_selftest_activation", "ba_set_profile_events", "ba_status_string", "ba_version",
     "block_attention_fwd", "block_attention_bwd", "sliding_window_attention_fwd", "sliding_window_attention_bwd",
     "rope_block_attention_fwd", "rope_block_attention_bwd",
     "ba_gdpa_workspace_size", "ba_gdpa_fwd", "ba_gdpa_bwd", "gdpa_fwd", "gdpa_bwd",
@@ -98,6 +98,8 @@ def _load():
     lib.ba_selftest_wait_timeout.restype = ctypes.c_int
     lib.ba_selftest_exp2.argtypes = [P, P, ctypes.c_int64, P]
     lib.ba_selftest_exp2.restype = ctypes.c_int
+    lib.ba_selftest_activation.argtypes = [ctypes.c_int, P, P, P, ctypes.c_int64, P]
+    lib.ba_selftest_activation.restype = ctypes.c_int
     lib.ba_swa_fwd_workspace_size.argtypes = [prob, i32]
     lib.ba_swa_fwd_workspace_size.restype = ctypes.c_size_t
     lib.ba_swa_bwd_workspace_size.argtypes = [prob, i32]
@@ -527,6 +529,15 @@ def ba_selftest_exp2(x, y, stream=None) -> int:
     if x.dtype != torch.float32 or y.dtype != torch.float32 or x.numel() != y.numel():
         raise ValueError("x and y must be float32 tensors of equal size")
     return int(_load().ba_selftest_exp2(_ptr(x), _ptr(y), int(x.numel()), _stream(stream)))
+
+
+def ba_selftest_activation(act, x, y, dy, stream=None) -> int:
+    """y = act(x), dy = act'(x) through the generalized attention's device
+    functions (act: BA_ACT_GELU or BA_ACT_SILU), float32 CUDA tensors of equal size."""
+    if any(t.dtype != torch.float32 or t.numel() != x.numel() for t in (x, y, dy)):
+        raise ValueError("x, y and dy must be float32 tensors of equal size")
+    return int(_load().ba_selftest_activation(int(act), _ptr(x), _ptr(y), _ptr(dy), int(x.numel()),
+                                              _stream(stream)))
 
 
 def ba_device_status(workspace, stream=None) -> int:

@@ -803,6 +803,17 @@ ba_status ba_selftest_wait_timeout(void *workspace, size_t workspace_bytes, int3
     return BA_OK;
 }
 
+ba_status ba_selftest_activation(ba_activation act, const float *x, float *y, float *dy, int64_t n,
+                                 ba_stream_t stream_)
+{
+    if (act != BA_ACT_GELU && act != BA_ACT_SILU) return BA_ERR_INVALID_ARG;
+    if (n < 0 || (n > 0 && (!x || !y || !dy || !aligned(x, 4) || !aligned(y, 4) || !aligned(dy, 4))))
+        return BA_ERR_INVALID_ARG;
+    BA_TRY(launch_activation_selftest(act == BA_ACT_GELU ? kGelu : kSilu, x, y, dy, n,
+                                      reinterpret_cast<cudaStream_t>(stream_)));
+    return BA_OK;
+}
+
 ba_status ba_selftest_exp2(const float *x, float *y, int64_t n, ba_stream_t stream_)
 {
     if (n < 0 || (n > 0 && (!x || !y || !aligned(x, 4) || !aligned(y, 4)))) return BA_ERR_INVALID_ARG;

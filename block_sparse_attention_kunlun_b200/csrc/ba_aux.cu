@@ -9,8 +9,10 @@
 //   wait_selftest_kernel  one warp waits on a barrier nothing completes, with a
 //                     short limit, through the same bounded wait the attention
 //                     kernels use, and reports the timeout in the status word
-//   exp2_selftest_kernel  the attention kernels' FMA-pipe 2^x on a caller's array
+//   exp2_selftest_kernel  the forward's FMA-pipe 2^x on a caller's array
 //                     (its accuracy is tested against 2^x computed on the host)
+//   activation_selftest_kernel  the generalized attention's GELU / SiLU and
+//                     their derivatives on a caller's array (tested likewise)
 //   skip_*_kernel     component skip: flagged examples pass v through
 //                     ("Meta Scales GEM Ads Model Across Platforms and
 //                     Thousands of GPUs", section "Kunlun changes how GEM
@@ -361,6 +363,32 @@ cudaError_t launch_exp2_selftest(const float *x, float *y, int64_t n, cudaStream
     if (n == 0) return cudaSuccess;
     const int64_t g = (n + 255) / 256;
     exp2_selftest_kernel<<<int(g < 4096 ? g : 4096), 256, 0, stream>>>(x, y, n);
+    return cudaGetLastError();
+}
+
+// The generalized attention's activation A on a caller's array: y = act(x)
+// and dy = act'(x) through the same device functions the kernels use.
+template <int A>
+__global__ void __launch_bounds__(256)
+    activation_selftest_kernel(const float *__restrict__ x, float *__restrict__ y, float *__restrict__ dy, int64_t n)
+{
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+        const float2 vg = act_value_grad<A>(x[i]);
+        // the kernels call all three forms; they must agree bit for bit
+        const bool same = __float_as_uint(vg.x) == __float_as_uint(act_value<A>(x[i])) &&
+                          __float_as_uint(vg.y) == __float_as_uint(act_grad<A>(x[i]));
+        y[i] = vg.x;
+        dy[i] = same ? vg.y : __int_as_float(0x7fc00000); // a disagreement shows as NaN
+    }
+}
+
+cudaError_t launch_activation_selftest(int act, const float *x, float *y, float *dy, int64_t n, cudaStream_t stream)
+{
+    if (n == 0) return cudaSuccess;
+    const int64_t g = (n + 255) / 256;
+    const int grid = int(g < 4096 ? g : 4096);
+    if (act == kGelu) activation_selftest_kernel<kGelu><<<grid, 256, 0, stream>>>(x, y, dy, n);
+    else activation_selftest_kernel<kSilu><<<grid, 256, 0, stream>>>(x, y, dy, n);
     return cudaGetLastError();
 }
 

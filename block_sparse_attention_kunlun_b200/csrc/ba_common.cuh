@@ -184,28 +184,68 @@ __device__ __forceinline__ void rope_transpose_bits(const Problem &p, int64_t po
 // so no running maximum and no lse.
 enum Act : int { kSoftmax = 0, kGelu = 1, kSilu = 2 };
 
-// GELU (exact form x Phi(x), Phi the standard normal distribution function)
-// and SiLU (x sigma(x)).
+// 2^x and 1/x on the special-function unit (ex2.approx / rcp.approx, relative
+// errors near 2^-22 and 2^-23; 2^-inf = 0 and 1/inf = 0). The attention's
+// warps are bound by instruction issue, so the activations below use one
+// instruction for each rather than the library's full-precision forms.
+__device__ __forceinline__ float act_ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float act_rcp(float x)
+{
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// GELU(x) = x Phi(x), Phi the standard normal distribution function, with
+// Phi from erf by Abramowitz & Stegun, Handbook of Mathematical Functions,
+// formula 7.1.26 (Hastings' approximation): for z >= 0,
+//   erf(z) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) e^(-z^2) + eps(z),
+//   t = 1 / (1 + p z), |eps(z)| <= 1.5e-7,
+// p = 0.3275911, a1..a5 = 0.254829592, -0.284496736, 1.421413741,
+// -1.453152027, 1.061405429. With z = |x| / sqrt(2), e^(-z^2) = e^(-x^2/2) is
+// also the exponential of the normal density phi, which GELU' = Phi + x phi
+// shares. Returns {Phi(x), e^(-x^2/2)}.
+__device__ __forceinline__ float2 gelu_parts(float x)
+{
+    const float z = fabsf(x) * 0.70710678118654752f;
+    const float t = act_rcp(fmaf(0.3275911f, z, 1.f));
+    const float poly =
+        t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f), -0.284496736f),
+                 0.254829592f);
+    const float e = act_ex2(x * x * -0.72134752044448170f); // e^(-x^2/2) = 2^(-x^2 / (2 ln 2))
+    const float tail = 0.5f * poly * e;                     // Phi(-|x|) = (1 - erf(z)) / 2
+    return make_float2(x >= 0.f ? 1.f - tail : tail, e);
+}
+
+// sigma(x) = 1 / (1 + 2^(-x log2 e)) for SiLU(x) = x sigma(x).
+__device__ __forceinline__ float silu_sigma(float x) { return act_rcp(1.f + act_ex2(x * -1.4426950408889634f)); }
+
+// The activation: GELU (the erf form above) or SiLU.
 template <int A>
 __device__ __forceinline__ float act_value(float x)
 {
     static_assert(A == kGelu || A == kSilu, "an activation");
-    if constexpr (A == kGelu) return 0.5f * x * (1.f + erff(x * 0.70710678118654752f));
-    else return x / (1.f + __expf(-x));
+    if constexpr (A == kGelu) return x * gelu_parts(x).x;
+    else return x * silu_sigma(x);
 }
 
-// The activation and its derivative: GELU' = Phi(x) + x phi(x) with phi the
-// standard normal density; SiLU' = sigma(x) (1 + x (1 - sigma(x))).
+// The activation and its derivative: GELU' = Phi(x) + x phi(x) with
+// phi(x) = e^(-x^2/2) / sqrt(2 pi); SiLU' = sigma(x) (1 + x (1 - sigma(x))).
 template <int A>
 __device__ __forceinline__ float2 act_value_grad(float x)
 {
     static_assert(A == kGelu || A == kSilu, "an activation");
     if constexpr (A == kGelu) {
-        const float cdf = 0.5f * (1.f + erff(x * 0.70710678118654752f));
-        const float pdf = 0.39894228040143268f * __expf(-0.5f * x * x);
-        return make_float2(x * cdf, fmaf(x, pdf, cdf));
+        const float2 g = gelu_parts(x);
+        return make_float2(x * g.x, fmaf(x, 0.39894228040143268f * g.y, g.x));
     } else {
-        const float sg = 1.f / (1.f + __expf(-x));
+        const float sg = silu_sigma(x);
         return make_float2(x * sg, sg * fmaf(x, 1.f - sg, 1.f));
     }
 }
@@ -216,10 +256,10 @@ __device__ __forceinline__ float act_grad(float x)
 {
     static_assert(A == kGelu || A == kSilu, "an activation");
     if constexpr (A == kGelu) {
-        const float cdf = 0.5f * (1.f + erff(x * 0.70710678118654752f));
-        return fmaf(x, 0.39894228040143268f * __expf(-0.5f * x * x), cdf);
+        const float2 g = gelu_parts(x);
+        return fmaf(x, 0.39894228040143268f * g.y, g.x);
     } else {
-        const float sg = 1.f / (1.f + __expf(-x));
+        const float sg = silu_sigma(x);
         return sg * fmaf(x, 1.f - sg, 1.f);
     }
 }

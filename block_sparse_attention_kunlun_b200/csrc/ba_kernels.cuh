@@ -20,6 +20,7 @@ cudaError_t launch_stage_query_tails(const int32_t *offs, const uint8_t *skip, i
                                      const void *a, const void *b, void *ta, void *tb, cudaStream_t stream);
 cudaError_t launch_wait_selftest(int *status, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_exp2_selftest(const float *x, float *y, int64_t n, cudaStream_t stream);
+cudaError_t launch_activation_selftest(int act, const float *x, float *y, float *dy, int64_t n, cudaStream_t stream);
 
 template <typename T>
 cudaError_t launch_bwd_pre(const Problem &p, const void *out, const void *dout, float *delta, int num_sms,

@@ -382,7 +382,7 @@ ba_status ba_selftest_wait_timeout(void *workspace, size_t workspace_bytes, int3
 /*
  * Self-test of the attention kernels' FMA-pipe 2^x (the pages have no
  * counterpart). To take load off the special-function unit, the softmax in
- * the bf16 kernels evaluates some of its exponentials on the fused
+ * the bf16 forward evaluates one exponential pair in eight on the fused
  * multiply-add pipe: x is split into the nearest integer n and f = x - n in
  * [-1/2, 1/2], 2^f comes from a cubic fitted to it (relative error below
  * 1e-4), and n is added to the exponent field; x below -125 is first raised
@@ -392,6 +392,21 @@ ba_status ba_selftest_wait_timeout(void *workspace, size_t workspace_bytes, int3
  * Returns BA_ERR_INVALID_ARG for n < 0 or null/misaligned pointers.
  */
 ba_status ba_selftest_exp2(const float *x, float *y, int64_t n, ba_stream_t stream);
+
+/*
+ * Self-test of the generalized attention's activations (ba_gdpa_*): writes
+ * y[i] = act(x[i]) and dy[i] = act'(x[i]) for the n DEVICE floats x (y, dy:
+ * DEVICE, n floats each, aliasing nothing), asynchronously on stream, through
+ * the device functions the kernels use. GELU's Phi comes from erf by
+ * Abramowitz & Stegun's formula 7.1.26 (absolute error at most 1.5e-7);
+ * e^(-x^2/2), 2^x and reciprocals come from the special-function unit.
+ * SiLU's sigma(x) = 1 / (1 + 2^(-x log2 e)) likewise. dy[i] is NaN if the
+ * kernels' three forms of the activation (value, derivative, both at once)
+ * disagree for x[i]. BA_ERR_INVALID_ARG for an unknown act, n < 0 or
+ * null/misaligned pointers.
+ */
+ba_status ba_selftest_activation(ba_activation act, const float *x, float *y, float *dy, int64_t n,
+                                 ba_stream_t stream);
 
 /*
  * Profiling hook. Until changed, calls made from THIS host thread record

@@ -112,6 +112,10 @@ int main(void)
     CHECK(ba_selftest_exp2(NULL, NULL, 5, NULL) == BA_ERR_INVALID_ARG);
     CHECK(ba_selftest_exp2((const float *)fake, (float *)fake, -1, NULL) == BA_ERR_INVALID_ARG);
     CHECK(ba_selftest_exp2(NULL, NULL, 0, NULL) == BA_OK); /* nothing to do, nothing launched */
+    CHECK(ba_selftest_activation((ba_activation)0, (const float *)fake, (float *)fake, (float *)fake, 4, NULL) ==
+          BA_ERR_INVALID_ARG); /* not an activation */
+    CHECK(ba_selftest_activation(BA_ACT_GELU, NULL, NULL, NULL, 4, NULL) == BA_ERR_INVALID_ARG);
+    CHECK(ba_selftest_activation(BA_ACT_SILU, NULL, NULL, NULL, 0, NULL) == BA_OK); /* nothing launched */
     CHECK(ba_set_profile_events(3, NULL, NULL) == BA_ERR_INVALID_ARG);
     CHECK(ba_device_status(NULL, NULL) == BA_ERR_INVALID_ARG);
 
