@@ -474,6 +474,22 @@ __global__ void __launch_bounds__(384, 1)
                 if (lane == 0) mbar_arrive(&sb.ds_full[g]);
             }
             if (!ok) break;
+            // rotary embedding: this row's cos / sin for the epilogue, read now so that they
+            // arrive while the next item's Q / dO go into TMEM
+            constexpr int kRopeVec = kRope ? D / 16 : 1; // float4s of the group's D / 4 pairs
+            float4 rcos[kRopeVec], rsin[kRopeVec];
+            const bool rope_in = !kRope || !valid || i < p.rope_rows;
+            if constexpr (kRope) {
+                if (valid && rope_in) {
+                    const float4 *cs = reinterpret_cast<const float4 *>(p.rope_cos + i * (D / 2) + (D / 4) * g);
+                    const float4 *sn = reinterpret_cast<const float4 *>(p.rope_sin + i * (D / 2) + (D / 4) * g);
+#pragma unroll
+                    for (int u = 0; u < kRopeVec; ++u) {
+                        rcos[u] = ld_nc_early(cs + u);
+                        rsin[u] = ld_nc_early(sn + u);
+                    }
+                }
+            }
             // the next item's Q / dO go into TMEM now: this item's last S and dP have completed
             TileRef rn;
             const bool have_next = items.advance(rn, sb.ring, abort, ok);
@@ -495,7 +511,23 @@ __global__ void __launch_bounds__(384, 1)
                     if (valid) {
                         // rotary embedding: the accumulator is the gradient of the rotated q; turn
                         // its 16 pairs back (transposed rotation at this row's position)
-                        if constexpr (kRope) rope_transpose_bits<4>(p, i, (D / 4) * g + 16 * c, a);
+                        if constexpr (kRope) {
+                            // this chunk's 16 pairs, picked with constant indices (the arrays stay in registers)
+                            float4 cc[4], ss[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                cc[u] = rcos[u];
+                                ss[u] = rsin[u];
+#pragma unroll
+                                for (int cq = 1; cq < D / 64; ++cq)
+                                    if (c == cq) {
+                                        cc[u] = rcos[4 * cq + u];
+                                        ss[u] = rsin[4 * cq + u];
+                                    }
+                            }
+                            if (rope_in) rope_transpose_loaded<4>(cc, ss, a);
+                            else if (c == 0) atomicOr(p.status, kStatusRopeRange); // past the tables
+                        }
                         uint4 *dst = reinterpret_cast<uint4 *>(qrow + 32 * c);
 #pragma unroll
                         for (int x = 0; x < 4; ++x)

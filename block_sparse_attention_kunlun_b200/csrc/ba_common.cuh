@@ -148,6 +148,35 @@ __device__ __forceinline__ float2 rope_pair_t(float g0, float g1, float c, float
     return make_float2(fmaf(g0, c, g1 * s), fmaf(g1, c, -g0 * s));
 }
 
+// 16 bytes of a read-only table, read through the non-coherent path with the
+// load kept where it is written (ahead of the code that waits for other work).
+__device__ __forceinline__ float4 ld_nc_early(const float4 *ptr)
+{
+    float4 v;
+    asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(ptr));
+    return v;
+}
+
+// Transposed rotation, in place, of 4 NQ adjacent pairs (bit patterns v[2m],
+// v[2m+1]) with their cos and sin already loaded (c[u], s[u]: pairs 4u .. 4u + 3).
+template <int NQ>
+__device__ __forceinline__ void rope_transpose_loaded(const float4 *c, const float4 *s, uint32_t *v)
+{
+#pragma unroll
+    for (int u = 0; u < NQ; ++u) {
+        const float cc[4] = {c[u].x, c[u].y, c[u].z, c[u].w}, ss[4] = {s[u].x, s[u].y, s[u].z, s[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int m = 4 * u + e;
+            const float2 r = rope_pair_t(__uint_as_float(v[2 * m]), __uint_as_float(v[2 * m + 1]), cc[e], ss[e]);
+            v[2 * m] = __float_as_uint(r.x);
+            v[2 * m + 1] = __float_as_uint(r.y);
+        }
+    }
+}
+
 // Transposed rotation, in place, of 4 * NQ adjacent pairs held as float bit
 // patterns v[2m], v[2m+1] (m < 4 * NQ), pair indices k0 .. k0 + 4 NQ - 1 of
 // the row at local position pos (k0 a multiple of 4). A position past the

@@ -83,6 +83,40 @@ def test_gdpa_examples_are_isolated_and_deterministic():
             assert torch.equal(got[n][sl], alone[n]), (e, n)
 
 
+def _poison(t, s0, n):
+    pattern = torch.tensor([float("inf"), float("nan"), float("-inf")], dtype=t.dtype)
+    rows = t[s0:s0 + n]
+    rows.copy_(pattern.repeat(rows.numel() // 3 + 1)[: rows.numel()].view_as(rows))
+
+
+@pytest.mark.parametrize("act", ["gelu", "silu"])
+def test_gdpa_examples_are_isolated_from_non_finite_neighbours(act):
+    """Inf / NaN in the first rows of a neighbour's q, k, v and dout (or in all
+    of a short example's rows) leave every other example's out, dq, dk and dv
+    bit-equal to a clean run: the partial tiles at example ends never multiply
+    a neighbour's rows by zero activations."""
+    lengths = [300, 200, 1000, 129, 777, 90, 128, 5]
+    w = CONFIGS[3].replace(heads=2, batch=len(lengths))
+    inp = make_inputs(w, lengths=lengths, seed=4343)
+    offs = inp["seq_offsets"].numpy()
+    poisoned = {1: 40, 3: lengths[3], 5: lengths[5], 7: lengths[7]}
+    dirty = dict(inp)
+    for n in ("q", "k", "v", "dout"):
+        dirty[n] = inp[n].clone()
+        for e, rows in poisoned.items():
+            _poison(dirty[n], int(offs[e]), rows)
+    clean = run_gpu(inp, w.block, w.window, act)
+    got = run_gpu(dirty, w.block, w.window, act)
+    ref = run_oracle(inp, w.block, w.window, act)
+    for e in range(len(lengths)):
+        if e in poisoned:
+            continue
+        sl = slice(int(offs[e]), int(offs[e + 1]))
+        for n in ("out", "dq", "dk", "dv"):
+            assert torch.equal(got[n][sl], clean[n][sl]), f"example {e} {n} changed by a neighbour"
+            check_bf16(f"{act} e{e} {n}", got[n][sl], ref[n][sl])
+
+
 def test_gdpa_rejects_fp32_and_unknown_activations():
     q = torch.zeros((128, 2, 64), device="cuda")
     offs = torch.tensor([0, 128], dtype=torch.int32, device="cuda")
@@ -141,3 +175,31 @@ def test_gdpa_cross_matches_oracle(act, head_dim, lq, lk, peaked):
             assert not out[qs].any() and not dq[qs].any()
         if lq[e] == 0:
             assert not dk[ks].any() and not dv[ks].any()
+
+
+def test_gdpa_cross_examples_are_isolated_from_non_finite_neighbours():
+    """Cross-attention: Inf / NaN in one example's queries, keys, values and
+    dout leave the other examples' results bit-equal to a clean run (each side's
+    partial tiles end inside a neighbour's rows)."""
+    lq, lk = [300, 100, 1000, 129], [64, 200, 17, 130]
+    q, k, v, dout, qo, ko = _cross_inputs(128, lq, lk, 91, 128 ** -0.5)
+
+    def run(q_, k_, v_, do_):
+        dev = [t.cuda() for t in (q_, k_, v_, do_, qo, ko)]
+        out = ba.gdpa_cross_fwd(*dev[:3], dev[4], dev[5], "silu")
+        dq, dk, dv = ba.gdpa_cross_bwd(*dev[:4], dev[4], dev[5], "silu")
+        torch.cuda.synchronize()
+        return out.cpu(), dq.cpu(), dk.cpu(), dv.cpu()
+
+    clean = run(q, k, v, dout)
+    d = [t.clone() for t in (q, k, v, dout)]
+    _poison(d[0], int(qo[1]), lq[1])
+    _poison(d[3], int(qo[1]), lq[1])
+    _poison(d[1], int(ko[1]), lk[1])
+    _poison(d[2], int(ko[1]), lk[1])
+    got = run(*d)
+    for e in (0, 2, 3):
+        qs, ks = slice(int(qo[e]), int(qo[e + 1])), slice(int(ko[e]), int(ko[e + 1]))
+        for name, a, b, sl in (("out", got[0], clean[0], qs), ("dq", got[1], clean[1], qs),
+                               ("dk", got[2], clean[2], ks), ("dv", got[3], clean[3], ks)):
+            assert torch.equal(a[sl], b[sl]), f"example {e} {name} changed by a neighbour"
