@@ -449,14 +449,18 @@ __global__ void __launch_bounds__(384, 1)
                 if (!mbar_wait(&sb.dp_full, s_cnt & 1, abort)) { ok = false; break; }
                 tc_fence_after();
                 const float2 ndl = make_float2(-dl, -dl);
+                // both 32-key halves of dP in one round trip (one TMEM wait, not two)
+                uint32_t drr[2][32];
+                tmem_ld32(tmem + lane_base + Lay::kColDP + 64 * g, drr[0]);
+                tmem_ld32(tmem + lane_base + Lay::kColDP + 64 * g + 32, drr[1]);
+                tmem_wait_ld();
+                reg_fence(drr[0]);
+                reg_fence(drr[1]);
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
                     // 32 keys at a time; their dS (16 columns) lands in [64g+16h2, +16),
                     // inside the dP columns this thread has already read
-                    uint32_t dr[32];
-                    tmem_ld32(tmem + lane_base + Lay::kColDP + 64 * g + 32 * h2, dr);
-                    tmem_wait_ld();
-                    reg_fence(dr);
+                    uint32_t(&dr)[32] = drr[h2];
                     uint32_t pk[16];
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
