@@ -95,7 +95,9 @@ __device__ __forceinline__ int first_key_tile(int t, int64_t B, int64_t W)
 
 } // namespace
 
-template <int D, int A, bool kCross, bool kMx>
+// kFmaExp: one exponential pair in eight goes through the FMA pipe (the
+// launcher's choice for long items; short ones keep every exponential on MUFU)
+template <int D, int A, bool kCross, bool kMx, bool kFmaExp = true>
 __global__ void __launch_bounds__(512, 1)
     fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -470,9 +472,9 @@ __global__ void __launch_bounds__(512, 1)
                             const float2 x = ffma2(make_float2(__uint_as_float(sr[c0 / 32][c0 % 32]),
                                                                __uint_as_float(sr[c0 / 32][c0 % 32 + 1])),
                                                    sc2, nm2);
-                            // one pair in eight goes through the FMA pipe to offload the MUFU unit
-                            float p0 = (c % 8 == 7) ? exp2_fma(x.x) : ex2_approx(x.x);
-                            float p1 = (c % 8 == 7) ? exp2_fma(x.y) : ex2_approx(x.y);
+                            // with kFmaExp one pair in eight goes through the FMA pipe to offload MUFU
+                            float p0 = (kFmaExp && c % 8 == 7) ? exp2_fma(x.x) : ex2_approx(x.x);
+                            float p1 = (kFmaExp && c % 8 == 7) ? exp2_fma(x.y) : ex2_approx(x.y);
                             if (!FULL) {
                                 p0 = x.x > -INFINITY ? p0 : 0.f;
                                 p1 = x.y > -INFINITY ? p1 : 0.f;
@@ -661,6 +663,12 @@ cudaError_t launch_fwd_bf16_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
     auto kern = mx ? fwd_bf16_sm100_kernel<D, A, false, kCanMx>
                    : (A != kSoftmax && p.other_offsets) ? fwd_bf16_sm100_kernel<D, A, A != kSoftmax, false>
                                                         : fwd_bf16_sm100_kernel<D, A, false, false>;
+    if constexpr (A == kSoftmax) {
+        // Items that see fewer than 1024 keys (block x window) are short: their softmax warps are
+        // bound by instruction issue, and MUFU's one-instruction 2^x beats the FMA-pipe form's nine
+        // (measured: config-3 forward 4% faster; with 16-tile items the 1-in-8 mix is 3% faster).
+        if (!mx && int64_t(p.block) * p.window < 1024) kern = fwd_bf16_sm100_kernel<D, A, false, false, false>;
+    }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
     // the register split only works if the CTA is launched with at least the budgets' sum

@@ -162,6 +162,25 @@ def test_mx_backward_with_skip_and_isolation():
                 assert torch.equal(a[sl], b2[sl]), e
 
 
+def test_mx_backward_direct_call_and_status_word():
+    """ba_mx_bwd through the C entry point with a caller-sized workspace; the
+    status word ba_device_status reads sits at the workspace's start."""
+    w = CONFIGS[3].replace(heads=2, batch=3)
+    inp = make_inputs(w, lengths=[300, 129, 64], seed=21)
+    q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "dout"))
+    offs = inp["seq_offsets"].cuda()
+    out, lse = ba.mx_block_attention_fwd(q, k, v, offs, w.block, w.window)
+    prob = ba.make_problem(q, offs)
+    ws = ba.workspace_for(ba.ba_mx_bwd_workspace_size(prob, w.block, w.window), q.device)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    assert ba.ba_mx_bwd(prob, q, k, v, out, lse, do, offs, w.block, w.window, None, dq, dk, dv, ws) == ba.BA_OK
+    assert ba.ba_device_status(ws) == ba.BA_OK
+    ref = ba.mx_block_attention_bwd(q, k, v, out, lse, do, offs, w.block, w.window)
+    torch.cuda.synchronize()
+    for a, b in zip((dq, dk, dv), ref):
+        assert torch.equal(a, b)
+
+
 def test_mx_backward_rejects_head_dim_64_and_small_workspace():
     q = torch.zeros((128, 2, 64), dtype=torch.bfloat16, device="cuda")
     offs = torch.tensor([0, 128], dtype=torch.int32, device="cuda")
