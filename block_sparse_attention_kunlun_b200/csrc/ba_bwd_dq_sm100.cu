@@ -401,8 +401,9 @@ __global__ void __launch_bounds__(384, 1)
                 // phase A: P from S
                 if (!mbar_wait(&sb.s_full, s_cnt & 1, abort)) { ok = false; break; }
                 tc_fence_after();
-                // P of this group's 64 keys as bf16 pairs (phase B only needs it to form dS)
-                uint32_t pp[4][8];
+                // P of this group's 64 keys, kept in float32: phase B only needs it to form dS, so
+                // it is never packed (packing and unpacking cost three instructions a pair)
+                float2 pf[4][8];
                 const float2 sc2 = make_float2(scale_log2, scale_log2), nl2 = make_float2(-l2, -l2);
                 {
                     uint32_t sr[2][16];
@@ -440,7 +441,7 @@ __global__ void __launch_bounds__(384, 1)
                                 e0 = (cc >= lo_c && cc <= hi_c) ? e0 : 0.f;
                                 e1 = (cc + 1 >= lo_c && cc + 1 <= hi_c) ? e1 : 0.f;
                             }
-                            pp[q4][c2] = pack_bf16x2(e0, e1);
+                            pf[q4][c2] = make_float2(e0, e1);
                         }
                         if (q4 < 3) tmem_wait_ld();
                     }
@@ -464,9 +465,7 @@ __global__ void __launch_bounds__(384, 1)
                     uint32_t pk[16];
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        const uint32_t pw = pp[2 * h2 + c / 8][c % 8];
-                        const float2 p2 = make_float2(__uint_as_float(pw << 16), __uint_as_float(pw & 0xffff0000u));
-                        const float2 ds = fmul2(p2, fadd2(make_float2(__uint_as_float(dr[2 * c]),
+                        const float2 ds = fmul2(pf[2 * h2 + c / 8][c % 8], fadd2(make_float2(__uint_as_float(dr[2 * c]),
                                                                       __uint_as_float(dr[2 * c + 1])), ndl));
                         pk[c] = pack_bf16x2(ds.x, ds.y);
                     }
