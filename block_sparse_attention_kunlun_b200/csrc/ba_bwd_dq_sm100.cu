@@ -504,6 +504,9 @@ __global__ void __launch_bounds__(384, 1)
             if (!mbar_wait(&sb.dq_done, item_cnt & 1, abort)) break;
             tc_fence_after();
             {
+                // dq rows start on 32-byte boundaries whenever dq itself does (a row is head_dim
+                // bf16, 128 or 256 bytes); a 16-byte-aligned dq takes 16-byte stores
+                const bool dq32 = (reinterpret_cast<uintptr_t>(dq) & 31) == 0;
                 __nv_bfloat16 *qrow = dq + ((int64_t(r.s0) + i) * p.heads + r.h) * D + (D / 2) * g;
 #pragma unroll 1
                 for (int c = 0; c < D / 64; ++c) {
@@ -531,14 +534,18 @@ __global__ void __launch_bounds__(384, 1)
                             if (rope_in) rope_transpose_loaded<4>(cc, ss, a);
                             else if (c == 0) atomicOr(p.status, kStatusRopeRange); // past the tables
                         }
-                        uint4 *dst = reinterpret_cast<uint4 *>(qrow + 32 * c);
+                        uint32_t pk[16];
 #pragma unroll
-                        for (int x = 0; x < 4; ++x)
-                            dst[x] = make_uint4(
-                                pack_bf16x2(__uint_as_float(a[8 * x + 0]) * p.scale, __uint_as_float(a[8 * x + 1]) * p.scale),
-                                pack_bf16x2(__uint_as_float(a[8 * x + 2]) * p.scale, __uint_as_float(a[8 * x + 3]) * p.scale),
-                                pack_bf16x2(__uint_as_float(a[8 * x + 4]) * p.scale, __uint_as_float(a[8 * x + 5]) * p.scale),
-                                pack_bf16x2(__uint_as_float(a[8 * x + 6]) * p.scale, __uint_as_float(a[8 * x + 7]) * p.scale));
+                        for (int x = 0; x < 16; ++x)
+                            pk[x] = pack_bf16x2(__uint_as_float(a[2 * x]) * p.scale, __uint_as_float(a[2 * x + 1]) * p.scale);
+                        if (dq32) { // 32-byte stores: half the store instructions, each writing whole sectors
+                            st_global_32b(qrow + 32 * c, pk);
+                            st_global_32b(qrow + 32 * c + 16, pk + 8);
+                        } else {
+                            uint4 *dst = reinterpret_cast<uint4 *>(qrow + 32 * c);
+#pragma unroll
+                            for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+                        }
                     }
                 }
                 tc_fence_before();

@@ -497,6 +497,16 @@ __device__ __forceinline__ float exp2_fma(float x)
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// 32 bytes (eight words) to global memory in one instruction; dst must be
+// 32-byte aligned. A warp storing one row per lane then writes whole 32-byte
+// sectors with half the instructions of 16-byte stores.
+__device__ __forceinline__ void st_global_32b(void *dst, const uint32_t *w)
+{
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

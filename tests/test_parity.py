@@ -318,3 +318,27 @@ def test_examples_are_isolated_from_non_finite_neighbours(dtype, head_dim, block
                 check_bf16(f"e{e} {n}", dirty_got[n][sl], ref[n][sl])
         assert torch.equal(dirty_got["lse"][:, sl], clean_got["lse"][:, sl]), f"example {e} lse changed"
         check_abs(f"e{e} lse", dirty_got["lse"][:, sl], ref["lse"][:, sl], 1e-5 if dtype == torch.float32 else 2e-3)
+
+
+@pytest.mark.parametrize("head_dim", [128, 64])
+def test_gradients_into_16_byte_aligned_outputs(head_dim):
+    """dq, dk and dv at addresses that are 16-byte but not 32-byte aligned (the
+    dQ epilogue then takes 16-byte stores instead of 32-byte ones) get the same
+    bits as into freshly allocated (256-byte aligned) tensors."""
+    w = CONFIGS[3].replace(head_dim=head_dim, heads=2, batch=3)
+    inp = make_inputs(w, lengths=[300, 129, 64], seed=77 + head_dim)
+    q, k, v, dout = (inp[n].to(DEV) for n in ("q", "k", "v", "dout"))
+    offs = inp["seq_offsets"].to(DEV)
+    out, lse = ba.block_attention_fwd(q, k, v, offs, w.block, w.window)
+    ref = ba.block_attention_bwd(q, k, v, out, lse, dout, offs, w.block, w.window)
+    shifted = []
+    for _ in range(3):
+        buf = torch.empty(q.numel() + 8, dtype=q.dtype, device=DEV)
+        t = buf[8:].view(q.shape)                  # 16 bytes past a 256-byte boundary
+        assert t.data_ptr() % 32 == 16
+        shifted.append(t)
+    got = ba.block_attention_bwd(q, k, v, out, lse, dout, offs, w.block, w.window,
+                                 dq=shifted[0], dk=shifted[1], dv=shifted[2])
+    torch.cuda.synchronize()
+    for name, a, b in zip(("dq", "dk", "dv"), got, ref):
+        assert torch.equal(a, b), name
