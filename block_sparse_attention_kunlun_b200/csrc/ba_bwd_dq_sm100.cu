@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(384, 1)
             const uint8_t *dsrc = staging + Lay::kTileBytes;
             const uint8_t *osrc = staging + 2 * Lay::kTileBytes;
             const uint32_t col0 = g == 0 ? Lay::kColQ : Lay::kColDO;
-            float dl = 0.f;
+            float2 dl2 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int c = 0; c < Lay::kChunks; ++c) {
 #pragma unroll
@@ -339,7 +339,7 @@ __global__ void __launch_bounds__(384, 1)
                                     __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&dw[e]));
                                 const float2 of =
                                     __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ow[e]));
-                                dl = fmaf(df.x, of.x, fmaf(df.y, of.y, dl));
+                                dl2 = ffma2(df, of, dl2);
                             }
                         }
                         const uint4 a = g == 0 ? *reinterpret_cast<const uint4 *>(qsrc + off) : d4;
@@ -352,6 +352,7 @@ __global__ void __launch_bounds__(384, 1)
                     tmem_st16(tmem + lane_base + col0 + 32 * c + 16 * hh, w);
                 }
             }
+            const float dl = dl2.x + dl2.y;
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
