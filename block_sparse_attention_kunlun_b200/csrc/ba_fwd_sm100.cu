@@ -475,7 +475,9 @@ __global__ void __launch_bounds__(512, 1)
                             // with kFmaExp one pair in eight goes through the FMA pipe to offload MUFU
                             float p0 = (kFmaExp && c % 8 == 7) ? exp2_fma(x.x) : ex2_approx(x.x);
                             float p1 = (kFmaExp && c % 8 == 7) ? exp2_fma(x.y) : ex2_approx(x.y);
-                            if (!FULL) {
+                            // masked scores are -inf here and ex2.approx(-inf) is 0; only the
+                            // FMA-pipe form (which floors x at -125) needs them zeroed again
+                            if (!FULL && kFmaExp && c % 8 == 7) {
                                 p0 = x.x > -INFINITY ? p0 : 0.f;
                                 p1 = x.y > -INFINITY ? p1 : 0.f;
                             }
