@@ -387,6 +387,14 @@ __global__ void __launch_bounds__(448, 1)
                 const int lo_c = int(lo64 < -1 ? -1 : (lo64 > 64 ? 64 : lo64));
                 const int hi_c = int(hi64 < -1 ? -1 : (hi64 > 64 ? 64 : hi64));
                 const bool full = __all_sync(0xffffffffu, lo_c <= 0 && hi_c >= 63);
+                uint32_t vis[2] = {0u, 0u}; // visible columns [lo_c, hi_c] of the group's 64, as bits
+                if (!full) {
+#pragma unroll
+                    for (int w = 0; w < 2; ++w) {
+                        const int lo = max(lo_c - 32 * w, 0), hi = min(hi_c - 32 * w, 31);
+                        vis[w] = lo <= hi ? (0xffffffffu >> (31 - hi)) & (0xffffffffu << lo) : 0u;
+                    }
+                }
                 // -lse (log2 units) and -Delta of this group's queries, staged with the Q tile
                 // (complete once S^T is: the S^T product waited for the same barrier phase)
                 if (!mbar_wait(&sb.q_full[qs], (it / QS) & 1, abort)) { ok = false; break; }
@@ -423,7 +431,7 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
                                     const int cc = 16 * q4 + 4 * c4 + e;
-                                    ev[e] = (cc >= lo_c && cc <= hi_c) ? ev[e] : 0.f;
+                                    ev[e] = (vis[cc / 32] & (1u << (cc % 32))) ? ev[e] : 0.f;
                                 }
                             }
                             pp[q4][2 * c4] = pack_bf16x2(ev[0], ev[1]);
@@ -440,8 +448,8 @@ __global__ void __launch_bounds__(448, 1)
                             float2 v1 = act_value_grad<A>(__uint_as_float(cur[2 * c2 + 1]) * p.scale);
                             if (!full) {
                                 const int cc = 16 * q4 + 2 * c2;
-                                if (!(cc >= lo_c && cc <= hi_c)) v0 = make_float2(0.f, 0.f);
-                                if (!(cc + 1 >= lo_c && cc + 1 <= hi_c)) v1 = make_float2(0.f, 0.f);
+                                if (!(vis[cc / 32] & (1u << (cc % 32)))) v0 = make_float2(0.f, 0.f);
+                                if (!(vis[cc / 32] & (1u << (cc % 32 + 1)))) v1 = make_float2(0.f, 0.f);
                             }
                             pa[c2] = pack_bf16x2(v0.x, v1.x);
                             pp[q4][c2] = pack_bf16x2(v0.y, v1.y);

@@ -399,6 +399,14 @@ __global__ void __launch_bounds__(384, 1)
                 const int lo_c = int(lo64 < -1 ? -1 : (lo64 > 64 ? 64 : lo64));
                 const int hi_c = int(hi64 < -1 ? -1 : (hi64 > 64 ? 64 : hi64));
                 const bool full = __all_sync(0xffffffffu, lo_c <= 0 && hi_c >= 63);
+                uint32_t vis[2] = {0u, 0u}; // visible columns [lo_c, hi_c] of the group's 64, as bits
+                if (!full) {
+#pragma unroll
+                    for (int w = 0; w < 2; ++w) {
+                        const int lo = max(lo_c - 32 * w, 0), hi = min(hi_c - 32 * w, 31);
+                        vis[w] = lo <= hi ? (0xffffffffu >> (31 - hi)) & (0xffffffffu << lo) : 0u;
+                    }
+                }
                 // phase A: P from S
                 if (!mbar_wait(&sb.s_full, s_cnt & 1, abort)) { ok = false; break; }
                 tc_fence_after();
@@ -439,8 +447,8 @@ __global__ void __launch_bounds__(384, 1)
                             }
                             if (!full) {
                                 const int cc = 16 * q4 + 2 * c2;
-                                e0 = (cc >= lo_c && cc <= hi_c) ? e0 : 0.f;
-                                e1 = (cc + 1 >= lo_c && cc + 1 <= hi_c) ? e1 : 0.f;
+                                e0 = (vis[cc / 32] & (1u << (cc % 32))) ? e0 : 0.f;
+                                e1 = (vis[cc / 32] & (1u << (cc % 32 + 1))) ? e1 : 0.f;
                             }
                             pf[q4][c2] = make_float2(e0, e1);
                         }

@@ -437,6 +437,16 @@ __global__ void __launch_bounds__(512, 1)
                 // positive), one for P; a tile visible to the whole warp skips masking.
                 float alpha = 1.f, rs = 0.f;
                 bool grow = false;
+                // this row's visible columns [lo_c, hi_c] as four 32-bit masks (partial tiles only),
+                // so that each column's test is one bit test
+                uint32_t vis[4] = {0u, 0u, 0u, 0u};
+                if (!full) {
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const int lo = max(lo_c - 32 * w, 0), hi = min(hi_c - 32 * w, 31);
+                        vis[w] = lo <= hi ? (0xffffffffu >> (31 - hi)) & (0xffffffffu << lo) : 0u;
+                    }
+                }
                 auto softmax_tile = [&](auto full_t) {
                     constexpr bool FULL = decltype(full_t)::value;
                     float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -444,8 +454,8 @@ __global__ void __launch_bounds__(512, 1)
                     for (int c = 0; c < 128; c += 2) {
                         float a = __uint_as_float(sr[c / 32][c % 32]), b = __uint_as_float(sr[c / 32][c % 32 + 1]);
                         if (!FULL) {
-                            a = (c >= lo_c && c <= hi_c) ? a : -INFINITY;
-                            b = (c + 1 >= lo_c && c + 1 <= hi_c) ? b : -INFINITY;
+                            a = (vis[c / 32] & (1u << (c % 32))) ? a : -INFINITY;
+                            b = (vis[c / 32] & (1u << (c % 32 + 1))) ? b : -INFINITY;
                             sr[c / 32][c % 32] = __float_as_uint(a);
                             sr[c / 32][c % 32 + 1] = __float_as_uint(b);
                         }
@@ -505,8 +515,8 @@ __global__ void __launch_bounds__(512, 1)
                                 p1 = act_value<A>(__uint_as_float(sr[c0 / 32][c0 % 32 + 1]) * p.scale);
                             }
                             if (!FULL) {
-                                p0 = (c0 >= lo_c && c0 <= hi_c) ? p0 : 0.f;
-                                p1 = (c0 + 1 >= lo_c && c0 + 1 <= hi_c) ? p1 : 0.f;
+                                p0 = (vis[c0 / 32] & (1u << (c0 % 32))) ? p0 : 0.f;
+                                p1 = (vis[c0 / 32] & (1u << (c0 % 32 + 1))) ? p1 : 0.f;
                             }
                             pk[c] = pack_bf16x2(p0, p1);
                         }
