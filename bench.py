@@ -16,8 +16,10 @@ inputs resident in HBM; ``e2e`` is the same metric with pinned-host inputs
 copied in and the results copied out inside the timed region.
 
 The same line carries ``other_configs``: the long-context workload (8 x 32768,
-block 512, window 4) and the jagged workload with component skip, each timed
-the same way (N = 1 only).
+block 512, window 4), the jagged workload with component skip, and the jagged
+histories with independent 64-token blocks (block 64, window 1), each timed
+the same way (N = 1 only), each with its step's HBM bytes against the copy
+bandwidth.
 
 Multi-GPU: every rank runs its own batch (seeded per rank) with no
 collective on the data path; the step time is the max over ranks. Launched
@@ -458,10 +460,16 @@ class Runner:
                 for n in KERNEL_NAMES}
 
 
-def other_config_line(ba, cfg, dev, K, warmup, local):
+def other_config_line(ba, cfg, dev, K, warmup, local, hbm_gbs, block=None, window=None):
     """One more workload timed like the main one (its own process memory is
-    released afterwards)."""
+    released afterwards); block/window replace the workload's block rule.
+    Its ``hbm`` entry sets the step's algorithmic bytes (each input read once,
+    each result written once) against the copy bandwidth: the roof of a mask so
+    sparse that a step is bound by HBM, not by the tensor cores."""
     w = CONFIGS[cfg]
+    if block is not None:
+        w = w.replace(block=block, window=window,
+                      name=w.name.replace(f"block {w.block}, window {w.window}", f"block {block}, window {window}"))
     inp = make_inputs(w)
     run = Runner(ba, w, inp, dev)
     clocks = ClockSampler(local)
@@ -472,6 +480,10 @@ def other_config_line(ba, cfg, dev, K, warmup, local):
          "tokens_per_s": run.T / (ms / 1e3), "total_tokens": int(run.T),
          "visible_pairs_per_head": run.pairs, "useful_flops_per_step": run.flops["step"],
          "steps": K, "warmup": warmup, "kernels": run.kernel_stats(ms_k), "clocks": clk}
+    step_bytes = run.bytes["fwd"] + run.bytes["bwd"]
+    d["hbm"] = {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_bytes / (ms / 1e3) / 1e9,
+                "peak_gbs": hbm_gbs, "frac": step_bytes / (ms / 1e3) / 1e9 / hbm_gbs,
+                "floor_ms": step_bytes / (hbm_gbs * 1e9) * 1e3}
     if run.skip_np is not None:
         d["live_tokens"] = F.live_tokens(run.lens, run.skip_np)
         d["skipped_examples"] = int(run.skip_np.sum())
@@ -666,8 +678,11 @@ def main(argv=None, runner_cls=None):
         del run
         torch.cuda.empty_cache()
         Ko = max(5, min(K, 20))
-        line["other_configs"] = {f"config{c}": other_config_line(ba, c, dev, Ko, max(3, args.warmup), local)
+        line["other_configs"] = {f"config{c}": other_config_line(ba, c, dev, Ko, max(3, args.warmup), local, hbm)
                                  for c in (4, 5) if c != args.config}
+        # the pages' independent 64-token blocks on the same jagged histories
+        line["other_configs"]["config3_block64_window1"] = other_config_line(
+            ba, 3, dev, Ko, max(3, args.warmup), local, hbm, block=64, window=1)
     if not args.no_cpu_baseline and world == 1 and on_gpu and not args.gdpa and not args.mx:
         line["cpu_baseline"] = cpu_baseline(w, inp, pairs, tables=tables_for(lens, D) if args.rope else None)
     print(json.dumps(line), flush=True)
