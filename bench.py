@@ -337,6 +337,13 @@ class Runner:
 
     def __init__(self, ba, w, inp, dev, rope=False, gdpa=None, mx=False):
         self.ba, self.w, self.inp, self.dev, self.rope, self.gdpa, self.mx = ba, w, inp, dev, rope, gdpa, mx
+        # window 1 with blocks dividing 128: the bf16 backward is one fused pass (dQ, dK and dV)
+        # after a per-row statistics pass, which take the dQ and dK/dV profile slots
+        self.fused = (w.dtype == torch.bfloat16 and not rope and not gdpa and w.window == 1
+                      and w.block <= 128 and 128 % w.block == 0)
+        self.kernel_names = dict(KERNEL_NAMES)
+        if self.fused:
+            self.kernel_names.update(bwd_dq="bwd_stats_kernel", bwd_dkdv="bwd_dkdv_sm100_kernel (fused dQ)")
         self.lens = inp["lengths"].numpy()
         self.skip_np = inp["skip"].numpy() if inp["skip"] is not None else None
         T, H, D = inp["q"].shape
@@ -453,10 +460,14 @@ class Runner:
 
     def kernel_stats(self, ms_k):
         # Per kernel, the FLOPs its own tensor-core work does on visible pairs: forward 4 D (S, PV),
-        # dQ pass 6 D (S, dP, dQ), dK/dV pass 8 D (S, dP, dV, dK); per visible pair and head.
+        # dQ pass 6 D (S, dP, dQ), dK/dV pass 8 D (S, dP, dV, dK); per visible pair and head. The
+        # fused backward does 10 D (S, dP, dV, dK, dQ); its statistics pass none.
         unit = self.pairs * self.H * self.D
         fl = {"fwd": 4 * unit, "bwd_dq": 6 * unit, "bwd_dkdv": 8 * unit}
-        return {n: {"ms": ms_k[n], "tflops": fl[n] / (ms_k[n] / 1e3) / 1e12, "flops_per_launch": fl[n]}
+        if self.fused:
+            fl.update(bwd_dq=0, bwd_dkdv=10 * unit)
+        return {n: {"kernel": self.kernel_names[n], "ms": ms_k[n], "tflops": fl[n] / (ms_k[n] / 1e3) / 1e12,
+                    "flops_per_launch": fl[n]}
                 for n in KERNEL_NAMES}
 
 
@@ -629,7 +640,7 @@ def main(argv=None, runner_cls=None):
     try:
         with open(args.traffic_file) as f:
             tr = json.load(f)
-        key = f"{KERNEL_NAMES[dom]}:config{args.config}" + (f":block{w.block}:window{w.window}"
+        key = f"{run.kernel_names[dom]}:config{args.config}" + (f":block{w.block}:window{w.window}"
                                                             if (args.swa or args.block or args.window) else "")
         key += ":rope" if args.rope else ""
         key += f":gdpa-{args.gdpa}" if args.gdpa else ""
@@ -640,7 +651,7 @@ def main(argv=None, runner_cls=None):
         pass
     achieved = kstats[dom]["tflops"]
     flops_launch = kstats[dom]["flops_per_launch"]
-    roofline = {"kernel": KERNEL_NAMES[dom], "bound": "tensor", "achieved": achieved, "peak": tensor_peak,
+    roofline = {"kernel": run.kernel_names[dom], "bound": "tensor", "achieved": achieved, "peak": tensor_peak,
                 "unit": "TFLOP/s", "frac": achieved / tensor_peak, "traffic": traffic,
                 "peak_source": f"{peaks_src} {'bf16_tflops_sustained' if long_region else 'bf16_tflops (burst)'};"
                                f" timed region {timed_s:.2f} s",

@@ -105,14 +105,30 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 // the pass reads them through (rows 128 b .. 128 b + 127 for example b).
 bool stage_query_tails(const ba_problem &P, const int32_t *offs, const uint8_t *skip, const void *q,
                        const void *dout, uint8_t *ws, const WorkspaceLayout &lay, CUtensorMap &tqt, CUtensorMap &tdot,
-                       cudaStream_t stream)
+                       cudaStream_t stream, const void *k = nullptr, CUtensorMap *tkt = nullptr)
 {
     const int64_t rows = int64_t(P.batch) * kTile;
     if (!encode_bf16_rows(&tqt, ws + lay.tail_q, rows, P.heads, P.head_dim) ||
-        !encode_bf16_rows(&tdot, ws + lay.tail_do, rows, P.heads, P.head_dim))
+        !encode_bf16_rows(&tdot, ws + lay.tail_do, rows, P.heads, P.head_dim) ||
+        (k && !encode_bf16_rows(tkt, ws + lay.tail_k, rows, P.heads, P.head_dim)))
         return false;
     return launch_stage_query_tails(offs, skip, P.batch, size_t(P.heads) * P.head_dim * 2, q, dout, ws + lay.tail_q,
-                                    ws + lay.tail_do, stream) == cudaSuccess;
+                                    ws + lay.tail_do, stream, k, k ? ws + lay.tail_k : nullptr) == cudaSuccess;
+}
+
+// The bf16 backward runs fused (one pass for dQ, dK and dV) when every query
+// tile sees only its own key tile, for block attention without rotation.
+bool fused_backward(const ba_problem &P, int32_t block, int32_t window, bool with_rope)
+{
+    return P.dtype == BA_BF16 && !with_rope && diagonal_tiles(block, window);
+}
+
+// The backward's workspace: the per-row statistics, the staged partial tiles
+// (bf16), and for the fused backward the staged partial key tiles.
+WorkspaceLayout bwd_layout(const ba_problem &P, int32_t block, int32_t window, bool with_rope)
+{
+    return workspace_layout(P.batch, P.total_tokens, P.heads, P.head_dim, true, P.dtype == BA_BF16,
+                            fused_backward(P, block, window, with_rope));
 }
 
 bool head_dim_supported(const ba_problem &p)
@@ -278,7 +294,8 @@ ba_status bwd_impl(const ba_problem *pp, const ba_rope *rope, const void *q, con
         return BA_ERR_INVALID_ARG;
     if (with_rope && (st = check_rope(rope, P)) != BA_OK) return st;
     const bool bf16 = P.dtype == BA_BF16;
-    const WorkspaceLayout lay = workspace_layout(P.batch, T, P.heads, P.head_dim, true, bf16);
+    const bool fused = fused_backward(P, block, window, with_rope);
+    const WorkspaceLayout lay = bwd_layout(P, block, window, with_rope);
     const RopeLayout rl = rope_layout(P, lay.total);
     const size_t need = with_rope && !caller_rotated(rope) ? rl.total : lay.total;
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return BA_ERR_INVALID_ARG;
@@ -320,13 +337,29 @@ ba_status bwd_impl(const ba_problem *pp, const ba_rope *rope, const void *q, con
         if (with_rope) BA_TRY(launch_rope_rows(p, esz, true, dq, dk, dq, dk, num_sms, stream));
         return BA_OK;
     }
-    CUtensorMap tq, tk, tv, tdo, to, tdk, tdv, tqt, tdot;
+    CUtensorMap tq, tk, tv, tdo, to, tdk, tdv, tqt, tdot, tkt, tdq;
     if (!encode_bf16_rows(&tq, q, T, P.heads, P.head_dim) || !encode_bf16_rows(&tk, k, T, P.heads, P.head_dim) ||
         !encode_bf16_rows(&tv, v, T, P.heads, P.head_dim) || !encode_bf16_rows(&tdo, dout, T, P.heads, P.head_dim) ||
         !encode_bf16_rows(&to, out, T, P.heads, P.head_dim) || !encode_bf16_rows(&tdk, dk, T, P.heads, P.head_dim) ||
         !encode_bf16_rows(&tdv, dv, T, P.heads, P.head_dim) ||
-        !stage_query_tails(P, seq_offsets, skip, q, dout, ws, lay, tqt, tdot, stream))
+        (fused && !encode_bf16_rows(&tdq, dq, T, P.heads, P.head_dim)) ||
+        !stage_query_tails(P, seq_offsets, skip, q, dout, ws, lay, tqt, tdot, stream, fused ? k : nullptr, &tkt))
         return BA_ERR_CUDA;
+    if (fused) {
+        // one pass for dQ, dK and dV; its per-row statistics first (profile slot 1)
+        BA_TRY(prof_mark(1, 0, stream));
+        BA_TRY(launch_bwd_stats(p, out, dout, lse, delta, nlse2, num_sms, stream));
+        BA_TRY(prof_mark(1, 1, stream));
+        BA_TRY(prof_mark(2, 0, stream));
+        if (P.head_dim == 64)
+            BA_TRY(launch_bwd_fused_sm100<64>(tq, tk, tv, tdo, tdk, tdv, tqt, tdot, tkt, tdq, p, nlse2, delta, dq, dk,
+                                              dv, num_sms, stream));
+        else
+            BA_TRY(launch_bwd_fused_sm100<128>(tq, tk, tv, tdo, tdk, tdv, tqt, tdot, tkt, tdq, p, nlse2, delta, dq,
+                                               dk, dv, num_sms, stream));
+        BA_TRY(prof_mark(2, 1, stream));
+        return BA_OK;
+    }
     BA_TRY(prof_mark(1, 0, stream));
     if (P.head_dim == 64)
         BA_TRY(launch_bwd_dq_sm100<64, kSoftmax>(tq, tk, tv, tdo, to, p, lse, delta, nlse2, dq, num_sms, stream));
@@ -586,7 +619,7 @@ ba_status mx_bwd_impl(const ba_problem *pp, const void *q, const void *k, const 
         return BA_ERR_INVALID_ARG;
     if (P.dtype != BA_BF16 || P.head_dim != 128) return BA_ERR_UNSUPPORTED;
     const size_t rt = mx_bwd_operand_bytes(P);
-    const size_t base = workspace_layout(P.batch, T, P.heads, P.head_dim, true, true).total;
+    const size_t base = bwd_layout(P, block, window, false).total;
     const size_t need = base + 2 * rt;
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return BA_ERR_INVALID_ARG;
     int num_sms = 0, cc = 0;
@@ -614,7 +647,7 @@ size_t ba_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
 size_t ba_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
 {
     if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
-    return workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, true, p->dtype == BA_BF16).total;
+    return bwd_layout(*p, block, window, false).total;
 }
 
 ba_status ba_fwd(const ba_problem *p, const void *q, const void *k, const void *v, const int32_t *seq_offsets,
@@ -767,8 +800,7 @@ ba_status ba_mx_fwd(const ba_problem *p, const void *q, const void *k, const voi
 size_t ba_mx_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window)
 {
     if (check_problem(p, block, window) == BA_ERR_INVALID_ARG) return 0;
-    return 2 * mx_bwd_operand_bytes(*p) +
-           workspace_layout(p->batch, p->total_tokens, p->heads, p->head_dim, true, p->dtype == BA_BF16).total;
+    return 2 * mx_bwd_operand_bytes(*p) + bwd_layout(*p, block, window, false).total;
 }
 
 ba_status ba_mx_bwd(const ba_problem *p, const void *q, const void *k, const void *v, const void *out,

@@ -6,6 +6,9 @@
 //                     (q and dout), zero-padded, for the dK/dV pass
 //   bwd_pre_kernel    Delta = rowsum(dout * out) in fp32 (the fp32 path; the
 //                     bf16 dQ pass computes Delta itself)
+//   bwd_stats_kernel  -Delta and -lse log2(e) per row for the fused bf16
+//                     backward (masks whose query tiles see only their own
+//                     key tile), which has no dQ pass
 //   wait_selftest_kernel  one warp waits on a barrier nothing completes, with a
 //                     short limit, through the same bounded wait the attention
 //                     kernels use, and reports the timeout in the status word
@@ -245,12 +248,15 @@ cudaError_t launch_zero_unpaired_rows(const int32_t *offs, const int32_t *other,
 // has fewer than 128 rows, is copied from a (q) and b (dout) to rows
 // [128 b, 128 b + 128) of ta and tb with zeros in the rows past the example,
 // so that the pass never multiplies a neighbour's rows, finite or not, by its
-// zero probabilities. Examples whose length is a multiple of 128 (or zero) or
-// that are skipped are left alone. grid = (example, 8 slices of 16 rows).
+// zero probabilities. The fused backward also stages c (k) into tc, since its
+// dQ = dS K sums over the partial key tile's rows. Examples whose length is a
+// multiple of 128 (or zero) or that are skipped are left alone. grid =
+// (example, 8 slices of 16 rows).
 __global__ void __launch_bounds__(256)
     stage_query_tails_kernel(const int32_t *__restrict__ offs, const uint8_t *__restrict__ skip, int64_t row_bytes,
-                             const uint8_t *__restrict__ a, const uint8_t *__restrict__ b, uint8_t *__restrict__ ta,
-                             uint8_t *__restrict__ tb)
+                             const uint8_t *__restrict__ a, const uint8_t *__restrict__ b,
+                             const uint8_t *__restrict__ c, uint8_t *__restrict__ ta, uint8_t *__restrict__ tb,
+                             uint8_t *__restrict__ tc)
 {
     const int e = blockIdx.x;
     if (skip && skip[e]) return;
@@ -263,24 +269,84 @@ __global__ void __launch_bounds__(256)
     for (int64_t x = threadIdx.x; x < (kTile / 8) * units; x += blockDim.x) {
         const int64_t r = r0 + x / units, u = x % units;
         const int64_t dst = (int64_t(e) * kTile + r) * units + u;
-        uint4 va = make_uint4(0, 0, 0, 0), vb = va;
+        uint4 va = make_uint4(0, 0, 0, 0), vb = va, vc = va;
         if (r < valid) {
             va = reinterpret_cast<const uint4 *>(a)[(first + r) * units + u];
             vb = reinterpret_cast<const uint4 *>(b)[(first + r) * units + u];
+            if (c) vc = reinterpret_cast<const uint4 *>(c)[(first + r) * units + u];
         }
         reinterpret_cast<uint4 *>(ta)[dst] = va;
         reinterpret_cast<uint4 *>(tb)[dst] = vb;
+        if (c) reinterpret_cast<uint4 *>(tc)[dst] = vc;
     }
 }
 
 cudaError_t launch_stage_query_tails(const int32_t *offs, const uint8_t *skip, int32_t batch, size_t row_bytes,
-                                     const void *a, const void *b, void *ta, void *tb, cudaStream_t stream)
+                                     const void *a, const void *b, void *ta, void *tb, cudaStream_t stream,
+                                     const void *c, void *tc)
 {
     if (batch == 0) return cudaSuccess;
+    if ((c == nullptr) != (tc == nullptr)) return cudaErrorInvalidValue;
     stage_query_tails_kernel<<<dim3(batch, 8), 256, 0, stream>>>(
         offs, skip, int64_t(row_bytes), static_cast<const uint8_t *>(a), static_cast<const uint8_t *>(b),
-        static_cast<uint8_t *>(ta), static_cast<uint8_t *>(tb));
+        static_cast<const uint8_t *>(c), static_cast<uint8_t *>(ta), static_cast<uint8_t *>(tb),
+        static_cast<uint8_t *>(tc));
     return cudaGetLastError();
+}
+
+// The fused backward's per-row statistics, which the dQ pass computes
+// otherwise: -Delta = -(dout . out) and -lse log2(e) of every (token, head)
+// row, written [heads, total_tokens]. D / 8 lanes per row, one 16-byte vector
+// of each operand per lane and row, two rows per lane in flight; rows of
+// skipped examples are computed too (nothing reads them).
+__device__ __forceinline__ float bf16x8_dot(const uint4 a, const uint4 b)
+{
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 af = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&aw[e]));
+        const float2 bf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bw[e]));
+        acc.x = fmaf(af.x, bf.x, acc.x);
+        acc.y = fmaf(af.y, bf.y, acc.y);
+    }
+    return acc.x + acc.y;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256)
+    bwd_stats_kernel(const __nv_bfloat16 *__restrict__ out, const __nv_bfloat16 *__restrict__ dout,
+                     const float *__restrict__ lse, int32_t total_tokens, int32_t heads,
+                     float *__restrict__ neg_delta, float *__restrict__ nlse2)
+{
+    constexpr int LPR = D / 8, RPW = 32 / LPR; // lanes per row, rows per warp and step
+    const int lane = threadIdx.x & 31, u = lane % LPR;
+    const int64_t nrows = int64_t(total_tokens) * heads;
+    const int64_t step = int64_t(gridDim.x) * (blockDim.x >> 5) * (2 * RPW);
+    for (int64_t base = (int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * (2 * RPW); base < nrows;
+         base += step) {
+        const int64_t rw[2] = {base + lane / LPR, base + RPW + lane / LPR};
+        uint4 o[2], g[2];
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            o[x] = g[x] = make_uint4(0u, 0u, 0u, 0u);
+            if (rw[x] < nrows) {
+                o[x] = __ldg(reinterpret_cast<const uint4 *>(out + rw[x] * D) + u);
+                g[x] = __ldg(reinterpret_cast<const uint4 *>(dout + rw[x] * D) + u);
+            }
+        }
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            float sum = bf16x8_dot(o[x], g[x]);
+#pragma unroll
+            for (int d = LPR / 2; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
+            if (u == 0 && rw[x] < nrows) {
+                const int64_t t = rw[x] / heads, h = rw[x] % heads, hr = h * int64_t(total_tokens) + t;
+                neg_delta[hr] = -sum;
+                nlse2[hr] = -lse[hr] * 1.4426950408889634f;
+            }
+        }
+    }
 }
 
 static int grid_for_rows(int64_t nrows, int num_sms)
@@ -290,6 +356,25 @@ static int grid_for_rows(int64_t nrows, int num_sms)
     const int64_t cap = int64_t(num_sms) * 16;
     if (g > cap) g = cap;
     return int(g < 1 ? 1 : g);
+}
+
+cudaError_t launch_bwd_stats(const Problem &p, const void *out, const void *dout, const float *lse,
+                             float *neg_delta, float *nlse2, int num_sms, cudaStream_t stream)
+{
+    const int64_t nrows = int64_t(p.total_tokens) * p.heads;
+    if (nrows == 0) return cudaSuccess;
+    const int g = grid_for_rows(nrows, num_sms);
+    const auto *o = static_cast<const __nv_bfloat16 *>(out), *d = static_cast<const __nv_bfloat16 *>(dout);
+    switch (p.head_dim) {
+    case 64:
+        bwd_stats_kernel<64><<<g, 256, 0, stream>>>(o, d, lse, p.total_tokens, p.heads, neg_delta, nlse2);
+        break;
+    case 128:
+        bwd_stats_kernel<128><<<g, 256, 0, stream>>>(o, d, lse, p.total_tokens, p.heads, neg_delta, nlse2);
+        break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
 }
 
 template <typename T>

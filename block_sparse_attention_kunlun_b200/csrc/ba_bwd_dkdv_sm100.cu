@@ -39,6 +39,17 @@
 //   warp 13    MMA issuer.
 // TMEM columns: S^T / P^T [0,128), dP^T / dS^T [128,256), dV [256, 256+D),
 // dK [256+D, 256+2D).
+//
+// Fused backward (kDq; masks under which every query tile sees only its own key
+// tile, so each item has one query tile, the key tile's own rows): the same pass
+// also forms dQ = (1/sqrt(D)) dS K. The compute warps write dS a second time, as
+// bf16 into shared memory with the keys as rows (the MN-major A operand of
+// dQ = dS K; TMEM holds dS^T with the keys on the lanes, the wrong way round for
+// an A operand), and dQ accumulates over the dS^T columns after the dK product
+// has read them. The epilogue stores dQ first, which frees those columns for the
+// next item's dP^T. Keys past the example enter the dQ sum, so their dS is
+// written as zero and an example's partial key tile is read from a zero-padded
+// copy. -Delta and -lse log2(e) come from a separate per-row pass.
 #include "ba_common.cuh"
 #include "ba_kernels.cuh"
 #include "ba_ptx.cuh"
@@ -50,7 +61,7 @@ namespace ba {
 
 namespace {
 
-template <int D>
+template <int D, bool kDq = false>
 struct DkvLayout {
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     static constexpr int kChunks = D / 64;
@@ -59,22 +70,27 @@ struct DkvLayout {
     // Q ring and dO ring. Q(m) is read until dK(m), late in tile m's step, and
     // S^T(m+1) needs Q(m+1): three Q slots keep its load well ahead. dO(m) is free
     // after dV(m), early in the step, so at D = 128 one dO slot is enough.
-    static constexpr int kQSlots = D == 64 ? 4 : 3;
-    static constexpr int kOSlots = D == 64 ? 4 : 1;
+    // The fused backward has one query tile per item, and its dS buffer takes a slot's room.
+    static constexpr int kQSlots = kDq ? 2 : (D == 64 ? 4 : 3);
+    static constexpr int kOSlots = kDq ? (D == 64 ? 2 : 1) : (D == 64 ? 4 : 1);
     static constexpr int kK = 0;
     static constexpr int kV = kTileBytes;
     static constexpr int kQ0 = 2 * kTileBytes;           // Q slot s at kQ0 + s tile
     static constexpr int kO0 = kQ0 + kQSlots * kTileBytes; // dO slot s at kO0 + s tile
     static constexpr int kStage = kO0 + kOSlots * kTileBytes; // epilogue staging: 128 rows x 64 columns
-    static constexpr int kBytes = kStage + kChunkBytes;
+    // fused backward: dS (bf16) as two 64-query chunks of 128 key rows, 128-byte swizzled
+    static constexpr int kDS = kStage + kChunkBytes;
+    static constexpr int kDSChunkBytes = kTile * 128;
+    static constexpr int kBytes = kDS + (kDq ? 2 * kDSChunkBytes : 0);
     static constexpr int kAlloc = kBytes + 1024;
     static constexpr int kThreads = 448;
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+    static constexpr uint32_t kColDQ = kColDP; // fused backward: over dS^T once dK has read it
     static constexpr uint32_t kTmemCols = 512;
 };
 
 struct DkvBarriers {
-    uint64_t k_full, k_empty, v_full, v_empty, dkv_full, dv_free, dk_free;
+    uint64_t k_full, k_empty, v_full, v_empty, dkv_full, dv_free, dk_free, dq_free;
     uint64_t q_full[4], q_empty[4], o_full[4], o_empty[4];
     uint64_t s_full, dp_full, pa_done[2], pb_done[2];
     uint64_t epi_sync; // group barrier of the epilogue warps
@@ -101,16 +117,18 @@ __device__ __forceinline__ void query_tile_range(const TileRef &r, int64_t B, in
 
 } // namespace
 
-template <int D, bool kRope, int A, bool kCross>
+template <int D, bool kRope, int A, bool kCross, bool kDq>
 __global__ void __launch_bounds__(448, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                           const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                           const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_dot,
                           const Problem p, const float *__restrict__ nlse2, const float *__restrict__ neg_delta,
-                          __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv)
+                          __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv,
+                          const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_dq,
+                          __nv_bfloat16 *__restrict__ dq)
 {
-    using Lay = DkvLayout<D>;
+    using Lay = DkvLayout<D, kDq>;
     constexpr int QS = Lay::kQSlots, OS = Lay::kOSlots;
     extern __shared__ uint8_t smem_raw[];
     __shared__ DkvBarriers sb;
@@ -127,6 +145,7 @@ __global__ void __launch_bounds__(448, 1)
         mbar_init(&sb.dkv_full, 1);
         mbar_init(&sb.dv_free, 4);
         mbar_init(&sb.dk_free, 4);
+        mbar_init(&sb.dq_free, 4);
         for (int i = 0; i < 4; ++i) {
             mbar_init(&sb.q_full[i], 1 + 32); // the Q tile's expect_tx arrival + one per lane's copies
             mbar_init(&sb.q_empty[i], 1);
@@ -216,11 +235,20 @@ __global__ void __launch_bounds__(448, 1)
                         ok = false;
                         break;
                     }
+                    const CUtensorMap *mk = &tm_k;
+                    int32_t ky = r.s0 + r.t * kTile;
+                    if constexpr (kDq) {
+                        // dQ sums over the key rows: an example's partial key tile comes from its
+                        // zero-padded copy
+                        if (r.L - r.t * kTile < kTile) {
+                            mk = &tm_kt;
+                            ky = r.b * kTile;
+                        }
+                    }
                     if (lane == 0) {
                         mbar_arrive_expect_tx(&sb.k_full, Lay::kTileBytes);
                         for (int c = 0; c < Lay::kChunks; ++c)
-                            tma_load_2d(smem + Lay::kK + c * Lay::kChunkBytes, &tm_k, &sb.k_full, r.h * D + c * 64,
-                                        r.s0 + r.t * kTile);
+                            tma_load_2d(smem + Lay::kK + c * Lay::kChunkBytes, mk, &sb.k_full, r.h * D + c * 64, ky);
                     }
                     __syncwarp();
                     if (!mbar_wait(&sb.v_empty, (item_cnt & 1) ^ 1, abort)) {
@@ -294,7 +322,7 @@ __global__ void __launch_bounds__(448, 1)
                                sdesc_sw128(q_addr + off, 16, 1024), idesc_sp, kk > 0 ? 1u : 0u);
                     }
                     tc_commit(&sb.s_full);
-                    if (m == nq - 1) tc_commit(&sb.k_empty);
+                    if (!kDq && m == nq - 1) tc_commit(&sb.k_empty); // the fused backward reads K again for dQ
                 }
                 __syncwarp();
                 return true;
@@ -303,6 +331,10 @@ __global__ void __launch_bounds__(448, 1)
             auto issue_dp = [&](int m) -> bool {
                 const uint32_t it = it0 + m, os = it % OS;
                 if (!mbar_wait(&sb.o_full[os], (it / OS) & 1, abort)) return false;
+                if constexpr (kDq) {
+                    // dP^T overwrites the previous item's dQ: the epilogue must have read it
+                    if (m == 0 && !mbar_wait(&sb.dq_free, (item_cnt & 1) ^ 1, abort)) return false;
+                }
                 tc_fence_after();
                 {
                     const uint32_t o_addr = smem_base + Lay::kO0 + os * Lay::kTileBytes;
@@ -357,6 +389,20 @@ __global__ void __launch_bounds__(448, 1)
                      (m + 1 >= nq || issue_dp(m + 1));
             }
             if (!ok) break;
+            if constexpr (kDq) {
+                // dQ = dS K (scaled in the epilogue). A = dS from shared memory, written by the
+                // compute warps before their phase-B arrivals (waited for in issue_acc), MN-major
+                // with 16 keys (2 KB of rows) per step; B = K, MN-major. It accumulates over the
+                // dS^T columns, which the dK product issued before it has read.
+                constexpr uint32_t idesc_q = idesc_bf16(128, D, true, true);
+                const uint32_t ds_addr = smem_base + Lay::kDS;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    mma_ss(tmem + Lay::kColDQ, sdesc_sw128(ds_addr + kk * 2048, Lay::kDSChunkBytes, 1024),
+                           sdesc_sw128(k_addr + kk * 2048, Lay::kChunkBytes, 1024), idesc_q, kk > 0 ? 1u : 0u);
+                tc_commit(&sb.k_empty);
+            }
             tc_commit(&sb.dkv_full);
             __syncwarp();
             it0 += nq;
@@ -483,7 +529,19 @@ __global__ void __launch_bounds__(448, 1)
                         dk16[c2] = pack_bf16x2(ds.x, ds.y);
                     }
                     tmem_st16(tmem + lane_base + Lay::kColDP + 64 * g + 16 * h2, dk16);
+                    if constexpr (kDq) {
+                        // the same dS for dQ = dS K: row `row` (this key) of query chunk g, 16-byte
+                        // units 4 h2 .. 4 h2 + 3; zero for a key past the example, whose dP^T row
+                        // may hold a neighbour's non-finite values
+                        uint8_t *drow = smem + Lay::kDS + g * Lay::kDSChunkBytes + row * 128;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<uint4 *>(drow + (((4 * h2 + j) ^ (row & 7)) << 4)) =
+                                valid_k ? make_uint4(dk16[4 * j], dk16[4 * j + 1], dk16[4 * j + 2], dk16[4 * j + 3])
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                    }
                 }
+                if constexpr (kDq) fence_proxy_async_smem(); // dS written for the tensor core
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -510,6 +568,49 @@ __global__ void __launch_bounds__(448, 1)
             const int64_t grow = (int64_t(r.s0) + k) * p.heads + r.h;
             if (!mbar_wait(&sb.dkv_full, item_cnt & 1, abort)) break;
             tc_fence_after();
+            if constexpr (kDq) {
+                // dQ first (the tile's query rows are its key rows), 64 columns at a time, scaled
+                // by 1/sqrt(D): reading it frees the columns the next item's dP^T writes
+#pragma unroll 1
+                for (int c = 0; c < Lay::kChunks; ++c) {
+                    uint32_t rr[2][32], pk[32];
+                    tmem_ld32(tmem + lane_base + Lay::kColDQ + 64 * c, rr[0]);
+                    tmem_ld32(tmem + lane_base + Lay::kColDQ + 64 * c + 32, rr[1]);
+                    tmem_wait_ld();
+                    reg_fence(rr[0]);
+                    reg_fence(rr[1]);
+                    if (c == Lay::kChunks - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sb.dq_free);
+                    }
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                        pk[x] = pack_bf16x2(__uint_as_float(rr[x / 16][2 * (x % 16)]) * p.scale,
+                                            __uint_as_float(rr[x / 16][2 * (x % 16) + 1]) * p.scale);
+                    if (full_tile) {
+                        if (leader) bulk_wait_group_read<0>();
+                        if (!group_sync(&sb.epi_sync, sync_phase, abort)) { ok = false; break; }
+                        uint8_t *srow = stage + row * 128;
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            *reinterpret_cast<uint4 *>(srow + ((u ^ (row & 7)) << 4)) =
+                                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                        fence_proxy_async_smem();
+                        if (!group_sync(&sb.epi_sync, sync_phase, abort)) { ok = false; break; }
+                        if (leader) {
+                            tma_store_2d(&tm_dq, stage, r.h * D + 64 * c, r.s0 + r.t * kTile);
+                            bulk_commit_group();
+                        }
+                    } else if (valid_k) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(dq + grow * D + 64 * c);
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                    }
+                }
+                if (!ok) break;
+            }
             // 64 columns at a time: dV chunks, then dK chunks (scaled by 1/sqrt(D))
 #pragma unroll 1
             for (int part = 0; part < 2 * Lay::kChunks; ++part) {
@@ -594,16 +695,46 @@ cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, 
 {
     using Lay = DkvLayout<D>;
     // the rotary epilogue exists for block attention only, cross-attention for the generalized one
-    auto kern = (A == kSoftmax && p.rope_cos)        ? bwd_dkdv_sm100_kernel<D, A == kSoftmax, A, false>
-                : (A != kSoftmax && p.other_offsets) ? bwd_dkdv_sm100_kernel<D, false, A, A != kSoftmax>
-                                                     : bwd_dkdv_sm100_kernel<D, false, A, false>;
+    auto kern = (A == kSoftmax && p.rope_cos)        ? bwd_dkdv_sm100_kernel<D, A == kSoftmax, A, false, false>
+                : (A != kSoftmax && p.other_offsets) ? bwd_dkdv_sm100_kernel<D, false, A, A != kSoftmax, false>
+                                                     : bwd_dkdv_sm100_kernel<D, false, A, false, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
+    if (e != cudaSuccess) return e;
+    // the last three arguments belong to the fused backward; valid maps stand in, unread
+    kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, tdk, tdv, tqt, tdot, p, nlse2, neg_delta,
+                                                          static_cast<__nv_bfloat16 *>(dk),
+                                                          static_cast<__nv_bfloat16 *>(dv), tk, tdk, nullptr);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_bwd_fused_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                   const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
+                                   const CUtensorMap &tqt, const CUtensorMap &tdot, const CUtensorMap &tkt,
+                                   const CUtensorMap &tdq, const Problem &p, const float *nlse2,
+                                   const float *neg_delta, void *dq, void *dk, void *dv, int num_sms,
+                                   cudaStream_t stream)
+{
+    using Lay = DkvLayout<D, true>;
+    auto kern = bwd_dkdv_sm100_kernel<D, false, kSoftmax, false, true>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess) return e;
     kern<<<num_sms, Lay::kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, tdo, tdk, tdv, tqt, tdot, p, nlse2, neg_delta,
                                                           static_cast<__nv_bfloat16 *>(dk),
-                                                          static_cast<__nv_bfloat16 *>(dv));
+                                                          static_cast<__nv_bfloat16 *>(dv), tkt, tdq,
+                                                          static_cast<__nv_bfloat16 *>(dq));
     return cudaGetLastError();
 }
+template cudaError_t launch_bwd_fused_sm100<64>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
+                                                const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
+                                                const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
+                                                const CUtensorMap &, const Problem &, const float *, const float *,
+                                                void *, void *, void *, int, cudaStream_t);
+template cudaError_t launch_bwd_fused_sm100<128>(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
+                                                 const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
+                                                 const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
+                                                 const CUtensorMap &, const Problem &, const float *, const float *,
+                                                 void *, void *, void *, int, cudaStream_t);
 
 #define BA_DKDV_INST(D, A)                                                                                   \
     template cudaError_t launch_bwd_dkdv_sm100<D, A>(const CUtensorMap &, const CUtensorMap &,                \

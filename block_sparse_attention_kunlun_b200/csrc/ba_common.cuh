@@ -64,8 +64,15 @@ __host__ __device__ __forceinline__ bool visible(int64_t i, int64_t j, int64_t b
 //                       partial query tile of q (dout), zeros past the example
 //                       (the dK/dV pass reads that tile from here)
 struct WorkspaceLayout {
-    size_t status, tile_prefix, tile_info, pair_prefix, pair_info, delta, nlse2, tail_q, tail_do, total;
+    size_t status, tile_prefix, tile_info, pair_prefix, pair_info, delta, nlse2, tail_q, tail_do, tail_k, total;
 };
+
+// Masks under which every 128-row query tile sees only its own key tile: window 1
+// with blocks that divide the tile. The bf16 backward then runs as one fused pass.
+__host__ __device__ inline bool diagonal_tiles(int64_t block, int64_t window)
+{
+    return window == 1 && block <= kTile && kTile % block == 0;
+}
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -81,7 +88,8 @@ __host__ __device__ inline int64_t max_pairs(int64_t batch, int64_t total_tokens
 
 __host__ __device__ inline WorkspaceLayout workspace_layout(int64_t batch, int64_t total_tokens,
                                                             int64_t heads, int64_t head_dim,
-                                                            bool with_delta, bool tail_rows = false)
+                                                            bool with_delta, bool tail_rows = false,
+                                                            bool tail_k = false)
 {
     WorkspaceLayout w;
     w.status = 0;
@@ -99,9 +107,12 @@ __host__ __device__ inline WorkspaceLayout workspace_layout(int64_t batch, int64
     w.nlse2 = off;
     if (with_delta) off = align256(off + sizeof(float) * size_t(heads * total_tokens));
     const size_t tail_bytes = tail_rows ? align256(size_t(batch) * kTile * size_t(heads * head_dim) * 2) : 0;
+    // the partial tiles staged zero-padded: query tiles (q, dout) for the dK/dV pass, and the
+    // key tile (k) for the fused backward
     w.tail_q = off;
     w.tail_do = off + tail_bytes;
-    w.total = off + 2 * tail_bytes;
+    w.tail_k = off + 2 * tail_bytes;
+    w.total = off + (tail_k ? 3 : 2) * tail_bytes;
     return w;
 }
 

@@ -77,7 +77,12 @@ struct FwdBarriers {
     uint64_t q_full[2], q_empty[2]; // query tile of group w, released after its last S
     uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
     uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-    uint64_t o_ready[2]; // group w's softmax is done with its item: inv_l[w] holds 1 / l
+    // group w's softmax is done with its item: inv_l[w] holds 1 / l. A group may finish its next
+    // item (whose S needs nothing from the epilogue) before the epilogue has taken this one, so it
+    // writes inv_l[w] and arrives on o_ready[w] only once the epilogue has read the previous value
+    // (l_free[w]); o_ready[w] is then never two phases ahead of the epilogue's wait.
+    uint64_t o_ready[2], l_free[2];
+    uint32_t handed[8]; // per softmax warp: items handed to the epilogue (kept here, not in registers)
     uint64_t epi_sync;   // group barrier of the epilogue warpgroup
     uint64_t tail;       // the TMA warp's own barrier for a V tile whose last rows it clears
     uint64_t sf_ready;   // MXFP8: the item's scale factors (Q tile and first K tile) are in TMEM
@@ -125,6 +130,7 @@ __global__ void __launch_bounds__(512, 1)
             mbar_init(&sb.o_final[w], 1);
             mbar_init(&sb.o_free[w], 4);
             mbar_init(&sb.o_ready[w], 4);
+            mbar_init(&sb.l_free[w], 4);
         }
         for (int i = 0; i < S; ++i) {
             mbar_init(&sb.k_full[i], 1);
@@ -135,6 +141,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(&sb.epi_sync, 128);
         mbar_init(&sb.tail, 1);
         mbar_init(&sb.sf_ready, 4);
+        for (int i = 0; i < 8; ++i) sb.handed[i] = 0;
         sb.abort = 0;
         fence_mbar_init();
     }
@@ -559,7 +566,10 @@ __global__ void __launch_bounds__(512, 1)
                 if (lane == 0) mbar_arrive(&sb.p_full[w]);
             }
             if (!ok) break;
-            // hand 1 / l to the epilogue warps, write lse, and go on with the next item
+            // hand 1 / l to the epilogue warps (once they have read the previous item's), write lse,
+            // and go on with the next item
+            const uint32_t gi = sb.handed[warp];
+            if (!mbar_wait(&sb.l_free[w], (gi & 1) ^ 1, abort)) { ok = false; break; }
             if constexpr (A == kSoftmax) {
                 sb.inv_l[w][row] = valid ? 1.f / l : 0.f;
                 if (valid)
@@ -568,7 +578,10 @@ __global__ void __launch_bounds__(512, 1)
                 sb.inv_l[w][row] = valid ? 1.f : 0.f;
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sb.o_ready[w]);
+            if (lane == 0) {
+                mbar_arrive(&sb.o_ready[w]);
+                sb.handed[warp] = gi + 1;
+            }
         }
     } else {
         warpgroup_regs_dec<Lay::kRegsEpi>();
@@ -587,14 +600,21 @@ __global__ void __launch_bounds__(512, 1)
         while (ok && items.advance(r, sb.ring, abort, ok)) {
             const bool second = !kMx && pair_has_second(r);
             for (int w = 0; w < (second ? 2 : 1) && ok; ++w) {
-                if (!mbar_wait(&sb.o_ready[w], done[w] & 1, abort) ||
-                    !mbar_wait(&sb.o_final[w], done[w] & 1, abort)) {
+                // 1 / l first, released at once so the softmax may write the next item's, then
+                // the item's last P V
+                if (!mbar_wait(&sb.o_ready[w], done[w] & 1, abort)) {
+                    ok = false;
+                    break;
+                }
+                const float inv_l = sb.inv_l[w][row];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sb.l_free[w]);
+                if (!mbar_wait(&sb.o_final[w], done[w] & 1, abort)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 ++done[w];
-                const float inv_l = sb.inv_l[w][row];
                 const int t = r.t + w;
                 const int64_t i = int64_t(t) * kTile + row;
                 const bool valid = i < r.L;

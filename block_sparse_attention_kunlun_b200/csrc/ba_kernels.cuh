@@ -15,9 +15,14 @@ cudaError_t launch_worklist(const Problem &p, cudaStream_t stream, bool reset_st
 // Cross-attention: zero the rows (of a, and of b unless nullptr) of examples whose other side is empty.
 cudaError_t launch_zero_unpaired_rows(const int32_t *offs, const int32_t *other, int32_t batch, size_t row_bytes,
                                       void *a, void *b, cudaStream_t stream);
-// The dK/dV pass's partial query tiles of a (q) and b (dout), zero-padded to 128 rows, into ta and tb.
+// The dK/dV pass's partial query tiles of a (q) and b (dout), zero-padded to 128 rows, into ta and tb;
+// with c (k) and tc given, the partial key tiles too (the fused backward).
 cudaError_t launch_stage_query_tails(const int32_t *offs, const uint8_t *skip, int32_t batch, size_t row_bytes,
-                                     const void *a, const void *b, void *ta, void *tb, cudaStream_t stream);
+                                     const void *a, const void *b, void *ta, void *tb, cudaStream_t stream,
+                                     const void *c = nullptr, void *tc = nullptr);
+// -Delta and -lse log2(e) of every row, [heads, total_tokens] (bf16 out and dout).
+cudaError_t launch_bwd_stats(const Problem &p, const void *out, const void *dout, const float *lse,
+                             float *neg_delta, float *nlse2, int num_sms, cudaStream_t stream);
 cudaError_t launch_wait_selftest(int *status, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_exp2_selftest(const float *x, float *y, int64_t n, cudaStream_t stream);
 cudaError_t launch_activation_selftest(int act, const float *x, float *y, float *dy, int64_t n, cudaStream_t stream);
@@ -61,6 +66,16 @@ template <int D, int A>
 cudaError_t launch_bwd_dq_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const CUtensorMap &tdo, const CUtensorMap &to, const Problem &p, const float *lse,
                                 float *neg_delta, float *nlse2, void *dq, int num_sms, cudaStream_t stream);
+// The fused backward (masks with diagonal_tiles(block, window); block attention,
+// no rotary): dQ, dK and dV in one pass. tkt maps the staged partial key tiles,
+// tdq the dq output.
+template <int D>
+cudaError_t launch_bwd_fused_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                   const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
+                                   const CUtensorMap &tqt, const CUtensorMap &tdot, const CUtensorMap &tkt,
+                                   const CUtensorMap &tdq, const Problem &p, const float *nlse2,
+                                   const float *neg_delta, void *dq, void *dk, void *dv, int num_sms,
+                                   cudaStream_t stream);
 template <int D, int A>
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,

@@ -96,8 +96,13 @@ typedef struct {
  * forward's lse in the form the dK/dV pass reads, and (bf16) 128 rows of q
  * and 128 of dout per example, 2 * batch * 128 * heads * head_dim bf16
  * values in all: each example's last query tile, when partial, staged with
- * zeros past the example's end for the key-side gradient pass. A batch of
- * more than 2^31 / 128 examples is BA_ERR_UNSUPPORTED.
+ * zeros past the example's end for the key-side gradient pass. With window 1
+ * and a block that divides 128 (every 128-row query tile then sees only its
+ * own key tile) the bf16 backward runs as one fused pass for dq, dk and dv,
+ * and the workspace also holds 128 staged rows of k per example (batch * 128
+ * * heads * head_dim more bf16 values), since that pass's dq sums over the
+ * partial key tile's rows. A batch of more than 2^31 / 128 examples is
+ * BA_ERR_UNSUPPORTED.
  */
 size_t ba_fwd_workspace_size(const ba_problem *p, int32_t block, int32_t window);
 size_t ba_bwd_workspace_size(const ba_problem *p, int32_t block, int32_t window);
@@ -138,9 +143,9 @@ ba_status ba_bwd(const ba_problem *p, const void *q, const void *k, const void *
  * writes the exact gradients dq, dk, dv of sum(out * dout).
  *  - BF16 only (BA_ERR_UNSUPPORTED for BA_F32); head_dim 64 or 128; no skip
  *    flags. Same tensor layouts, ownership and errors as ba_fwd / ba_bwd.
- *  - Workspace: ba_gdpa_workspace_size bytes, for either direction (the
- *    backward's size, which includes the staged query tiles described at
- *    ba_bwd_workspace_size).
+ *  - Workspace: ba_gdpa_workspace_size bytes, for either direction: the
+ *    staged query tiles described at ba_bwd_workspace_size, never its
+ *    staged k rows (the generalized attention has no fused backward).
  *  - act outside the enumeration: BA_ERR_INVALID_ARG.
  */
 typedef enum { BA_ACT_GELU = 1, BA_ACT_SILU = 2 } ba_activation;

@@ -47,10 +47,18 @@ def test_workspace_sizes():
     # and (bf16) 128 staged rows of q and of dout per example
     staged = 2 * 3 * 128 * 2 * 128 * 2
     assert f + 2 * 4 * 2 * 1000 + staged <= b <= f + 2 * 4 * 2 * 1000 + staged + 1024
+    # window 1 with blocks dividing 128 (each query tile sees only its own key tile): the fused
+    # backward stages the partial key tiles (k) as well; other masks do not
+    for blk in (1, 16, 64, 128):
+        assert ba.ba_bwd_workspace_size(p, blk, 1) == b + staged // 2
+        assert ba.ba_mx_bwd_workspace_size(p, blk, 1) == ba.ba_mx_bwd_workspace_size(p, 128, 2) + staged // 2
+    for blk, win in ((96, 1), (256, 1), (64, 2)):
+        assert ba.ba_bwd_workspace_size(p, blk, win) == b
     # float32 has no staged rows
     p32 = prob(batch=3, T=1000, H=2, D=64, dt=ba.BA_F32)
     f32, b32 = ba.ba_fwd_workspace_size(p32, 128, 2), ba.ba_bwd_workspace_size(p32, 128, 2)
     assert f32 + 2 * 4 * 2 * 1000 <= b32 <= f32 + 2 * 4 * 2 * 1000 + 512
+    assert ba.ba_bwd_workspace_size(p32, 64, 1) == b32
     # the generalized attention's workspace (either direction) is the backward's
     assert ba.ba_gdpa_workspace_size(p, 128, 2) == f + staged
     # the work table grows with the number of 128-row tiles

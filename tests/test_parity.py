@@ -114,6 +114,12 @@ EDGE = [
     (64, 1000000, 1, [700, 300]),        # one block: full causal attention
     (128, 64, 1000000, [600, 190]),      # window covers everything: full causal
     (64, 128, 2, [0, 0, 0, 200]),        # leading empty examples
+    # window 1 with blocks dividing 128: every query tile sees only its own key
+    # tile, and the backward runs as one fused pass
+    (64, 64, 1, [1, 127, 129, 640, 65, 300]),
+    (128, 32, 1, [1000, 33, 128, 257]),
+    (128, 128, 1, [129, 1, 500, 384]),
+    (64, 16, 1, [77, 256, 3]),
 ]
 
 
@@ -162,6 +168,34 @@ def test_forward_is_deterministic_and_status_ok():
     b = ba.block_attention_fwd(q, k, v, offs, w.block, w.window, workspace=ws)
     assert ba.ba_device_status(ws) == ba.BA_OK
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_repeated_steps_with_one_key_tile_per_item(block):
+    """Items of one key tile (window 1) make the forward's softmax fast next to its
+    epilogue, so a softmax group can finish its next item before the epilogue has
+    taken this one. Thirty fwd + bwd steps on 32 jagged histories must all report
+    a clean status and give bit-identical results (no item interferes with another)."""
+    w = CONFIGS[3].replace(block=block, window=1, batch=32)
+    lengths = make_inputs(CONFIGS[3])["lengths"][:32].tolist()
+    inp = make_inputs(w, lengths=lengths)
+    q, k, v, dout = (inp[n].cuda() for n in ("q", "k", "v", "dout"))
+    offs = inp["seq_offsets"].cuda()
+    prob = ba.make_problem(q, offs)
+    wf = ba.workspace_for(ba.ba_fwd_workspace_size(prob, block, 1), q.device)
+    wb = ba.workspace_for(ba.ba_bwd_workspace_size(prob, block, 1), q.device)
+    first = None
+    for step in range(30):
+        out, lse = ba.block_attention_fwd(q, k, v, offs, block, 1, workspace=wf)
+        assert ba.ba_device_status(wf) == ba.BA_OK, f"forward, step {step}"
+        dq, dk, dv = ba.block_attention_bwd(q, k, v, out, lse, dout, offs, block, 1, workspace=wb)
+        assert ba.ba_device_status(wb) == ba.BA_OK, f"backward, step {step}"
+        res = (out, lse, dq, dk, dv)
+        if first is None:
+            first = tuple(t.clone() for t in res)
+        else:
+            for name, a, b in zip(("out", "lse", "dq", "dk", "dv"), first, res):
+                assert torch.equal(a, b), f"{name} differs at step {step}"
 
 
 # ------------------------------------------------ full sizes, sampled rows ---
