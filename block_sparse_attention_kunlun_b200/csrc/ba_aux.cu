@@ -296,9 +296,10 @@ cudaError_t launch_stage_query_tails(const int32_t *offs, const uint8_t *skip, i
 
 // The fused backward's per-row statistics, which the dQ pass computes
 // otherwise: -Delta = -(dout . out) and -lse log2(e) of every (token, head)
-// row, written [heads, total_tokens]. D / 8 lanes per row, one 16-byte vector
-// of each operand per lane and row, two rows per lane in flight; rows of
-// skipped examples are computed too (nothing reads them).
+// row, written [heads, total_tokens]. One warp per (head, 32 consecutive
+// tokens): D / 8 lanes per token row, one 16-byte vector of each operand per
+// lane, and each output written as one 128-byte line. Rows of skipped
+// examples are computed too (nothing reads them).
 __device__ __forceinline__ float bf16x8_dot(const uint4 a, const uint4 b)
 {
     const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
@@ -319,32 +320,38 @@ __global__ void __launch_bounds__(256)
                      const float *__restrict__ lse, int32_t total_tokens, int32_t heads,
                      float *__restrict__ neg_delta, float *__restrict__ nlse2)
 {
-    constexpr int LPR = D / 8, RPW = 32 / LPR; // lanes per row, rows per warp and step
-    const int lane = threadIdx.x & 31, u = lane % LPR;
-    const int64_t nrows = int64_t(total_tokens) * heads;
-    const int64_t step = int64_t(gridDim.x) * (blockDim.x >> 5) * (2 * RPW);
-    for (int64_t base = (int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * (2 * RPW); base < nrows;
-         base += step) {
-        const int64_t rw[2] = {base + lane / LPR, base + RPW + lane / LPR};
-        uint4 o[2], g[2];
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            o[x] = g[x] = make_uint4(0u, 0u, 0u, 0u);
-            if (rw[x] < nrows) {
-                o[x] = __ldg(reinterpret_cast<const uint4 *>(out + rw[x] * D) + u);
-                g[x] = __ldg(reinterpret_cast<const uint4 *>(dout + rw[x] * D) + u);
+    constexpr int LPR = D / 8;      // lanes per row: one 16-byte vector each
+    constexpr int RPS = 32 / LPR;   // rows per load step
+    constexpr int STEPS = 32 / RPS; // load steps per task of 32 tokens
+    const int lane = threadIdx.x & 31, u = lane % LPR, sub = lane / LPR;
+    const int64_t T = total_tokens;
+    const int64_t ntasks = (T + 31) / 32 * heads;
+    const int64_t rs = int64_t(heads) * D; // elements from one token's row of a head to the next token's
+    // task = (32-token block, head), heads fastest: the warps of one token block read whole token rows
+    for (int64_t task = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); task < ntasks;
+         task += int64_t(gridDim.x) * (blockDim.x >> 5)) {
+        const int64_t tb = task / heads, h = task - tb * heads, t0 = tb * 32;
+        float mine = 0.f; // lane j ends with token t0 + j's dout . out
+#pragma unroll 4
+        for (int k = 0; k < STEPS; ++k) {
+            const int64_t t = t0 + k * RPS + sub;
+            float sum = 0.f;
+            if (t < T) {
+                const uint4 o4 = __ldg(reinterpret_cast<const uint4 *>(out + t * rs + h * D) + u);
+                const uint4 g4 = __ldg(reinterpret_cast<const uint4 *>(dout + t * rs + h * D) + u);
+                sum = bf16x8_dot(o4, g4);
             }
-        }
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            float sum = bf16x8_dot(o[x], g[x]);
 #pragma unroll
             for (int d = LPR / 2; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
-            if (u == 0 && rw[x] < nrows) {
-                const int64_t t = rw[x] / heads, h = rw[x] % heads, hr = h * int64_t(total_tokens) + t;
-                neg_delta[hr] = -sum;
-                nlse2[hr] = -lse[hr] * 1.4426950408889634f;
-            }
+            // token t0 + j was row j % RPS of step j / RPS, whose sum sits in lanes (j % RPS) * LPR ..
+            const float b = __shfl_sync(0xffffffffu, sum, (lane % RPS) * LPR);
+            if (lane / RPS == k) mine = b;
+        }
+        const int64_t t = t0 + lane;
+        if (t < T) {
+            const int64_t hr = h * T + t;
+            neg_delta[hr] = -mine;
+            nlse2[hr] = -lse[hr] * 1.4426950408889634f;
         }
     }
 }
@@ -361,9 +368,9 @@ static int grid_for_rows(int64_t nrows, int num_sms)
 cudaError_t launch_bwd_stats(const Problem &p, const void *out, const void *dout, const float *lse,
                              float *neg_delta, float *nlse2, int num_sms, cudaStream_t stream)
 {
-    const int64_t nrows = int64_t(p.total_tokens) * p.heads;
-    if (nrows == 0) return cudaSuccess;
-    const int g = grid_for_rows(nrows, num_sms);
+    const int64_t ntasks = (int64_t(p.total_tokens) + 31) / 32 * p.heads; // warps' tasks
+    if (ntasks == 0) return cudaSuccess;
+    const int g = grid_for_rows(ntasks, num_sms); // one task per warp, 8 warps per block, capped
     const auto *o = static_cast<const __nv_bfloat16 *>(out), *d = static_cast<const __nv_bfloat16 *>(dout);
     switch (p.head_dim) {
     case 64:
