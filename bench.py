@@ -331,16 +331,22 @@ KERNEL_NAMES = {"fwd": "fwd_bf16_sm100_kernel", "bwd_dq": "bwd_dq_sm100_kernel",
                 "bwd_dkdv": "bwd_dkdv_sm100_kernel"}
 
 
+def fused_backward(w, rope=False, gdpa=None):
+    """Whether ba_bwd runs this workload's backward as one fused pass (dQ, dK and dV)
+    after a per-row statistics pass, which then take the dQ and dK/dV profile slots:
+    bf16 block attention without rotation, window 1 and a block dividing 128 (every
+    128-row query tile sees only its own key tile)."""
+    return (w.dtype == torch.bfloat16 and not rope and not gdpa and w.window == 1
+            and w.block <= 128 and 128 % w.block == 0)
+
+
 class Runner:
     """Device buffers and one training step (ba_fwd + ba_bwd, or the rotary
     entry points) of one workload through the library's public API."""
 
     def __init__(self, ba, w, inp, dev, rope=False, gdpa=None, mx=False):
         self.ba, self.w, self.inp, self.dev, self.rope, self.gdpa, self.mx = ba, w, inp, dev, rope, gdpa, mx
-        # window 1 with blocks dividing 128: the bf16 backward is one fused pass (dQ, dK and dV)
-        # after a per-row statistics pass, which take the dQ and dK/dV profile slots
-        self.fused = (w.dtype == torch.bfloat16 and not rope and not gdpa and w.window == 1
-                      and w.block <= 128 and 128 % w.block == 0)
+        self.fused = fused_backward(w, rope, gdpa)
         self.kernel_names = dict(KERNEL_NAMES)
         if self.fused:
             self.kernel_names.update(bwd_dq="bwd_stats_kernel", bwd_dkdv="bwd_dkdv_sm100_kernel (fused dQ)")
