@@ -10,7 +10,7 @@ import torch
 
 import block_sparse_attention_kunlun_b200 as ba
 import oracle
-from block_sparse_attention_kunlun_b200.workloads import CONFIGS, make_inputs
+from block_sparse_attention_kunlun_b200.workloads import CONFIGS, draw_lengths, make_inputs
 from parity_util import check_abs, check_bf16, f64
 
 pytestmark = pytest.mark.gpu
@@ -177,7 +177,9 @@ def test_repeated_steps_with_one_key_tile_per_item(block):
     taken this one. Thirty fwd + bwd steps on 32 jagged histories must all report
     a clean status and give bit-identical results (no item interferes with another)."""
     w = CONFIGS[3].replace(block=block, window=1, batch=32)
-    lengths = make_inputs(CONFIGS[3])["lengths"][:32].tolist()
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(CONFIGS[3].seed)
+    lengths = draw_lengths(CONFIGS[3], gen)[:32].tolist()  # config 3's first 32 histories
     inp = make_inputs(w, lengths=lengths)
     q, k, v, dout = (inp[n].cuda() for n in ("q", "k", "v", "dout"))
     offs = inp["seq_offsets"].cuda()
